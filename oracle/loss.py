@@ -1,0 +1,121 @@
+"""Oracle for the multi-exit LM-head loss with online distillation.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+Definition followed.
+  * Logits per exit: l_m = W^m h_m with W^m in R^{V x D_m} ("Editing the methods
+    of sub-models are made of blocks", Modeling paragraph: every sub-model ends
+    in its own LM head; h_m is the block-m output o_m).
+  * Next-token cross-entropy at every exit (same paragraph).
+  * Distillation: the largest exit's softmax is the teacher and every smaller
+    exit gets a token-level cross-entropy against it, mixed with its own LM loss
+    with weight alpha_d ("Matryoshka Language Model Suites", agihunt.info
+    summary, distillation paragraph); the mix is (1 - alpha_d) next-token loss
+    + alpha_d cross-entropy to the largest exit ("Is nesting the cheapest way to
+    build a model suite?", section 4: 0.7 and 0.3 at alpha_d = 0.3); the
+    distillation term exists only for the smaller exits ("Visualizing Core
+    ideas", bullet (b)).
+  * Per-exit losses are summed with equal weight ("Matryoshka Language Model
+    Suites", limitations paragraph).
+
+Readings where the pages are silent: the teacher is stop-gradient; the
+distillation temperature is 1; every term is a mean over the T tokens;
+``grad_scale`` multiplies dL (so a caller can fold in a global token count).
+
+    CE_LM,m = mean_t ( lse(l_{m,t}) - l_{m,t,y_t} )
+    CE_KD,m = mean_t ( - sum_v p_{M,t,v} log q_{m,t,v} ),  m < M
+    L = sum_{m<M} [ (1 - alpha_d) CE_LM,m + alpha_d CE_KD,m ] + CE_LM,M
+
+Backward (derived by hand; the pages give no gradient), with q_m = softmax(l_m):
+    G_m = grad_scale/T * (q_m - (1 - alpha_d) onehot(y) - alpha_d p_M),  m < M
+    G_M = grad_scale/T * (q_M - onehot(y))
+    dh_m = G_m W^m,     dW^m = G_m^T h_m
+
+Tokens are independent, so the token loop below processes a block of rows at
+a time only to bound memory; each block is the plain definition.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        import torch
+        return a.detach().to(torch.float64).numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def logsumexp_rows(l: np.ndarray) -> np.ndarray:
+    """log sum_v exp(l[t, v]) per row, with the row max factored out."""
+    mx = np.max(l, axis=1)
+    return mx + np.log(np.sum(np.exp(l - mx[:, None]), axis=1))
+
+
+def softmax_rows(l: np.ndarray) -> np.ndarray:
+    return np.exp(l - logsumexp_rows(l)[:, None])
+
+
+def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
+                   rows=None, token_block=256):
+    """Multi-exit loss, per-token statistics and (optionally) gradients, fp64.
+
+    y: int [T] targets; h: list of M arrays [T, D_m]; W: list of M arrays [V, D_m].
+    rows: optional int array of token indices; when given, only those tokens are
+    evaluated (their per-token statistics and dh rows; the means and dW are then
+    over the selected tokens, normalised by the full T).
+
+    Returns a dict with
+      ce_lm [M], ce_kd [M-1], loss (scalar)         -- means over the tokens
+      lse [M, T'], tgt [M, T'], S [M-1, T']          -- per-token statistics,
+          S_m,t = sum_v p_{M,t,v} l_{m,t,v}
+      dh (list of [T', D_m]) and dW (list of [V, D_m]) when need_grad.
+    """
+    y = np.asarray(y, dtype=np.int64)
+    M = len(h)
+    T = y.shape[0]
+    idx = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    Tn = idx.shape[0]
+    Ws = [_f64(w) for w in W]
+    V = Ws[0].shape[0]
+    out = {
+        "lse": np.zeros((M, Tn)), "tgt": np.zeros((M, Tn)), "S": np.zeros((max(M - 1, 0), Tn)),
+        "ce_lm_sum": np.zeros(M), "ce_kd_sum": np.zeros(max(M - 1, 0)),
+    }
+    if need_grad:
+        out["dh"] = [np.zeros((Tn, w.shape[1])) for w in Ws]
+        out["dW"] = [np.zeros_like(w) for w in Ws]
+    g = grad_scale / T
+    for b0 in range(0, Tn, token_block):
+        sel = idx[b0:b0 + token_block]
+        n = sel.shape[0]
+        yb = y[sel]
+        hb = [_f64(hm[sel]) for hm in h]
+        logits = [hb[m] @ Ws[m].T for m in range(M)]           # [n, V] each
+        lse = [logsumexp_rows(l) for l in logits]
+        logq = [logits[m] - lse[m][:, None] for m in range(M)]
+        pM = np.exp(logq[M - 1])                                # teacher softmax
+        ar = np.arange(n)
+        for m in range(M):
+            out["lse"][m, b0:b0 + n] = lse[m]
+            out["tgt"][m, b0:b0 + n] = logits[m][ar, yb]
+            out["ce_lm_sum"][m] += np.sum(lse[m] - logits[m][ar, yb])
+        for m in range(M - 1):
+            out["S"][m, b0:b0 + n] = np.sum(pM * logits[m], axis=1)
+            out["ce_kd_sum"][m] += np.sum(-np.sum(pM * logq[m], axis=1))
+        if need_grad:
+            onehot = np.zeros((n, V))
+            onehot[ar, yb] = 1.0
+            for m in range(M):
+                q = np.exp(logq[m])
+                if m < M - 1:
+                    G = g * (q - (1.0 - alpha_d) * onehot - alpha_d * pM)
+                else:
+                    G = g * (q - onehot)
+                out["dh"][m][b0:b0 + n] = G @ Ws[m]
+                out["dW"][m] += G.T @ hb[m]
+    out["ce_lm"] = out["ce_lm_sum"] / T
+    out["ce_kd"] = out["ce_kd_sum"] / T
+    out["loss"] = float(np.sum((1.0 - alpha_d) * out["ce_lm"][:M - 1])
+                        + np.sum(alpha_d * out["ce_kd"]) + out["ce_lm"][M - 1])
+    return out

@@ -1,0 +1,232 @@
+"""Pins for the multi-exit loss oracle.
+
+Closed forms, special cases, brute-force enumeration on V <= 16 and finite
+differences, chosen so a dropped term, a swapped mixing weight, a wrong sign or
+a transposed operand in the oracle fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import multiexit_loss, softmax_rows
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_figures.json")
+
+
+def _rand_suite(M=3, T=6, D=(3, 5, 8), V=11, seed=0, scale=1.0):
+    rng = np.random.default_rng(seed)
+    y = rng.integers(0, V, size=T)
+    h = [rng.normal(0, 2.0, size=(T, d)) for d in D[:M]]
+    W = [scale * rng.normal(0, 1.0 / math.sqrt(d), size=(V, d)) for d in D[:M]]
+    return y, h, W
+
+
+def _softplus(z):
+    return math.log1p(math.exp(z))
+
+
+def _sig(z):
+    return 1.0 / (1.0 + math.exp(-z))
+
+
+def test_two_class_closed_form_with_page_mix():
+    # V=2, one token, target 0; teacher logits (a, 0), student logits (b, 0).
+    # With the pages' mix (0.7 next-token + 0.3 cross-entropy to the largest exit):
+    #   CE_LM = softplus(-logit gap), CE_KD = -(s(a) log s(b) + s(-a) log s(-b)).
+    fig = json.load(open(GOLDEN))
+    alpha = fig["alpha_d"]["value"]
+    assert (fig["mix_weights"]["lm"], fig["mix_weights"]["kd"]) == (0.7, 0.3)
+    a, b = 2.0, -1.0
+    y = np.array([0])
+    h = [np.array([[b]]), np.array([[a]])]
+    W = [np.array([[1.0], [0.0]]), np.array([[1.0], [0.0]])]
+    r = multiexit_loss(y, h, W, alpha_d=alpha)
+    ce_lm1, ce_lm2 = _softplus(-b), _softplus(-a)
+    ce_kd1 = -(_sig(a) * math.log(_sig(b)) + _sig(-a) * math.log(_sig(-b)))
+    L = 0.7 * ce_lm1 + 0.3 * ce_kd1 + ce_lm2
+    np.testing.assert_allclose(r["ce_lm"], [ce_lm1, ce_lm2], rtol=1e-14)
+    np.testing.assert_allclose(r["ce_kd"], [ce_kd1], rtol=1e-14)
+    np.testing.assert_allclose(r["loss"], L, rtol=1e-14)
+    # dL/dh_1 = d/db: s(b) - 0.7 - 0.3 s(a); teacher is stop-gradient:
+    # dL/dh_2 = d/da of CE_LM,2 only: s(a) - 1
+    np.testing.assert_allclose(r["dh"][0][0, 0], _sig(b) - 0.7 - 0.3 * _sig(a), rtol=1e-13)
+    np.testing.assert_allclose(r["dh"][1][0, 0], _sig(a) - 1.0, rtol=1e-13)
+    # dW^1 rows: row 0 gets (q0 - 0.7 - 0.3 p0) * h, row 1 gets (q1 - 0.3 p1) * h
+    np.testing.assert_allclose(r["dW"][0][:, 0],
+                               [(_sig(b) - 0.7 - 0.3 * _sig(a)) * b,
+                                (_sig(-b) - 0.3 * _sig(-a)) * b], rtol=1e-13)
+
+
+def test_zero_heads_closed_form():
+    # W = 0 -> every softmax is uniform: lse = log V, CE_LM = CE_KD = log V,
+    # L = M log V; dh = 0; dW^m[v] = c_m/T sum_t (1/V - [y_t = v]) h_t with
+    # c_m = 1 - alpha_d for students and 1 for the teacher.
+    M, T, V, D = 3, 7, 13, (2, 3, 4)
+    rng = np.random.default_rng(1)
+    y = rng.integers(0, V, size=T)
+    h = [rng.normal(size=(T, d)) for d in D]
+    W = [np.zeros((V, d)) for d in D]
+    alpha = 0.3
+    r = multiexit_loss(y, h, W, alpha_d=alpha, grad_scale=1.0)
+    logV = math.log(V)
+    np.testing.assert_allclose(r["lse"], logV, rtol=1e-14)
+    np.testing.assert_allclose(r["ce_lm"], logV, rtol=1e-14)
+    np.testing.assert_allclose(r["ce_kd"], logV, rtol=1e-14)
+    np.testing.assert_allclose(r["loss"], M * logV, rtol=1e-14)
+    for m in range(M):
+        assert np.all(r["dh"][m] == 0.0)
+        c = (1 - alpha) if m < M - 1 else 1.0
+        exp = np.zeros((V, D[m]))
+        for t in range(T):
+            for v in range(V):
+                exp[v] += c / T * ((1.0 / V) - (1.0 if y[t] == v else 0.0)) * h[m][t]
+        np.testing.assert_allclose(r["dW"][m], exp, rtol=1e-12, atol=1e-15)
+
+
+def test_alpha_zero_is_plain_cross_entropy_textbook():
+    # alpha_d = 0: L = sum_m CE_LM,m, with CE written as log(sum exp) - l_y
+    # without any max shift (V <= 16 keeps exp in range).
+    y, h, W = _rand_suite(M=3, T=5, D=(2, 3, 4), V=9, seed=2)
+    r = multiexit_loss(y, h, W, alpha_d=0.0, need_grad=False)
+    tot = 0.0
+    for m in range(3):
+        s = 0.0
+        for t in range(5):
+            l = [sum(h[m][t, k] * W[m][v, k] for k in range(h[m].shape[1])) for v in range(9)]
+            s += math.log(sum(math.exp(z) for z in l)) - l[y[t]]
+        tot += s / 5
+    np.testing.assert_allclose(r["loss"], tot, rtol=1e-13)
+
+
+def test_student_equal_to_teacher_gives_teacher_entropy():
+    y, h, W = _rand_suite(M=2, T=8, D=(6, 6), V=15, seed=3)
+    h[0], W[0] = h[1].copy(), W[1].copy()
+    r = multiexit_loss(y, h, W, alpha_d=0.3)
+    H = 0.0
+    for t in range(8):
+        l = [float(np.dot(h[1][t], W[1][v])) for v in range(15)]
+        z = sum(math.exp(v) for v in l)
+        p = [math.exp(v) / z for v in l]
+        H += -sum(pi * math.log(pi) for pi in p)
+    np.testing.assert_allclose(r["ce_kd"][0], H / 8, rtol=1e-13)
+    # KD part of the student gradient vanishes: G_student = (1 - alpha) G_teacher
+    np.testing.assert_allclose(r["dh"][0], 0.7 * r["dh"][1], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(r["dW"][0], 0.7 * r["dW"][1], rtol=1e-12, atol=1e-15)
+
+
+def test_probabilities_sum_to_one():
+    rng = np.random.default_rng(4)
+    l = rng.normal(0, 30, size=(20, 50))
+    p = softmax_rows(l)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(p >= 0)
+
+
+def test_brute_force_enumeration_small_vocab():
+    # V <= 16, T <= 8, D <= 8: every quantity by explicit loops over v.
+    M, T, D, V, alpha = 3, 6, (2, 5, 8), 16, 0.3
+    y, h, W = _rand_suite(M=M, T=T, D=D, V=V, seed=5)
+    r = multiexit_loss(y, h, W, alpha_d=alpha)
+    ce_lm = [0.0] * M
+    ce_kd = [0.0] * (M - 1)
+    for t in range(T):
+        logits = [[sum(h[m][t, k] * W[m][v, k] for k in range(D[m])) for v in range(V)]
+                  for m in range(M)]
+        Z = [sum(math.exp(l) for l in logits[m]) for m in range(M)]
+        lse = [math.log(z) for z in Z]
+        pM = [math.exp(l) / Z[M - 1] for l in logits[M - 1]]
+        for m in range(M):
+            np.testing.assert_allclose(r["lse"][m, t], lse[m], rtol=1e-13)
+            np.testing.assert_allclose(r["tgt"][m, t], logits[m][y[t]], rtol=1e-13)
+            ce_lm[m] += lse[m] - logits[m][y[t]]
+        for m in range(M - 1):
+            Sm = sum(pM[v] * logits[m][v] for v in range(V))
+            np.testing.assert_allclose(r["S"][m, t], Sm, rtol=1e-12, atol=1e-14)
+            ce_kd[m] += -sum(pM[v] * (logits[m][v] - lse[m]) for v in range(V))
+    ce_lm = [c / T for c in ce_lm]
+    ce_kd = [c / T for c in ce_kd]
+    np.testing.assert_allclose(r["ce_lm"], ce_lm, rtol=1e-13)
+    np.testing.assert_allclose(r["ce_kd"], ce_kd, rtol=1e-13)
+    L = sum((1 - alpha) * ce_lm[m] + alpha * ce_kd[m] for m in range(M - 1)) + ce_lm[M - 1]
+    np.testing.assert_allclose(r["loss"], L, rtol=1e-13)
+
+
+def _teacher_fixed_loss(y, h, W, alpha, hM_fixed, WM_fixed, m_var):
+    """Loss with the teacher's softmax held at the given (fixed) parameters.
+
+    The teacher is stop-gradient, so finite differences of the student terms
+    must hold the teacher's distribution fixed while the student moves.
+    """
+    M = len(h)
+    r_t = multiexit_loss(y, h[:M - 1] + [hM_fixed], W[:M - 1] + [WM_fixed], alpha_d=alpha,
+                         need_grad=False)
+    return r_t["loss"]
+
+
+def test_gradients_match_finite_differences():
+    M, T, D, V, alpha, gs = 3, 4, (2, 3, 5), 7, 0.3, 1.7
+    y, h, W = _rand_suite(M=M, T=T, D=D, V=V, seed=6)
+    r = multiexit_loss(y, h, W, alpha_d=alpha, grad_scale=gs)
+    eps = 1e-6
+    # students: the teacher enters L through CE_LM,M (independent of students)
+    # and through p_M inside CE_KD (held fixed because it is stop-gradient;
+    # moving a student parameter does not change it anyway).
+    for m in range(M - 1):
+        for arr, grad in ((h, r["dh"][m]), (W, r["dW"][m])):
+            num = np.zeros_like(arr[m])
+            for idx in np.ndindex(arr[m].shape):
+                base = arr[m][idx]
+                arr[m][idx] = base + eps
+                lp = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False)["loss"]
+                arr[m][idx] = base - eps
+                lm = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False)["loss"]
+                arr[m][idx] = base
+                num[idx] = gs * (lp - lm) / (2 * eps)
+            np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-9)
+    # teacher: stop-gradient means only CE_LM,M depends on it -> a 1-exit loss
+    m = M - 1
+    for which in ("h", "W"):
+        arr = h if which == "h" else W
+        grad = r["dh"][m] if which == "h" else r["dW"][m]
+        num = np.zeros_like(arr[m])
+        for idx in np.ndindex(arr[m].shape):
+            base = arr[m][idx]
+            arr[m][idx] = base + eps
+            lp = multiexit_loss(y, [h[m]], [W[m]], need_grad=False)["loss"]
+            arr[m][idx] = base - eps
+            lm = multiexit_loss(y, [h[m]], [W[m]], need_grad=False)["loss"]
+            arr[m][idx] = base
+            num[idx] = gs * (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-9)
+
+
+def test_head_gradient_columns_sum_to_zero():
+    # sum_v G[t, v] = 0 for every token, hence sum_v dW^m[v, :] = 0.
+    y, h, W = _rand_suite(M=3, T=9, D=(4, 6, 8), V=21, seed=7)
+    r = multiexit_loss(y, h, W, alpha_d=0.3)
+    for m in range(3):
+        np.testing.assert_allclose(r["dW"][m].sum(axis=0), 0.0, atol=1e-14)
+
+
+def test_token_blocking_and_row_selection_do_not_change_results():
+    y, h, W = _rand_suite(M=3, T=23, D=(4, 6, 8), V=19, seed=8)
+    a = multiexit_loss(y, h, W, token_block=1)
+    b = multiexit_loss(y, h, W, token_block=256)
+    np.testing.assert_allclose(a["loss"], b["loss"], rtol=1e-13)
+    for m in range(3):
+        np.testing.assert_allclose(a["dW"][m], b["dW"][m], rtol=1e-12, atol=1e-15)
+    rows = np.array([3, 0, 22, 7])
+    c = multiexit_loss(y, h, W, rows=rows)
+    for m in range(3):
+        np.testing.assert_allclose(c["dh"][m], b["dh"][m][rows], rtol=1e-13)
+        np.testing.assert_allclose(c["lse"][m], b["lse"][m][rows], rtol=1e-13)
+
+
+def test_single_exit_has_no_distillation():
+    y, h, W = _rand_suite(M=1, T=5, D=(4,), V=10, seed=9)
+    r = multiexit_loss(y, h, W, alpha_d=0.3)
+    assert r["ce_kd"].shape == (0,)
+    np.testing.assert_allclose(r["loss"], r["ce_lm"][0], rtol=1e-15)
