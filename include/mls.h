@@ -1,0 +1,216 @@
+/*
+ * mls.h -- C ABI of libmls: the Matryoshka LM-suite junction and the
+ * multi-exit LM-head loss with online distillation, on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Matryoshka Language Model Suites", Godey & Artzi, 2026) stacks
+ * M blocks of strictly increasing width D_1 < ... < D_M.  Block m+1's input is
+ * the junction of block m's output with a fresh residual embedding, and every
+ * block ends in an exit with its own LM head.  This library implements the
+ * data-parallel hot path of one training step on those pieces:
+ *
+ *   mls_junction_fwd / mls_junction_bwd       -- the parameter-free junction
+ *   mls_multiexit_loss_fwd / _bwd             -- per-exit logits, next-token CE,
+ *                                                distillation from the largest
+ *                                                exit, and their gradients
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are row-major with tokens outermost, on the current CUDA
+ *     device, and owned by the caller.  The library keeps no pointer after a
+ *     call returns and allocates no device memory: scratch space is a caller
+ *     buffer sized by the matching *_workspace query.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on that stream; results are valid once the stream has
+ *     reached the end of the call.
+ *   - Argument errors (NULL pointers, non-positive sizes, widths that do not
+ *     increase, unsupported shapes or dtypes, misaligned pointers, workspace
+ *     too small) are reported synchronously and nothing is launched.
+ *   - Data errors found on the device (a token id or target outside [0, V))
+ *     never cause an out-of-range access: the affected token's outputs are
+ *     written as zeros and bit MLS_DEVFLAG_BAD_ID is OR-ed into *dev_status.
+ *     A device-side wait that runs past its limit sets MLS_DEVFLAG_TIMEOUT and
+ *     the kernel returns.  `dev_status` may be NULL (then nothing is recorded);
+ *     mls_status_read() collects it.
+ *   - Dtypes: MLS_F32 or MLS_BF16 inputs; accumulation is always fp32.
+ *   - Reentrant: no global mutable state besides one-time kernel attributes.
+ */
+#ifndef MLS_H_
+#define MLS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLS_OK = 0,
+  MLS_ERR_INVALID_ARG = 1,     /* NULL pointer, size <= 0, widths not increasing   */
+  MLS_ERR_UNSUPPORTED = 2,     /* shape/dtype/alignment outside the supported set */
+  MLS_ERR_WORKSPACE = 3,       /* workspace NULL or smaller than the query result */
+  MLS_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed            */
+  MLS_ERR_BAD_ID = 5,          /* reported by mls_status_read: id/target not in [0,V) */
+  MLS_ERR_DEVICE_TIMEOUT = 6,  /* reported by mls_status_read: a device wait gave up */
+  MLS_ERR_NO_DEVICE = 7        /* no sm_100 device is current                       */
+} mls_status;
+
+typedef enum { MLS_F32 = 0, MLS_BF16 = 1 } mls_dtype;
+
+/* Bits of the device status word. */
+#define MLS_DEVFLAG_BAD_ID  1
+#define MLS_DEVFLAG_TIMEOUT 2
+
+/* ------------------------------------------------------------------------ */
+/* Junction                                                                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * mls_junction_fwd -- block m output -> block m+1 input.
+ *
+ * Defined by "Visualizing the core idea of Matryoshka LM Suites" (How to read
+ * it, bottom panel: the junction) and "Matryoshka Language Model Suites"
+ * (agihunt.info summary, junction paragraph): the block output is rescaled to
+ * the L2 norm of the fresh residual embedding of the same token and the two
+ * are concatenated along channels; the junction has no parameters.  The
+ * residual table e_{m+1} has width delta = D_{m+1} - D_m and is indexed by the
+ * original token ids ("Editing the methods of sub-models are made of blocks",
+ * Modeling paragraph, after version).
+ *
+ * For every token t:
+ *   s_t = ||e_next[x_t]||_2 / max(||o_m[t]||_2, 1e-12)           (fp32)
+ *   y[t, 0:D_m]          = s_t * o_m[t]        (rounded to dt, nearest-even)
+ *   y[t, D_m:D_m+delta]  = e_next[x_t]         (bit-exact copy)
+ *
+ *   x         device int32 [T]           token ids, each in [0, V)
+ *   o_m       device dt [T, D_m]          block-m output
+ *   e_next    device dt [V, delta]        residual table of block m+1
+ *   y         device dt [T, D_m+delta]    output (must not alias the inputs)
+ *   scale_out device f32 [T] or NULL      s_t
+ *   Supported: D_m and delta multiples of 8 (bf16) or 4 (f32); every pointer
+ *   16-byte aligned.  Otherwise MLS_ERR_UNSUPPORTED.
+ */
+mls_status mls_junction_fwd(const int32_t* x, int64_t T,
+                            const void* o_m, int64_t D_m,
+                            const void* e_next, int64_t V, int64_t delta,
+                            void* y, float* scale_out,
+                            mls_dtype dt, int32_t* dev_status, void* stream);
+
+/*
+ * mls_junction_bwd -- gradients of mls_junction_fwd (derived from its
+ * definition; the pages give no gradient).  With u = o/||o||, e_hat = e/||e||
+ * (e_hat = 0 when ||e|| = 0), s as above and dy = [g_o ; g_e]:
+ *   do_m[t]    = s_t (g_o - u (u . g_o))
+ *   de_rows[t] = g_e + (u . g_o) e_hat
+ *   dE_table[v] (+)= sum over t with x_t = v of de_rows[t], summed in
+ *                    ascending t (deterministic; no floating-point atomics)
+ *
+ *   dy        device dt [T, D_m+delta]    gradient w.r.t. y
+ *   do_m      device dt [T, D_m]          output
+ *   de_rows   device dt [T, delta] or NULL
+ *   dE_table  device f32 [V, delta] or NULL;  accumulate_dE != 0 adds into it,
+ *             0 overwrites every row (rows of unused ids become 0)
+ *   workspace device, >= mls_junction_bwd_workspace(T, V) bytes when dE_table
+ *             is non-NULL (may be NULL otherwise)
+ * Supported shapes as for the forward pass.
+ */
+mls_status mls_junction_bwd(const int32_t* x, int64_t T,
+                            const void* o_m, int64_t D_m,
+                            const void* e_next, int64_t V, int64_t delta,
+                            const void* dy, void* do_m, void* de_rows,
+                            float* dE_table, int accumulate_dE,
+                            void* workspace, size_t ws_bytes,
+                            mls_dtype dt, int32_t* dev_status, void* stream);
+
+/* Scratch bytes mls_junction_bwd needs for the dE_table scatter. */
+mls_status mls_junction_bwd_workspace(int64_t T, int64_t V, size_t* bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Multi-exit LM-head loss                                                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Loss definition.  Logits per exit l_m = W^m h_m with W^m in R^{V x D_m}
+ * ("Editing the methods of sub-models are made of blocks", Modeling
+ * paragraph); next-token cross-entropy at every exit; the largest exit's
+ * softmax p_M teaches every smaller exit through a token-level cross-entropy
+ * mixed with weight alpha_d ("Matryoshka Language Model Suites", agihunt.info
+ * summary, distillation paragraph) as (1 - alpha_d) CE_LM + alpha_d CE_KD
+ * ("Is nesting the cheapest way to build a model suite?", section 4: 0.7 and
+ * 0.3); per-exit losses summed with equal weight (same summary, limitations
+ * paragraph).  Each term is a mean over the T tokens; the teacher is
+ * stop-gradient; the distillation temperature is 1.
+ *
+ *   CE_LM,m = mean_t ( lse_m,t - l_m,t,y_t )
+ *   CE_KD,m = mean_t ( lse_m,t - S_m,t ),  S_m,t = sum_v p_M,t,v l_m,t,v   (m < M)
+ *   L = sum_{m<M} [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m] + CE_LM,M
+ *
+ * The T x V logits are never written to memory.
+ *
+ * Common arguments
+ *   M          number of exits, 1 <= M <= 4
+ *   D          HOST int64 [M], strictly increasing widths
+ *   y_targets  device int32 [T] next-token targets in [0, V)
+ *   h          HOST array of M device pointers, h[m] is dt [T, D[m]]
+ *   W          HOST array of M device pointers, W[m] is dt [V, D[m]]
+ *   Supported: MLS_BF16 needs every D[m] % 64 == 0 and V % 128 == 0 (tensor
+ *   core path); MLS_F32 accepts any positive sizes (CUDA-core path).  All
+ *   device pointers 16-byte aligned.
+ */
+
+/* Workspace bytes for the forward and backward calls of this shape. */
+mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int64_t V,
+                                        mls_dtype dt, size_t* fwd_bytes, size_t* bwd_bytes);
+
+/*
+ * mls_multiexit_loss_fwd
+ *   losses  device f32 [2M]: CE_LM[0..M-1], CE_KD[0..M-2], L
+ *   stats   device f32 [3M-1, T]: rows 0..M-1 lse_m, rows M..2M-1 the target
+ *           logits l_m,y, rows 2M..3M-2 S_m.  Kept for the backward pass.
+ */
+mls_status mls_multiexit_loss_fwd(int M, int64_t T, int64_t V, const int64_t* D,
+                                  const int32_t* y_targets,
+                                  const void* const* h, const void* const* W,
+                                  float alpha_d, mls_dtype dt,
+                                  float* losses, float* stats,
+                                  void* workspace, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream);
+
+/*
+ * mls_multiexit_loss_bwd -- gradients of L times grad_scale.  With
+ * q_m = softmax(l_m):
+ *   G_m = grad_scale/T (q_m - (1 - alpha_d) onehot(y) - alpha_d p_M),  m < M
+ *   G_M = grad_scale/T (q_M - onehot(y))
+ *   dh[m] = G_m W^m           device dt [T, D[m]], overwritten
+ *   dW[m] (+)= G_m^T h_m      device f32 [V, D[m]]; accumulate_dW != 0 adds
+ *   stats is the forward call's output for the same inputs.
+ */
+mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
+                                  const int32_t* y_targets,
+                                  const void* const* h, const void* const* W,
+                                  float alpha_d, mls_dtype dt,
+                                  const float* stats, float grad_scale,
+                                  void* const* dh, float* const* dW, int accumulate_dW,
+                                  void* workspace, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Status                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Synchronises `stream`, copies *dev_status to *host_out and clears the device
+ * word.  Returns MLS_ERR_BAD_ID or MLS_ERR_DEVICE_TIMEOUT when the matching
+ * flag was set (timeout wins), MLS_OK when the word was 0.
+ */
+mls_status mls_status_read(int32_t* dev_status, void* stream, int32_t* host_out);
+
+/* Static English text for a status code. */
+const char* mls_status_string(mls_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int mls_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLS_H_ */

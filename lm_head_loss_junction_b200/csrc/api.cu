@@ -1,0 +1,249 @@
+// C ABI of libmls: argument checking, workspace sizing and kernel launch on
+// the caller's stream.  Every declaration, its meaning and its error behaviour
+// is documented in include/mls.h.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+
+#include "kernels.h"
+#include "mls.h"
+
+namespace {
+
+using mls::LossProblem;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Returns MLS_OK when the current device is a compute-capability 10.0 GPU
+// (the only target this library is built for).
+mls_status device_ok() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MLS_ERR_NO_DEVICE;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MLS_ERR_NO_DEVICE;
+  }
+  if (major != 10 || minor != 0) return MLS_ERR_NO_DEVICE;
+  return MLS_OK;
+}
+
+mls_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MLS_OK : MLS_ERR_CUDA; }
+
+mls_status check_junction_shape(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
+                                int64_t V, int64_t delta, mls_dtype dt) {
+  if (x == nullptr || o_m == nullptr || e_next == nullptr) return MLS_ERR_INVALID_ARG;
+  if (T <= 0 || D_m <= 0 || V <= 0 || delta <= 0) return MLS_ERR_INVALID_ARG;
+  if (dt != MLS_F32 && dt != MLS_BF16) return MLS_ERR_INVALID_ARG;
+  const int64_t per_vec = dt == MLS_BF16 ? 8 : 4;
+  if (D_m % per_vec != 0 || delta % per_vec != 0) return MLS_ERR_UNSUPPORTED;
+  if ((D_m + delta) / per_vec > INT_MAX || V > INT_MAX || T > (int64_t(1) << 40)) return MLS_ERR_UNSUPPORTED;
+  if (!aligned16(o_m) || !aligned16(e_next)) return MLS_ERR_UNSUPPORTED;
+  return MLS_OK;
+}
+
+mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y, const void* const* h,
+                         const void* const* W, float alpha_d, mls_dtype dt, int32_t* status, LossProblem* p) {
+  if (M < 1 || M > mls::kMaxExits) return M < 1 ? MLS_ERR_INVALID_ARG : MLS_ERR_UNSUPPORTED;
+  if (D == nullptr || h == nullptr || W == nullptr || y == nullptr) return MLS_ERR_INVALID_ARG;
+  if (T <= 0 || V <= 0) return MLS_ERR_INVALID_ARG;
+  if (dt != MLS_F32 && dt != MLS_BF16) return MLS_ERR_INVALID_ARG;
+  if (!(alpha_d == alpha_d)) return MLS_ERR_INVALID_ARG;   // NaN
+  for (int m = 0; m < M; ++m) {
+    if (D[m] <= 0) return MLS_ERR_INVALID_ARG;
+    if (m > 0 && D[m] <= D[m - 1]) return MLS_ERR_INVALID_ARG;   // widths strictly increase
+    if (h[m] == nullptr || W[m] == nullptr) return MLS_ERR_INVALID_ARG;
+    if (!aligned16(h[m]) || !aligned16(W[m])) return MLS_ERR_UNSUPPORTED;
+  }
+  if (T > INT_MAX || V > INT_MAX) return MLS_ERR_UNSUPPORTED;
+  if (dt == MLS_BF16) {
+    if (V % 128 != 0) return MLS_ERR_UNSUPPORTED;
+    for (int m = 0; m < M; ++m)
+      if (D[m] % 64 != 0 || D[m] > 65536) return MLS_ERR_UNSUPPORTED;
+    if (static_cast<double>(V) * static_cast<double>(T) >= 9.0e15) return MLS_ERR_UNSUPPORTED;
+  }
+  p->M = M;
+  p->T = T;
+  p->V = V;
+  for (int m = 0; m < M; ++m) {
+    p->D[m] = D[m];
+    p->h[m] = h[m];
+    p->W[m] = W[m];
+  }
+  p->y = y;
+  p->alpha_d = alpha_d;
+  p->status = status;
+  return MLS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mls_version(void) { return 100; }
+
+const char* mls_status_string(mls_status s) {
+  switch (s) {
+    case MLS_OK: return "ok";
+    case MLS_ERR_INVALID_ARG: return "invalid argument";
+    case MLS_ERR_UNSUPPORTED: return "unsupported shape, dtype or alignment";
+    case MLS_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLS_ERR_CUDA: return "CUDA runtime error";
+    case MLS_ERR_BAD_ID: return "token id or target outside [0, V)";
+    case MLS_ERR_DEVICE_TIMEOUT: return "a device-side wait ran past its limit";
+    case MLS_ERR_NO_DEVICE: return "no compute-capability 10.0 device is current";
+  }
+  return "unknown status";
+}
+
+mls_status mls_junction_fwd(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
+                            int64_t V, int64_t delta, void* y, float* scale_out, mls_dtype dt,
+                            int32_t* dev_status, void* stream) {
+  mls_status st = check_junction_shape(x, T, o_m, D_m, e_next, V, delta, dt);
+  if (st != MLS_OK) return st;
+  if (y == nullptr) return MLS_ERR_INVALID_ARG;
+  if (!aligned16(y)) return MLS_ERR_UNSUPPORTED;
+  if ((st = device_ok()) != MLS_OK) return st;
+  mls::JunctionArgs a{};
+  a.bf16 = dt == MLS_BF16;
+  a.x = x;
+  a.T = T;
+  a.D = D_m;
+  a.V = V;
+  a.delta = delta;
+  a.o = o_m;
+  a.E = e_next;
+  a.y = y;
+  a.scale_out = scale_out;
+  a.status = dev_status;
+  return from_cuda(mls::launch_junction_fwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+mls_status mls_junction_bwd_workspace(int64_t T, int64_t V, size_t* bytes) {
+  if (bytes == nullptr || T <= 0 || V <= 0) return MLS_ERR_INVALID_ARG;
+  *bytes = mls::junction_scatter_bytes(T);
+  return MLS_OK;
+}
+
+mls_status mls_junction_bwd(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
+                            int64_t V, int64_t delta, const void* dy, void* do_m, void* de_rows, float* dE_table,
+                            int accumulate_dE, void* workspace, size_t ws_bytes, mls_dtype dt,
+                            int32_t* dev_status, void* stream) {
+  mls_status st = check_junction_shape(x, T, o_m, D_m, e_next, V, delta, dt);
+  if (st != MLS_OK) return st;
+  if (dy == nullptr || do_m == nullptr) return MLS_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(do_m) || (de_rows != nullptr && !aligned16(de_rows)) ||
+      (dE_table != nullptr && !aligned16(dE_table)))
+    return MLS_ERR_UNSUPPORTED;
+  if (T > INT_MAX) return MLS_ERR_UNSUPPORTED;
+  if (dE_table != nullptr) {
+    if (workspace == nullptr || ws_bytes < mls::junction_scatter_bytes(T)) return MLS_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
+  }
+  if ((st = device_ok()) != MLS_OK) return st;
+  mls::JunctionArgs a{};
+  a.bf16 = dt == MLS_BF16;
+  a.x = x;
+  a.T = T;
+  a.D = D_m;
+  a.V = V;
+  a.delta = delta;
+  a.o = o_m;
+  a.E = e_next;
+  a.dy = dy;
+  a.do_out = do_m;
+  a.de_out = de_rows;
+  a.dE = dE_table;
+  a.accumulate_dE = accumulate_dE;
+  a.workspace = workspace;
+  a.status = dev_status;
+  return from_cuda(mls::launch_junction_bwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int64_t V, mls_dtype dt,
+                                        size_t* fwd_bytes, size_t* bwd_bytes) {
+  if (fwd_bytes == nullptr || bwd_bytes == nullptr) return MLS_ERR_INVALID_ARG;
+  const void* dummy[mls::kMaxExits] = {&fwd_bytes, &fwd_bytes, &fwd_bytes, &fwd_bytes};
+  // The pointer arrays only need to be non-null and aligned for the shape check.
+  alignas(16) static const char probe[16] = {0};
+  for (auto& d : dummy) d = probe;
+  LossProblem p{};
+  mls_status st = build_problem(M, T, V, D, reinterpret_cast<const int32_t*>(probe), dummy, dummy, 0.f, dt,
+                                nullptr, &p);
+  if (st != MLS_OK) return st;
+  if (dt == MLS_BF16) {
+    *fwd_bytes = mls::loss_tc_fwd_bytes(p);
+    *bwd_bytes = mls::loss_tc_bwd_bytes(p);
+  } else {
+    *fwd_bytes = mls::loss_simt_fwd_bytes(p);
+    *bwd_bytes = mls::loss_simt_bwd_bytes(p);
+  }
+  return MLS_OK;
+}
+
+mls_status mls_multiexit_loss_fwd(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y_targets,
+                                  const void* const* h, const void* const* W, float alpha_d, mls_dtype dt,
+                                  float* losses, float* stats, void* workspace, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream) {
+  LossProblem p{};
+  mls_status st = build_problem(M, T, V, D, y_targets, h, W, alpha_d, dt, dev_status, &p);
+  if (st != MLS_OK) return st;
+  if (losses == nullptr || stats == nullptr) return MLS_ERR_INVALID_ARG;
+  if (!aligned16(stats)) return MLS_ERR_UNSUPPORTED;
+  const size_t need = dt == MLS_BF16 ? mls::loss_tc_fwd_bytes(p) : mls::loss_simt_fwd_bytes(p);
+  if (workspace == nullptr || ws_bytes < need) return MLS_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
+  if ((st = device_ok()) != MLS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dt == MLS_BF16) {
+    if (!mls::tensor_map_encoder_available()) return MLS_ERR_CUDA;
+    return from_cuda(mls::loss_tc_fwd(p, losses, stats, workspace, s));
+  }
+  return from_cuda(mls::loss_simt_fwd(p, losses, stats, workspace, s));
+}
+
+mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y_targets,
+                                  const void* const* h, const void* const* W, float alpha_d, mls_dtype dt,
+                                  const float* stats, float grad_scale, void* const* dh, float* const* dW,
+                                  int accumulate_dW, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                  void* stream) {
+  LossProblem p{};
+  mls_status st = build_problem(M, T, V, D, y_targets, h, W, alpha_d, dt, dev_status, &p);
+  if (st != MLS_OK) return st;
+  if (stats == nullptr || dh == nullptr || dW == nullptr) return MLS_ERR_INVALID_ARG;
+  for (int m = 0; m < M; ++m) {
+    if (dh[m] == nullptr || dW[m] == nullptr) return MLS_ERR_INVALID_ARG;
+    if (!aligned16(dh[m]) || !aligned16(dW[m])) return MLS_ERR_UNSUPPORTED;
+  }
+  if (!(grad_scale == grad_scale)) return MLS_ERR_INVALID_ARG;
+  const size_t need = dt == MLS_BF16 ? mls::loss_tc_bwd_bytes(p) : mls::loss_simt_bwd_bytes(p);
+  if (workspace == nullptr || ws_bytes < need) return MLS_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
+  if ((st = device_ok()) != MLS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dt == MLS_BF16) {
+    if (!mls::tensor_map_encoder_available()) return MLS_ERR_CUDA;
+    return from_cuda(mls::loss_tc_bwd(p, stats, grad_scale, dh, dW, accumulate_dW, workspace, s));
+  }
+  return from_cuda(mls::loss_simt_bwd(p, stats, grad_scale, dh, dW, accumulate_dW, workspace, s));
+}
+
+mls_status mls_status_read(int32_t* dev_status, void* stream, int32_t* host_out) {
+  if (dev_status == nullptr || host_out == nullptr) return MLS_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MLS_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return MLS_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MLS_ERR_CUDA;
+  *host_out = v;
+  if (v & MLS_DEVFLAG_TIMEOUT) return MLS_ERR_DEVICE_TIMEOUT;
+  if (v & MLS_DEVFLAG_BAD_ID) return MLS_ERR_BAD_ID;
+  return MLS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,325 @@
+// fp32 CUDA-core path of the multi-exit loss (used for MLS_F32 inputs, where
+// bf16 tensor cores would change the arithmetic), plus the fixed-order loss
+// reduction shared with the tensor-core path.
+//
+// One thread block per token: every thread walks a strided subset of the
+// vocabulary, computes the logits of all exits for its entries, and keeps
+// online softmax statistics.  The teacher (largest exit) keeps its running
+// max m_T and sum z_T; every student also keeps A_s = sum_v exp(l_T,v - m_T)
+// l_s,v so that S_s = sum_v p_T,v l_s,v = A_s / z_T.  Partials are merged by a
+// fixed tree, so results are deterministic.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mls {
+
+namespace {
+
+constexpr int kSimtThreads = 256;
+
+struct SimtDev {
+  int M;
+  int64_t T, V;
+  int64_t D[kMaxExits];
+  int64_t Doff[kMaxExits];   // offsets of each exit's row in the staged h row
+  const int32_t* y;
+  const float* h[kMaxExits];
+  const float* W[kMaxExits];
+  float alpha_d;
+  int32_t* status;
+  float* dh[kMaxExits];
+  float* dW[kMaxExits];
+};
+
+__device__ __forceinline__ void merge_max_sum(float& m1, float& z1, float m2, float z2) {
+  const float m = fmaxf(m1, m2);
+  if (m == -INFINITY) return;
+  z1 = z1 * __expf(m1 - m) + z2 * __expf(m2 - m);
+  m1 = m;
+}
+
+// Quantities per thread, in shared memory for the tree merge:
+//   [0] m_T  [1] z_T  [2..2+M-2] A_s  then per student (m_s, z_s), then tgt[M]
+__global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev p, float* __restrict__ stats,
+                                                                  float* __restrict__ terms) {
+  extern __shared__ float sm[];
+  const int M = p.M;
+  const int S = M - 1;
+  const int64_t t = blockIdx.x;
+  const int tid = threadIdx.x;
+  float* hrow = sm;
+  int64_t hsum = 0;
+  for (int m = 0; m < M; ++m) hsum += p.D[m];
+  float* red = sm + hsum;  // [Q][kSimtThreads]
+  const int Q = 2 + S + 2 * S + M;
+  for (int m = 0; m < M; ++m)
+    for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) hrow[p.Doff[m] + k] = p.h[m][t * p.D[m] + k];
+  __syncthreads();
+
+  const int32_t yt = p.y[t];
+  const bool bad = yt < 0 || yt >= p.V;
+  float mT = -INFINITY, zT = 0.f;
+  float A[kMaxExits - 1], ms[kMaxExits - 1], zs[kMaxExits - 1], tgt[kMaxExits];
+  for (int s = 0; s < kMaxExits - 1; ++s) { A[s] = 0.f; ms[s] = -INFINITY; zs[s] = 0.f; }
+  for (int m = 0; m < kMaxExits; ++m) tgt[m] = 0.f;
+
+  for (int64_t v = tid; v < p.V; v += kSimtThreads) {
+    float l[kMaxExits];
+    for (int m = 0; m < M; ++m) {
+      const float* w = p.W[m] + v * p.D[m];
+      const float* hh = hrow + p.Doff[m];
+      float acc = 0.f;
+      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
+      l[m] = acc;
+    }
+    const float lT = l[M - 1];
+    if (lT > mT) {
+      const float r = __expf(mT - lT);
+      zT *= r;
+      for (int s = 0; s < S; ++s) A[s] *= r;
+      mT = lT;
+    }
+    const float pt = __expf(lT - mT);
+    zT += pt;
+    for (int s = 0; s < S; ++s) {
+      A[s] = fmaf(pt, l[s], A[s]);
+      if (l[s] > ms[s]) { zs[s] = zs[s] * __expf(ms[s] - l[s]); ms[s] = l[s]; }
+      zs[s] += __expf(l[s] - ms[s]);
+    }
+    if (v == yt)
+      for (int m = 0; m < M; ++m) tgt[m] = l[m];
+  }
+
+  // stage per-thread partials
+  red[0 * kSimtThreads + tid] = mT;
+  red[1 * kSimtThreads + tid] = zT;
+  for (int s = 0; s < S; ++s) red[(2 + s) * kSimtThreads + tid] = A[s];
+  for (int s = 0; s < S; ++s) {
+    red[(2 + S + 2 * s) * kSimtThreads + tid] = ms[s];
+    red[(2 + S + 2 * s + 1) * kSimtThreads + tid] = zs[s];
+  }
+  for (int m = 0; m < M; ++m) red[(2 + 3 * S + m) * kSimtThreads + tid] = tgt[m];
+  __syncthreads();
+  for (int stride = kSimtThreads / 2; stride > 0; stride >>= 1) {
+    if (tid < stride) {
+      const int o = tid + stride;
+      float m1 = red[tid], z1 = red[kSimtThreads + tid];
+      const float m2 = red[o], z2 = red[kSimtThreads + o];
+      const float mm = fmaxf(m1, m2);
+      const float r1 = (m1 == -INFINITY) ? 0.f : __expf(m1 - mm);
+      const float r2 = (m2 == -INFINITY) ? 0.f : __expf(m2 - mm);
+      red[tid] = mm;
+      red[kSimtThreads + tid] = z1 * r1 + z2 * r2;
+      for (int s = 0; s < S; ++s) {
+        float* a = red + (2 + s) * kSimtThreads;
+        a[tid] = a[tid] * r1 + a[o] * r2;
+        float* msp = red + (2 + S + 2 * s) * kSimtThreads;
+        float* zsp = msp + kSimtThreads;
+        float mA = msp[tid], zA = zsp[tid];
+        merge_max_sum(mA, zA, msp[o], zsp[o]);
+        msp[tid] = mA;
+        zsp[tid] = zA;
+      }
+      for (int m = 0; m < M; ++m) red[(2 + 3 * S + m) * kSimtThreads + tid] += red[(2 + 3 * S + m) * kSimtThreads + o];
+    }
+    __syncthreads();
+  }
+  (void)Q;
+  if (tid == 0) {
+    const float lseT = red[0] + logf(red[kSimtThreads]);
+    const float T_ = static_cast<float>(p.T);
+    (void)T_;
+    for (int m = 0; m < M; ++m) {
+      float lse;
+      if (m == M - 1) {
+        lse = lseT;
+      } else {
+        lse = red[(2 + S + 2 * m) * kSimtThreads] + logf(red[(2 + S + 2 * m + 1) * kSimtThreads]);
+      }
+      const float tg = red[(2 + 3 * S + m) * kSimtThreads];
+      stats[m * p.T + t] = lse;
+      stats[(M + m) * p.T + t] = bad ? 0.f : tg;
+      terms[m * p.T + t] = bad ? 0.f : lse - tg;
+    }
+    for (int s = 0; s < S; ++s) {
+      const float Sv = red[(2 + s) * kSimtThreads] / red[kSimtThreads];
+      const float lse = red[(2 + S + 2 * s) * kSimtThreads] + logf(red[(2 + S + 2 * s + 1) * kSimtThreads]);
+      stats[(2 * M + s) * p.T + t] = Sv;
+      terms[(M + s) * p.T + t] = bad ? 0.f : lse - Sv;
+    }
+    if (bad) set_flag(p.status, MLS_DEVFLAG_BAD_ID);
+  }
+}
+
+// Backward, one block per token: G'_m[t, :] into the workspace, then
+// dh_m[t] = alpha * G'_m[t, :] W^m.
+__global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p, const float* __restrict__ stats,
+                                                                 float alpha, float* __restrict__ G) {
+  extern __shared__ float sm[];
+  const int M = p.M;
+  const int64_t t = blockIdx.x;
+  const int tid = threadIdx.x;
+  float* hrow = sm;
+  for (int m = 0; m < M; ++m)
+    for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) hrow[p.Doff[m] + k] = p.h[m][t * p.D[m] + k];
+  __syncthreads();
+  const int32_t yt = p.y[t];
+  const bool bad = yt < 0 || yt >= p.V;
+  float lse[kMaxExits];
+  for (int m = 0; m < M; ++m) lse[m] = stats[m * p.T + t];
+  const float a = p.alpha_d;
+  for (int64_t v = tid; v < p.V; v += kSimtThreads) {
+    float l[kMaxExits];
+    for (int m = 0; m < M; ++m) {
+      const float* w = p.W[m] + v * p.D[m];
+      const float* hh = hrow + p.Doff[m];
+      float acc = 0.f;
+      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
+      l[m] = acc;
+    }
+    const float pT = __expf(l[M - 1] - lse[M - 1]);
+    const float hot = (v == yt) ? 1.f : 0.f;
+    for (int m = 0; m < M; ++m) {
+      float g;
+      if (m == M - 1) g = pT - hot;
+      else g = __expf(l[m] - lse[m]) - a * pT - (1.f - a) * hot;
+      G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : g;
+    }
+  }
+  __syncthreads();
+  for (int m = 0; m < M; ++m) {
+    const float* g = G + (static_cast<int64_t>(m) * p.T + t) * p.V;
+    for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) {
+      float acc = 0.f;
+      for (int64_t v = 0; v < p.V; ++v) acc = fmaf(g[v], p.W[m][v * p.D[m] + k], acc);
+      p.dh[m][t * p.D[m] + k] = bad ? 0.f : alpha * acc;
+    }
+  }
+  if (tid == 0 && bad) set_flag(p.status, MLS_DEVFLAG_BAD_ID);
+}
+
+// dW^m[v] (+)= alpha * sum_t G'_m[t, v] h_m[t], one block per (v, m).
+__global__ void __launch_bounds__(kSimtThreads) simt_dw_kernel(const SimtDev p, float alpha, const float* __restrict__ G,
+                                                               int accumulate) {
+  const int64_t v = blockIdx.x;
+  const int m = blockIdx.y;
+  const float* g = G + static_cast<int64_t>(m) * p.T * p.V + v;
+  for (int64_t k = threadIdx.x; k < p.D[m]; k += kSimtThreads) {
+    float acc = 0.f;
+    for (int64_t t = 0; t < p.T; ++t) acc = fmaf(g[t * p.V], p.h[m][t * p.D[m] + k], acc);
+    float* out = p.dW[m] + v * p.D[m] + k;
+    *out = accumulate ? *out + alpha * acc : alpha * acc;
+  }
+}
+
+// Fixed-order sum of the per-token loss terms; one block.
+__global__ void __launch_bounds__(1024) loss_reduce_kernel(const float* __restrict__ terms, int M, int64_t T,
+                                                           float alpha_d, float* __restrict__ losses) {
+  __shared__ float part[1024];
+  __shared__ float tot[2 * kMaxExits];
+  const int tid = threadIdx.x;
+  const int Q = 2 * M - 1;
+  for (int q = 0; q < Q; ++q) {
+    float s = 0.f;
+    for (int64_t i = tid; i < T; i += 1024) s += terms[q * T + i];
+    part[tid] = s;
+    __syncthreads();
+    for (int stride = 512; stride > 0; stride >>= 1) {
+      if (tid < stride) part[tid] += part[tid + stride];
+      __syncthreads();
+    }
+    if (tid == 0) tot[q] = part[0] / static_cast<float>(T);
+    __syncthreads();
+  }
+  if (tid == 0) {
+    float L = tot[M - 1];
+    for (int m = 0; m < M; ++m) losses[m] = tot[m];
+    for (int s = 0; s < M - 1; ++s) {
+      losses[M + s] = tot[M + s];
+      L += (1.f - alpha_d) * tot[s] + alpha_d * tot[M + s];
+    }
+    losses[2 * M - 1] = L;
+  }
+}
+
+SimtDev make_dev(const LossProblem& p) {
+  SimtDev d{};
+  d.M = p.M;
+  d.T = p.T;
+  d.V = p.V;
+  int64_t off = 0;
+  for (int m = 0; m < p.M; ++m) {
+    d.D[m] = p.D[m];
+    d.Doff[m] = off;
+    off += p.D[m];
+    d.h[m] = static_cast<const float*>(p.h[m]);
+    d.W[m] = static_cast<const float*>(p.W[m]);
+  }
+  d.y = p.y;
+  d.alpha_d = p.alpha_d;
+  d.status = p.status;
+  return d;
+}
+
+int64_t sum_d(const LossProblem& p) {
+  int64_t s = 0;
+  for (int m = 0; m < p.M; ++m) s += p.D[m];
+  return s;
+}
+
+cudaError_t ensure_smem(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+}  // namespace
+
+size_t loss_simt_fwd_bytes(const LossProblem& p) {
+  return static_cast<size_t>(2 * p.M - 1) * p.T * sizeof(float);
+}
+
+size_t loss_simt_bwd_bytes(const LossProblem& p) {
+  return static_cast<size_t>(p.M) * p.T * p.V * sizeof(float);
+}
+
+cudaError_t launch_loss_reduce(const float* terms, int M, int64_t T, float alpha_d, float* losses,
+                               cudaStream_t st) {
+  loss_reduce_kernel<<<1, 1024, 0, st>>>(terms, M, T, alpha_d, losses);
+  return cudaGetLastError();
+}
+
+cudaError_t loss_simt_fwd(const LossProblem& p, float* losses, float* stats, void* ws, cudaStream_t st) {
+  const SimtDev d = make_dev(p);
+  const int S = p.M - 1;
+  const int Q = 2 + S + 2 * S + p.M;
+  const size_t smem = (sum_d(p) + static_cast<size_t>(Q) * kSimtThreads) * sizeof(float);
+  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(simt_stats_kernel), smem);
+  if (err != cudaSuccess) return err;
+  float* terms = static_cast<float*>(ws);
+  simt_stats_kernel<<<static_cast<unsigned>(p.T), kSimtThreads, smem, st>>>(d, stats, terms);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  return launch_loss_reduce(terms, p.M, p.T, p.alpha_d, losses, st);
+}
+
+cudaError_t loss_simt_bwd(const LossProblem& p, const float* stats, float grad_scale, void* const* dh,
+                          float* const* dW, int accumulate, void* ws, cudaStream_t st) {
+  SimtDev d = make_dev(p);
+  for (int m = 0; m < p.M; ++m) {
+    d.dh[m] = static_cast<float*>(dh[m]);
+    d.dW[m] = dW[m];
+  }
+  const float alpha = grad_scale / static_cast<float>(p.T);
+  float* G = static_cast<float*>(ws);
+  const size_t smem = sum_d(p) * sizeof(float);
+  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(simt_grad_kernel), smem);
+  if (err != cudaSuccess) return err;
+  simt_grad_kernel<<<static_cast<unsigned>(p.T), kSimtThreads, smem, st>>>(d, stats, alpha, G);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  dim3 grid(static_cast<unsigned>(p.V), static_cast<unsigned>(p.M));
+  simt_dw_kernel<<<grid, kSimtThreads, 0, st>>>(d, alpha, G, accumulate);
+  return cudaGetLastError();
+}
+
+}  // namespace mls

@@ -1,0 +1,808 @@
+// Tensor-core (tcgen05 + TMEM + TMA) path of the multi-exit LM-head loss, bf16.
+//
+// Forward.  A persistent kernel walks (token tile of 128) x (vocab tile of 128)
+// output tiles.  For each tile it computes the logits of every exit into its
+// own TMEM region (teacher = largest exit first), and a 4-warp epilogue turns
+// them into per-row softmax statistics without ever writing logits out:
+//   teacher: lse_T over the tile and p~ = exp(l_T - max_T) kept in registers;
+//   student s: lse_s over the tile and Abar_s = sum_v p~_v l_s,v / sum_v p~_v.
+// A merge kernel combines the per-tile partials of every token exactly (log-
+// sum-exp merge, teacher-weighted mean of Abar), which gives lse_m and
+// S_m = sum_v p_T,v l_m,v; a fixed-order reduction gives the losses.
+//
+// Backward.  The same mainloop recomputes each tile's logits; the epilogue forms
+//   G'_m = q_m - (1 - alpha_d) onehot(y) - alpha_d p_T   (students)
+//   G'_T = p_T - onehot(y)                               (teacher, stop-gradient)
+// in bf16 into a workspace, and two tensor-core GEMMs per exit produce
+//   dh_m = (grad_scale/T) G'_m W^m   and   dW^m (+)= (grad_scale/T) G'_m^T h_m.
+//
+// Definitions: "Matryoshka Language Model Suites" (agihunt.info summary,
+// distillation paragraph), "Is nesting the cheapest way to build a model
+// suite?" (section 4, the 0.7/0.3 mix), "Editing the methods of sub-models are
+// made of blocks" (Modeling paragraph: one LM head W^m in R^{V x D_m} per exit).
+#include <cuda.h>
+#include <mutex>
+
+#include "kernels.h"
+#include "umma.cuh"
+
+namespace mls {
+
+namespace {
+
+constexpr int kBM = 128;          // token rows per tile (UMMA M)
+constexpr int kBK = 64;           // K per stage: one 128-byte swizzle row of bf16
+constexpr int kUK = 16;           // K per tcgen05.mma (kind::f16)
+constexpr int kLossBN = 128;      // vocabulary columns per tile
+constexpr int kLossStages = 6;
+constexpr int kThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ shared layouts
+struct LossMaps {
+  CUtensorMap h[kMaxExits];
+  CUtensorMap w[kMaxExits];
+};
+
+struct LossArgs {
+  int M;
+  int T;
+  int V;
+  int kblocks[kMaxExits];      // D_m / kBK
+  int n_tt, n_vt, num_tiles, group_tt;
+  const int32_t* y;
+  float alpha;                 // alpha_d
+  float* partial;              // forward: [n_vt][2M-1][T]
+  float* stats;                // forward: target rows written; backward: lse read
+  __nv_bfloat16* G;            // backward: [M][T][V]
+  int32_t* status;
+};
+
+struct __align__(1024) LossSmem {
+  uint8_t a[kLossStages][kBM * kBK * 2];
+  uint8_t b[kLossStages][kLossBN * kBK * 2];
+  uint64_t full[kLossStages];
+  uint64_t empty[kLossStages];
+  uint64_t tfull[kMaxExits];
+  uint64_t tempty[kMaxExits];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+enum LossMode { kModeStats = 0, kModeGrad = 1 };
+
+__device__ __forceinline__ void loss_tile_coords(int i, const LossArgs& a, int& tt, int& vt) {
+  const int per_group = a.group_tt * a.n_vt;
+  const int g = i / per_group;
+  const int first = g * a.group_tt;
+  const int gt = min(a.group_tt, a.n_tt - first);
+  const int r = i - g * per_group;
+  vt = r / gt;
+  tt = first + r % gt;
+}
+
+// All lanes of a warp wait; the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status) {
+  const bool ok = mbar_wait(bar, parity, abort, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Time-bounded wait that ignores the abort flag (used while draining).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+  int dummy = 0;
+  (void)mbar_wait(bar, parity, &dummy, status);
+}
+
+// ------------------------------------------------------------------ loss tile kernel
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_constant__ LossMaps maps,
+                                                                const LossArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  LossSmem& s = *reinterpret_cast<LossSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile int* abort = &s.abort;
+  const int M = a.M;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kLossStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int m = 0; m < kMaxExits; ++m) {
+      mbar_init(&s.tfull[m], 1);
+      mbar_init(&s.tempty[m], 4);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int m = 0; m < M; ++m) {
+      tma_prefetch_desc(&maps.h[m]);
+      tma_prefetch_desc(&maps.w[m]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        int tt, vt;
+        loss_tile_coords(tile, a, tt, vt);
+        for (int j = 0; j < M && ok; ++j) {
+          const int m = M - 1 - j;
+          for (int kb = 0; kb < a.kblocks[m]; ++kb) {
+            if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, a.status)) { ok = false; break; }
+            mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
+            tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, tt * kBM);
+            tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, vt * kLossBN);
+            ++issued;
+            if (++stage == kLossStages) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      if (!ok) {
+        // Let every load already issued land before the CTA can exit.
+        const uint32_t n = issued < kLossStages ? issued : kLossStages;
+        uint32_t st = stage, ph = phase;
+        for (uint32_t i = 0; i < n; ++i) {
+          if (st == 0) { st = kLossStages - 1; ph ^= 1; } else { --st; }
+          drain_wait(&s.full[st], ph, a.status);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kBM, kLossBN, false, false);
+      uint32_t stage = 0, phase = 0, iter = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x, ++iter) {
+        for (int j = 0; j < M && ok; ++j) {
+          const int m = M - 1 - j;
+          if (!mbar_wait(&s.tempty[m], (iter & 1) ^ 1, abort, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + static_cast<uint32_t>(m * kLossBN);
+          for (int kb = 0; kb < a.kblocks[m]; ++kb) {
+            if (!mbar_wait(&s.full[stage], phase, abort, a.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t da = smem_desc_sw128(smem_u32(s.a[stage]), 16, 1024);
+            const uint64_t db = smem_desc_sw128(smem_u32(s.b[stage]), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < kBK / kUK; ++k) {
+              // +32 bytes along K inside the 128-byte swizzled row
+              umma_bf16(d, da + static_cast<uint64_t>(k * 2), db + static_cast<uint64_t>(k * 2), idesc,
+                        (kb | k) != 0);
+            }
+            umma_commit(&s.empty[stage]);
+            if (++stage == kLossStages) { stage = 0; phase ^= 1; }
+          }
+          if (ok) umma_commit(&s.tfull[m]);
+        }
+      }
+      // Make sure every MMA issued has finished before TMEM is released.
+      umma_commit(&s.drain);
+      drain_wait(&s.drain, 0, a.status);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (4 warps)
+    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int Q = 2 * M - 1;
+    uint32_t iter = 0;
+    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x, ++iter) {
+      int tt, vt;
+      loss_tile_coords(tile, a, tt, vt);
+      const int t = tt * kBM + row;
+      const bool valid = t < a.T;
+      const int v0 = vt * kLossBN;
+      const int yt = valid ? __ldg(a.y + t) : -1;
+      const int yl = yt - v0;                  // target column inside this tile, if any
+      const bool has_tgt = valid && yl >= 0 && yl < kLossBN;
+
+      // ---------------- teacher
+      if (!warp_wait(&s.tfull[M - 1], iter & 1, abort, a.status)) break;
+      tc_fence_after();
+      float p[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + (M - 1) * kLossBN + c * 32, p[c]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tempty[M - 1]);
+
+      if (MODE == kModeStats) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mx = fmaxf(mx, p[c][j]);
+        if (has_tgt) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c * 32 + j == yl) a.stats[static_cast<int64_t>(M + M - 1) * a.T + t] = p[c][j];
+        }
+        const float mxs = mx * kLog2e;
+        float z = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            p[c][j] = exp2f(fmaf(p[c][j], kLog2e, -mxs));
+            z += p[c][j];
+          }
+        const float inv_z = 1.f / z;
+        if (valid) a.partial[(static_cast<int64_t>(vt) * Q + (M - 1)) * a.T + t] = mx + logf(z);
+
+        // ---------------- students, largest first
+        for (int sidx = M - 2; sidx >= 0; --sidx) {
+          if (!warp_wait(&s.tfull[sidx], iter & 1, abort, a.status)) break;
+          tc_fence_after();
+          float ms = -INFINITY, zs = 0.f, A = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float r[32];
+            tmem_ld32(lane_base + sidx * kLossBN + c * 32, r);
+            float cm = r[0];
+#pragma unroll
+            for (int j = 1; j < 32; ++j) cm = fmaxf(cm, r[j]);
+            const float mn = fmaxf(ms, cm);
+            const float mns = mn * kLog2e;
+            float zc = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              zc += exp2f(fmaf(r[j], kLog2e, -mns));
+              A = fmaf(p[c][j], r[j], A);
+            }
+            zs = zs * exp2f((ms - mn) * kLog2e) + zc;
+            ms = mn;
+            if (has_tgt && (yl >> 5) == c) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j == (yl & 31)) a.stats[static_cast<int64_t>(M + sidx) * a.T + t] = r[j];
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tempty[sidx]);
+          if (valid) {
+            a.partial[(static_cast<int64_t>(vt) * Q + sidx) * a.T + t] = ms + logf(zs);
+            a.partial[(static_cast<int64_t>(vt) * Q + M + sidx) * a.T + t] = A * inv_z;
+          }
+        }
+        if (*abort) break;
+      } else {
+        // ---------------- backward: G' tiles in bf16
+        const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
+        const float lTs = lseT * kLog2e;
+        const bool bad = valid && (yt < 0 || yt >= a.V);
+        const int64_t g_row = (static_cast<int64_t>(M - 1) * a.T + t) * a.V + v0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) p[c][j] = exp2f(fmaf(p[c][j], kLog2e, -lTs));
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float g0 = p[c][j] - ((c * 32 + j) == yl ? 1.f : 0.f);
+            float g1 = p[c][j + 1] - ((c * 32 + j + 1) == yl ? 1.f : 0.f);
+            if (bad) { g0 = 0.f; g1 = 0.f; }
+            packed[j / 2] = pack_bf16x2(g0, g1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(a.G + g_row + c * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+          }
+        }
+        const float al = a.alpha, one_m_al = 1.f - a.alpha;
+        for (int sidx = M - 2; sidx >= 0; --sidx) {
+          if (!warp_wait(&s.tfull[sidx], iter & 1, abort, a.status)) break;
+          tc_fence_after();
+          const float lse = valid ? a.stats[static_cast<int64_t>(sidx) * a.T + t] : 0.f;
+          const float ls = lse * kLog2e;
+          const int64_t row_off = (static_cast<int64_t>(sidx) * a.T + t) * a.V + v0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float r[32];
+            tmem_ld32(lane_base + sidx * kLossBN + c * 32, r);
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float g0 = exp2f(fmaf(r[j], kLog2e, -ls)) - al * p[c][j] -
+                         ((c * 32 + j) == yl ? one_m_al : 0.f);
+              float g1 = exp2f(fmaf(r[j + 1], kLog2e, -ls)) - al * p[c][j + 1] -
+                         ((c * 32 + j + 1) == yl ? one_m_al : 0.f);
+              if (bad) { g0 = 0.f; g1 = 0.f; }
+              packed[j / 2] = pack_bf16x2(g0, g1);
+            }
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(a.G + row_off + c * 32);
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tempty[sidx]);
+        }
+        if (*abort) break;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ merge kernel
+// Per token: combine the per-vocab-tile partials into lse_m and S_m, write the
+// stats rows and the per-token loss terms.
+__global__ void __launch_bounds__(256) loss_merge_kernel(const float* __restrict__ partial, int n_vt, int M,
+                                                         int T, int V, const int32_t* __restrict__ y,
+                                                         float* __restrict__ stats, float* __restrict__ terms,
+                                                         int32_t* status) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int Q = 2 * M - 1;
+  const int yt = y[t];
+  const bool bad = yt < 0 || yt >= V;
+  // teacher, with the teacher-weighted means of every student
+  float mT = -INFINITY, zT = 0.f;
+  float Sacc[kMaxExits - 1] = {0.f, 0.f, 0.f};
+  for (int i = 0; i < n_vt; ++i) {
+    const float l = partial[(static_cast<int64_t>(i) * Q + (M - 1)) * T + t];
+    if (l > mT) {
+      const float r = __expf(mT - l);
+      zT *= r;
+      for (int s = 0; s < M - 1; ++s) Sacc[s] *= r;
+      mT = l;
+    }
+    const float w = __expf(l - mT);
+    zT += w;
+    for (int s = 0; s < M - 1; ++s) Sacc[s] = fmaf(w, partial[(static_cast<int64_t>(i) * Q + M + s) * T + t], Sacc[s]);
+  }
+  const float lseT = mT + logf(zT);
+  stats[static_cast<int64_t>(M - 1) * T + t] = lseT;
+  if (bad) stats[static_cast<int64_t>(M + M - 1) * T + t] = 0.f;
+  terms[static_cast<int64_t>(M - 1) * T + t] = bad ? 0.f : lseT - stats[static_cast<int64_t>(2 * M - 1) * T + t];
+  for (int s = 0; s < M - 1; ++s) {
+    float ms = -INFINITY, zs = 0.f;
+    for (int i = 0; i < n_vt; ++i) {
+      const float l = partial[(static_cast<int64_t>(i) * Q + s) * T + t];
+      if (l > ms) { zs *= __expf(ms - l); ms = l; }
+      zs += __expf(l - ms);
+    }
+    const float lse = ms + logf(zs);
+    const float Sv = Sacc[s] / zT;
+    stats[static_cast<int64_t>(s) * T + t] = lse;
+    stats[static_cast<int64_t>(2 * M + s) * T + t] = Sv;
+    if (bad) stats[static_cast<int64_t>(M + s) * T + t] = 0.f;
+    terms[static_cast<int64_t>(s) * T + t] = bad ? 0.f : lse - stats[static_cast<int64_t>(M + s) * T + t];
+    terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : lse - Sv;
+  }
+  if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
+}
+
+// ------------------------------------------------------------------ GEMM kernel (dh, dW)
+// out[M x N] (+)= alpha * A[M x K] B[N x K]^T with bf16 operands in TMA boxes,
+// fp32 accumulation in TMEM (two accumulator buffers so the epilogue of one
+// tile overlaps the mainloop of the next).
+//   A_MN: A stored with M contiguous (boxes of 64 M x 64 K), else K contiguous
+//   B_MN: B stored with N contiguous, else K contiguous
+constexpr int kGemmStages = 4;
+
+struct GemmArgs {
+  int Mdim, Ndim, Kdim;
+  int n_mt, n_nt, num_tiles, group_m, kblocks;
+  void* out;
+  float alpha;
+  int accumulate;
+  int32_t* status;
+};
+
+template <int BN>
+struct __align__(1024) GemmSmem {
+  uint8_t a[kGemmStages][kBM * kBK * 2];
+  uint8_t b[kGemmStages][BN * kBK * 2];
+  uint64_t full[kGemmStages];
+  uint64_t empty[kGemmStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <bool A_MN, bool B_MN, int BN, bool OUT_BF16>
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                                                           const __grid_constant__ CUtensorMap map_b,
+                                                           const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  using Smem = GemmSmem<BN>;
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile int* abort = &s.abort;
+  constexpr uint32_t kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGemmStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 4);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  auto coords = [&](int i, int& mt, int& nt) {
+    const int per_group = g.group_m * g.n_nt;
+    const int gi = i / per_group;
+    const int first = gi * g.group_m;
+    const int gm = min(g.group_m, g.n_mt - first);
+    const int r = i - gi * per_group;
+    nt = r / gm;
+    mt = first + r % gm;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x) {
+        int mt, nt;
+        coords(tile, mt, nt);
+        for (int kb = 0; kb < g.kblocks; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, g.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&s.full[stage], (kBM + BN) * kBK * 2);
+          if (A_MN) {
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              tma_load_2d(&map_a, &s.full[stage], s.a[stage] + j * (64 * kBK * 2), mt * kBM + j * 64, kb * kBK);
+          } else {
+            tma_load_2d(&map_a, &s.full[stage], s.a[stage], kb * kBK, mt * kBM);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(&map_b, &s.full[stage], s.b[stage] + j * (64 * kBK * 2), nt * BN + j * 64, kb * kBK);
+          } else {
+            tma_load_2d(&map_b, &s.full[stage], s.b[stage], kb * kBK, nt * BN);
+          }
+          ++issued;
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        const uint32_t n = issued < kGemmStages ? issued : kGemmStages;
+        uint32_t st = stage, ph = phase;
+        for (uint32_t i = 0; i < n; ++i) {
+          if (st == 0) { st = kGemmStages - 1; ph ^= 1; } else { --st; }
+          drain_wait(&s.full[st], ph, g.status);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kBM, BN, A_MN, B_MN);
+      // K step of one tcgen05.mma: +32 B inside the swizzled row (K-major) or
+      // +16 rows of 128 B (MN-major).
+      constexpr uint32_t a_step = A_MN ? (kUK * 128) >> 4 : (kUK * 2) >> 4;
+      constexpr uint32_t b_step = B_MN ? (kUK * 128) >> 4 : (kUK * 2) >> 4;
+      constexpr uint32_t a_lbo = A_MN ? 64 * kBK * 2 : 16;
+      constexpr uint32_t b_lbo = B_MN ? 64 * kBK * 2 : 16;
+      uint32_t stage = 0, phase = 0, iter = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x, ++iter) {
+        const uint32_t buf = iter & 1;
+        if (!mbar_wait(&s.tempty[buf], ((iter >> 1) & 1) ^ 1, abort, g.status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * BN;
+        for (int kb = 0; kb < g.kblocks; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort, g.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(smem_u32(s.a[stage]), a_lbo, 1024);
+          const uint64_t db = smem_desc_sw128(smem_u32(s.b[stage]), b_lbo, 1024);
+#pragma unroll
+          for (int k = 0; k < kBK / kUK; ++k)
+            umma_bf16(d, da + static_cast<uint64_t>(k * a_step), db + static_cast<uint64_t>(k * b_step), idesc,
+                      (kb | k) != 0);
+          umma_commit(&s.empty[stage]);
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
+        }
+        if (ok) umma_commit(&s.tfull[buf]);
+      }
+      umma_commit(&s.drain);
+      drain_wait(&s.drain, 0, g.status);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t iter = 0;
+    for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++iter) {
+      int mt, nt;
+      coords(tile, mt, nt);
+      const uint32_t buf = iter & 1;
+      if (!warp_wait(&s.tfull[buf], (iter >> 1) & 1, abort, g.status)) break;
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(mt) * kBM + row_in_tile;
+      const bool valid = row < g.Mdim;
+      const int64_t col0 = static_cast<int64_t>(nt) * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float r[32];
+        tmem_ld32(lane_base + buf * BN + c * 32, r);
+        if (c == BN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tempty[buf]);
+        }
+        if (!valid) continue;
+        const int64_t off = row * g.Ndim + col0 + c * 32;
+        if (OUT_BF16) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + off);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = r[8 * u + e] * g.alpha;
+            dst[u] = f32_to_bf16x8(f);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + off);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float4 v = make_float4(r[4 * u] * g.alpha, r[4 * u + 1] * g.alpha, r[4 * u + 2] * g.alpha,
+                                   r[4 * u + 3] * g.alpha);
+            if (g.accumulate) {
+              const float4 o = dst[u];
+              v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+            }
+            dst[u] = v;
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] (inner contiguous), 128-byte swizzled boxes.
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer) {
+  EncodeTiledFn enc = get_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+size_t align_up(size_t b) { return (b + 255) & ~size_t(255); }
+
+struct TcWs {
+  float* partial;
+  float* terms;
+};
+
+TcWs fwd_layout(const LossProblem& p, void* ws) {
+  const int n_vt = static_cast<int>(p.V / kLossBN);
+  const size_t part = static_cast<size_t>(n_vt) * (2 * p.M - 1) * p.T * sizeof(float);
+  TcWs w;
+  w.partial = static_cast<float*>(ws);
+  w.terms = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(part));
+  return w;
+}
+
+template <int MODE>
+cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaStream_t st) {
+  LossMaps maps;
+  for (int m = 0; m < p.M; ++m) {
+    if (!make_map(&maps.h[m], p.h[m], p.D[m], p.T, kBK, kBM)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.w[m], p.W[m], p.D[m], p.V, kBK, kLossBN)) return cudaErrorInvalidValue;
+  }
+  LossArgs a = args_in;
+  const size_t smem = sizeof(LossSmem) + 1024;
+  auto fn = loss_tile_kernel<MODE>;
+  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+  fn<<<grid, kThreads, smem, st>>>(maps, a);
+  return cudaGetLastError();
+}
+
+LossArgs base_args(const LossProblem& p) {
+  LossArgs a{};
+  a.M = p.M;
+  a.T = static_cast<int>(p.T);
+  a.V = static_cast<int>(p.V);
+  for (int m = 0; m < p.M; ++m) a.kblocks[m] = static_cast<int>(p.D[m] / kBK);
+  a.n_tt = static_cast<int>((p.T + kBM - 1) / kBM);
+  a.n_vt = static_cast<int>(p.V / kLossBN);
+  a.num_tiles = a.n_tt * a.n_vt;
+  a.group_tt = 16;
+  a.y = p.y;
+  a.alpha = p.alpha_d;
+  a.status = p.status;
+  return a;
+}
+
+template <bool A_MN, bool B_MN, int BN, bool OUT_BF16>
+cudaError_t run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int Mdim, int Ndim, int Kdim, void* out,
+                     float alpha, int accumulate, int32_t* status, cudaStream_t st) {
+  GemmArgs g{};
+  g.Mdim = Mdim;
+  g.Ndim = Ndim;
+  g.Kdim = Kdim;
+  g.n_mt = (Mdim + kBM - 1) / kBM;
+  g.n_nt = Ndim / BN;
+  g.num_tiles = g.n_mt * g.n_nt;
+  g.group_m = 16;
+  g.kblocks = (Kdim + kBK - 1) / kBK;
+  g.out = out;
+  g.alpha = alpha;
+  g.accumulate = accumulate;
+  g.status = status;
+  const size_t smem = sizeof(GemmSmem<BN>) + 1024;
+  auto fn = gemm_kernel<A_MN, B_MN, BN, OUT_BF16>;
+  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int grid = g.num_tiles < num_sms() ? g.num_tiles : num_sms();
+  fn<<<grid, kThreads, smem, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+int pick_bn(int64_t D) { return (D % 256 == 0) ? 256 : (D % 128 == 0) ? 128 : 64; }
+
+// dh_m[T x D] = alpha * G'_m[T x V] W^m[V x D]: A = G' (K = V contiguous), B = W^m (N = D contiguous)
+template <int BN>
+cudaError_t run_dh(const __nv_bfloat16* G, const void* W, void* dh, int T, int V, int D, float alpha,
+                   int32_t* status, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, G, V, T, kBK, kBM)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, W, D, V, 64, kBK)) return cudaErrorInvalidValue;
+  return run_gemm<false, true, BN, true>(ma, mb, T, D, V, dh, alpha, 0, status, st);
+}
+
+// dW^m[V x D] (+)= alpha * G'_m^T h_m: A = G'^T (M = V contiguous), B = h_m (N = D contiguous), K = T
+template <int BN>
+cudaError_t run_dw(const __nv_bfloat16* G, const void* h, float* dW, int T, int V, int D, float alpha,
+                   int accumulate, int32_t* status, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, G, V, T, 64, kBK)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, h, D, T, 64, kBK)) return cudaErrorInvalidValue;
+  return run_gemm<true, true, BN, false>(ma, mb, V, D, T, dW, alpha, accumulate, status, st);
+}
+
+}  // namespace
+
+bool tensor_map_encoder_available() { return get_encoder() != nullptr; }
+
+size_t loss_tc_fwd_bytes(const LossProblem& p) {
+  const int64_t n_vt = p.V / kLossBN;
+  const size_t part = static_cast<size_t>(n_vt) * (2 * p.M - 1) * p.T * sizeof(float);
+  const size_t terms = static_cast<size_t>(2 * p.M - 1) * p.T * sizeof(float);
+  return align_up(part) + align_up(terms);
+}
+
+size_t loss_tc_bwd_bytes(const LossProblem& p) {
+  return static_cast<size_t>(p.M) * p.T * p.V * sizeof(__nv_bfloat16);
+}
+
+cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void* ws, cudaStream_t st) {
+  const TcWs w = fwd_layout(p, ws);
+  LossArgs a = base_args(p);
+  a.partial = w.partial;
+  a.stats = stats;
+  cudaError_t err = run_loss_tiles<kModeStats>(p, a, st);
+  if (err != cudaSuccess) return err;
+  const int T = static_cast<int>(p.T);
+  loss_merge_kernel<<<(T + 255) / 256, 256, 0, st>>>(w.partial, a.n_vt, p.M, T, static_cast<int>(p.V), p.y,
+                                                      stats, w.terms, p.status);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  return launch_loss_reduce(w.terms, p.M, p.T, p.alpha_d, losses, st);
+}
+
+cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_scale, void* const* dh,
+                        float* const* dW, int accumulate, void* ws, cudaStream_t st) {
+  __nv_bfloat16* G = static_cast<__nv_bfloat16*>(ws);
+  LossArgs a = base_args(p);
+  a.stats = const_cast<float*>(stats);
+  a.G = G;
+  cudaError_t err = run_loss_tiles<kModeGrad>(p, a, st);
+  if (err != cudaSuccess) return err;
+  const float alpha = grad_scale / static_cast<float>(p.T);
+  const int T = static_cast<int>(p.T), V = static_cast<int>(p.V);
+  for (int m = 0; m < p.M; ++m) {
+    const __nv_bfloat16* Gm = G + static_cast<int64_t>(m) * p.T * p.V;
+    const int D = static_cast<int>(p.D[m]);
+    switch (pick_bn(D)) {
+      case 256: err = run_dh<256>(Gm, p.W[m], dh[m], T, V, D, alpha, p.status, st); break;
+      case 128: err = run_dh<128>(Gm, p.W[m], dh[m], T, V, D, alpha, p.status, st); break;
+      default: err = run_dh<64>(Gm, p.W[m], dh[m], T, V, D, alpha, p.status, st); break;
+    }
+    if (err != cudaSuccess) return err;
+    switch (pick_bn(D)) {
+      case 256: err = run_dw<256>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
+      case 128: err = run_dw<128>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
+      default: err = run_dw<64>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
+    }
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace mls

@@ -1,0 +1,66 @@
+"""Comparison helpers and tolerances for the GPU-vs-oracle parity tests.
+
+Tolerances (fixed by the method's problem statement for this path):
+  * gather/copy/index results: bit-exact;
+  * losses and per-token loss statistics: 2e-3 relative;
+  * gradients: 1e-2 relative, per tensor in Frobenius norm and per element as
+    |g - g*| <= 1e-2 |g*| + 1e-2 rms(g*) (elementwise relative error alone is
+    ill-posed near zero);
+  * the rescaled junction output, a stored activation, is the exact value
+    rounded once to the storage dtype: |y - y*| <= u |y*| (1 + 1e-5) + tiny,
+    u = 2^-8 for bf16 (unit roundoff of an 8-bit significand), 2^-23 for f32,
+    plus the fp32 error of the scale (a few ulp).
+"""
+import numpy as np
+import torch
+
+LOSS_RTOL = 2e-3
+GRAD_RTOL = 1e-2
+
+
+def f64(t) -> np.ndarray:
+    if isinstance(t, torch.Tensor):
+        return t.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def unit_roundoff(dtype) -> float:
+    return 2.0 ** -8 if dtype == torch.bfloat16 else 2.0 ** -23
+
+
+def assert_grad_close(got, exp, name="grad", rtol=GRAD_RTOL):
+    got = f64(got)
+    exp = f64(exp)
+    assert got.shape == exp.shape, (name, got.shape, exp.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    nrm = np.linalg.norm(exp)
+    err = np.linalg.norm(got - exp)
+    assert err <= rtol * nrm + 1e-30, f"{name}: Frobenius rel err {err / max(nrm, 1e-300):.3e} > {rtol}"
+    rms = np.sqrt(np.mean(exp * exp)) if exp.size else 0.0
+    bad = np.abs(got - exp) > rtol * np.abs(exp) + rtol * rms
+    assert not bad.any(), (f"{name}: {int(bad.sum())} elements outside tolerance; worst "
+                           f"{np.max(np.abs(got - exp)):.3e} (rms {rms:.3e})")
+
+
+def assert_loss_close(got, exp, name="loss", rtol=LOSS_RTOL):
+    got = f64(got)
+    exp = f64(exp)
+    assert got.shape == exp.shape, (name, got.shape, exp.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    rel = np.abs(got - exp) / np.maximum(np.abs(exp), 1e-30)
+    assert np.all(rel <= rtol), f"{name}: max rel err {rel.max():.3e} > {rtol}"
+
+
+def assert_stats_close(got, exp, name="stats", rtol=LOSS_RTOL):
+    """Per-token statistics (lse, target logit, teacher-weighted mean).
+
+    Individual target logits and S values can sit near zero, so the bound is
+    relative to the row's typical magnitude: |g - e| <= rtol (|e| + rms(row)).
+    """
+    got = f64(got)
+    exp = f64(exp)
+    assert got.shape == exp.shape, (name, got.shape, exp.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    rms = np.sqrt(np.mean(exp * exp, axis=-1, keepdims=True))
+    bad = np.abs(got - exp) > rtol * (np.abs(exp) + rms)
+    assert not bad.any(), f"{name}: {int(bad.sum())} outside; worst {np.max(np.abs(got - exp)):.3e}"

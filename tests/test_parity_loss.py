@@ -1,0 +1,123 @@
+"""GPU multi-exit loss (forward and backward) against the fp64 oracle.
+
+Small cases compare every output element; they span several 128x128 tiles
+with ragged token tails.  All calls go through the C ABI (libmls).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lm_head_loss_junction_b200 import multiexit_loss_bwd, multiexit_loss_fwd, new_status, status_read
+from lm_head_loss_junction_b200 import workloads as wl
+from tests.helpers import assert_grad_close, assert_loss_close, assert_stats_close, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_inputs(d):
+    y = torch.from_numpy(d.y).cuda()
+    h = [t.cuda() for t in d.o]
+    W = [t.cuda() for t in d.W]
+    return y, h, W
+
+
+def _oracle(d, alpha, grad_scale=1.0, rows=None, need_grad=True):
+    return oracle.multiexit_loss(d.y, d.o, d.W, alpha_d=alpha, grad_scale=grad_scale, rows=rows,
+                                 need_grad=need_grad)
+
+
+def _losses_expected(r, M):
+    return np.concatenate([r["ce_lm"], r["ce_kd"], [r["loss"]]])
+
+
+def _check_all(d, alpha, grad_scale=1.0):
+    cfg = d.cfg
+    M = cfg.M
+    y, h, W = _gpu_inputs(d)
+    st = new_status()
+    losses, stats = multiexit_loss_fwd(y, h, W, alpha, status=st)
+    dh, dW = multiexit_loss_bwd(y, h, W, stats, alpha, grad_scale, status=st)
+    assert status_read(st) == (0, 0)
+    r = _oracle(d, alpha, grad_scale)
+    assert_loss_close(losses, _losses_expected(r, M), "losses")
+    s = f64(stats)
+    assert_stats_close(s[:M], r["lse"], "lse")
+    assert_stats_close(s[M:2 * M], r["tgt"], "target logits")
+    if M > 1:
+        assert_stats_close(s[2 * M:], r["S"], "teacher-weighted logits")
+    for m in range(M):
+        assert_grad_close(dh[m], r["dh"][m], f"dh[{m}]")
+        assert_grad_close(dW[m], r["dW"][m], f"dW[{m}]")
+
+
+def test_tiny_fp32_suite_full():
+    d = wl.make_inputs(wl.CONFIGS["tiny3"])
+    _check_all(d, 0.3)
+
+
+SMALL_BF16 = [
+    ("main3", dict(batch=1, seq=300, V=1024)),
+    ("proxy2", dict(batch=2, seq=97, V=2048)),
+    ("suite4", dict(batch=1, seq=200, V=512)),
+    ("main3_aligned", dict(batch=1, seq=256, V=640)),
+]
+
+
+@pytest.mark.parametrize("name,small", SMALL_BF16)
+def test_bf16_tensor_core_path_small(name, small):
+    cfg = wl.small_variant(wl.CONFIGS[name], **small)
+    d = wl.make_inputs(cfg, with_tables=False)
+    _check_all(d, cfg.alpha_d, grad_scale=1.0)
+
+
+def test_alpha_and_grad_scale_are_runtime_arguments():
+    cfg = wl.small_variant(wl.CONFIGS["proxy2"], batch=1, seq=130, V=256)
+    d = wl.make_inputs(cfg, with_tables=False)
+    for alpha, gs in ((0.0, 1.0), (0.7, 3.5)):
+        _check_all(d, alpha, gs)
+
+
+def test_single_exit_and_accumulate():
+    cfg = wl.small_variant(wl.CONFIGS["main3"], batch=1, seq=130, V=256)
+    d = wl.make_inputs(cfg, with_tables=False)
+    y, h, W = _gpu_inputs(d)
+    losses, stats = multiexit_loss_fwd(y, h[:1], W[:1], 0.3)
+    r = oracle.multiexit_loss(d.y, d.o[:1], d.W[:1], alpha_d=0.3)
+    assert_loss_close(losses, [r["ce_lm"][0], r["loss"]])
+    base = [torch.randn(w.shape, dtype=torch.float32, device="cuda") for w in W[:1]]
+    dW = [b.clone() for b in base]
+    multiexit_loss_bwd(y, h[:1], W[:1], stats, 0.3, dW=dW, accumulate_dW=True)
+    assert_grad_close(dW[0] - base[0], r["dW"][0], "accumulated dW")
+
+
+def test_bad_targets_are_flagged():
+    cfg = wl.small_variant(wl.CONFIGS["proxy2"], batch=1, seq=128, V=256)
+    d = wl.make_inputs(cfg, with_tables=False)
+    y, h, W = _gpu_inputs(d)
+    y = y.clone()
+    y[3] = -5
+    y[77] = cfg.V + 1
+    st = new_status()
+    losses, stats = multiexit_loss_fwd(y, h, W, 0.3, status=st)
+    code, word = status_read(st)
+    assert code == 5 and word & 1
+    assert torch.isfinite(losses).all()
+    dh, dW = multiexit_loss_bwd(y, h, W, stats, 0.3, status=st)
+    assert status_read(st)[0] == 5
+    for m in range(cfg.M):
+        assert torch.all(dh[m][3] == 0) and torch.all(dh[m][77] == 0)
+        assert torch.isfinite(dW[m]).all()
+
+
+def test_repeated_calls_are_deterministic():
+    cfg = wl.small_variant(wl.CONFIGS["main3"], batch=1, seq=257, V=512)
+    d = wl.make_inputs(cfg, with_tables=False)
+    y, h, W = _gpu_inputs(d)
+    l1, s1 = multiexit_loss_fwd(y, h, W, 0.3)
+    l2, s2 = multiexit_loss_fwd(y, h, W, 0.3)
+    assert torch.equal(l1, l2) and torch.equal(s1, s2)
+    g1 = multiexit_loss_bwd(y, h, W, s1, 0.3)
+    g2 = multiexit_loss_bwd(y, h, W, s1, 0.3)
+    for a, b in zip(g1[0] + g1[1], g2[0] + g2[1]):
+        assert torch.equal(a, b)
