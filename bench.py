@@ -1,0 +1,418 @@
+"""Benchmark of one Matryoshka-suite hot-path step on B200.
+
+A step is one pass of the whole path over one batch of synthetic input:
+    junction fwd (block m -> m+1, for m < M)
+    multi-exit loss fwd (per-exit CE + distillation from the largest exit)
+    multi-exit loss bwd (dh_m, dW^m)
+    junction bwd (do_m, de rows, deterministic dE scatter), fed with dh_{m+1}
+    as the incoming gradient of block m+1's input (the blocks themselves are
+    not part of this path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload main3] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own batch
+(weak scaling, no collective on the data path) and the reported time is the
+max over ranks.  ``--impl reference`` times the fp64 CPU oracle on a bounded
+sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lm_head_loss_junction_b200 import workloads as wl  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the step
+class Step:
+    """Device-resident inputs, outputs and workspaces of one hot-path step."""
+
+    def __init__(self, cfg: wl.SuiteConfig, device, seed_offset: int = 0):
+        import dataclasses
+        from lm_head_loss_junction_b200 import api
+        self.api = api
+        self.cfg = dataclasses.replace(cfg, seed=cfg.seed + seed_offset)
+        c = self.cfg
+        d = wl.make_inputs(c)
+        self.host = d
+        self.dev = device
+        self.x = torch.from_numpy(d.x).to(device)
+        self.y = torch.from_numpy(d.y).to(device)
+        self.o = [t.to(device) for t in d.o]
+        self.E = [t.to(device) for t in d.E]
+        self.W = [t.to(device) for t in d.W]
+        dt = self.o[0].dtype
+        T, V, M = c.T, c.V, c.M
+        self.jy = [torch.empty((T, c.D[j + 1]), dtype=dt, device=device) for j in range(M - 1)]
+        self.jscale = [torch.empty(T, dtype=torch.float32, device=device) for _ in range(M - 1)]
+        self.losses = torch.empty(2 * M, dtype=torch.float32, device=device)
+        self.stats = torch.empty((3 * M - 1, T), dtype=torch.float32, device=device)
+        self.dh = [torch.empty_like(t) for t in self.o]
+        self.dW = [torch.empty((V, c.D[m]), dtype=torch.float32, device=device) for m in range(M)]
+        self.do = [torch.empty_like(self.o[j]) for j in range(M - 1)]
+        self.de = [torch.empty((T, c.deltas[j + 1]), dtype=dt, device=device) for j in range(M - 1)]
+        self.dE = [torch.empty((V, c.deltas[j + 1]), dtype=torch.float32, device=device) for j in range(M - 1)]
+        fb, bb = api.multiexit_loss_workspace(T, list(c.D), V, dt)
+        self.ws_loss = torch.empty(max(fb, bb), dtype=torch.uint8, device=device)
+        self.ws_j = torch.empty(api.junction_bwd_workspace(T, V), dtype=torch.uint8, device=device)
+        self.status = api.new_status(device)
+
+    def run(self, stream=None, marks=None):
+        a, c = self.api, self.cfg
+        M = c.M
+
+        def mark(i):
+            if marks is not None:
+                marks[i].record(stream)
+
+        mark(0)
+        for j in range(M - 1):
+            a.junction_fwd(self.x, self.o[j], self.E[j + 1], out=self.jy[j], scale_out=self.jscale[j],
+                           status=self.status, stream=stream)
+        mark(1)
+        a.multiexit_loss_fwd(self.y, self.o, self.W, c.alpha_d, losses=self.losses, stats=self.stats,
+                             workspace=self.ws_loss, status=self.status, stream=stream)
+        mark(2)
+        a.multiexit_loss_bwd(self.y, self.o, self.W, self.stats, c.alpha_d, 1.0, dh=self.dh, dW=self.dW,
+                             workspace=self.ws_loss, status=self.status, stream=stream)
+        mark(3)
+        for j in range(M - 1):
+            a.junction_bwd(self.x, self.o[j], self.E[j + 1], self.dh[j + 1], do_out=self.do[j],
+                           de_out=self.de[j], dE=self.dE[j], accumulate_dE=False, workspace=self.ws_j,
+                           status=self.status, stream=stream)
+        mark(4)
+
+    def working_set_gb(self):
+        ts = [self.x, self.y] + self.o + self.E[1:] + self.W + self.dh + self.dW + self.jy + self.do + self.de + \
+            self.dE
+        return (sum(t.numel() * t.element_size() for t in ts) + self.ws_loss.numel()) / 1e9
+
+    # algorithmic work
+    def loss_flops_algorithmic(self):
+        c = self.cfg
+        return 6.0 * c.T * c.V * sum(c.D)
+
+    def loss_flops_executed(self):
+        c = self.cfg
+        return 8.0 * c.T * c.V * sum(c.D)
+
+    def junction_bytes(self):
+        """(forward, backward) algorithmic HBM bytes over all junctions of the step."""
+        c = self.cfg
+        b = 2 if c.dtype == "bf16" else 4
+        fwd = bwd = 0
+        for j in range(c.M - 1):
+            D, dl, Dn = c.D[j], c.deltas[j + 1], c.D[j + 1]
+            fwd += c.T * ((D + dl + Dn) * b + 4 + 4)                 # o, e row, y; id; scale
+            bwd += c.T * ((Dn + D + dl + D + dl) * b + 4 + 4)        # dy, o, e row, do, de; id; coef
+        return fwd, bwd
+
+
+def _dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _max_over_ranks(v: float, ws: int, device) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(d: wl.SuiteInputs, n_tokens: int):
+    """Times the fp64 oracle on the first n_tokens tokens of the workload (full
+    V and full dW work for those tokens, both junctions).  Returns (seconds, tokens)."""
+    import oracle
+    c = d.cfg
+    rows = np.arange(n_tokens)
+    sub_o = [t[:n_tokens] for t in d.o]
+    t0 = time.perf_counter()
+    for j in range(c.M - 1):
+        oracle.junction_fwd(d.x[rows], sub_o[j], d.E[j + 1])
+    r = oracle.multiexit_loss(d.y[:n_tokens], sub_o, d.W, alpha_d=c.alpha_d, grad_scale=1.0)
+    for j in range(c.M - 1):
+        oracle.junction_bwd(d.x[rows], sub_o[j], d.E[j + 1], r["dh"][j + 1])
+    return time.perf_counter() - t0, n_tokens
+
+
+def _cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info if i.get("internal_api") in ("openblas", "mkl", "blis")),
+                default=None)
+        if n:
+            return int(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, cfg):
+    ws, rank, _ = _dist_env()
+    if rank != 0:
+        return
+    n = args.ref_tokens
+    d = wl.make_inputs(cfg)
+    times = []
+    for i in range(args.warmup + args.steps):
+        sec, _ = cpu_oracle_sample(d, n)
+        if i >= args.warmup:
+            times.append(sec)
+    tot = sum(times)
+    value = n * len(times) / tot
+    line = {
+        "impl": "reference", "metric": "multi-exit head-loss fwd+bwd tokens/s (1 B200) and % bf16 tensor peak; "
+        "junction GB/s", "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * tot / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, **cfg.describe(), "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+                         "sample": f"first {n} tokens of {cfg.name} per step: both junctions fwd+bwd and the "
+                                   f"{cfg.M}-exit loss fwd+bwd over the full vocabulary, fp64 numpy"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="main3", choices=wl.CONFIG_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=64)
+    ap.add_argument("--cpu-tokens", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = wl.CONFIGS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    ws, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    from lm_head_loss_junction_b200 import _lib
+    step = Step(cfg, device, seed_offset=rank)
+    stream = torch.cuda.current_stream(device)
+    peaks, peak_kind = load_peaks()
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    for _ in range(args.warmup):
+        step.run(stream)
+    barrier()
+    code, word = step.api.status_read(step.status, stream)
+    if code != 0:
+        raise RuntimeError(f"device status after warm-up: {code} ({word})")
+
+    # ---------------- timed region: K steps, events between phases
+    K = args.steps
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    launches0 = _lib.lib().mls_kernel_launches()
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for k in range(K):
+            step.run(stream, marks[k])
+        end.record(stream)
+        barrier()
+    launches = _lib.lib().mls_kernel_launches() - launches0
+    ms_total = start.elapsed_time(end)
+    ms_total = _max_over_ranks(ms_total, ws, device)
+    ms_step = ms_total / K
+    phase_ms = [statistics.mean(marks[k][i].elapsed_time(marks[k][i + 1]) for k in range(K)) for i in range(4)]
+    code, word = step.api.status_read(step.status, stream)
+    if code != 0:
+        raise RuntimeError(f"device status after timing: {code} ({word})")
+
+    c = step.cfg
+    tokens_all = c.T * ws
+    value = tokens_all * K / (ms_total / 1000.0)
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = [torch.from_numpy(step.host.x).pin_memory(), torch.from_numpy(step.host.y).pin_memory()] + \
+                  [t.pin_memory() for t in step.host.o]
+        dev_in = [step.x, step.y] + step.o
+        host_out = torch.empty(step.losses.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = host_out.numel() * host_out.element_size()
+        for _ in range(2):
+            for hsrc, ddst in zip(host_in, dev_in):
+                ddst.copy_(hsrc, non_blocking=True)
+            step.run(stream)
+            host_out.copy_(step.losses, non_blocking=True)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            for hsrc, ddst in zip(host_in, dev_in):
+                ddst.copy_(hsrc, non_blocking=True)
+            step.run(stream)
+            host_out.copy_(step.losses, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        ms_e2e = _max_over_ranks(e0.elapsed_time(e1), ws, device)
+        e2e = {"value": tokens_all * K / (ms_e2e / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    # ---------------- roofline of the dominant kernel and phase rates
+    ms_fwd, ms_bwd = phase_ms[1], phase_ms[2]
+    flops_fwd = 2.0 * c.T * c.V * sum(c.D)
+    peak_tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    ach_fwd = flops_fwd / (ms_fwd / 1000.0) / 1e12
+    jf_bytes, jb_bytes = step.junction_bytes()
+    hbm = peaks.get("hbm_gbs")
+    phases = {
+        "junction_fwd_ms": phase_ms[0], "loss_fwd_ms": ms_fwd, "loss_bwd_ms": ms_bwd, "junction_bwd_ms": phase_ms[3],
+        "loss_fwd_bwd_tokens_per_s": c.T / ((ms_fwd + ms_bwd) / 1000.0),
+        "loss_executed_tflops": step.loss_flops_executed() / ((ms_fwd + ms_bwd) / 1000.0) / 1e12,
+        "loss_executed_frac_of_peak": step.loss_flops_executed() / ((ms_fwd + ms_bwd) / 1000.0) / 1e12 / peak_tc,
+        "loss_algorithmic_frac_of_peak": step.loss_flops_algorithmic() / ((ms_fwd + ms_bwd) / 1000.0) / 1e12 / peak_tc,
+        "junction_fwd_gbs": jf_bytes / (phase_ms[0] / 1000.0) / 1e9 if c.M > 1 else None,
+        "junction_fwd_frac_of_hbm": jf_bytes / (phase_ms[0] / 1000.0) / 1e9 / hbm if c.M > 1 else None,
+        "junction_bwd_gbs_incl_scatter": jb_bytes / (phase_ms[3] / 1000.0) / 1e9 if c.M > 1 else None,
+    }
+    roofline = {"bound": "tensor", "achieved": ach_fwd, "peak": peak_tc, "unit": "TFLOP/s",
+                "frac": ach_fwd / peak_tc, "traffic": None,
+                "kernel": "loss_tile_kernel<stats> (mls_multiexit_loss_fwd call: tile kernel + merge + reduce)",
+                "algorithmic_per_launch": f"2*T*V*sum(D) = {flops_fwd:.4g} flop",
+                "peak_source": f"{peak_kind} bf16_tflops_sustained"}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        sec, n = cpu_oracle_sample(step.host, args.cpu_tokens)
+        cpu = {"value": n / sec, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+               "sample": f"first {n} tokens of {cfg.name}: both junctions fwd+bwd and the {c.M}-exit loss "
+                         f"fwd+bwd over the full vocabulary, fp64 numpy ({sec:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": "multi-exit head-loss fwd+bwd tokens/s (1 B200) and % bf16 tensor peak; junction GB/s",
+            "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if c.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": c.name, "global_batch": c.batch * ws, "seq_len": c.seq, "tokens_per_gpu": c.T,
+                       "M": c.M, "D": list(c.D), "V": c.V, "alpha_d": c.alpha_d,
+                       "parallelism": f"dp{ws} (independent batches)",
+                       "l2": f"no flush; per-step working set {step.working_set_gb():.2f} GB > 126 MB L2"},
+            "e2e": e2e, "gpu_launches": int(launches), "roofline": roofline, "cpu_baseline": cpu,
+            "phases": phases, "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

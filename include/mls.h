@@ -210,6 +210,10 @@ const char* mls_status_string(mls_status s);
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int mls_version(void);
 
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all threads).  Diagnostics only; the count never resets. */
+uint64_t mls_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

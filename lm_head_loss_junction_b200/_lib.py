@@ -47,6 +47,7 @@ PROTOTYPES = {
     "mls_status_read": (_int, [_vp, _vp, ctypes.POINTER(_i32)]),
     "mls_status_string": (ctypes.c_char_p, [_int]),
     "mls_version": (_int, []),
+    "mls_kernel_launches": (ctypes.c_uint64, []),
 }
 
 

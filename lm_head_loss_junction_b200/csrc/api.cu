@@ -3,11 +3,19 @@
 // is documented in include/mls.h.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cstdint>
 
 #include "kernels.h"
 #include "mls.h"
+
+namespace mls {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+}  // namespace mls
 
 namespace {
 
@@ -86,6 +94,8 @@ mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const in
 extern "C" {
 
 int mls_version(void) { return 100; }
+
+uint64_t mls_kernel_launches(void) { return mls::g_launches.load(std::memory_order_relaxed); }
 
 const char* mls_status_string(mls_status s) {
   switch (s) {

@@ -392,6 +392,7 @@ cudaError_t launch_fwd_t(const JunctionArgs& a, cudaStream_t st) {
     default: MLS_JF(16); break;
   }
 #undef MLS_JF
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -422,6 +423,7 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
     default: MLS_JB(16); break;
   }
 #undef MLS_JB
+  note_launches(1);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || a.dE == nullptr) return err;
 
@@ -442,6 +444,7 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
                                                      kbuf[p & 1], vbuf[p & 1]);
     kin = kbuf[p & 1];
     vin = vbuf[p & 1];
+    note_launches(3);
   }
   if (!a.accumulate_dE) {
     err = cudaMemsetAsync(a.dE, 0, static_cast<size_t>(a.V) * a.delta * sizeof(float), st);
@@ -452,6 +455,7 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   const int64_t blocks = (warps + 7) / 8;
   table_scatter_kernel<BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
       kin, vin, n, a.V, dy, d_vec, dl_vec, coef, E, a.dE, n_slices);
+  note_launches(1);
   return cudaGetLastError();
 }
 

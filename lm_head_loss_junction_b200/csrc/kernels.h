@@ -69,6 +69,9 @@ cudaError_t loss_simt_bwd(const LossProblem& p, const float* stats, float grad_s
 cudaError_t launch_loss_reduce(const float* terms, int M, int64_t T, float alpha_d, float* losses,
                                cudaStream_t st);
 
+// Counts kernel launches issued by the library (diagnostics).
+void note_launches(int n);
+
 // Set when the tensor-map encoder could not be obtained from the driver.
 bool tensor_map_encoder_available();
 

@@ -51,7 +51,6 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
   int64_t hsum = 0;
   for (int m = 0; m < M; ++m) hsum += p.D[m];
   float* red = sm + hsum;  // [Q][kSimtThreads]
-  const int Q = 2 + S + 2 * S + M;
   for (int m = 0; m < M; ++m)
     for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) hrow[p.Doff[m] + k] = p.h[m][t * p.D[m] + k];
   __syncthreads();
@@ -124,11 +123,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
     }
     __syncthreads();
   }
-  (void)Q;
   if (tid == 0) {
     const float lseT = red[0] + logf(red[kSimtThreads]);
-    const float T_ = static_cast<float>(p.T);
-    (void)T_;
     for (int m = 0; m < M; ++m) {
       float lse;
       if (m == M - 1) {
@@ -285,18 +281,20 @@ size_t loss_simt_bwd_bytes(const LossProblem& p) {
 cudaError_t launch_loss_reduce(const float* terms, int M, int64_t T, float alpha_d, float* losses,
                                cudaStream_t st) {
   loss_reduce_kernel<<<1, 1024, 0, st>>>(terms, M, T, alpha_d, losses);
+  note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t loss_simt_fwd(const LossProblem& p, float* losses, float* stats, void* ws, cudaStream_t st) {
   const SimtDev d = make_dev(p);
   const int S = p.M - 1;
-  const int Q = 2 + S + 2 * S + p.M;
+  const int Q = 2 + S + 2 * S + p.M;   // per-thread quantities merged by the tree
   const size_t smem = (sum_d(p) + static_cast<size_t>(Q) * kSimtThreads) * sizeof(float);
   cudaError_t err = ensure_smem(reinterpret_cast<const void*>(simt_stats_kernel), smem);
   if (err != cudaSuccess) return err;
   float* terms = static_cast<float*>(ws);
   simt_stats_kernel<<<static_cast<unsigned>(p.T), kSimtThreads, smem, st>>>(d, stats, terms);
+  note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   return launch_loss_reduce(terms, p.M, p.T, p.alpha_d, losses, st);
@@ -315,10 +313,12 @@ cudaError_t loss_simt_bwd(const LossProblem& p, const float* stats, float grad_s
   cudaError_t err = ensure_smem(reinterpret_cast<const void*>(simt_grad_kernel), smem);
   if (err != cudaSuccess) return err;
   simt_grad_kernel<<<static_cast<unsigned>(p.T), kSimtThreads, smem, st>>>(d, stats, alpha, G);
+  note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   dim3 grid(static_cast<unsigned>(p.V), static_cast<unsigned>(p.M));
   simt_dw_kernel<<<grid, kSimtThreads, 0, st>>>(d, alpha, G, accumulate);
+  note_launches(1);
   return cudaGetLastError();
 }
 

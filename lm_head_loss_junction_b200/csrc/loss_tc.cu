@@ -680,6 +680,7 @@ cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaSt
   if (err != cudaSuccess) return err;
   const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
   fn<<<grid, kThreads, smem, st>>>(maps, a);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -721,6 +722,7 @@ cudaError_t run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int Mdim, int
   if (err != cudaSuccess) return err;
   const int grid = g.num_tiles < num_sms() ? g.num_tiles : num_sms();
   fn<<<grid, kThreads, smem, st>>>(ma, mb, g);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -771,6 +773,7 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   const int T = static_cast<int>(p.T);
   loss_merge_kernel<<<(T + 255) / 256, 256, 0, st>>>(w.partial, a.n_vt, p.M, T, static_cast<int>(p.V), p.y,
                                                       stats, w.terms, p.status);
+  note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   return launch_loss_reduce(w.terms, p.M, p.T, p.alpha_d, losses, st);
