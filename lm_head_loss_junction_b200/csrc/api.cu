@@ -136,7 +136,7 @@ mls_status mls_junction_fwd(const int32_t* x, int64_t T, const void* o_m, int64_
 
 mls_status mls_junction_bwd_workspace(int64_t T, int64_t V, size_t* bytes) {
   if (bytes == nullptr || T <= 0 || V <= 0) return MLS_ERR_INVALID_ARG;
-  *bytes = mls::junction_scatter_bytes(T);
+  *bytes = mls::junction_scatter_bytes(T, V);
   return MLS_OK;
 }
 
@@ -152,7 +152,7 @@ mls_status mls_junction_bwd(const int32_t* x, int64_t T, const void* o_m, int64_
     return MLS_ERR_UNSUPPORTED;
   if (T > INT_MAX) return MLS_ERR_UNSUPPORTED;
   if (dE_table != nullptr) {
-    if (workspace == nullptr || ws_bytes < mls::junction_scatter_bytes(T)) return MLS_ERR_WORKSPACE;
+    if (workspace == nullptr || ws_bytes < mls::junction_scatter_bytes(T, V)) return MLS_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
   }
   if ((st = device_ok()) != MLS_OK) return st;

@@ -1,5 +1,5 @@
-// Junction kernels: forward (rescale + gather + concat), backward (do, de rows)
-// and the deterministic scatter of de into the residual-embedding table.
+// Junction kernels: forward (rescale + gather + concat) and backward (do, de
+// rows, and the residual-table gradient through the id-grouped row sums).
 //
 // The junction maps block m's output o_m[t] (width D_m) and the fresh residual
 // embedding e_{m+1}[x_t] (width delta = D_{m+1} - D_m) to block m+1's input
@@ -216,144 +216,6 @@ __global__ void __launch_bounds__(256) junction_bwd_kernel(
   }
 }
 
-// ---------------------------------------------------------------- table scatter
-// dE[v] (+)= sum_{t: x_t = v} de_t with de_t = g_e,t + c_t E[v]; so the row sum is
-//   dE[v] (+)= (sum_t g_e,t) + (sum_t c_t) E[v],
-// both sums taken over the tokens of v in ascending t.  Tokens are grouped by
-// id with a stable LSD radix sort (8-bit digits), so the order is fixed and
-// the result is deterministic.
-
-constexpr int kSortBlock = 1024;  // keys per sort block (one per thread)
-
-__global__ void __launch_bounds__(kSortBlock) sort_hist_kernel(const int32_t* __restrict__ keys,
-                                                               const int32_t* __restrict__ x, int64_t n,
-                                                               int64_t V, int shift,
-                                                               int32_t* __restrict__ hist, int nblk) {
-  __shared__ int32_t h[256];
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
-  __syncthreads();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * kSortBlock + threadIdx.x;
-  if (i < n) {
-    int32_t k;
-    if (keys != nullptr) {
-      k = keys[i];
-    } else {  // first pass reads ids directly; invalid ids sort last as key V
-      const int32_t id = x[i];
-      k = (id < 0 || id >= V) ? static_cast<int32_t>(V) : id;
-    }
-    atomicAdd(&h[(k >> shift) & 255], 1);
-  }
-  __syncthreads();
-  for (int d = threadIdx.x; d < 256; d += blockDim.x) hist[d * nblk + blockIdx.x] = h[d];
-}
-
-// Exclusive prefix sum over hist[0..n) in one block (digit-major, block-minor order).
-__global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t* __restrict__ hist, int n) {
-  __shared__ int32_t part[1024];
-  const int tid = threadIdx.x;
-  const int per = (n + 1023) / 1024;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
-  int32_t s = 0;
-  for (int i = lo; i < hi; ++i) s += hist[i];
-  part[tid] = s;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {   // inclusive Hillis-Steele scan
-    const int32_t v = (tid >= off) ? part[tid - off] : 0;
-    __syncthreads();
-    part[tid] += v;
-    __syncthreads();
-  }
-  int32_t run = part[tid] - s;
-  for (int i = lo; i < hi; ++i) {
-    const int32_t c = hist[i];
-    hist[i] = run;
-    run += c;
-  }
-}
-
-__global__ void __launch_bounds__(kSortBlock) sort_scatter_kernel(
-    const int32_t* __restrict__ kin, const int32_t* __restrict__ vin, const int32_t* __restrict__ x,
-    int64_t n, int64_t V, int shift, const int32_t* __restrict__ hist, int nblk, int32_t* __restrict__ kout,
-    int32_t* __restrict__ vout) {
-  __shared__ int32_t wcnt[kSortBlock / 32][256];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < (kSortBlock / 32) * 256; i += blockDim.x) (&wcnt[0][0])[i] = 0;
-  __syncthreads();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * kSortBlock + tid;
-  const bool valid = i < n;
-  int32_t k = 0, v = 0;
-  if (valid) {
-    if (kin != nullptr) {
-      k = kin[i];
-      v = vin[i];
-    } else {
-      const int32_t id = x[i];
-      k = (id < 0 || id >= V) ? static_cast<int32_t>(V) : id;
-      v = static_cast<int32_t>(i);
-    }
-  }
-  const int d = (k >> shift) & 255;
-  const unsigned peers = __match_any_sync(0xffffffffu, valid ? d : 256 + lane);
-  const int rank = __popc(peers & ((1u << lane) - 1u));
-  if (valid && rank == 0) wcnt[warp][d] = __popc(peers);
-  __syncthreads();
-  if (tid < 256) {
-    int32_t run = 0;
-    for (int w = 0; w < kSortBlock / 32; ++w) {
-      const int32_t c = wcnt[w][tid];
-      wcnt[w][tid] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  if (valid) {
-    const int32_t pos = hist[d * nblk + blockIdx.x] + wcnt[warp][d] + rank;
-    kout[pos] = k;
-    vout[pos] = v;
-  }
-}
-
-// One warp per (sorted position, column slice of 32 vectors).  Only the first
-// position of each id segment does work; it walks the segment in order.
-template <bool BF16>
-__global__ void __launch_bounds__(256) table_scatter_kernel(
-    const int32_t* __restrict__ keys, const int32_t* __restrict__ toks, int64_t n, int64_t V,
-    const uint4* __restrict__ dy, int d_vec, int dl_vec, const float* __restrict__ coef,
-    const uint4* __restrict__ E, float* __restrict__ dE, int n_slices) {
-  constexpr int N = Elt<BF16>::kPerVec;
-  const int lane = threadIdx.x & 31;
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t pos = w / n_slices;
-  const int slice = static_cast<int>(w % n_slices);
-  if (pos >= n) return;
-  const int32_t key = keys[pos];
-  if (key >= V) return;                                   // invalid ids sort last
-  if (pos > 0 && keys[pos - 1] == key) return;           // not a segment start
-  const int vi = slice * 32 + lane;
-  const bool active = vi < dl_vec;
-  const int dp_vec = d_vec + dl_vec;
-  float acc[N];
-#pragma unroll
-  for (int k = 0; k < N; ++k) acc[k] = 0.f;
-  float csum = 0.f;
-  for (int64_t p = pos; p < n && keys[p] == key; ++p) {
-    const int64_t t = toks[p];
-    csum += coef[t];
-    if (active) {
-      float g[N];
-      Elt<BF16>::load(__ldg(dy + t * dp_vec + d_vec + vi), g);
-#pragma unroll
-      for (int k = 0; k < N; ++k) acc[k] += g[k];
-    }
-  }
-  if (!active) return;
-  float e[N];
-  Elt<BF16>::load(__ldg(E + static_cast<int64_t>(key) * dl_vec + vi), e);
-  float* out = dE + static_cast<int64_t>(key) * dl_vec * N + static_cast<int64_t>(vi) * N;
-#pragma unroll
-  for (int k = 0; k < N; ++k) out[k] += fmaf(csum, e[k], acc[k]);
-}
-
 int pick_cap(int nvec) {
   const int per_lane = (nvec + 31) / 32;
   if (per_lane <= 1) return 1;
@@ -408,11 +270,7 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   auto* dout = static_cast<uint4*>(a.do_out);
   auto* deo = static_cast<uint4*>(a.de_out);
   float* coef = nullptr;
-  JunctionScatterWs ws{};
-  if (a.dE != nullptr) {
-    ws = junction_scatter_layout(a.T, a.workspace);
-    coef = ws.coef;
-  }
+  if (a.dE != nullptr) coef = static_cast<float*>(a.workspace);
 #define MLS_JB(C) junction_bwd_kernel<BF16, C><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status)
   switch (cap) {
     case 1: MLS_JB(1); break;
@@ -427,61 +285,18 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || a.dE == nullptr) return err;
 
-  // Stable radix sort of the ids, then the per-id segment sums.
-  const int64_t n = a.T;
-  const int nblk = static_cast<int>((n + kSortBlock - 1) / kSortBlock);
-  int bits = 1;
-  while ((int64_t(1) << bits) <= a.V) ++bits;          // keys live in [0, V]
-  const int passes = (bits + 7) / 8;
-  const int32_t* kin = nullptr;
-  const int32_t* vin = nullptr;
-  int32_t* kbuf[2] = {ws.keys0, ws.keys1};
-  int32_t* vbuf[2] = {ws.vals0, ws.vals1};
-  for (int p = 0; p < passes; ++p) {
-    sort_hist_kernel<<<nblk, kSortBlock, 0, st>>>(kin, a.x, n, a.V, 8 * p, ws.hist, nblk);
-    sort_scan_kernel<<<1, 1024, 0, st>>>(ws.hist, 256 * nblk);
-    sort_scatter_kernel<<<nblk, kSortBlock, 0, st>>>(kin, vin, a.x, n, a.V, 8 * p, ws.hist, nblk,
-                                                     kbuf[p & 1], vbuf[p & 1]);
-    kin = kbuf[p & 1];
-    vin = vbuf[p & 1];
-    note_launches(3);
-  }
-  if (!a.accumulate_dE) {
-    err = cudaMemsetAsync(a.dE, 0, static_cast<size_t>(a.V) * a.delta * sizeof(float), st);
-    if (err != cudaSuccess) return err;
-  }
-  const int n_slices = (dl_vec + 31) / 32;
-  const int64_t warps = n * n_slices;
-  const int64_t blocks = (warps + 7) / 8;
-  table_scatter_kernel<BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      kin, vin, n, a.V, dy, d_vec, dl_vec, coef, E, a.dE, n_slices);
-  note_launches(1);
-  return cudaGetLastError();
+  // Table gradient: tokens grouped by id, fixed-order row sums.
+  SegIndexDev ix;
+  void* ix_ws = static_cast<char*>(a.workspace) + ((static_cast<size_t>(a.T) * 4 + 255) & ~size_t(255));
+  err = build_segindex(a.x, a.T, a.V, ix_ws, &ix, st);
+  if (err != cudaSuccess) return err;
+  return scatter_table_grad(ix, BF16, a.dy, d_vec, dl_vec, coef, a.E, a.dE, a.accumulate_dE != 0, st);
 }
 
 }  // namespace
 
-size_t junction_scatter_bytes(int64_t T) {
-  const int64_t nblk = (T + kSortBlock - 1) / kSortBlock;
-  const size_t t4 = static_cast<size_t>(T) * 4;
-  auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
-  return up(t4) * 5 + up(static_cast<size_t>(256) * nblk * 4);
-}
-
-JunctionScatterWs junction_scatter_layout(int64_t T, void* base) {
-  const int64_t nblk = (T + kSortBlock - 1) / kSortBlock;
-  const size_t t4 = static_cast<size_t>(T) * 4;
-  auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
-  char* p = static_cast<char*>(base);
-  JunctionScatterWs w;
-  w.coef = reinterpret_cast<float*>(p); p += up(t4);
-  w.keys0 = reinterpret_cast<int32_t*>(p); p += up(t4);
-  w.keys1 = reinterpret_cast<int32_t*>(p); p += up(t4);
-  w.vals0 = reinterpret_cast<int32_t*>(p); p += up(t4);
-  w.vals1 = reinterpret_cast<int32_t*>(p); p += up(t4);
-  w.hist = reinterpret_cast<int32_t*>(p);
-  (void)nblk;
-  return w;
+size_t junction_scatter_bytes(int64_t T, int64_t V) {
+  return ((static_cast<size_t>(T) * 4 + 255) & ~size_t(255)) + segindex_bytes(T, V);
 }
 
 cudaError_t launch_junction_fwd(const JunctionArgs& a, cudaStream_t st) {

@@ -27,15 +27,31 @@ struct JunctionArgs {
   int32_t* status;
 };
 
-struct JunctionScatterWs {
-  float* coef;
-  int32_t *keys0, *keys1, *vals0, *vals1, *hist;
-};
-
-size_t junction_scatter_bytes(int64_t T);
-JunctionScatterWs junction_scatter_layout(int64_t T, void* base);
+size_t junction_scatter_bytes(int64_t T, int64_t V);
 cudaError_t launch_junction_fwd(const JunctionArgs& a, cudaStream_t st);
 cudaError_t launch_junction_bwd(const JunctionArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------------------ id-grouped row sums
+// Tokens grouped by id (stable in t): the tokens of id v are
+// toks[offsets[v] .. offsets[v] + counts[v]).  Ids outside [0, V) are left out.
+struct SegIndexDev {
+  int64_t V;
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* toks;
+  const int32_t* heavy;      // ids with many tokens
+  const int32_t* n_heavy;
+  int64_t max_heavy;
+};
+
+size_t segindex_bytes(int64_t T, int64_t V);
+cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, SegIndexDev* out, cudaStream_t st);
+// dE[v] (+)= sum_t g_e,t + (sum_t coef_t) E[v]; g_e is the tail of each dy row.
+cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
+                               const float* coef, const void* E, float* dE, bool accumulate, cudaStream_t st);
+// dW[v] -= scale * sum_t h_t (bf16 rows of d_vec 16-byte vectors).
+cudaError_t scatter_target_rows(const SegIndexDev& ix, const void* h, int d_vec, float* dW, float scale,
+                                cudaStream_t st);
 
 // ------------------------------------------------------------------ loss
 struct LossProblem {

@@ -11,10 +11,13 @@
 // S_m = sum_v p_T,v l_m,v; a fixed-order reduction gives the losses.
 //
 // Backward.  The same mainloop recomputes each tile's logits; the epilogue forms
-//   G'_m = q_m - (1 - alpha_d) onehot(y) - alpha_d p_T   (students)
-//   G'_T = p_T - onehot(y)                               (teacher, stop-gradient)
+// the dense part of the logit gradient
+//   G'_m = q_m - alpha_d p_T   (students),   G'_T = p_T   (teacher, stop-gradient)
 // in bf16 into a workspace, and two tensor-core GEMMs per exit produce
-//   dh_m = (grad_scale/T) G'_m W^m   and   dW^m (+)= (grad_scale/T) G'_m^T h_m.
+//   dh_m = a (G'_m W^m - c_m W^m[y_t])   and   dW^m (+)= a G'_m^T h_m - a c_m sum_{t: y_t = v} h_t,
+// a = grad_scale/T, c_m = 1 - alpha_d (students) or 1 (teacher).  The one-hot
+// term is applied exactly in fp32 (a row gather in the dh epilogue and an
+// id-grouped row sum for dW) instead of being rounded into the bf16 G'.
 //
 // Definitions: "Matryoshka Language Model Suites" (agihunt.info summary,
 // distillation paragraph), "Is nesting the cheapest way to build a model
@@ -297,12 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
 #pragma unroll
           for (int j = 0; j < 32; ++j) p[c][j] = exp2f(fmaf(p[c][j], kLog2e, -lTs));
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float g0 = p[c][j] - ((c * 32 + j) == yl ? 1.f : 0.f);
-            float g1 = p[c][j + 1] - ((c * 32 + j + 1) == yl ? 1.f : 0.f);
-            if (bad) { g0 = 0.f; g1 = 0.f; }
-            packed[j / 2] = pack_bf16x2(g0, g1);
-          }
+          for (int j = 0; j < 32; j += 2) packed[j / 2] = bad ? 0u : pack_bf16x2(p[c][j], p[c][j + 1]);
           if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(a.G + g_row + c * 32);
 #pragma unroll
@@ -310,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
               dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
           }
         }
-        const float al = a.alpha, one_m_al = 1.f - a.alpha;
+        const float al = a.alpha;
         for (int sidx = M - 2; sidx >= 0; --sidx) {
           if (!warp_wait(&s.tfull[sidx], iter & 1, abort, a.status)) break;
           tc_fence_after();
@@ -324,12 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
             uint32_t packed[16];
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              float g0 = exp2f(fmaf(r[j], kLog2e, -ls)) - al * p[c][j] -
-                         ((c * 32 + j) == yl ? one_m_al : 0.f);
-              float g1 = exp2f(fmaf(r[j + 1], kLog2e, -ls)) - al * p[c][j + 1] -
-                         ((c * 32 + j + 1) == yl ? one_m_al : 0.f);
-              if (bad) { g0 = 0.f; g1 = 0.f; }
-              packed[j / 2] = pack_bf16x2(g0, g1);
+              const float g0 = fmaf(-al, p[c][j], exp2f(fmaf(r[j], kLog2e, -ls)));
+              const float g1 = fmaf(-al, p[c][j + 1], exp2f(fmaf(r[j + 1], kLog2e, -ls)));
+              packed[j / 2] = bad ? 0u : pack_bf16x2(g0, g1);
             }
             if (valid) {
               uint4* dst = reinterpret_cast<uint4*>(a.G + row_off + c * 32);
@@ -419,6 +414,12 @@ struct GemmArgs {
   float alpha;
   int accumulate;
   int32_t* status;
+  // Optional exact one-hot term (bf16 output only): row r additionally gets
+  //   - alpha * onehot_coef * onehot_rows[onehot_idx[r], :]   when onehot_idx[r] in [0, onehot_limit)
+  const int32_t* onehot_idx;
+  const __nv_bfloat16* onehot_rows;
+  float onehot_coef;
+  int onehot_limit;
 };
 
 template <int BN>
@@ -566,6 +567,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       const int64_t row = static_cast<int64_t>(mt) * kBM + row_in_tile;
       const bool valid = row < g.Mdim;
       const int64_t col0 = static_cast<int64_t>(nt) * BN;
+      int64_t onehot_row = -1;
+      if (OUT_BF16 && valid && g.onehot_idx != nullptr) {
+        const int32_t k = __ldg(g.onehot_idx + row);
+        if (k >= 0 && k < g.onehot_limit) onehot_row = k;
+      }
+      const float oh_scale = g.alpha * g.onehot_coef;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float r[32];
@@ -579,11 +586,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const int64_t off = row * g.Ndim + col0 + c * 32;
         if (OUT_BF16) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + off);
+          const uint4* oh = (onehot_row >= 0)
+                                ? reinterpret_cast<const uint4*>(g.onehot_rows + onehot_row * g.Ndim + col0 + c * 32)
+                                : nullptr;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = r[8 * u + e] * g.alpha;
+            if (oh != nullptr) {
+              float w[8];
+              bf16x8_to_f32(__ldg(oh + u), w);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = fmaf(-oh_scale, w[e], f[e]);
+            }
             dst[u] = f32_to_bf16x8(f);
           }
         } else {
@@ -652,6 +668,9 @@ int num_sms() {
 
 size_t align_up(size_t b) { return (b + 255) & ~size_t(255); }
 
+// bf16 G' of every exit: [M][T][V]
+size_t g_bytes(const LossProblem& p) { return static_cast<size_t>(p.M) * p.T * p.V * sizeof(__nv_bfloat16); }
+
 struct TcWs {
   float* partial;
   float* terms;
@@ -702,8 +721,9 @@ LossArgs base_args(const LossProblem& p) {
 
 template <bool A_MN, bool B_MN, int BN, bool OUT_BF16>
 cudaError_t run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int Mdim, int Ndim, int Kdim, void* out,
-                     float alpha, int accumulate, int32_t* status, cudaStream_t st) {
+                     float alpha, int accumulate, int32_t* status, cudaStream_t st, const GemmArgs* extra = nullptr) {
   GemmArgs g{};
+  if (extra != nullptr) g = *extra;
   g.Mdim = Mdim;
   g.Ndim = Ndim;
   g.Kdim = Kdim;
@@ -728,14 +748,20 @@ cudaError_t run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int Mdim, int
 
 int pick_bn(int64_t D) { return (D % 256 == 0) ? 256 : (D % 128 == 0) ? 128 : 64; }
 
-// dh_m[T x D] = alpha * G'_m[T x V] W^m[V x D]: A = G' (K = V contiguous), B = W^m (N = D contiguous)
+// dh_m[T x D] = alpha * (G'_m[T x V] W^m[V x D] - c_m W^m[y_t]): A = G' (K = V contiguous),
+// B = W^m (N = D contiguous); the one-hot row of W^m is subtracted exactly in the epilogue.
 template <int BN>
 cudaError_t run_dh(const __nv_bfloat16* G, const void* W, void* dh, int T, int V, int D, float alpha,
-                   int32_t* status, cudaStream_t st) {
+                   const int32_t* y, float c_onehot, int32_t* status, cudaStream_t st) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, G, V, T, kBK, kBM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, W, D, V, 64, kBK)) return cudaErrorInvalidValue;
-  return run_gemm<false, true, BN, true>(ma, mb, T, D, V, dh, alpha, 0, status, st);
+  GemmArgs extra{};
+  extra.onehot_idx = y;
+  extra.onehot_rows = static_cast<const __nv_bfloat16*>(W);
+  extra.onehot_coef = c_onehot;
+  extra.onehot_limit = V;
+  return run_gemm<false, true, BN, true>(ma, mb, T, D, V, dh, alpha, 0, status, st, &extra);
 }
 
 // dW^m[V x D] (+)= alpha * G'_m^T h_m: A = G'^T (M = V contiguous), B = h_m (N = D contiguous), K = T
@@ -760,7 +786,7 @@ size_t loss_tc_fwd_bytes(const LossProblem& p) {
 }
 
 size_t loss_tc_bwd_bytes(const LossProblem& p) {
-  return static_cast<size_t>(p.M) * p.T * p.V * sizeof(__nv_bfloat16);
+  return align_up(g_bytes(p)) + segindex_bytes(p.T, p.V);
 }
 
 cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void* ws, cudaStream_t st) {
@@ -787,15 +813,21 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   a.G = G;
   cudaError_t err = run_loss_tiles<kModeGrad>(p, a, st);
   if (err != cudaSuccess) return err;
+  // Tokens grouped by target, for the exact one-hot part of dW.
+  SegIndexDev ix;
+  err = build_segindex(p.y, p.T, p.V, static_cast<char*>(ws) + align_up(g_bytes(p)), &ix, st);
+  if (err != cudaSuccess) return err;
   const float alpha = grad_scale / static_cast<float>(p.T);
   const int T = static_cast<int>(p.T), V = static_cast<int>(p.V);
   for (int m = 0; m < p.M; ++m) {
     const __nv_bfloat16* Gm = G + static_cast<int64_t>(m) * p.T * p.V;
     const int D = static_cast<int>(p.D[m]);
+    // one-hot weight of exit m: (1 - alpha_d) for students, 1 for the teacher
+    const float c = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
     switch (pick_bn(D)) {
-      case 256: err = run_dh<256>(Gm, p.W[m], dh[m], T, V, D, alpha, p.status, st); break;
-      case 128: err = run_dh<128>(Gm, p.W[m], dh[m], T, V, D, alpha, p.status, st); break;
-      default: err = run_dh<64>(Gm, p.W[m], dh[m], T, V, D, alpha, p.status, st); break;
+      case 256: err = run_dh<256>(Gm, p.W[m], dh[m], T, V, D, alpha, p.y, c, p.status, st); break;
+      case 128: err = run_dh<128>(Gm, p.W[m], dh[m], T, V, D, alpha, p.y, c, p.status, st); break;
+      default: err = run_dh<64>(Gm, p.W[m], dh[m], T, V, D, alpha, p.y, c, p.status, st); break;
     }
     if (err != cudaSuccess) return err;
     switch (pick_bn(D)) {
@@ -803,6 +835,8 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
       case 128: err = run_dw<128>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
       default: err = run_dw<64>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
     }
+    if (err != cudaSuccess) return err;
+    err = scatter_target_rows(ix, p.h[m], D / 8, dW[m], alpha * c, st);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;

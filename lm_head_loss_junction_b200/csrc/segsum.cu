@@ -1,0 +1,343 @@
+// Deterministic row scatters grouped by token id: the residual-table gradient
+// of the junction (dE[v] (+)= sum over tokens with x_t = v) and the one-hot
+// part of the head gradient (dW^m[v] -= c sum over tokens with y_t = v of h_t).
+//
+// Tokens are grouped by id with a stable LSD radix sort (8-bit digits), so
+// each id's tokens are visited in ascending t and every sum is taken in a
+// fixed order: results are bitwise reproducible, with no floating-point
+// atomics.  Rows with few tokens are reduced by one warp; rows with many
+// (Zipf-frequent ids) by a whole block whose warps split the tokens and are
+// combined in warp order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mls {
+
+namespace {
+
+constexpr int kSortBlock = 1024;     // keys per sort block (one per thread)
+constexpr int kHeavy = 32;           // rows with more tokens than this use a block
+constexpr int kHeavyWarps = 16;
+
+size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
+
+__device__ __forceinline__ int32_t clamp_key(int32_t id, int64_t V) {
+  return (id < 0 || id >= V) ? static_cast<int32_t>(V) : id;   // invalid ids sort last
+}
+
+__global__ void __launch_bounds__(kSortBlock) sort_hist_kernel(const int32_t* __restrict__ keys,
+                                                               const int32_t* __restrict__ ids, int64_t n,
+                                                               int64_t V, int shift, int32_t* __restrict__ hist,
+                                                               int nblk) {
+  __shared__ int32_t h[256];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kSortBlock + threadIdx.x;
+  if (i < n) {
+    const int32_t k = keys != nullptr ? keys[i] : clamp_key(ids[i], V);
+    atomicAdd(&h[(k >> shift) & 255], 1);
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < 256; d += blockDim.x) hist[d * nblk + blockIdx.x] = h[d];
+}
+
+// out[i] = sum_{j < i} in[i] over n entries, one block; in may equal out.
+__global__ void __launch_bounds__(1024) exclusive_scan_kernel(const int32_t* in, int32_t* out, int n) {
+  __shared__ int32_t part[1024];
+  const int tid = threadIdx.x;
+  const int per = (n + 1023) / 1024;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  int32_t s = 0;
+  for (int i = lo; i < hi; ++i) s += in[i];
+  part[tid] = s;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const int32_t v = (tid >= off) ? part[tid - off] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  int32_t run = part[tid] - s;
+  for (int i = lo; i < hi; ++i) {
+    const int32_t c = in[i];
+    out[i] = run;
+    run += c;
+  }
+}
+
+__global__ void __launch_bounds__(kSortBlock) sort_scatter_kernel(
+    const int32_t* __restrict__ kin, const int32_t* __restrict__ vin, const int32_t* __restrict__ ids, int64_t n,
+    int64_t V, int shift, const int32_t* __restrict__ hist, int nblk, int32_t* __restrict__ kout,
+    int32_t* __restrict__ vout) {
+  __shared__ int32_t wcnt[kSortBlock / 32][256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < (kSortBlock / 32) * 256; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kSortBlock + tid;
+  const bool valid = i < n;
+  int32_t k = 0, v = 0;
+  if (valid) {
+    if (kin != nullptr) {
+      k = kin[i];
+      v = vin[i];
+    } else {
+      k = clamp_key(ids[i], V);
+      v = static_cast<int32_t>(i);
+    }
+  }
+  const int d = (k >> shift) & 255;
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? d : 256 + lane);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank == 0) wcnt[warp][d] = __popc(peers);
+  __syncthreads();
+  if (tid < 256) {
+    int32_t run = 0;
+    for (int w = 0; w < kSortBlock / 32; ++w) {
+      const int32_t c = wcnt[w][tid];
+      wcnt[w][tid] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (valid) {
+    const int32_t pos = hist[d * nblk + blockIdx.x] + wcnt[warp][d] + rank;
+    kout[pos] = k;
+    vout[pos] = v;
+  }
+}
+
+__global__ void count_ids_kernel(const int32_t* __restrict__ ids, int64_t n, int64_t V, int32_t* __restrict__ counts) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int32_t id = ids[i];
+  if (id >= 0 && id < V) atomicAdd(counts + id, 1);
+}
+
+// Rows with more than kHeavy tokens go to a list (its order does not matter:
+// every row is reduced independently in a fixed order).
+__global__ void heavy_list_kernel(const int32_t* __restrict__ counts, int64_t V, int32_t* __restrict__ heavy,
+                                  int32_t* __restrict__ n_heavy) {
+  const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (v >= V) return;
+  if (counts[v] > kHeavy) heavy[atomicAdd(n_heavy, 1)] = static_cast<int32_t>(v);
+}
+
+template <bool BF16>
+struct Vec8;
+template <>
+struct Vec8<true> {
+  static constexpr int N = 8;
+  __device__ static void add(float (&acc)[8], const uint4& u) {
+    float f[8];
+    bf16x8_to_f32(u, f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] += f[k];
+  }
+  __device__ static void load(const uint4& u, float (&f)[8]) { bf16x8_to_f32(u, f); }
+};
+template <>
+struct Vec8<false> {
+  static constexpr int N = 4;
+  __device__ static void add(float (&acc)[4], const uint4& u) {
+    acc[0] += __uint_as_float(u.x); acc[1] += __uint_as_float(u.y);
+    acc[2] += __uint_as_float(u.z); acc[3] += __uint_as_float(u.w);
+  }
+  __device__ static void load(const uint4& u, float (&f)[4]) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
+};
+
+// Writes one row slice: out = base + acc + cs*E (table mode) or out -= scale*acc (target mode).
+template <bool BF16, bool TABLE>
+__device__ __forceinline__ void emit(float* out_row, int vi, const float (&acc)[Vec8<BF16>::N], float cs,
+                                     const uint4* E_row, float scale, bool accumulate) {
+  constexpr int N = Vec8<BF16>::N;
+  float* o = out_row + static_cast<int64_t>(vi) * N;
+  if (TABLE) {
+    float e[N];
+    Vec8<BF16>::load(__ldg(E_row + vi), e);
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+      const float val = fmaf(cs, e[k], acc[k]);
+      o[k] = accumulate ? o[k] + val : val;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < N; ++k) o[k] = fmaf(-scale, acc[k], o[k]);
+  }
+}
+
+// One warp per id row (light rows, and the zero rows of table mode).
+//   src row of token t: src + t*src_ld + src_off (16-byte vectors)
+template <bool BF16, bool TABLE>
+__global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix, const uint4* __restrict__ src,
+                                                           int64_t src_ld, int src_off, int n_vec,
+                                                           const float* __restrict__ coef,
+                                                           const uint4* __restrict__ E, float* __restrict__ out,
+                                                           float scale, int accumulate) {
+  constexpr int N = Vec8<BF16>::N;
+  const int lane = threadIdx.x & 31;
+  const int64_t v = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (v >= ix.V) return;
+  const int32_t cnt = ix.counts[v];
+  if (cnt > kHeavy) return;                   // handled by the heavy kernel
+  if (cnt == 0 && (!TABLE || accumulate)) return;   // nothing to add
+  const int32_t off = ix.offsets[v];
+  float* out_row = out + v * static_cast<int64_t>(n_vec) * N;
+  const uint4* E_row = TABLE ? E + v * static_cast<int64_t>(n_vec) : nullptr;
+  float cs = 0.f;
+  if (TABLE)
+    for (int p = 0; p < cnt; ++p) cs += coef[ix.toks[off + p]];
+  for (int vi = lane; vi < n_vec; vi += 32) {
+    float acc[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) acc[k] = 0.f;
+    for (int p = 0; p < cnt; ++p) {
+      const int64_t t = ix.toks[off + p];
+      Vec8<BF16>::add(acc, __ldg(src + t * src_ld + src_off + vi));
+    }
+    emit<BF16, TABLE>(out_row, vi, acc, cs, E_row, scale, accumulate != 0);
+  }
+}
+
+// One block per (heavy row, slice of 32 vectors); warps split the row's tokens
+// round-robin and are combined in warp order.
+template <bool BF16, bool TABLE>
+__global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(
+    const SegIndexDev ix, const uint4* __restrict__ src, int64_t src_ld, int src_off, int n_vec,
+    const float* __restrict__ coef, const uint4* __restrict__ E, float* __restrict__ out, float scale,
+    int accumulate) {
+  constexpr int N = Vec8<BF16>::N;
+  __shared__ float part[kHeavyWarps][32 * N];
+  __shared__ float cpart[kHeavyWarps];
+  if (static_cast<int>(blockIdx.x) >= *ix.n_heavy) return;
+  const int64_t v = ix.heavy[blockIdx.x];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int vi = blockIdx.y * 32 + lane;
+  const bool active = vi < n_vec;
+  const int32_t cnt = ix.counts[v];
+  const int32_t off = ix.offsets[v];
+  float acc[N];
+#pragma unroll
+  for (int k = 0; k < N; ++k) acc[k] = 0.f;
+  float cs = 0.f;
+  for (int p = warp; p < cnt; p += kHeavyWarps) {
+    const int64_t t = ix.toks[off + p];
+    if (TABLE) cs += coef[t];
+    if (active) Vec8<BF16>::add(acc, __ldg(src + t * src_ld + src_off + vi));
+  }
+#pragma unroll
+  for (int k = 0; k < N; ++k) part[warp][lane * N + k] = acc[k];
+  if (lane == 0) cpart[warp] = cs;
+  __syncthreads();
+  if (warp == 0) {
+    float tot[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) tot[k] = 0.f;
+    float ctot = 0.f;
+    for (int w = 0; w < kHeavyWarps; ++w) {
+#pragma unroll
+      for (int k = 0; k < N; ++k) tot[k] += part[w][lane * N + k];
+      ctot += cpart[w];
+    }
+    if (active) {
+      float* out_row = out + v * static_cast<int64_t>(n_vec) * N;
+      const uint4* E_row = TABLE ? E + v * static_cast<int64_t>(n_vec) : nullptr;
+      emit<BF16, TABLE>(out_row, vi, tot, ctot, E_row, scale, accumulate != 0);
+    }
+  }
+}
+
+template <bool BF16, bool TABLE>
+cudaError_t launch_segsum(const SegIndexDev& ix, const uint4* src, int64_t src_ld, int src_off, int n_vec,
+                          const float* coef, const uint4* E, float* out, float scale, int accumulate,
+                          cudaStream_t st) {
+  const int64_t blocks = (ix.V * 32 + 255) / 256;
+  segsum_light_kernel<BF16, TABLE><<<static_cast<unsigned>(blocks), 256, 0, st>>>(ix, src, src_ld, src_off, n_vec,
+                                                                                 coef, E, out, scale, accumulate);
+  dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>((n_vec + 31) / 32));
+  segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, src, src_ld, src_off, n_vec, coef, E,
+                                                                      out, scale, accumulate);
+  note_launches(2);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t segindex_bytes(int64_t T, int64_t V) {
+  const int64_t nblk = (T + kSortBlock - 1) / kSortBlock;
+  const size_t t4 = static_cast<size_t>(T) * 4;
+  const int64_t max_heavy = T / (kHeavy + 1) + 1;
+  return up256(t4) * 4 + up256(static_cast<size_t>(256) * nblk * 4) + up256(static_cast<size_t>(V + 1) * 4) * 2 +
+         up256(static_cast<size_t>(max_heavy) * 4) + 256;
+}
+
+cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, SegIndexDev* out, cudaStream_t st) {
+  const int64_t nblk = (T + kSortBlock - 1) / kSortBlock;
+  const size_t t4 = static_cast<size_t>(T) * 4;
+  char* p = static_cast<char*>(ws);
+  int32_t* keys0 = reinterpret_cast<int32_t*>(p); p += up256(t4);
+  int32_t* keys1 = reinterpret_cast<int32_t*>(p); p += up256(t4);
+  int32_t* vals0 = reinterpret_cast<int32_t*>(p); p += up256(t4);
+  int32_t* vals1 = reinterpret_cast<int32_t*>(p); p += up256(t4);
+  int32_t* hist = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(256) * nblk * 4);
+  int32_t* counts = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V + 1) * 4);
+  int32_t* offsets = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V + 1) * 4);
+  const int64_t max_heavy = T / (kHeavy + 1) + 1;
+  int32_t* heavy = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(max_heavy) * 4);
+  int32_t* n_heavy = reinterpret_cast<int32_t*>(p);
+
+  // per-id counts and their exclusive prefix (segment offsets in sorted order)
+  cudaError_t err = cudaMemsetAsync(counts, 0, static_cast<size_t>(V + 1) * 4, st);
+  if (err == cudaSuccess) err = cudaMemsetAsync(n_heavy, 0, 4, st);
+  if (err != cudaSuccess) return err;
+  count_ids_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(ids, T, V, counts);
+  exclusive_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, static_cast<int>(V + 1));
+  heavy_list_kernel<<<static_cast<unsigned>((V + 255) / 256), 256, 0, st>>>(counts, V, heavy, n_heavy);
+  note_launches(3);
+
+  // stable radix sort of the ids carrying token indices
+  int bits = 1;
+  while ((int64_t(1) << bits) <= V) ++bits;          // keys live in [0, V]
+  const int passes = (bits + 7) / 8;
+  const int32_t* kin = nullptr;
+  const int32_t* vin = nullptr;
+  int32_t* kbuf[2] = {keys0, keys1};
+  int32_t* vbuf[2] = {vals0, vals1};
+  for (int pass = 0; pass < passes; ++pass) {
+    sort_hist_kernel<<<static_cast<unsigned>(nblk), kSortBlock, 0, st>>>(kin, ids, T, V, 8 * pass, hist,
+                                                                         static_cast<int>(nblk));
+    exclusive_scan_kernel<<<1, 1024, 0, st>>>(hist, hist, static_cast<int>(256 * nblk));
+    sort_scatter_kernel<<<static_cast<unsigned>(nblk), kSortBlock, 0, st>>>(
+        kin, vin, ids, T, V, 8 * pass, hist, static_cast<int>(nblk), kbuf[pass & 1], vbuf[pass & 1]);
+    note_launches(3);
+    kin = kbuf[pass & 1];
+    vin = vbuf[pass & 1];
+  }
+  out->V = V;
+  out->counts = counts;
+  out->offsets = offsets;
+  out->toks = vin;
+  out->heavy = heavy;
+  out->n_heavy = n_heavy;
+  out->max_heavy = max_heavy;
+  return cudaGetLastError();
+}
+
+cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
+                               const float* coef, const void* E, float* dE, bool accumulate, cudaStream_t st) {
+  const uint4* src = static_cast<const uint4*>(dy);
+  const int64_t ld = d_vec + dl_vec;
+  const uint4* e = static_cast<const uint4*>(E);
+  return bf16 ? launch_segsum<true, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, 0.f, accumulate, st)
+              : launch_segsum<false, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, 0.f, accumulate, st);
+}
+
+cudaError_t scatter_target_rows(const SegIndexDev& ix, const void* h, int d_vec, float* dW, float scale,
+                                cudaStream_t st) {
+  const uint4* src = static_cast<const uint4*>(h);
+  return launch_segsum<true, false>(ix, src, d_vec, 0, d_vec, nullptr, nullptr, dW, scale, 1, st);
+}
+
+}  // namespace mls

@@ -119,3 +119,48 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     out["loss"] = float(np.sum((1.0 - alpha_d) * out["ce_lm"][:M - 1])
                         + np.sum(alpha_d * out["ce_kd"]) + out["ce_lm"][M - 1])
     return out
+
+
+def multiexit_loss_vocab_rows(y, h, W, alpha_d=0.3, grad_scale=1.0, vrows=None, token_block=256):
+    """Losses over all tokens and the head-gradient rows dW^m[v] for v in vrows.
+
+    Same definitions as ``multiexit_loss``; the logits of every token are
+    computed (for the softmax normalisers), but the gradient is formed only in
+    the requested vocabulary columns:  dW^m[v] = sum_t G_m[t, v] h_m[t].
+    Returns a dict with ce_lm, ce_kd, loss and dW_rows (list of [len(vrows), D_m]).
+    """
+    y = np.asarray(y, dtype=np.int64)
+    vrows = np.asarray(vrows, dtype=np.int64)
+    M = len(h)
+    T = y.shape[0]
+    Ws = [_f64(w) for w in W]
+    g = grad_scale / T
+    ce_lm = np.zeros(M)
+    ce_kd = np.zeros(max(M - 1, 0))
+    dW_rows = [np.zeros((vrows.shape[0], w.shape[1])) for w in Ws]
+    for b0 in range(0, T, token_block):
+        yb = y[b0:b0 + token_block]
+        n = yb.shape[0]
+        ar = np.arange(n)
+        hb = [_f64(hm[b0:b0 + token_block]) for hm in h]
+        logits = [hb[m] @ Ws[m].T for m in range(M)]
+        lse = [logsumexp_rows(l) for l in logits]
+        logq = [logits[m] - lse[m][:, None] for m in range(M)]
+        pM = np.exp(logq[M - 1])
+        for m in range(M):
+            ce_lm[m] += np.sum(lse[m] - logits[m][ar, yb])
+        for m in range(M - 1):
+            ce_kd[m] += np.sum(-np.sum(pM * logq[m], axis=1))
+        onehot = (yb[:, None] == vrows[None, :]).astype(np.float64)
+        pM_sel = pM[:, vrows]
+        for m in range(M):
+            q_sel = np.exp(logq[m][:, vrows])
+            if m < M - 1:
+                G = g * (q_sel - (1.0 - alpha_d) * onehot - alpha_d * pM_sel)
+            else:
+                G = g * (q_sel - onehot)
+            dW_rows[m] += G.T @ hb[m]
+    ce_lm /= T
+    ce_kd /= T
+    loss = float(np.sum((1.0 - alpha_d) * ce_lm[:M - 1]) + np.sum(alpha_d * ce_kd) + ce_lm[M - 1])
+    return {"ce_lm": ce_lm, "ce_kd": ce_kd, "loss": loss, "dW_rows": dW_rows}

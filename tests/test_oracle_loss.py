@@ -11,7 +11,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle import multiexit_loss, softmax_rows
+from oracle import multiexit_loss, multiexit_loss_vocab_rows, softmax_rows
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_figures.json")
 
@@ -230,3 +230,15 @@ def test_single_exit_has_no_distillation():
     r = multiexit_loss(y, h, W, alpha_d=0.3)
     assert r["ce_kd"].shape == (0,)
     np.testing.assert_allclose(r["loss"], r["ce_lm"][0], rtol=1e-15)
+
+
+def test_vocab_row_restriction_matches_full_gradient():
+    # the restricted form must agree with the full definition on every requested row
+    y, h, W = _rand_suite(M=3, T=37, D=(4, 6, 8), V=29, seed=10)
+    full = multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=2.0, token_block=5)
+    rows = np.array([0, 28, 3, int(y[0]), 17])
+    r = multiexit_loss_vocab_rows(y, h, W, alpha_d=0.3, grad_scale=2.0, vrows=rows, token_block=8)
+    np.testing.assert_allclose(r["loss"], full["loss"], rtol=1e-13)
+    np.testing.assert_allclose(r["ce_kd"], full["ce_kd"], rtol=1e-13)
+    for m in range(3):
+        np.testing.assert_allclose(r["dW_rows"][m], full["dW"][m][rows], rtol=1e-12, atol=1e-15)

@@ -121,3 +121,54 @@ def test_repeated_calls_are_deterministic():
     g2 = multiexit_loss_bwd(y, h, W, s1, 0.3)
     for a, b in zip(g1[0] + g1[1], g2[0] + g2[1]):
         assert torch.equal(a, b)
+
+
+FULL = ["proxy2", "main3", "main3_aligned", "suite4"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    """Full-size workloads in the benchmark's launch configuration.
+
+    Sampled tokens: the per-token statistics and dh rows against the oracle.
+    Sampled vocabulary rows of dW against the oracle over all tokens (main3 and
+    proxy2; that needs the full fp64 forward).  At any size: the reported
+    losses equal the token means of the reported statistics, and the columns of
+    every dW sum to zero up to rounding.
+    """
+    cfg = wl.CONFIGS[name]
+    d = wl.make_inputs(cfg, with_tables=False)
+    y, h, W = _gpu_inputs(d)
+    M = cfg.M
+    st = new_status()
+    losses, stats = multiexit_loss_fwd(y, h, W, cfg.alpha_d, status=st)
+    dh, dW = multiexit_loss_bwd(y, h, W, stats, cfg.alpha_d, 1.0, status=st)
+    assert status_read(st) == (0, 0)
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(cfg.T, size=64, replace=False))
+    r = oracle.multiexit_loss(d.y, d.o, d.W, alpha_d=cfg.alpha_d, rows=rows)
+    s = f64(stats)
+    assert_stats_close(s[:M, rows], r["lse"], "lse")
+    assert_stats_close(s[M:2 * M, rows], r["tgt"], "target logits")
+    assert_stats_close(s[2 * M:, rows], r["S"], "teacher-weighted logits")
+    for m in range(M):
+        assert_grad_close(dh[m][torch.from_numpy(rows).cuda()], r["dh"][m], f"dh[{m}] rows")
+    # losses are the token means of the statistics
+    L = f64(losses)
+    ce_lm = (s[:M] - s[M:2 * M]).mean(axis=1)
+    ce_kd = (s[:M - 1] - s[2 * M:]).mean(axis=1)
+    assert_loss_close(L[:M], ce_lm, "CE_LM vs stats")
+    assert_loss_close(L[M:2 * M - 1], ce_kd, "CE_KD vs stats")
+    tot = np.sum((1 - cfg.alpha_d) * ce_lm[:M - 1]) + np.sum(cfg.alpha_d * ce_kd) + ce_lm[M - 1]
+    assert_loss_close(L[-1:], [tot], "L vs stats")
+    # sum over the vocabulary of every dW column vanishes (softmax rows sum to one)
+    for m in range(M):
+        col = dW[m].double().sum(dim=0)
+        scale = dW[m].double().abs().sum(dim=0)
+        assert float((col.abs() / scale.clamp_min(1e-30)).max()) < 2e-3, f"dW[{m}] column sums"
+    if name in ("proxy2", "main3"):
+        vrows = np.unique(np.concatenate([rng.choice(cfg.V, size=48, replace=False), d.y[:16]]))
+        rv = oracle.multiexit_loss_vocab_rows(d.y, d.o, d.W, alpha_d=cfg.alpha_d, vrows=vrows)
+        assert_loss_close(losses, np.concatenate([rv["ce_lm"], rv["ce_kd"], [rv["loss"]]]), "losses")
+        for m in range(M):
+            assert_grad_close(dW[m][torch.from_numpy(vrows).cuda()], rv["dW_rows"][m], f"dW[{m}] rows")
