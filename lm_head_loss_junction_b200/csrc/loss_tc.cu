@@ -1,12 +1,13 @@
 // Tensor-core (tcgen05 + TMEM + TMA) path of the multi-exit LM-head loss, bf16.
 //
-// Forward.  A persistent kernel walks (token tile of 128) x (vocab tile of 128)
-// output tiles.  For each tile it computes the logits of every exit into its
-// own TMEM region (teacher = largest exit first), and a 4-warp epilogue turns
-// them into per-row softmax statistics without ever writing logits out:
-//   teacher: lse_T over the tile and p~ = exp(l_T - max_T) kept in registers;
-//   student s: lse_s over the tile and Abar_s = sum_v p~_v l_s,v / sum_v p~_v.
-// A merge kernel combines the per-tile partials of every token exactly (log-
+// Forward.  A persistent kernel walks (token tile of 128) x (vocab tile of 256)
+// output tiles.  For each tile it computes the logits of every exit, teacher
+// (largest exit) first, into two alternating TMEM regions, and an 8-warp
+// epilogue turns each 128-column half ("split") into per-row softmax
+// statistics without ever writing logits out:
+//   teacher: lse_T over the split and p~ = exp(l_T - max_T) kept in registers;
+//   student s: lse_s over the split and Abar_s = sum_v p~_v l_s,v / sum_v p~_v.
+// A merge kernel combines the per-split partials of every token exactly (log-
 // sum-exp merge, teacher-weighted mean of Abar), which gives lse_m and
 // S_m = sum_v p_T,v l_m,v; a fixed-order reduction gives the losses.
 //
@@ -24,6 +25,7 @@
 // suite?" (section 4, the 0.7/0.3 mix), "Editing the methods of sub-models are
 // made of blocks" (Modeling paragraph: one LM head W^m in R^{V x D_m} per exit).
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <mutex>
 
 #include "kernels.h"
@@ -36,10 +38,19 @@ namespace {
 constexpr int kBM = 128;          // token rows per tile (UMMA M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle row of bf16
 constexpr int kUK = 16;           // K per tcgen05.mma (kind::f16)
-constexpr int kLossBN = 128;      // vocabulary columns per tile
-constexpr int kLossStages = 6;
-constexpr int kThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kThreads = 192;     // GEMM: warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Loss tile kernel geometry.  One tile = 128 tokens x 256 vocabulary columns;
+// each exit's logits of the tile are one accumulation "job" in TMEM.  Two
+// 256-column TMEM regions alternate between consecutive jobs, so the epilogue
+// of one job overlaps the MMAs of the next.  Eight epilogue warps: two per
+// TMEM lane quadrant, each owning one 128-column half ("split") of the tile.
+constexpr int kLossBN = 256;
+constexpr int kSplitCols = 128;
+constexpr int kLossStages = 4;
+constexpr int kLossEpiWarps = 8;
+constexpr int kLossThreads = 64 + 32 * kLossEpiWarps;
 
 // ------------------------------------------------------------------ shared layouts
 struct LossMaps {
@@ -55,7 +66,7 @@ struct LossArgs {
   int n_tt, n_vt, num_tiles, group_tt;
   const int32_t* y;
   float alpha;                 // alpha_d
-  float* partial;              // forward: [n_vt][2M-1][T]
+  float* partial;              // forward: [2 n_vt][2M-1][T]
   float* stats;                // forward: target rows written; backward: lse read
   __nv_bfloat16* G;            // backward: [M][T][V]
   int32_t* status;
@@ -66,8 +77,8 @@ struct __align__(1024) LossSmem {
   uint8_t b[kLossStages][kLossBN * kBK * 2];
   uint64_t full[kLossStages];
   uint64_t empty[kLossStages];
-  uint64_t tfull[kMaxExits];
-  uint64_t tempty[kMaxExits];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -97,10 +108,19 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32
   (void)mbar_wait(bar, parity, &dummy, status);
 }
 
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_half2(uint32_t u) {
+  return __half22float2(*reinterpret_cast<__half2*>(&u));
+}
+
 // ------------------------------------------------------------------ loss tile kernel
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_constant__ LossMaps maps,
-                                                                const LossArgs a) {
+__global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid_constant__ LossMaps maps,
+                                                                    const LossArgs a) {
   extern __shared__ uint8_t smem_raw[];
   LossSmem& s = *reinterpret_cast<LossSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -113,9 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    for (int m = 0; m < kMaxExits; ++m) {
-      mbar_init(&s.tfull[m], 1);
-      mbar_init(&s.tempty[m], 4);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&s.tfull[r], 1);
+      mbar_init(&s.tempty[r], kLossEpiWarps);
     }
     mbar_init(&s.drain, 1);
     s.abort = 0;
@@ -145,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
         int tt, vt;
         loss_tile_coords(tile, a, tt, vt);
         for (int j = 0; j < M && ok; ++j) {
-          const int m = M - 1 - j;
+          const int m = M - 1 - j;                // teacher first, then students
           for (int kb = 0; kb < a.kblocks[m]; ++kb) {
             if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, a.status)) { ok = false; break; }
             mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
@@ -170,14 +190,15 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kBM, kLossBN, false, false);
-      uint32_t stage = 0, phase = 0, iter = 0;
+      uint32_t stage = 0, phase = 0, job = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x, ++iter) {
-        for (int j = 0; j < M && ok; ++j) {
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+        for (int j = 0; j < M && ok; ++j, ++job) {
           const int m = M - 1 - j;
-          if (!mbar_wait(&s.tempty[m], (iter & 1) ^ 1, abort, a.status)) { ok = false; break; }
+          const uint32_t region = job & 1;
+          if (!mbar_wait(&s.tempty[region], ((job >> 1) & 1) ^ 1, abort, a.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d = tmem + static_cast<uint32_t>(m * kLossBN);
+          const uint32_t d = tmem + region * kLossBN;
           for (int kb = 0; kb < a.kblocks[m]; ++kb) {
             if (!mbar_wait(&s.full[stage], phase, abort, a.status)) { ok = false; break; }
             tc_fence_after();
@@ -192,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
             umma_commit(&s.empty[stage]);
             if (++stage == kLossStages) { stage = 0; phase ^= 1; }
           }
-          if (ok) umma_commit(&s.tfull[m]);
+          if (ok) umma_commit(&s.tfull[region]);
         }
       }
       // Make sure every MMA issued has finished before TMEM is released.
@@ -200,145 +221,150 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
       drain_wait(&s.drain, 0, a.status);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (4 warps)
-    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    // ---------------------------------------------------------------- epilogue (8 warps)
+    const int q = warp & 3;                          // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;                // which 128-column split of the tile
     const int row = q * 32 + lane;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * kSplitCols;
     const int Q = 2 * M - 1;
-    uint32_t iter = 0;
-    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x, ++iter) {
+    const float al = a.alpha;
+    uint32_t job = 0;
+    // teacher probabilities of this thread's row and split, packed fp16 pairs
+    uint32_t pt[4][16];
+    float inv_z = 0.f;
+    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
       int tt, vt;
       loss_tile_coords(tile, a, tt, vt);
       const int t = tt * kBM + row;
       const bool valid = t < a.T;
-      const int v0 = vt * kLossBN;
+      const int c0 = vt * kLossBN + half * kSplitCols;     // first vocabulary column of the split
+      const bool live = c0 < a.V;                           // the last tile may be half outside V
+      const int split = vt * 2 + half;
       const int yt = valid ? __ldg(a.y + t) : -1;
-      const int yl = yt - v0;                  // target column inside this tile, if any
-      const bool has_tgt = valid && yl >= 0 && yl < kLossBN;
-
-      // ---------------- teacher
-      if (!warp_wait(&s.tfull[M - 1], iter & 1, abort, a.status)) break;
-      tc_fence_after();
-      float p[4][32];
+      const int yl = yt - c0;                               // target column inside this split, if any
+      const bool has_tgt = valid && yl >= 0 && yl < kSplitCols;
+      const bool bad = valid && (yt < 0 || yt >= a.V);
+      bool stop = false;
+      for (int j = 0; j < M; ++j, ++job) {
+        const int m = M - 1 - j;
+        const uint32_t region = job & 1;
+        const uint32_t base = lane_base + region * kLossBN;
+        if (!warp_wait(&s.tfull[region], (job >> 1) & 1, abort, a.status)) { stop = true; break; }
+        tc_fence_after();
+        if (MODE == kModeStats) {
+          float lse_part = -INFINITY, abar = 0.f;
+          if (live) {
+            if (j == 0) {
+              // teacher: split max, then p~ = exp(l - max) (fp16 in registers) and their sum
+              float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + (M - 1) * kLossBN + c * 32, p[c]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.tempty[M - 1]);
-
-      if (MODE == kModeStats) {
-        float mx = -INFINITY;
+              for (int c = 0; c < 4; ++c) {
+                float r[32];
+                tmem_ld32(base + c * 32, r);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+                for (int k = 0; k < 32; ++k) mx = fmaxf(mx, r[k]);
+                if (has_tgt && (yl >> 5) == c) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) mx = fmaxf(mx, p[c][j]);
-        if (has_tgt) {
+                  for (int k = 0; k < 32; ++k)
+                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.T + t] = r[k];
+                }
+              }
+              const float mxs = mx * kLog2e;
+              float z = 0.f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+              for (int c = 0; c < 4; ++c) {
+                float r[32];
+                tmem_ld32(base + c * 32, r);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c * 32 + j == yl) a.stats[static_cast<int64_t>(M + M - 1) * a.T + t] = p[c][j];
-        }
-        const float mxs = mx * kLog2e;
-        float z = 0.f;
+                for (int k = 0; k < 32; k += 2) {
+                  const float e0 = exp2f(fmaf(r[k], kLog2e, -mxs));
+                  const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -mxs));
+                  z += e0 + e1;
+                  pt[c][k / 2] = pack_half2(e0, e1);
+                }
+              }
+              inv_z = 1.f / z;
+              lse_part = mx + logf(z);
+            } else {
+              // student: online max/sum over the split and the teacher-weighted sum of its logits
+              float ms = -INFINITY, zs = 0.f, A = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+              for (int c = 0; c < 4; ++c) {
+                float r[32];
+                tmem_ld32(base + c * 32, r);
+                float cm = r[0];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            p[c][j] = exp2f(fmaf(p[c][j], kLog2e, -mxs));
-            z += p[c][j];
-          }
-        const float inv_z = 1.f / z;
-        if (valid) a.partial[(static_cast<int64_t>(vt) * Q + (M - 1)) * a.T + t] = mx + logf(z);
-
-        // ---------------- students, largest first
-        for (int sidx = M - 2; sidx >= 0; --sidx) {
-          if (!warp_wait(&s.tfull[sidx], iter & 1, abort, a.status)) break;
-          tc_fence_after();
-          float ms = -INFINITY, zs = 0.f, A = 0.f;
+                for (int k = 1; k < 32; ++k) cm = fmaxf(cm, r[k]);
+                const float mn = fmaxf(ms, cm);
+                const float mns = mn * kLog2e;
+                float zc = 0.f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float r[32];
-            tmem_ld32(lane_base + sidx * kLossBN + c * 32, r);
-            float cm = r[0];
+                for (int k = 0; k < 32; k += 2) {
+                  zc += exp2f(fmaf(r[k], kLog2e, -mns)) + exp2f(fmaf(r[k + 1], kLog2e, -mns));
+                  const float2 pp = unpack_half2(pt[c][k / 2]);
+                  A = fmaf(pp.x, r[k], A);
+                  A = fmaf(pp.y, r[k + 1], A);
+                }
+                zs = zs * exp2f((ms - mn) * kLog2e) + zc;
+                ms = mn;
+                if (has_tgt && (yl >> 5) == c) {
 #pragma unroll
-            for (int j = 1; j < 32; ++j) cm = fmaxf(cm, r[j]);
-            const float mn = fmaxf(ms, cm);
-            const float mns = mn * kLog2e;
-            float zc = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              zc += exp2f(fmaf(r[j], kLog2e, -mns));
-              A = fmaf(p[c][j], r[j], A);
-            }
-            zs = zs * exp2f((ms - mn) * kLog2e) + zc;
-            ms = mn;
-            if (has_tgt && (yl >> 5) == c) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j == (yl & 31)) a.stats[static_cast<int64_t>(M + sidx) * a.T + t] = r[j];
-            }
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[sidx]);
-          if (valid) {
-            a.partial[(static_cast<int64_t>(vt) * Q + sidx) * a.T + t] = ms + logf(zs);
-            a.partial[(static_cast<int64_t>(vt) * Q + M + sidx) * a.T + t] = A * inv_z;
-          }
-        }
-        if (*abort) break;
-      } else {
-        // ---------------- backward: G' tiles in bf16
-        const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
-        const float lTs = lseT * kLog2e;
-        const bool bad = valid && (yt < 0 || yt >= a.V);
-        const int64_t g_row = (static_cast<int64_t>(M - 1) * a.T + t) * a.V + v0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t packed[16];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) p[c][j] = exp2f(fmaf(p[c][j], kLog2e, -lTs));
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) packed[j / 2] = bad ? 0u : pack_bf16x2(p[c][j], p[c][j + 1]);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(a.G + g_row + c * 32);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
-          }
-        }
-        const float al = a.alpha;
-        for (int sidx = M - 2; sidx >= 0; --sidx) {
-          if (!warp_wait(&s.tfull[sidx], iter & 1, abort, a.status)) break;
-          tc_fence_after();
-          const float lse = valid ? a.stats[static_cast<int64_t>(sidx) * a.T + t] : 0.f;
-          const float ls = lse * kLog2e;
-          const int64_t row_off = (static_cast<int64_t>(sidx) * a.T + t) * a.V + v0;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float r[32];
-            tmem_ld32(lane_base + sidx * kLossBN + c * 32, r);
-            uint32_t packed[16];
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float g0 = fmaf(-al, p[c][j], exp2f(fmaf(r[j], kLog2e, -ls)));
-              const float g1 = fmaf(-al, p[c][j + 1], exp2f(fmaf(r[j + 1], kLog2e, -ls)));
-              packed[j / 2] = bad ? 0u : pack_bf16x2(g0, g1);
-            }
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(a.G + row_off + c * 32);
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+                  for (int k = 0; k < 32; ++k)
+                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.T + t] = r[k];
+                }
+              }
+              lse_part = ms + logf(zs);
+              abar = A * inv_z;
             }
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[sidx]);
+          if (lane == 0) mbar_arrive(&s.tempty[region]);
+          if (valid) {
+            a.partial[(static_cast<int64_t>(split) * Q + m) * a.T + t] = lse_part;
+            if (j > 0) a.partial[(static_cast<int64_t>(split) * Q + M + m) * a.T + t] = abar;
+          }
+        } else {
+          // ---------------- backward: dense part of the logit gradient, bf16
+          if (live) {
+            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
+            const float ls = lse * kLog2e;
+            __nv_bfloat16* grow = a.G + (static_cast<int64_t>(m) * a.T + t) * a.V + c0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float r[32];
+              tmem_ld32(base + c * 32, r);
+              uint32_t packed[16];
+#pragma unroll
+              for (int k = 0; k < 32; k += 2) {
+                const float e0 = exp2f(fmaf(r[k], kLog2e, -ls));
+                const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -ls));
+                float g0, g1;
+                if (j == 0) {                      // teacher: G' = p_T
+                  pt[c][k / 2] = pack_half2(e0, e1);
+                  g0 = e0;
+                  g1 = e1;
+                } else {                           // student: G' = q - alpha_d p_T
+                  const float2 pp = unpack_half2(pt[c][k / 2]);
+                  g0 = fmaf(-al, pp.x, e0);
+                  g1 = fmaf(-al, pp.y, e1);
+                }
+                packed[k / 2] = bad ? 0u : pack_bf16x2(g0, g1);
+              }
+              if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tempty[region]);
         }
-        if (*abort) break;
       }
+      if (stop || *abort) break;
     }
   }
 
@@ -351,45 +377,82 @@ __global__ void __launch_bounds__(kThreads, 1) loss_tile_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------ merge kernel
-// Per token: combine the per-vocab-tile partials into lse_m and S_m, write the
-// stats rows and the per-token loss terms.
-__global__ void __launch_bounds__(256) loss_merge_kernel(const float* __restrict__ partial, int n_vt, int M,
-                                                         int T, int V, const int32_t* __restrict__ y,
-                                                         float* __restrict__ stats, float* __restrict__ terms,
-                                                         int32_t* status) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
+// Per token: combine the per-split partials into lse_m and S_m, write the stats
+// rows and the per-token loss terms.  A block covers 32 tokens; its 8 thread
+// rows each merge a contiguous range of splits, and the 8 results are combined
+// in row order (deterministic).
+constexpr int kMergeRows = 8;
+
+__global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float* __restrict__ partial, int n_splits,
+                                                                     int M, int T, int V,
+                                                                     const int32_t* __restrict__ y,
+                                                                     float* __restrict__ stats,
+                                                                     float* __restrict__ terms, int32_t* status) {
+  constexpr int S = kMaxExits - 1;
+  __shared__ float st_mT[kMergeRows][32], st_zT[kMergeRows][32];
+  __shared__ float st_A[kMergeRows][S][32], st_ms[kMergeRows][S][32], st_zs[kMergeRows][S][32];
+  const int lane = threadIdx.x, rowi = threadIdx.y;
+  const int t = blockIdx.x * 32 + lane;
   const int Q = 2 * M - 1;
+  const int per = (n_splits + kMergeRows - 1) / kMergeRows;
+  const int i0 = min(n_splits, rowi * per), i1 = min(n_splits, i0 + per);
+  float mT = -INFINITY, zT = 0.f;
+  float A[S] = {0.f, 0.f, 0.f}, ms[S] = {-INFINITY, -INFINITY, -INFINITY}, zs[S] = {0.f, 0.f, 0.f};
+  if (t < T) {
+    for (int i = i0; i < i1; ++i) {
+      const float* pi = partial + static_cast<int64_t>(i) * Q * T + t;
+      const float l = pi[static_cast<int64_t>(M - 1) * T];
+      if (l > mT) {
+        const float r = __expf(mT - l);
+        zT *= r;
+        for (int s = 0; s < M - 1; ++s) A[s] *= r;
+        mT = l;
+      }
+      const float w = (l == -INFINITY) ? 0.f : __expf(l - mT);
+      zT += w;
+      for (int s = 0; s < M - 1; ++s) {
+        A[s] = fmaf(w, pi[static_cast<int64_t>(M + s) * T], A[s]);
+        const float ls = pi[static_cast<int64_t>(s) * T];
+        if (ls > ms[s]) { zs[s] *= __expf(ms[s] - ls); ms[s] = ls; }
+        if (ls != -INFINITY) zs[s] += __expf(ls - ms[s]);
+      }
+    }
+  }
+  st_mT[rowi][lane] = mT;
+  st_zT[rowi][lane] = zT;
+  for (int s = 0; s < S; ++s) {
+    st_A[rowi][s][lane] = A[s];
+    st_ms[rowi][s][lane] = ms[s];
+    st_zs[rowi][s][lane] = zs[s];
+  }
+  __syncthreads();
+  if (rowi != 0 || t >= T) return;
+  for (int r = 1; r < kMergeRows; ++r) {
+    const float m2 = st_mT[r][lane], z2 = st_zT[r][lane];
+    const float mm = fmaxf(mT, m2);
+    const float r1 = (mT == -INFINITY) ? 0.f : __expf(mT - mm);
+    const float r2 = (m2 == -INFINITY) ? 0.f : __expf(m2 - mm);
+    zT = zT * r1 + z2 * r2;
+    for (int s = 0; s < M - 1; ++s) {
+      A[s] = A[s] * r1 + st_A[r][s][lane] * r2;
+      const float n2 = st_ms[r][s][lane], y2 = st_zs[r][s][lane];
+      const float mn = fmaxf(ms[s], n2);
+      const float q1 = (ms[s] == -INFINITY) ? 0.f : __expf(ms[s] - mn);
+      const float q2 = (n2 == -INFINITY) ? 0.f : __expf(n2 - mn);
+      zs[s] = zs[s] * q1 + y2 * q2;
+      ms[s] = mn;
+    }
+    mT = mm;
+  }
   const int yt = y[t];
   const bool bad = yt < 0 || yt >= V;
-  // teacher, with the teacher-weighted means of every student
-  float mT = -INFINITY, zT = 0.f;
-  float Sacc[kMaxExits - 1] = {0.f, 0.f, 0.f};
-  for (int i = 0; i < n_vt; ++i) {
-    const float l = partial[(static_cast<int64_t>(i) * Q + (M - 1)) * T + t];
-    if (l > mT) {
-      const float r = __expf(mT - l);
-      zT *= r;
-      for (int s = 0; s < M - 1; ++s) Sacc[s] *= r;
-      mT = l;
-    }
-    const float w = __expf(l - mT);
-    zT += w;
-    for (int s = 0; s < M - 1; ++s) Sacc[s] = fmaf(w, partial[(static_cast<int64_t>(i) * Q + M + s) * T + t], Sacc[s]);
-  }
   const float lseT = mT + logf(zT);
   stats[static_cast<int64_t>(M - 1) * T + t] = lseT;
-  if (bad) stats[static_cast<int64_t>(M + M - 1) * T + t] = 0.f;
+  if (bad) stats[static_cast<int64_t>(2 * M - 1) * T + t] = 0.f;
   terms[static_cast<int64_t>(M - 1) * T + t] = bad ? 0.f : lseT - stats[static_cast<int64_t>(2 * M - 1) * T + t];
   for (int s = 0; s < M - 1; ++s) {
-    float ms = -INFINITY, zs = 0.f;
-    for (int i = 0; i < n_vt; ++i) {
-      const float l = partial[(static_cast<int64_t>(i) * Q + s) * T + t];
-      if (l > ms) { zs *= __expf(ms - l); ms = l; }
-      zs += __expf(l - ms);
-    }
-    const float lse = ms + logf(zs);
-    const float Sv = Sacc[s] / zT;
+    const float lse = ms[s] + logf(zs[s]);
+    const float Sv = A[s] / zT;
     stats[static_cast<int64_t>(s) * T + t] = lse;
     stats[static_cast<int64_t>(2 * M + s) * T + t] = Sv;
     if (bad) stats[static_cast<int64_t>(M + s) * T + t] = 0.f;
@@ -676,9 +739,10 @@ struct TcWs {
   float* terms;
 };
 
+int loss_n_vt(const LossProblem& p) { return static_cast<int>((p.V + kLossBN - 1) / kLossBN); }
+
 TcWs fwd_layout(const LossProblem& p, void* ws) {
-  const int n_vt = static_cast<int>(p.V / kLossBN);
-  const size_t part = static_cast<size_t>(n_vt) * (2 * p.M - 1) * p.T * sizeof(float);
+  const size_t part = static_cast<size_t>(2 * loss_n_vt(p)) * (2 * p.M - 1) * p.T * sizeof(float);
   TcWs w;
   w.partial = static_cast<float*>(ws);
   w.terms = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(part));
@@ -698,7 +762,7 @@ cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaSt
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-  fn<<<grid, kThreads, smem, st>>>(maps, a);
+  fn<<<grid, kLossThreads, smem, st>>>(maps, a);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -710,7 +774,7 @@ LossArgs base_args(const LossProblem& p) {
   a.V = static_cast<int>(p.V);
   for (int m = 0; m < p.M; ++m) a.kblocks[m] = static_cast<int>(p.D[m] / kBK);
   a.n_tt = static_cast<int>((p.T + kBM - 1) / kBM);
-  a.n_vt = static_cast<int>(p.V / kLossBN);
+  a.n_vt = loss_n_vt(p);
   a.num_tiles = a.n_tt * a.n_vt;
   a.group_tt = 16;
   a.y = p.y;
@@ -779,8 +843,7 @@ cudaError_t run_dw(const __nv_bfloat16* G, const void* h, float* dW, int T, int 
 bool tensor_map_encoder_available() { return get_encoder() != nullptr; }
 
 size_t loss_tc_fwd_bytes(const LossProblem& p) {
-  const int64_t n_vt = p.V / kLossBN;
-  const size_t part = static_cast<size_t>(n_vt) * (2 * p.M - 1) * p.T * sizeof(float);
+  const size_t part = static_cast<size_t>(2 * loss_n_vt(p)) * (2 * p.M - 1) * p.T * sizeof(float);
   const size_t terms = static_cast<size_t>(2 * p.M - 1) * p.T * sizeof(float);
   return align_up(part) + align_up(terms);
 }
@@ -797,8 +860,9 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   cudaError_t err = run_loss_tiles<kModeStats>(p, a, st);
   if (err != cudaSuccess) return err;
   const int T = static_cast<int>(p.T);
-  loss_merge_kernel<<<(T + 255) / 256, 256, 0, st>>>(w.partial, a.n_vt, p.M, T, static_cast<int>(p.V), p.y,
-                                                      stats, w.terms, p.status);
+  loss_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
+                                                                     static_cast<int>(p.V), p.y, stats, w.terms,
+                                                                     p.status);
   note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;

@@ -153,18 +153,31 @@ template <bool BF16, bool TABLE>
 __device__ __forceinline__ void emit(float* out_row, int vi, const float (&acc)[Vec8<BF16>::N], float cs,
                                      const uint4* E_row, float scale, bool accumulate) {
   constexpr int N = Vec8<BF16>::N;
-  float* o = out_row + static_cast<int64_t>(vi) * N;
+  float4* o = reinterpret_cast<float4*>(out_row + static_cast<int64_t>(vi) * N);
+  float val[N];
   if (TABLE) {
     float e[N];
     Vec8<BF16>::load(__ldg(E_row + vi), e);
 #pragma unroll
-    for (int k = 0; k < N; ++k) {
-      const float val = fmaf(cs, e[k], acc[k]);
-      o[k] = accumulate ? o[k] + val : val;
-    }
-  } else {
+    for (int k = 0; k < N; ++k) val[k] = fmaf(cs, e[k], acc[k]);
+  }
 #pragma unroll
-    for (int k = 0; k < N; ++k) o[k] = fmaf(-scale, acc[k], o[k]);
+  for (int q = 0; q < N / 4; ++q) {
+    float4 r;
+    if (TABLE) {
+      r = make_float4(val[4 * q], val[4 * q + 1], val[4 * q + 2], val[4 * q + 3]);
+      if (accumulate) {
+        const float4 b = o[q];
+        r.x += b.x; r.y += b.y; r.z += b.z; r.w += b.w;
+      }
+    } else {
+      r = o[q];
+      r.x = fmaf(-scale, acc[4 * q], r.x);
+      r.y = fmaf(-scale, acc[4 * q + 1], r.y);
+      r.z = fmaf(-scale, acc[4 * q + 2], r.z);
+      r.w = fmaf(-scale, acc[4 * q + 3], r.w);
+    }
+    o[q] = r;
   }
 }
 
