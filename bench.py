@@ -141,30 +141,36 @@ class Step:
         self.ws_j = torch.empty(api.junction_bwd_workspace(T, V), dtype=torch.uint8, device=device)
         self.status = api.new_status(device)
 
-    def run(self, stream=None, marks=None):
+    def phases(self):
+        """The step as four stream-ordered callables f(stream): junction fwd,
+        loss fwd, loss bwd, junction bwd (fed with dh_{m+1})."""
         a, c = self.api, self.cfg
         M = c.M
 
-        def mark(i):
-            if marks is not None:
-                marks[i].record(stream)
+        def junction_fwd(stream):
+            for j in range(M - 1):
+                a.junction_fwd(self.x, self.o[j], self.E[j + 1], out=self.jy[j], scale_out=self.jscale[j],
+                               status=self.status, stream=stream)
 
-        mark(0)
-        for j in range(M - 1):
-            a.junction_fwd(self.x, self.o[j], self.E[j + 1], out=self.jy[j], scale_out=self.jscale[j],
-                           status=self.status, stream=stream)
-        mark(1)
-        a.multiexit_loss_fwd(self.y, self.o, self.W, c.alpha_d, losses=self.losses, stats=self.stats,
-                             workspace=self.ws_loss, status=self.status, stream=stream)
-        mark(2)
-        a.multiexit_loss_bwd(self.y, self.o, self.W, self.stats, c.alpha_d, 1.0, dh=self.dh, dW=self.dW,
-                             workspace=self.ws_loss, status=self.status, stream=stream)
-        mark(3)
-        for j in range(M - 1):
-            a.junction_bwd(self.x, self.o[j], self.E[j + 1], self.dh[j + 1], do_out=self.do[j],
-                           de_out=self.de[j], dE=self.dE[j], accumulate_dE=False, workspace=self.ws_j,
-                           status=self.status, stream=stream)
-        mark(4)
+        def loss_fwd(stream):
+            a.multiexit_loss_fwd(self.y, self.o, self.W, c.alpha_d, losses=self.losses, stats=self.stats,
+                                 workspace=self.ws_loss, status=self.status, stream=stream)
+
+        def loss_bwd(stream):
+            a.multiexit_loss_bwd(self.y, self.o, self.W, self.stats, c.alpha_d, 1.0, dh=self.dh, dW=self.dW,
+                                 workspace=self.ws_loss, status=self.status, stream=stream)
+
+        def junction_bwd(stream):
+            for j in range(M - 1):
+                a.junction_bwd(self.x, self.o[j], self.E[j + 1], self.dh[j + 1], do_out=self.do[j],
+                               de_out=self.de[j], dE=self.dE[j], accumulate_dE=False, workspace=self.ws_j,
+                               status=self.status, stream=stream)
+
+        return [junction_fwd, loss_fwd, loss_bwd, junction_bwd]
+
+    def run(self, stream=None):
+        for f in self.phases():
+            f(stream)
 
     def working_set_gb(self):
         ts = [self.x, self.y] + self.o + self.E[1:] + self.W + self.dh + self.dW + self.jy + self.do + self.de + \
@@ -275,9 +281,16 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload with this many tokens per GPU instead of its own batch")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every step from Python instead of replaying a captured CUDA graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = wl.CONFIGS[args.workload]
+    if args.tokens:
+        seq = min(cfg.seq, args.tokens)
+        cfg = wl.small_variant(cfg, batch=max(1, args.tokens // seq), seq=seq, name_suffix=f"T{args.tokens}")
 
     if args.impl == "reference":
         run_reference(args, cfg)
@@ -308,21 +321,45 @@ def main():
     code, word = step.api.status_read(step.status, stream)
     if code != 0:
         raise RuntimeError(f"device status after warm-up: {code} ({word})")
+    l0 = _lib.lib().mls_kernel_launches()
+    step.run(stream)
+    launches_per_step = _lib.lib().mls_kernel_launches() - l0
+
+    # The four phases of a step, each captured once as a CUDA graph and
+    # replayed (the library launches only stream-ordered work), so the timed
+    # region carries no Python launch overhead.  --eager launches from Python.
+    phase_fns = step.phases()
+    if args.eager:
+        runners = [lambda f=f: f(stream) for f in phase_fns]
+    else:
+        graphs = []
+        for f in phase_fns:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                f(None)
+            graphs.append(g)
+        runners = [g.replay for g in graphs]
+        for _ in range(2):
+            for r in runners:
+                r()
+    barrier()
 
     # ---------------- timed region: K steps, events between phases
     K = args.steps
     marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    launches0 = _lib.lib().mls_kernel_launches()
     barrier()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         start.record(stream)
         for k in range(K):
-            step.run(stream, marks[k])
+            for i, r in enumerate(runners):
+                marks[k][i].record(stream)
+                r()
+            marks[k][4].record(stream)
         end.record(stream)
         barrier()
-    launches = _lib.lib().mls_kernel_launches() - launches0
+    launches = launches_per_step * K
     ms_total = start.elapsed_time(end)
     ms_total = _max_over_ranks(ms_total, ws, device)
     ms_step = ms_total / K
@@ -344,20 +381,27 @@ def main():
         host_out = torch.empty(step.losses.shape, dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host_in)
         d2h = host_out.numel() * host_out.element_size()
-        for _ in range(2):
+        def e2e_step(s):
             for hsrc, ddst in zip(host_in, dev_in):
                 ddst.copy_(hsrc, non_blocking=True)
-            step.run(stream)
+            step.run(s)
             host_out.copy_(step.losses, non_blocking=True)
+
+        if args.eager:
+            e2e_run = lambda: e2e_step(stream)  # noqa: E731
+        else:
+            ge = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ge, capture_error_mode="relaxed"):
+                e2e_step(None)
+            e2e_run = ge.replay
+        for _ in range(2):
+            e2e_run()
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(K):
-            for hsrc, ddst in zip(host_in, dev_in):
-                ddst.copy_(hsrc, non_blocking=True)
-            step.run(stream)
-            host_out.copy_(step.losses, non_blocking=True)
+            e2e_run()
         e1.record(stream)
         barrier()
         ms_e2e = _max_over_ranks(e0.elapsed_time(e1), ws, device)
@@ -404,7 +448,8 @@ def main():
                        "M": c.M, "D": list(c.D), "V": c.V, "alpha_d": c.alpha_d,
                        "parallelism": f"dp{ws} (independent batches)",
                        "l2": f"no flush; per-step working set {step.working_set_gb():.2f} GB > 126 MB L2"},
-            "e2e": e2e, "gpu_launches": int(launches), "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": int(launches), "launch_mode": "eager" if args.eager else "cuda_graph",
+            "roofline": roofline, "cpu_baseline": cpu,
             "phases": phases, "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

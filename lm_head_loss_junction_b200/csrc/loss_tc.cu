@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           }
         } else {
           // ---------------- backward: dense part of the logit gradient, bf16
+          if (bad && j == 0 && vt == 0 && half == 0) set_flag(a.status, MLS_DEVFLAG_BAD_ID);
           if (live) {
             const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
             const float ls = lse * kLog2e;
