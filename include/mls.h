@@ -124,6 +124,35 @@ mls_status mls_junction_bwd(const int32_t* x, int64_t T,
 /* Scratch bytes mls_junction_bwd needs for the dE_table scatter. */
 mls_status mls_junction_bwd_workspace(int64_t T, int64_t V, size_t* bytes);
 
+/*
+ * mls_junction_bwd_noalloc -- mls_junction_bwd without a workspace argument.
+ * The paper has no counterpart: this is a convenience of this library.
+ *
+ * For callers that cannot allocate device memory where they call the junction
+ * backward pass: code running while a stream is captured into a CUDA graph
+ * (cudaMalloc cannot be captured), code that must not block on the device
+ * (cudaMalloc/cudaFree may synchronise), or programs whose device memory is
+ * all handed out by another allocator.  The table-gradient scratch comes from
+ * a fixed 4 MiB array in the library's own device memory, held by every GPU
+ * that loads the library until the process exits; nothing is allocated.
+ *
+ * Arguments, results and errors are those of mls_junction_bwd.  Additionally:
+ *   - with dE_table non-NULL, (T, V) must satisfy
+ *     mls_junction_bwd_workspace(T, V) <= 4 MiB (for example T <= 65536 with
+ *     V <= 262144); larger sizes return MLS_ERR_UNSUPPORTED and launch nothing;
+ *   - every call on a device shares the one array: calls whose work overlaps
+ *     on the GPU (different streams, or different host threads, without
+ *     ordering between them) race on it and give undefined results;
+ *   - the first call on each device looks the array's address up (once) and
+ *     must come before any stream capture on that device.
+ */
+mls_status mls_junction_bwd_noalloc(const int32_t* x, int64_t T,
+                                    const void* o_m, int64_t D_m,
+                                    const void* e_next, int64_t V, int64_t delta,
+                                    const void* dy, void* do_m, void* de_rows,
+                                    float* dE_table, int accumulate_dE,
+                                    mls_dtype dt, int32_t* dev_status, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Multi-exit LM-head loss                                                   */
 /* ------------------------------------------------------------------------ */

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmls.so")
-SOURCES = ["api.cu", "junction.cu", "segsum.cu", "loss_simt.cu", "loss_tc.cu"]
+SOURCES = ["api.cu", "junction.cu", "segsum.cu", "loss_simt.cu", "loss_tc.cu", "junction_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
