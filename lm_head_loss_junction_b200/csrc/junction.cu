@@ -94,10 +94,13 @@ __device__ __forceinline__ uint4 add_scaled_vec(const uint4& g, float c, const u
 }
 
 // ---------------------------------------------------------------- forward
-// CAP = 16-byte vectors per lane kept in registers; columns beyond
-// CAP*32 vectors are re-read in the second pass.
+// One warp per token.  Pass 1 streams the block-output row (kept in registers,
+// CAP 16-byte vectors per lane) and the embedding row (copied straight to the
+// output: it does not depend on the scale) while accumulating both squared
+// norms; pass 2 writes the rescaled block output from registers.  Columns
+// beyond CAP*32 vectors are re-read in pass 2.
 template <bool BF16, int CAP>
-__global__ void __launch_bounds__(256) junction_fwd_kernel(const int32_t* __restrict__ x, int64_t T,
+__global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __restrict__ x, int64_t T,
                                                            const uint4* __restrict__ o, int d_vec,
                                                            const uint4* __restrict__ E, int64_t V,
                                                            int dl_vec, uint4* __restrict__ y,
@@ -107,35 +110,41 @@ __global__ void __launch_bounds__(256) junction_fwd_kernel(const int32_t* __rest
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int dp_vec = d_vec + dl_vec;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
   for (int64_t t = warp0; t < T; t += nwarps) {
     const int32_t id = __ldg(x + t);
     const bool bad = (id < 0) || (static_cast<int64_t>(id) >= V);
     const uint4* orow = o + t * d_vec;
     const uint4* erow = E + static_cast<int64_t>(bad ? 0 : id) * dl_vec;
-    uint4 oc[CAP], ec[CAP];
+    uint4* yrow = y + t * dp_vec;
+    uint4 oc[CAP];
     float so = 0.f, se = 0.f;
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
       const int i = j * 32 + lane;
-      if (i < d_vec) { oc[j] = __ldcs(orow + i); so += sumsq<BF16>(oc[j]); }
-      if (i < dl_vec) { ec[j] = __ldg(erow + i); se += sumsq<BF16>(ec[j]); }
+      if (i < d_vec) oc[j] = __ldcs(orow + i);
+    }
+    for (int i = lane; i < dl_vec; i += 32) {
+      const uint4 ev = __ldg(erow + i);
+      se += sumsq<BF16>(ev);
+      yrow[d_vec + i] = bad ? zero : ev;
+    }
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < d_vec) so += sumsq<BF16>(oc[j]);
     }
     for (int i = CAP * 32 + lane; i < d_vec; i += 32) so += sumsq<BF16>(orow[i]);
-    for (int i = CAP * 32 + lane; i < dl_vec; i += 32) se += sumsq<BF16>(__ldg(erow + i));
     so = warp_sum(so);
     se = warp_sum(se);
     float s = sqrtf(se) / fmaxf(sqrtf(so), kJunctionEps);
     if (bad) s = 0.f;
-    uint4* yrow = y + t * dp_vec;
-    const uint4 zero = make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
       const int i = j * 32 + lane;
       if (i < d_vec) yrow[i] = scale_vec<BF16>(oc[j], s);
-      if (i < dl_vec) yrow[d_vec + i] = bad ? zero : ec[j];
     }
     for (int i = CAP * 32 + lane; i < d_vec; i += 32) yrow[i] = scale_vec<BF16>(orow[i], s);
-    for (int i = CAP * 32 + lane; i < dl_vec; i += 32) yrow[d_vec + i] = bad ? zero : __ldg(erow + i);
     if (lane == 0) {
       if (scale_out != nullptr) scale_out[t] = s;
       if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
@@ -146,9 +155,11 @@ __global__ void __launch_bounds__(256) junction_fwd_kernel(const int32_t* __rest
 // ---------------------------------------------------------------- backward
 // do = s (g_o - u (u.g_o)),  de = g_e + (u.g_o) e_hat, written as
 //   do = s g_o - (s ug / ||o||) o,   de = g_e + (ug / ||e||) e,   ug = o.g_o / ||o||.
+// o and g_o stay in registers between the reductions and the do store; the
+// embedding row is read again for de (it was just read, so from cache).
 // When coef_out is given, c_t = ug/||e|| is stored for the table scatter.
 template <bool BF16, int CAP>
-__global__ void __launch_bounds__(256) junction_bwd_kernel(
+__global__ void __launch_bounds__(256, 2) junction_bwd_kernel(
     const int32_t* __restrict__ x, int64_t T, const uint4* __restrict__ o, int d_vec,
     const uint4* __restrict__ E, int64_t V, int dl_vec, const uint4* __restrict__ dy,
     uint4* __restrict__ do_out, uint4* __restrict__ de_out, float* __restrict__ coef_out,
@@ -157,13 +168,14 @@ __global__ void __launch_bounds__(256) junction_bwd_kernel(
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int dp_vec = d_vec + dl_vec;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
   for (int64_t t = warp0; t < T; t += nwarps) {
     const int32_t id = __ldg(x + t);
     const bool bad = (id < 0) || (static_cast<int64_t>(id) >= V);
     const uint4* orow = o + t * d_vec;
     const uint4* grow = dy + t * dp_vec;
     const uint4* erow = E + static_cast<int64_t>(bad ? 0 : id) * dl_vec;
-    uint4 oc[CAP], gc[CAP], ec[CAP];
+    uint4 oc[CAP], gc[CAP];
     float so = 0.f, sog = 0.f, se = 0.f;
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
@@ -171,17 +183,22 @@ __global__ void __launch_bounds__(256) junction_bwd_kernel(
       if (i < d_vec) {
         oc[j] = __ldcs(orow + i);
         gc[j] = __ldcs(grow + i);
+      }
+    }
+    for (int i = lane; i < dl_vec; i += 32) se += sumsq<BF16>(__ldg(erow + i));
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < d_vec) {
         so += sumsq<BF16>(oc[j]);
         sog += dotv<BF16>(oc[j], gc[j]);
       }
-      if (i < dl_vec) { ec[j] = __ldg(erow + i); se += sumsq<BF16>(ec[j]); }
     }
     for (int i = CAP * 32 + lane; i < d_vec; i += 32) {
       const uint4 ov = orow[i], gv = grow[i];
       so += sumsq<BF16>(ov);
       sog += dotv<BF16>(ov, gv);
     }
-    for (int i = CAP * 32 + lane; i < dl_vec; i += 32) se += sumsq<BF16>(__ldg(erow + i));
     so = warp_sum(so);
     sog = warp_sum(sog);
     se = warp_sum(se);
@@ -192,7 +209,6 @@ __global__ void __launch_bounds__(256) junction_bwd_kernel(
     float a = s, b = s * ug / n_o, c = (n_e > 0.f) ? ug / n_e : 0.f;
     if (bad) { a = 0.f; b = 0.f; c = 0.f; }
     uint4* drow = do_out + t * d_vec;
-    const uint4 zero = make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
       const int i = j * 32 + lane;
@@ -201,13 +217,8 @@ __global__ void __launch_bounds__(256) junction_bwd_kernel(
     for (int i = CAP * 32 + lane; i < d_vec; i += 32) drow[i] = axpby_vec<BF16>(a, grow[i], b, orow[i]);
     if (de_out != nullptr) {
       uint4* erow_out = de_out + t * dl_vec;
-#pragma unroll
-      for (int j = 0; j < CAP; ++j) {
-        const int i = j * 32 + lane;
-        if (i < dl_vec) erow_out[i] = bad ? zero : add_scaled_vec<BF16>(__ldcs(grow + d_vec + i), c, ec[j]);
-      }
-      for (int i = CAP * 32 + lane; i < dl_vec; i += 32)
-        erow_out[i] = bad ? zero : add_scaled_vec<BF16>(grow[d_vec + i], c, __ldg(erow + i));
+      for (int i = lane; i < dl_vec; i += 32)
+        erow_out[i] = bad ? zero : add_scaled_vec<BF16>(__ldcs(grow + d_vec + i), c, __ldg(erow + i));
     }
     if (lane == 0) {
       if (coef_out != nullptr) coef_out[t] = c;
@@ -218,11 +229,9 @@ __global__ void __launch_bounds__(256) junction_bwd_kernel(
 
 int pick_cap(int nvec) {
   const int per_lane = (nvec + 31) / 32;
-  if (per_lane <= 1) return 1;
-  if (per_lane <= 2) return 2;
-  if (per_lane <= 4) return 4;
-  if (per_lane <= 8) return 8;
-  if (per_lane <= 12) return 12;
+  static const int caps[] = {1, 2, 4, 6, 8, 9, 12, 16};
+  for (int c : caps)
+    if (per_lane <= c) return c;
   return 16;
 }
 
@@ -239,7 +248,7 @@ template <bool BF16>
 cudaError_t launch_fwd_t(const JunctionArgs& a, cudaStream_t st) {
   constexpr int N = Elt<BF16>::kPerVec;
   const int d_vec = static_cast<int>(a.D / N), dl_vec = static_cast<int>(a.delta / N);
-  const int cap = pick_cap(d_vec > dl_vec ? d_vec : dl_vec);
+  const int cap = pick_cap(d_vec);
   const int grid = grid_for(a.T, 8);
   auto* o = static_cast<const uint4*>(a.o);
   auto* E = static_cast<const uint4*>(a.E);
@@ -249,7 +258,9 @@ cudaError_t launch_fwd_t(const JunctionArgs& a, cudaStream_t st) {
     case 1: MLS_JF(1); break;
     case 2: MLS_JF(2); break;
     case 4: MLS_JF(4); break;
+    case 6: MLS_JF(6); break;
     case 8: MLS_JF(8); break;
+    case 9: MLS_JF(9); break;
     case 12: MLS_JF(12); break;
     default: MLS_JF(16); break;
   }
@@ -262,7 +273,7 @@ template <bool BF16>
 cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   constexpr int N = Elt<BF16>::kPerVec;
   const int d_vec = static_cast<int>(a.D / N), dl_vec = static_cast<int>(a.delta / N);
-  const int cap = pick_cap(d_vec > dl_vec ? d_vec : dl_vec);
+  const int cap = pick_cap(d_vec);
   const int grid = grid_for(a.T, 8);
   auto* o = static_cast<const uint4*>(a.o);
   auto* E = static_cast<const uint4*>(a.E);
@@ -276,7 +287,9 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
     case 1: MLS_JB(1); break;
     case 2: MLS_JB(2); break;
     case 4: MLS_JB(4); break;
+    case 6: MLS_JB(6); break;
     case 8: MLS_JB(8); break;
+    case 9: MLS_JB(9); break;
     case 12: MLS_JB(12); break;
     default: MLS_JB(16); break;
   }

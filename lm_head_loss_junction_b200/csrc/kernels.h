@@ -33,10 +33,10 @@ cudaError_t launch_junction_bwd(const JunctionArgs& a, cudaStream_t st);
 
 // ------------------------------------------------------------------ id-grouped row sums
 // Tokens grouped by id (stable in t): the tokens of id v are
-// toks[offsets[v] .. offsets[v] + counts[v]).  Ids outside [0, V) are left out.
+// toks[offsets[v] .. ends[v]).  Ids outside [0, V) are left out.
 struct SegIndexDev {
   int64_t V;
-  const int32_t* counts;
+  const int32_t* ends;
   const int32_t* offsets;
   const int32_t* toks;
   const int32_t* heavy;      // ids with many tokens

@@ -41,27 +41,49 @@ __global__ void __launch_bounds__(kSortBlock) sort_hist_kernel(const int32_t* __
   for (int d = threadIdx.x; d < 256; d += blockDim.x) hist[d * nblk + blockIdx.x] = h[d];
 }
 
-// out[i] = sum_{j < i} in[i] over n entries, one block; in may equal out.
-__global__ void __launch_bounds__(1024) exclusive_scan_kernel(const int32_t* in, int32_t* out, int n) {
-  __shared__ int32_t part[1024];
-  const int tid = threadIdx.x;
-  const int per = (n + 1023) / 1024;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
-  int32_t s = 0;
-  for (int i = lo; i < hi; ++i) s += in[i];
-  part[tid] = s;
+// Exclusive prefix sum of n ints in place, one block of 1024 threads: chunks
+// of 4096 (4 consecutive values per thread, coalesced), warp-shuffle scans,
+// and a running carry between chunks.
+__global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t* data, int n) {
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t carry_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry_s = 0;
   __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    const int32_t v = (tid >= off) ? part[tid - off] : 0;
+  for (int base = 0; base < n; base += 4096) {
+    int32_t v[4];
+    const int i0 = base + 4 * tid;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = (i0 + k < n) ? data[i0 + k] : 0;
+    const int32_t own = v[0] + v[1] + v[2] + v[3];
+    int32_t incl = own;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += u;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
-    part[tid] += v;
+    if (warp == 0) {
+      int32_t w = warp_tot[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += u;
+      }
+      warp_tot[lane] = w;   // inclusive over warps
+    }
     __syncthreads();
-  }
-  int32_t run = part[tid] - s;
-  for (int i = lo; i < hi; ++i) {
-    const int32_t c = in[i];
-    out[i] = run;
-    run += c;
+    const int32_t carry = carry_s;
+    int32_t run = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + incl - own;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (i0 + k < n) data[i0 + k] = run;
+      run += v[k];
+    }
+    __syncthreads();
+    if (tid == 1023) carry_s = carry + warp_tot[31];
+    __syncthreads();
   }
 }
 
@@ -106,20 +128,22 @@ __global__ void __launch_bounds__(kSortBlock) sort_scatter_kernel(
   }
 }
 
-__global__ void count_ids_kernel(const int32_t* __restrict__ ids, int64_t n, int64_t V, int32_t* __restrict__ counts) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const int32_t id = ids[i];
-  if (id >= 0 && id < V) atomicAdd(counts + id, 1);
-}
-
-// Rows with more than kHeavy tokens go to a list (its order does not matter:
-// every row is reduced independently in a fixed order).
-__global__ void heavy_list_kernel(const int32_t* __restrict__ counts, int64_t V, int32_t* __restrict__ heavy,
-                                  int32_t* __restrict__ n_heavy) {
-  const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (v >= V) return;
-  if (counts[v] > kHeavy) heavy[atomicAdd(n_heavy, 1)] = static_cast<int32_t>(v);
+// Segment bounds from the sorted keys: offsets[v] = first position of id v,
+// ends[v] = one past its last (both 0 for absent ids, preset by a memset).
+// Ids with more than kHeavy tokens are appended to the heavy list; its order
+// does not matter, every row is reduced independently in a fixed order.
+__global__ void segment_bounds_kernel(const int32_t* __restrict__ keys, int64_t n, int64_t V,
+                                      int32_t* __restrict__ offsets, int32_t* __restrict__ ends,
+                                      int32_t* __restrict__ heavy, int32_t* __restrict__ n_heavy) {
+  const int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (p >= n) return;
+  const int32_t k = keys[p];
+  if (k >= V) return;                                    // invalid ids sort last
+  if (p == 0 || keys[p - 1] != k) {
+    offsets[k] = static_cast<int32_t>(p);
+    if (p + kHeavy < n && keys[p + kHeavy] == k) heavy[atomicAdd(n_heavy, 1)] = k;
+  }
+  if (p == n - 1 || keys[p + 1] != k) ends[k] = static_cast<int32_t>(p + 1);
 }
 
 template <bool BF16>
@@ -193,11 +217,17 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
   const int lane = threadIdx.x & 31;
   const int64_t v = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (v >= ix.V) return;
-  const int32_t cnt = ix.counts[v];
+  const int32_t off = ix.offsets[v];
+  const int32_t cnt = ix.ends[v] - off;
   if (cnt > kHeavy) return;                   // handled by the heavy kernel
   if (cnt == 0 && (!TABLE || accumulate)) return;   // nothing to add
-  const int32_t off = ix.offsets[v];
   float* out_row = out + v * static_cast<int64_t>(n_vec) * N;
+  if (cnt == 0) {                             // overwrite mode: the row of an unused id is zero
+    float4* o4 = reinterpret_cast<float4*>(out_row);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = lane; i < n_vec * (N / 4); i += 32) o4[i] = z;
+    return;
+  }
   const uint4* E_row = TABLE ? E + v * static_cast<int64_t>(n_vec) : nullptr;
   float cs = 0.f;
   if (TABLE)
@@ -229,8 +259,8 @@ __global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vi = blockIdx.y * 32 + lane;
   const bool active = vi < n_vec;
-  const int32_t cnt = ix.counts[v];
   const int32_t off = ix.offsets[v];
+  const int32_t cnt = ix.ends[v] - off;
   float acc[N];
 #pragma unroll
   for (int k = 0; k < N; ++k) acc[k] = 0.f;
@@ -282,7 +312,7 @@ size_t segindex_bytes(int64_t T, int64_t V) {
   const int64_t nblk = (T + kSortBlock - 1) / kSortBlock;
   const size_t t4 = static_cast<size_t>(T) * 4;
   const int64_t max_heavy = T / (kHeavy + 1) + 1;
-  return up256(t4) * 4 + up256(static_cast<size_t>(256) * nblk * 4) + up256(static_cast<size_t>(V + 1) * 4) * 2 +
+  return up256(t4) * 4 + up256(static_cast<size_t>(256) * nblk * 4) + up256(static_cast<size_t>(V) * 4) * 2 +
          up256(static_cast<size_t>(max_heavy) * 4) + 256;
 }
 
@@ -295,20 +325,11 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
   int32_t* vals0 = reinterpret_cast<int32_t*>(p); p += up256(t4);
   int32_t* vals1 = reinterpret_cast<int32_t*>(p); p += up256(t4);
   int32_t* hist = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(256) * nblk * 4);
-  int32_t* counts = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V + 1) * 4);
-  int32_t* offsets = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V + 1) * 4);
+  int32_t* offsets = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V) * 4);
+  int32_t* ends = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V) * 4);
   const int64_t max_heavy = T / (kHeavy + 1) + 1;
   int32_t* heavy = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(max_heavy) * 4);
   int32_t* n_heavy = reinterpret_cast<int32_t*>(p);
-
-  // per-id counts and their exclusive prefix (segment offsets in sorted order)
-  cudaError_t err = cudaMemsetAsync(counts, 0, static_cast<size_t>(V + 1) * 4, st);
-  if (err == cudaSuccess) err = cudaMemsetAsync(n_heavy, 0, 4, st);
-  if (err != cudaSuccess) return err;
-  count_ids_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(ids, T, V, counts);
-  exclusive_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, static_cast<int>(V + 1));
-  heavy_list_kernel<<<static_cast<unsigned>((V + 255) / 256), 256, 0, st>>>(counts, V, heavy, n_heavy);
-  note_launches(3);
 
   // stable radix sort of the ids carrying token indices
   int bits = 1;
@@ -321,15 +342,23 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
   for (int pass = 0; pass < passes; ++pass) {
     sort_hist_kernel<<<static_cast<unsigned>(nblk), kSortBlock, 0, st>>>(kin, ids, T, V, 8 * pass, hist,
                                                                          static_cast<int>(nblk));
-    exclusive_scan_kernel<<<1, 1024, 0, st>>>(hist, hist, static_cast<int>(256 * nblk));
+    exclusive_scan_kernel<<<1, 1024, 0, st>>>(hist, static_cast<int>(256 * nblk));
     sort_scatter_kernel<<<static_cast<unsigned>(nblk), kSortBlock, 0, st>>>(
         kin, vin, ids, T, V, 8 * pass, hist, static_cast<int>(nblk), kbuf[pass & 1], vbuf[pass & 1]);
     note_launches(3);
     kin = kbuf[pass & 1];
     vin = vbuf[pass & 1];
   }
+  // per-id segment bounds in sorted order, and the heavy ids
+  cudaError_t err = cudaMemsetAsync(offsets, 0, static_cast<size_t>(V) * 4, st);
+  if (err == cudaSuccess) err = cudaMemsetAsync(ends, 0, static_cast<size_t>(V) * 4, st);
+  if (err == cudaSuccess) err = cudaMemsetAsync(n_heavy, 0, 4, st);
+  if (err != cudaSuccess) return err;
+  segment_bounds_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(kin, T, V, offsets, ends, heavy,
+                                                                                n_heavy);
+  note_launches(1);
   out->V = V;
-  out->counts = counts;
+  out->ends = ends;
   out->offsets = offsets;
   out->toks = vin;
   out->heavy = heavy;
