@@ -124,10 +124,22 @@ __global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __r
       const int i = j * 32 + lane;
       if (i < d_vec) oc[j] = __ldcs(orow + i);
     }
-    for (int i = lane; i < dl_vec; i += 32) {
-      const uint4 ev = __ldg(erow + i);
-      se += sumsq<BF16>(ev);
-      yrow[d_vec + i] = bad ? zero : ev;
+    // loads first, then the copies, in groups of 4 vectors per lane
+    for (int i0 = lane; i0 < dl_vec; i0 += 4 * 32) {
+      uint4 ev[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 32;
+        if (i < dl_vec) ev[u] = __ldg(erow + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * 32;
+        if (i < dl_vec) {
+          se += sumsq<BF16>(ev[u]);
+          yrow[d_vec + i] = bad ? zero : ev[u];
+        }
+      }
     }
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
@@ -185,6 +197,7 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_kernel(
         gc[j] = __ldcs(grow + i);
       }
     }
+#pragma unroll 4
     for (int i = lane; i < dl_vec; i += 32) se += sumsq<BF16>(__ldg(erow + i));
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
@@ -217,8 +230,22 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_kernel(
     for (int i = CAP * 32 + lane; i < d_vec; i += 32) drow[i] = axpby_vec<BF16>(a, grow[i], b, orow[i]);
     if (de_out != nullptr) {
       uint4* erow_out = de_out + t * dl_vec;
-      for (int i = lane; i < dl_vec; i += 32)
-        erow_out[i] = bad ? zero : add_scaled_vec<BF16>(__ldcs(grow + d_vec + i), c, __ldg(erow + i));
+      for (int i0 = lane; i0 < dl_vec; i0 += 4 * 32) {
+        uint4 gv[4], ev[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * 32;
+          if (i < dl_vec) {
+            gv[u] = __ldcs(grow + d_vec + i);
+            ev[u] = __ldg(erow + i);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * 32;
+          if (i < dl_vec) erow_out[i] = bad ? zero : add_scaled_vec<BF16>(gv[u], c, ev[u]);
+        }
+      }
     }
     if (lane == 0) {
       if (coef_out != nullptr) coef_out[t] = c;

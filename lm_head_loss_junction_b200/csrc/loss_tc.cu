@@ -463,26 +463,38 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
   if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
 }
 
-// ------------------------------------------------------------------ GEMM kernel (dh, dW)
-// out[M x N] (+)= alpha * A[M x K] B[N x K]^T with bf16 operands in TMA boxes,
-// fp32 accumulation in TMEM (two accumulator buffers so the epilogue of one
-// tile overlaps the mainloop of the next).
+// ------------------------------------------------------------------ grouped GEMM kernel (dh, dW)
+// For every problem p of a group (one per exit; all share M and K):
+//   out_p[M x N_p] (+)= alpha * A_p[M x K] B_p[N_p x K]^T
+// with bf16 operands in TMA boxes and fp32 accumulation in TMEM (two
+// accumulator buffers so the epilogue of one tile overlaps the mainloop of the
+// next).  One persistent launch walks the tiles of all problems, so the grid
+// stays full across exits of different widths.
 //   A_MN: A stored with M contiguous (boxes of 64 M x 64 K), else K contiguous
 //   B_MN: B stored with N contiguous, else K contiguous
 constexpr int kGemmStages = 4;
 
+struct GemmMaps {
+  CUtensorMap a[kMaxExits];
+  CUtensorMap b[kMaxExits];
+};
+
 struct GemmArgs {
-  int Mdim, Ndim, Kdim;
-  int n_mt, n_nt, num_tiles, group_m, kblocks;
-  void* out;
+  int nprob;
+  int Mdim, Kdim;
+  int n_mt, kblocks, group_m;
+  int tile_start[kMaxExits + 1];   // prefix of tiles per problem
+  int Ndim[kMaxExits];
+  int n_nt[kMaxExits];
+  void* out[kMaxExits];
   float alpha;
   int accumulate;
   int32_t* status;
-  // Optional exact one-hot term (bf16 output only): row r additionally gets
-  //   - alpha * onehot_coef * onehot_rows[onehot_idx[r], :]   when onehot_idx[r] in [0, onehot_limit)
+  // Optional exact one-hot term (bf16 output only): row r of problem p also gets
+  //   - alpha * onehot_coef[p] * onehot_rows[p][onehot_idx[r], :]  when onehot_idx[r] in [0, onehot_limit)
   const int32_t* onehot_idx;
-  const __nv_bfloat16* onehot_rows;
-  float onehot_coef;
+  const __nv_bfloat16* onehot_rows[kMaxExits];
+  float onehot_coef[kMaxExits];
   int onehot_limit;
 };
 
@@ -499,9 +511,22 @@ struct __align__(1024) GemmSmem {
   int abort;
 };
 
+// tile index -> (problem, m tile, n tile); m tiles grouped for L2 reuse
+__device__ __forceinline__ void gemm_tile(const GemmArgs& g, int i, int& p, int& mt, int& nt) {
+  p = 0;
+  while (p + 1 < g.nprob && i >= g.tile_start[p + 1]) ++p;
+  const int r0 = i - g.tile_start[p];
+  const int per_group = g.group_m * g.n_nt[p];
+  const int gi = r0 / per_group;
+  const int first = gi * g.group_m;
+  const int gm = min(g.group_m, g.n_mt - first);
+  const int r = r0 - gi * per_group;
+  nt = r / gm;
+  mt = first + r % gm;
+}
+
 template <bool A_MN, bool B_MN, int BN, bool OUT_BF16>
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap map_a,
-                                                           const __grid_constant__ CUtensorMap map_b,
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmMaps maps,
                                                            const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
   using Smem = GemmSmem<BN>;
@@ -510,6 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort;
   constexpr uint32_t kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+  const int num_tiles = g.tile_start[g.nprob];
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGemmStages; ++i) {
@@ -525,8 +551,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&map_a);
-    tma_prefetch_desc(&map_b);
+    for (int p = 0; p < g.nprob; ++p) {
+      tma_prefetch_desc(&maps.a[p]);
+      tma_prefetch_desc(&maps.b[p]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&s.tmem_base, kTmemCols);
@@ -537,39 +565,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  auto coords = [&](int i, int& mt, int& nt) {
-    const int per_group = g.group_m * g.n_nt;
-    const int gi = i / per_group;
-    const int first = gi * g.group_m;
-    const int gm = min(g.group_m, g.n_mt - first);
-    const int r = i - gi * per_group;
-    nt = r / gm;
-    mt = first + r % gm;
-  };
-
   if (warp == 0) {
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x) {
-        int mt, nt;
-        coords(tile, mt, nt);
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int p, mt, nt;
+        gemm_tile(g, tile, p, mt, nt);
+        const CUtensorMap* ma = &maps.a[p];
+        const CUtensorMap* mb = &maps.b[p];
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, g.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&s.full[stage], (kBM + BN) * kBK * 2);
           if (A_MN) {
 #pragma unroll
             for (int j = 0; j < kBM / 64; ++j)
-              tma_load_2d(&map_a, &s.full[stage], s.a[stage] + j * (64 * kBK * 2), mt * kBM + j * 64, kb * kBK);
+              tma_load_2d(ma, &s.full[stage], s.a[stage] + j * (64 * kBK * 2), mt * kBM + j * 64, kb * kBK);
           } else {
-            tma_load_2d(&map_a, &s.full[stage], s.a[stage], kb * kBK, mt * kBM);
+            tma_load_2d(ma, &s.full[stage], s.a[stage], kb * kBK, mt * kBM);
           }
           if (B_MN) {
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(&map_b, &s.full[stage], s.b[stage] + j * (64 * kBK * 2), nt * BN + j * 64, kb * kBK);
+              tma_load_2d(mb, &s.full[stage], s.b[stage] + j * (64 * kBK * 2), nt * BN + j * 64, kb * kBK);
           } else {
-            tma_load_2d(&map_b, &s.full[stage], s.b[stage], kb * kBK, nt * BN);
+            tma_load_2d(mb, &s.full[stage], s.b[stage], kb * kBK, nt * BN);
           }
           ++issued;
           if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
@@ -595,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       constexpr uint32_t b_lbo = B_MN ? 64 * kBK * 2 : 16;
       uint32_t stage = 0, phase = 0, iter = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x, ++iter) {
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++iter) {
         const uint32_t buf = iter & 1;
         if (!mbar_wait(&s.tempty[buf], ((iter >> 1) & 1) ^ 1, abort, g.status)) break;
         tc_fence_after();
@@ -622,21 +642,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const int row_in_tile = q * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t iter = 0;
-    for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++iter) {
-      int mt, nt;
-      coords(tile, mt, nt);
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
+      int p, mt, nt;
+      gemm_tile(g, tile, p, mt, nt);
       const uint32_t buf = iter & 1;
       if (!warp_wait(&s.tfull[buf], (iter >> 1) & 1, abort, g.status)) break;
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mt) * kBM + row_in_tile;
       const bool valid = row < g.Mdim;
+      const int Ndim = g.Ndim[p];
       const int64_t col0 = static_cast<int64_t>(nt) * BN;
       int64_t onehot_row = -1;
       if (OUT_BF16 && valid && g.onehot_idx != nullptr) {
         const int32_t k = __ldg(g.onehot_idx + row);
         if (k >= 0 && k < g.onehot_limit) onehot_row = k;
       }
-      const float oh_scale = g.alpha * g.onehot_coef;
+      const float oh_scale = g.alpha * g.onehot_coef[p];
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float r[32];
@@ -647,11 +668,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           if (lane == 0) mbar_arrive(&s.tempty[buf]);
         }
         if (!valid) continue;
-        const int64_t off = row * g.Ndim + col0 + c * 32;
+        const int64_t off = row * Ndim + col0 + c * 32;
         if (OUT_BF16) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + off);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out[p]) + off);
           const uint4* oh = (onehot_row >= 0)
-                                ? reinterpret_cast<const uint4*>(g.onehot_rows + onehot_row * g.Ndim + col0 + c * 32)
+                                ? reinterpret_cast<const uint4*>(g.onehot_rows[p] + onehot_row * Ndim + col0 + c * 32)
                                 : nullptr;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -667,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             dst[u] = f32_to_bf16x8(f);
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + off);
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out[p]) + off);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             float4 v = make_float4(r[4 * u] * g.alpha, r[4 * u + 1] * g.alpha, r[4 * u + 2] * g.alpha,
@@ -785,58 +806,83 @@ LossArgs base_args(const LossProblem& p) {
 }
 
 template <bool A_MN, bool B_MN, int BN, bool OUT_BF16>
-cudaError_t run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int Mdim, int Ndim, int Kdim, void* out,
-                     float alpha, int accumulate, int32_t* status, cudaStream_t st, const GemmArgs* extra = nullptr) {
-  GemmArgs g{};
-  if (extra != nullptr) g = *extra;
-  g.Mdim = Mdim;
-  g.Ndim = Ndim;
-  g.Kdim = Kdim;
-  g.n_mt = (Mdim + kBM - 1) / kBM;
-  g.n_nt = Ndim / BN;
-  g.num_tiles = g.n_mt * g.n_nt;
+cudaError_t run_gemm(const GemmMaps& maps, GemmArgs g, cudaStream_t st) {
+  g.n_mt = (g.Mdim + kBM - 1) / kBM;
+  g.kblocks = (g.Kdim + kBK - 1) / kBK;
   g.group_m = 16;
-  g.kblocks = (Kdim + kBK - 1) / kBK;
-  g.out = out;
-  g.alpha = alpha;
-  g.accumulate = accumulate;
-  g.status = status;
+  g.tile_start[0] = 0;
+  for (int p = 0; p < g.nprob; ++p) {
+    g.n_nt[p] = g.Ndim[p] / BN;
+    g.tile_start[p + 1] = g.tile_start[p] + g.n_mt * g.n_nt[p];
+  }
   const size_t smem = sizeof(GemmSmem<BN>) + 1024;
   auto fn = gemm_kernel<A_MN, B_MN, BN, OUT_BF16>;
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int grid = g.num_tiles < num_sms() ? g.num_tiles : num_sms();
-  fn<<<grid, kThreads, smem, st>>>(ma, mb, g);
+  const int tiles = g.tile_start[g.nprob];
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  fn<<<grid, kThreads, smem, st>>>(maps, g);
   note_launches(1);
   return cudaGetLastError();
 }
 
-int pick_bn(int64_t D) { return (D % 256 == 0) ? 256 : (D % 128 == 0) ? 128 : 64; }
-
-// dh_m[T x D] = alpha * (G'_m[T x V] W^m[V x D] - c_m W^m[y_t]): A = G' (K = V contiguous),
-// B = W^m (N = D contiguous); the one-hot row of W^m is subtracted exactly in the epilogue.
-template <int BN>
-cudaError_t run_dh(const __nv_bfloat16* G, const void* W, void* dh, int T, int V, int D, float alpha,
-                   const int32_t* y, float c_onehot, int32_t* status, cudaStream_t st) {
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, G, V, T, kBK, kBM)) return cudaErrorInvalidValue;
-  if (!make_map(&mb, W, D, V, 64, kBK)) return cudaErrorInvalidValue;
-  GemmArgs extra{};
-  extra.onehot_idx = y;
-  extra.onehot_rows = static_cast<const __nv_bfloat16*>(W);
-  extra.onehot_coef = c_onehot;
-  extra.onehot_limit = V;
-  return run_gemm<false, true, BN, true>(ma, mb, T, D, V, dh, alpha, 0, status, st, &extra);
+// Largest N tile that divides every exit's width.
+int pick_bn(const LossProblem& p) {
+  bool d256 = true, d128 = true;
+  for (int m = 0; m < p.M; ++m) {
+    d256 = d256 && (p.D[m] % 256 == 0);
+    d128 = d128 && (p.D[m] % 128 == 0);
+  }
+  return d256 ? 256 : d128 ? 128 : 64;
 }
 
-// dW^m[V x D] (+)= alpha * G'_m^T h_m: A = G'^T (M = V contiguous), B = h_m (N = D contiguous), K = T
+// dh_m[T x D_m] = a (G'_m[T x V] W^m[V x D_m] - c_m W^m[y_t]) for every exit in one launch:
+// A = G'_m (K = V contiguous), B = W^m (N = D_m contiguous); the one-hot row of
+// W^m is subtracted exactly in the epilogue.
 template <int BN>
-cudaError_t run_dw(const __nv_bfloat16* G, const void* h, float* dW, int T, int V, int D, float alpha,
-                   int accumulate, int32_t* status, cudaStream_t st) {
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, G, V, T, 64, kBK)) return cudaErrorInvalidValue;
-  if (!make_map(&mb, h, D, T, 64, kBK)) return cudaErrorInvalidValue;
-  return run_gemm<true, true, BN, false>(ma, mb, V, D, T, dW, alpha, accumulate, status, st);
+cudaError_t run_dh_all(const LossProblem& p, const __nv_bfloat16* G, void* const* dh, float alpha, cudaStream_t st) {
+  GemmMaps maps;
+  GemmArgs g{};
+  g.nprob = p.M;
+  g.Mdim = static_cast<int>(p.T);
+  g.Kdim = static_cast<int>(p.V);
+  g.alpha = alpha;
+  g.status = p.status;
+  g.onehot_idx = p.y;
+  g.onehot_limit = static_cast<int>(p.V);
+  for (int m = 0; m < p.M; ++m) {
+    const __nv_bfloat16* Gm = G + static_cast<int64_t>(m) * p.T * p.V;
+    if (!make_map(&maps.a[m], Gm, p.V, p.T, kBK, kBM)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.b[m], p.W[m], p.D[m], p.V, 64, kBK)) return cudaErrorInvalidValue;
+    g.Ndim[m] = static_cast<int>(p.D[m]);
+    g.out[m] = dh[m];
+    g.onehot_rows[m] = static_cast<const __nv_bfloat16*>(p.W[m]);
+    g.onehot_coef[m] = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
+  }
+  return run_gemm<false, true, BN, true>(maps, g, st);
+}
+
+// dW^m[V x D_m] (+)= a G'_m^T h_m for every exit in one launch: A = G'^T (M = V
+// contiguous), B = h_m (N = D_m contiguous), K = T.
+template <int BN>
+cudaError_t run_dw_all(const LossProblem& p, const __nv_bfloat16* G, float* const* dW, float alpha, int accumulate,
+                       cudaStream_t st) {
+  GemmMaps maps;
+  GemmArgs g{};
+  g.nprob = p.M;
+  g.Mdim = static_cast<int>(p.V);
+  g.Kdim = static_cast<int>(p.T);
+  g.alpha = alpha;
+  g.accumulate = accumulate;
+  g.status = p.status;
+  for (int m = 0; m < p.M; ++m) {
+    const __nv_bfloat16* Gm = G + static_cast<int64_t>(m) * p.T * p.V;
+    if (!make_map(&maps.a[m], Gm, p.V, p.T, 64, kBK)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.b[m], p.h[m], p.D[m], p.T, 64, kBK)) return cudaErrorInvalidValue;
+    g.Ndim[m] = static_cast<int>(p.D[m]);
+    g.out[m] = dW[m];
+  }
+  return run_gemm<true, true, BN, false>(maps, g, st);
 }
 
 }  // namespace
@@ -883,25 +929,22 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   err = build_segindex(p.y, p.T, p.V, static_cast<char*>(ws) + align_up(g_bytes(p)), &ix, st);
   if (err != cudaSuccess) return err;
   const float alpha = grad_scale / static_cast<float>(p.T);
-  const int T = static_cast<int>(p.T), V = static_cast<int>(p.V);
+  switch (pick_bn(p)) {
+    case 256: err = run_dh_all<256>(p, G, dh, alpha, st); break;
+    case 128: err = run_dh_all<128>(p, G, dh, alpha, st); break;
+    default: err = run_dh_all<64>(p, G, dh, alpha, st); break;
+  }
+  if (err != cudaSuccess) return err;
+  switch (pick_bn(p)) {
+    case 256: err = run_dw_all<256>(p, G, dW, alpha, accumulate, st); break;
+    case 128: err = run_dw_all<128>(p, G, dW, alpha, accumulate, st); break;
+    default: err = run_dw_all<64>(p, G, dW, alpha, accumulate, st); break;
+  }
+  if (err != cudaSuccess) return err;
+  // one-hot part of dW: (1 - alpha_d) for students, 1 for the teacher
   for (int m = 0; m < p.M; ++m) {
-    const __nv_bfloat16* Gm = G + static_cast<int64_t>(m) * p.T * p.V;
-    const int D = static_cast<int>(p.D[m]);
-    // one-hot weight of exit m: (1 - alpha_d) for students, 1 for the teacher
     const float c = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
-    switch (pick_bn(D)) {
-      case 256: err = run_dh<256>(Gm, p.W[m], dh[m], T, V, D, alpha, p.y, c, p.status, st); break;
-      case 128: err = run_dh<128>(Gm, p.W[m], dh[m], T, V, D, alpha, p.y, c, p.status, st); break;
-      default: err = run_dh<64>(Gm, p.W[m], dh[m], T, V, D, alpha, p.y, c, p.status, st); break;
-    }
-    if (err != cudaSuccess) return err;
-    switch (pick_bn(D)) {
-      case 256: err = run_dw<256>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
-      case 128: err = run_dw<128>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
-      default: err = run_dw<64>(Gm, p.h[m], dW[m], T, V, D, alpha, accumulate, p.status, st); break;
-    }
-    if (err != cudaSuccess) return err;
-    err = scatter_target_rows(ix, p.h[m], D / 8, dW[m], alpha * c, st);
+    err = scatter_target_rows(ix, p.h[m], static_cast<int>(p.D[m] / 8), dW[m], alpha * c, st);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
