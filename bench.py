@@ -198,6 +198,24 @@ class Step:
         return fwd, bwd
 
 
+def measured_traffic(cfg):
+    """DRAM bytes per launch of the forward loss tile kernel from the committed
+    ncu capture, or None when the capture is for another workload or the kernel
+    source has changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic_loss_tile_stats_main3_T8192.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, rec["source"])
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except Exception:
+        return None
+    if sha != rec["source_sha256_16"] or cfg.name != wl.CONFIGS["main3"].name:
+        return None
+    return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
+
+
 def _dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -426,7 +444,7 @@ def main():
         "junction_bwd_gbs_incl_scatter": jb_bytes / (phase_ms[3] / 1000.0) / 1e9 if c.M > 1 else None,
     }
     roofline = {"bound": "tensor", "achieved": ach_fwd, "peak": peak_tc, "unit": "TFLOP/s",
-                "frac": ach_fwd / peak_tc, "traffic": None,
+                "frac": ach_fwd / peak_tc, "traffic": measured_traffic(c),
                 "kernel": "loss_tile_kernel<stats> (mls_multiexit_loss_fwd call: tile kernel + merge + reduce)",
                 "algorithmic_per_launch": f"2*T*V*sum(D) = {flops_fwd:.4g} flop",
                 "peak_source": f"{peak_kind} bf16_tflops_sustained"}
