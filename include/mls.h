@@ -121,6 +121,41 @@ mls_status mls_junction_bwd(const int32_t* x, int64_t T,
                             void* workspace, size_t ws_bytes,
                             mls_dtype dt, int32_t* dev_status, void* stream);
 
+/*
+ * Junction variants (bit flags, combinable) for the ablations the pages
+ * report: "Visualizing Core ideas", bullet (c) -- dropping the rescaling, and
+ * filling the new channels with zeros instead of the fresh embedding -- and
+ * "Is nesting the cheapest way to build a model suite?", section 5 (B) --
+ * stop-gradient at every junction, so each block learns only from its own exit.
+ *   MLS_JUNCTION_NO_RESCALE  s_t := 1:            y = [o ; e],   do = g_o, de = g_e
+ *   MLS_JUNCTION_ZERO_FILL   new channels zero:   y = [s o ; 0], de = (u . g_o) e_hat
+ *                            (the rescale still uses the fresh embedding's norm)
+ *   MLS_JUNCTION_STOP_GRAD   forward unchanged;   do = 0, de as for the variant without it
+ * Unknown bits return MLS_ERR_INVALID_ARG.  The _variant entry points take the
+ * same arguments as mls_junction_fwd / mls_junction_bwd plus `variant`;
+ * variant 0 is exactly the standard junction.
+ */
+typedef enum {
+  MLS_JUNCTION_STANDARD = 0,
+  MLS_JUNCTION_NO_RESCALE = 1,
+  MLS_JUNCTION_ZERO_FILL = 2,
+  MLS_JUNCTION_STOP_GRAD = 4
+} mls_junction_variant;
+
+mls_status mls_junction_fwd_variant(const int32_t* x, int64_t T,
+                                    const void* o_m, int64_t D_m,
+                                    const void* e_next, int64_t V, int64_t delta,
+                                    void* y, float* scale_out, uint32_t variant,
+                                    mls_dtype dt, int32_t* dev_status, void* stream);
+
+mls_status mls_junction_bwd_variant(const int32_t* x, int64_t T,
+                                    const void* o_m, int64_t D_m,
+                                    const void* e_next, int64_t V, int64_t delta,
+                                    const void* dy, void* do_m, void* de_rows,
+                                    float* dE_table, int accumulate_dE,
+                                    void* workspace, size_t ws_bytes, uint32_t variant,
+                                    mls_dtype dt, int32_t* dev_status, void* stream);
+
 /* Scratch bytes mls_junction_bwd needs for the dE_table scatter. */
 mls_status mls_junction_bwd_workspace(int64_t T, int64_t V, size_t* bytes);
 

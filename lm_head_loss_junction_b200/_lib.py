@@ -16,6 +16,10 @@ MLS_F32 = 0
 MLS_BF16 = 1
 MLS_DEVFLAG_BAD_ID = 1
 MLS_DEVFLAG_TIMEOUT = 2
+MLS_JUNCTION_STANDARD = 0
+MLS_JUNCTION_NO_RESCALE = 1
+MLS_JUNCTION_ZERO_FILL = 2
+MLS_JUNCTION_STOP_GRAD = 4
 
 STATUS_NAMES = {
     0: "MLS_OK", 1: "MLS_ERR_INVALID_ARG", 2: "MLS_ERR_UNSUPPORTED", 3: "MLS_ERR_WORKSPACE",
@@ -28,12 +32,16 @@ _i32 = ctypes.c_int32
 _int = ctypes.c_int
 _f32 = ctypes.c_float
 _sz = ctypes.c_size_t
+_u32 = ctypes.c_uint32
 
 # name -> (restype, argtypes), in the order of include/mls.h
 PROTOTYPES = {
     "mls_junction_fwd": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _int, _vp, _vp]),
     "mls_junction_bwd": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _int,
                                 _vp, _sz, _int, _vp, _vp]),
+    "mls_junction_fwd_variant": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _u32, _int, _vp, _vp]),
+    "mls_junction_bwd_variant": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _int,
+                                        _vp, _sz, _u32, _int, _vp, _vp]),
     "mls_junction_bwd_workspace": (_int, [_i64, _i64, ctypes.POINTER(_sz)]),
     "mls_junction_bwd_noalloc": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _int,
                                         _int, _vp, _vp]),

@@ -47,8 +47,9 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 # ---------------------------------------------------------------- junction
 def junction_fwd(x: torch.Tensor, o: torch.Tensor, E: torch.Tensor, *, out=None, scale_out=None,
-                 status=None, stream=None) -> torch.Tensor:
-    """y = [ (||E[x]|| / ||o||) o ; E[x] ] per token (see mls_junction_fwd)."""
+                 variant: int = 0, status=None, stream=None) -> torch.Tensor:
+    """y = [ (||E[x]|| / ||o||) o ; E[x] ] per token (see mls_junction_fwd; `variant`
+    selects an ablation, see mls_junction_fwd_variant)."""
     _need(x, "x", torch.int32, 1)
     _need(o, "o", ndim=2)
     _need(E, "E", o.dtype, 2)
@@ -60,8 +61,13 @@ def junction_fwd(x: torch.Tensor, o: torch.Tensor, E: torch.Tensor, *, out=None,
     _need(y, "out", o.dtype, 2)
     if scale_out is not None:
         _need(scale_out, "scale_out", torch.float32, 1)
-    code = lib().mls_junction_fwd(x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V, delta, y.data_ptr(),
-                                  _ptr(scale_out), _dtype_code(o), _ptr(status), _stream_ptr(stream))
+    if variant:
+        code = lib().mls_junction_fwd_variant(x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V, delta,
+                                              y.data_ptr(), _ptr(scale_out), int(variant), _dtype_code(o),
+                                              _ptr(status), _stream_ptr(stream))
+    else:
+        code = lib().mls_junction_fwd(x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V, delta, y.data_ptr(),
+                                      _ptr(scale_out), _dtype_code(o), _ptr(status), _stream_ptr(stream))
     check("mls_junction_fwd", code)
     return y
 
@@ -74,7 +80,7 @@ def junction_bwd_workspace(T: int, V: int) -> int:
 
 def junction_bwd(x: torch.Tensor, o: torch.Tensor, E: torch.Tensor, dy: torch.Tensor, *,
                  want_de_rows: bool = True, dE: Optional[torch.Tensor] = None, accumulate_dE: bool = False,
-                 do_out=None, de_out=None, workspace=None, status=None, stream=None):
+                 do_out=None, de_out=None, workspace=None, variant: int = 0, status=None, stream=None):
     """Returns (do, de_rows or None, dE or None) (see mls_junction_bwd)."""
     _need(x, "x", torch.int32, 1)
     _need(o, "o", ndim=2)
@@ -95,10 +101,16 @@ def junction_bwd(x: torch.Tensor, o: torch.Tensor, E: torch.Tensor, dy: torch.Te
         if workspace is None:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=o.device)
         ws_bytes = workspace.numel() * workspace.element_size()
-    code = lib().mls_junction_bwd(x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V, delta, dy.data_ptr(),
-                                  do.data_ptr(), _ptr(de), _ptr(dE), int(bool(accumulate_dE)),
-                                  _ptr(workspace), ws_bytes, _dtype_code(o), _ptr(status),
-                                  _stream_ptr(stream))
+    if variant:
+        code = lib().mls_junction_bwd_variant(x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V, delta,
+                                              dy.data_ptr(), do.data_ptr(), _ptr(de), _ptr(dE),
+                                              int(bool(accumulate_dE)), _ptr(workspace), ws_bytes, int(variant),
+                                              _dtype_code(o), _ptr(status), _stream_ptr(stream))
+    else:
+        code = lib().mls_junction_bwd(x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V, delta, dy.data_ptr(),
+                                      do.data_ptr(), _ptr(de), _ptr(dE), int(bool(accumulate_dE)),
+                                      _ptr(workspace), ws_bytes, _dtype_code(o), _ptr(status),
+                                      _stream_ptr(stream))
     check("mls_junction_bwd", code)
     return do, de, dE
 

@@ -23,6 +23,8 @@ using mls::LossProblem;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+constexpr uint32_t kKnownVariants = MLS_JUNCTION_NO_RESCALE | MLS_JUNCTION_ZERO_FILL | MLS_JUNCTION_STOP_GRAD;
+
 // Returns MLS_OK when the current device is a compute-capability 10.0 GPU
 // (the only target this library is built for).
 mls_status device_ok() {
@@ -114,6 +116,14 @@ const char* mls_status_string(mls_status s) {
 mls_status mls_junction_fwd(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
                             int64_t V, int64_t delta, void* y, float* scale_out, mls_dtype dt,
                             int32_t* dev_status, void* stream) {
+  return mls_junction_fwd_variant(x, T, o_m, D_m, e_next, V, delta, y, scale_out, MLS_JUNCTION_STANDARD, dt,
+                                  dev_status, stream);
+}
+
+mls_status mls_junction_fwd_variant(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
+                                    int64_t V, int64_t delta, void* y, float* scale_out, uint32_t variant,
+                                    mls_dtype dt, int32_t* dev_status, void* stream) {
+  if (variant & ~kKnownVariants) return MLS_ERR_INVALID_ARG;
   mls_status st = check_junction_shape(x, T, o_m, D_m, e_next, V, delta, dt);
   if (st != MLS_OK) return st;
   if (y == nullptr) return MLS_ERR_INVALID_ARG;
@@ -131,6 +141,7 @@ mls_status mls_junction_fwd(const int32_t* x, int64_t T, const void* o_m, int64_
   a.y = y;
   a.scale_out = scale_out;
   a.status = dev_status;
+  a.variant = variant;
   return from_cuda(mls::launch_junction_fwd(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -144,6 +155,15 @@ mls_status mls_junction_bwd(const int32_t* x, int64_t T, const void* o_m, int64_
                             int64_t V, int64_t delta, const void* dy, void* do_m, void* de_rows, float* dE_table,
                             int accumulate_dE, void* workspace, size_t ws_bytes, mls_dtype dt,
                             int32_t* dev_status, void* stream) {
+  return mls_junction_bwd_variant(x, T, o_m, D_m, e_next, V, delta, dy, do_m, de_rows, dE_table, accumulate_dE,
+                                  workspace, ws_bytes, MLS_JUNCTION_STANDARD, dt, dev_status, stream);
+}
+
+mls_status mls_junction_bwd_variant(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
+                                    int64_t V, int64_t delta, const void* dy, void* do_m, void* de_rows,
+                                    float* dE_table, int accumulate_dE, void* workspace, size_t ws_bytes,
+                                    uint32_t variant, mls_dtype dt, int32_t* dev_status, void* stream) {
+  if (variant & ~kKnownVariants) return MLS_ERR_INVALID_ARG;
   mls_status st = check_junction_shape(x, T, o_m, D_m, e_next, V, delta, dt);
   if (st != MLS_OK) return st;
   if (dy == nullptr || do_m == nullptr) return MLS_ERR_INVALID_ARG;
@@ -172,6 +192,7 @@ mls_status mls_junction_bwd(const int32_t* x, int64_t T, const void* o_m, int64_
   a.accumulate_dE = accumulate_dE;
   a.workspace = workspace;
   a.status = dev_status;
+  a.variant = variant;
   return from_cuda(mls::launch_junction_bwd(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -93,6 +93,21 @@ __device__ __forceinline__ uint4 add_scaled_vec(const uint4& g, float c, const u
   return Elt<BF16>::store(fg);
 }
 
+// ga*g + c*e, elementwise
+template <bool BF16>
+__device__ __forceinline__ uint4 lincomb_vec(float ga, const uint4& g, float c, const uint4& e) {
+  constexpr int N = Elt<BF16>::kPerVec;
+  float fg[N], fe[N];
+  Elt<BF16>::load(g, fg);
+  Elt<BF16>::load(e, fe);
+#pragma unroll
+  for (int i = 0; i < N; ++i) fg[i] = fmaf(c, fe[i], ga * fg[i]);
+  return Elt<BF16>::store(fg);
+}
+
+// Variant bits (see include/mls.h): 1 = no rescale, 2 = zero fill, 4 = stop-gradient.
+constexpr uint32_t kNoRescale = 1, kZeroFill = 2, kStopGrad = 4;
+
 // ---------------------------------------------------------------- forward
 // One warp per token.  Pass 1 streams the block-output row (kept in registers,
 // CAP 16-byte vectors per lane) and the embedding row (copied straight to the
@@ -105,8 +120,9 @@ __global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __r
                                                            const uint4* __restrict__ E, int64_t V,
                                                            int dl_vec, uint4* __restrict__ y,
                                                            float* __restrict__ scale_out,
-                                                           int32_t* __restrict__ status) {
+                                                           int32_t* __restrict__ status, uint32_t variant) {
   const int lane = threadIdx.x & 31;
+  const bool zero_fill = (variant & kZeroFill) != 0;
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int dp_vec = d_vec + dl_vec;
@@ -137,7 +153,7 @@ __global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __r
         const int i = i0 + u * 32;
         if (i < dl_vec) {
           se += sumsq<BF16>(ev[u]);
-          yrow[d_vec + i] = bad ? zero : ev[u];
+          yrow[d_vec + i] = (bad || zero_fill) ? zero : ev[u];
         }
       }
     }
@@ -149,7 +165,7 @@ __global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __r
     for (int i = CAP * 32 + lane; i < d_vec; i += 32) so += sumsq<BF16>(orow[i]);
     so = warp_sum(so);
     se = warp_sum(se);
-    float s = sqrtf(se) / fmaxf(sqrtf(so), kJunctionEps);
+    float s = (variant & kNoRescale) ? 1.f : sqrtf(se) / fmaxf(sqrtf(so), kJunctionEps);
     if (bad) s = 0.f;
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
@@ -175,7 +191,7 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_kernel(
     const int32_t* __restrict__ x, int64_t T, const uint4* __restrict__ o, int d_vec,
     const uint4* __restrict__ E, int64_t V, int dl_vec, const uint4* __restrict__ dy,
     uint4* __restrict__ do_out, uint4* __restrict__ de_out, float* __restrict__ coef_out,
-    int32_t* __restrict__ status) {
+    int32_t* __restrict__ status, uint32_t variant) {
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -220,6 +236,9 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_kernel(
     const float s = n_e / n_o;
     const float ug = sog / n_o;
     float a = s, b = s * ug / n_o, c = (n_e > 0.f) ? ug / n_e : 0.f;
+    if (variant & kNoRescale) { a = 1.f; b = 0.f; c = 0.f; }   // y = [o ; .]
+    if (variant & kStopGrad) { a = 0.f; b = 0.f; }              // nothing flows into o
+    const float ge = (variant & kZeroFill) ? 0.f : 1.f;         // the fill does not carry g_e
     if (bad) { a = 0.f; b = 0.f; c = 0.f; }
     uint4* drow = do_out + t * d_vec;
 #pragma unroll
@@ -243,7 +262,7 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_kernel(
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int i = i0 + u * 32;
-          if (i < dl_vec) erow_out[i] = bad ? zero : add_scaled_vec<BF16>(gv[u], c, ev[u]);
+          if (i < dl_vec) erow_out[i] = bad ? zero : lincomb_vec<BF16>(ge, gv[u], c, ev[u]);
         }
       }
     }
@@ -280,7 +299,7 @@ cudaError_t launch_fwd_t(const JunctionArgs& a, cudaStream_t st) {
   auto* o = static_cast<const uint4*>(a.o);
   auto* E = static_cast<const uint4*>(a.E);
   auto* y = static_cast<uint4*>(a.y);
-#define MLS_JF(C) junction_fwd_kernel<BF16, C><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, y, a.scale_out, a.status)
+#define MLS_JF(C) junction_fwd_kernel<BF16, C><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, y, a.scale_out, a.status, a.variant)
   switch (cap) {
     case 1: MLS_JF(1); break;
     case 2: MLS_JF(2); break;
@@ -309,7 +328,7 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   auto* deo = static_cast<uint4*>(a.de_out);
   float* coef = nullptr;
   if (a.dE != nullptr) coef = static_cast<float*>(a.workspace);
-#define MLS_JB(C) junction_bwd_kernel<BF16, C><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status)
+#define MLS_JB(C) junction_bwd_kernel<BF16, C><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status, a.variant)
   switch (cap) {
     case 1: MLS_JB(1); break;
     case 2: MLS_JB(2); break;
@@ -330,7 +349,8 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   void* ix_ws = static_cast<char*>(a.workspace) + ((static_cast<size_t>(a.T) * 4 + 255) & ~size_t(255));
   err = build_segindex(a.x, a.T, a.V, ix_ws, &ix, st);
   if (err != cudaSuccess) return err;
-  return scatter_table_grad(ix, BF16, a.dy, d_vec, dl_vec, coef, a.E, a.dE, a.accumulate_dE != 0, st);
+  const float ge = (a.variant & kZeroFill) ? 0.f : 1.f;
+  return scatter_table_grad(ix, BF16, a.dy, d_vec, dl_vec, coef, ge, a.E, a.dE, a.accumulate_dE != 0, st);
 }
 
 }  // namespace

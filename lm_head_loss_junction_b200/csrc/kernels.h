@@ -25,6 +25,7 @@ struct JunctionArgs {
   int accumulate_dE;
   void* workspace;
   int32_t* status;
+  uint32_t variant;   // junction variant bits (0 = the standard junction)
 };
 
 size_t junction_scatter_bytes(int64_t T, int64_t V);
@@ -46,9 +47,10 @@ struct SegIndexDev {
 
 size_t segindex_bytes(int64_t T, int64_t V);
 cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, SegIndexDev* out, cudaStream_t st);
-// dE[v] (+)= sum_t g_e,t + (sum_t coef_t) E[v]; g_e is the tail of each dy row.
+// dE[v] (+)= ge sum_t g_e,t + (sum_t coef_t) E[v]; g_e is the tail of each dy row.
 cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
-                               const float* coef, const void* E, float* dE, bool accumulate, cudaStream_t st);
+                               const float* coef, float ge, const void* E, float* dE, bool accumulate,
+                               cudaStream_t st);
 // dW[v] -= scale * sum_t h_t (bf16 rows of d_vec 16-byte vectors).
 cudaError_t scatter_target_rows(const SegIndexDev& ix, const void* h, int d_vec, float* dW, float scale,
                                 cudaStream_t st);

@@ -172,7 +172,7 @@ struct Vec8<false> {
   }
 };
 
-// Writes one row slice: out = base + acc + cs*E (table mode) or out -= scale*acc (target mode).
+// Writes one row slice: out = base + scale*acc + cs*E (table mode) or out -= scale*acc (target mode).
 template <bool BF16, bool TABLE>
 __device__ __forceinline__ void emit(float* out_row, int vi, const float (&acc)[Vec8<BF16>::N], float cs,
                                      const uint4* E_row, float scale, bool accumulate) {
@@ -183,7 +183,7 @@ __device__ __forceinline__ void emit(float* out_row, int vi, const float (&acc)[
     float e[N];
     Vec8<BF16>::load(__ldg(E_row + vi), e);
 #pragma unroll
-    for (int k = 0; k < N; ++k) val[k] = fmaf(cs, e[k], acc[k]);
+    for (int k = 0; k < N; ++k) val[k] = fmaf(cs, e[k], scale * acc[k]);
   }
 #pragma unroll
   for (int q = 0; q < N / 4; ++q) {
@@ -368,12 +368,13 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
 }
 
 cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
-                               const float* coef, const void* E, float* dE, bool accumulate, cudaStream_t st) {
+                               const float* coef, float ge, const void* E, float* dE, bool accumulate,
+                               cudaStream_t st) {
   const uint4* src = static_cast<const uint4*>(dy);
   const int64_t ld = d_vec + dl_vec;
   const uint4* e = static_cast<const uint4*>(E);
-  return bf16 ? launch_segsum<true, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, 0.f, accumulate, st)
-              : launch_segsum<false, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, 0.f, accumulate, st);
+  return bf16 ? launch_segsum<true, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, ge, accumulate, st)
+              : launch_segsum<false, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, ge, accumulate, st);
 }
 
 cudaError_t scatter_target_rows(const SegIndexDev& ix, const void* h, int d_vec, float* dW, float scale,

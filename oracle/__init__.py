@@ -13,6 +13,7 @@ Parity is pinned for every function here; nothing in this package is
 "parity unpinned".
 """
 from .junction import junction_fwd, junction_bwd, JUNCTION_EPS
+from . import junction as junction_variants
 from .loss import multiexit_loss, multiexit_loss_vocab_rows, softmax_rows, logsumexp_rows
 
 __all__ = ["junction_fwd", "junction_bwd", "JUNCTION_EPS", "multiexit_loss", "multiexit_loss_vocab_rows",

@@ -80,6 +80,8 @@ def test_junction_argument_errors():
     assert f(FAKE, 8, FAKE, 64, FAKE, 10, 62, FAKE, None, _lib.MLS_F32, None, None) == 2
     assert f(FAKE, 8, FAKE + 4, 64, FAKE, 10, 64, FAKE, None, _lib.MLS_BF16, None, None) == 2
     assert f(FAKE, 8, FAKE, 64, FAKE, 10, 64, None, None, _lib.MLS_BF16, None, None) == 1
+    fv = lib.mls_junction_fwd_variant
+    assert fv(FAKE, 8, FAKE, 64, FAKE, 10, 64, FAKE, None, 8, _lib.MLS_BF16, None, None) == 1   # unknown bit
     b = lib.mls_junction_bwd
     # dE requested without workspace
     assert b(FAKE, 8, FAKE, 64, FAKE, 10, 64, FAKE, FAKE, None, FAKE, 0, None, 0, _lib.MLS_BF16, None,

@@ -50,7 +50,7 @@ def test_no_parameters_and_scale_invariance():
     # The junction has no weight argument, and the output depends on o only
     # through its direction: y(c o) = y(o) for any c > 0.
     import inspect
-    assert list(inspect.signature(junction_fwd).parameters) == ["x", "o", "E"]
+    assert set(inspect.signature(junction_fwd).parameters) <= {"x", "o", "E", "variant"}
     x, o, E = _case(seed=3)
     y1, _ = junction_fwd(x, o, E)
     y2, _ = junction_fwd(x, 37.5 * o, E)
@@ -131,3 +131,69 @@ def test_table_gradient_is_one_hot_product():
     # tokens that never occur get exactly zero
     unused = np.setdiff1d(np.arange(7), x)
     assert np.all(dE[unused] == 0.0)
+
+
+# ------------------------------------------------------------------ variants
+from oracle import junction_variants as jv  # noqa: E402
+
+
+def _fd_check(x, o, E, R, variant, wrt_o=True):
+    do, de, dE = junction_bwd(x, o, E, R, variant=variant)
+    h = 1e-6
+
+    def L(oo, EE):
+        y, _ = junction_fwd(x, oo, EE, variant=variant)
+        return float(np.sum(y * R))
+    num_dE = np.zeros_like(E)
+    for idx in np.ndindex(E.shape):
+        Ep = E.copy(); Ep[idx] += h
+        Em = E.copy(); Em[idx] -= h
+        num_dE[idx] = (L(o, Ep) - L(o, Em)) / (2 * h)
+    np.testing.assert_allclose(dE, num_dE, rtol=1e-6, atol=1e-9)
+    if wrt_o:
+        num_do = np.zeros_like(o)
+        for idx in np.ndindex(o.shape):
+            op = o.copy(); op[idx] += h
+            om = o.copy(); om[idx] -= h
+            num_do[idx] = (L(op, E) - L(om, E)) / (2 * h)
+        np.testing.assert_allclose(do, num_do, rtol=1e-6, atol=1e-9)
+    return do, de, dE
+
+
+def test_variant_no_rescale_is_plain_concatenation():
+    x, o, E = _case(T=6, D=5, dl=3, V=4, seed=11)
+    y, s = junction_fwd(x, o, E, variant=jv.NO_RESCALE)
+    assert np.array_equal(y, np.concatenate([o, E[x]], axis=1)) and np.all(s == 1.0)
+    R = np.random.default_rng(1).normal(size=(6, 8))
+    do, de, _ = _fd_check(x, o, E, R, jv.NO_RESCALE)
+    np.testing.assert_array_equal(do, R[:, :5])
+    np.testing.assert_array_equal(de, R[:, 5:])
+
+
+def test_variant_zero_fill_keeps_the_rescale():
+    x, o, E = _case(T=6, D=5, dl=3, V=4, seed=12)
+    y, s = junction_fwd(x, o, E, variant=jv.ZERO_FILL)
+    assert np.all(y[:, 5:] == 0.0)
+    np.testing.assert_allclose(np.linalg.norm(y[:, :5], axis=1), np.linalg.norm(E[x], axis=1), rtol=1e-12)
+    R = np.random.default_rng(2).normal(size=(6, 8))
+    _fd_check(x, o, E, R, jv.ZERO_FILL)
+
+
+def test_variant_zero_fill_without_rescale():
+    x, o, E = _case(T=4, D=3, dl=2, V=3, seed=13)
+    y, _ = junction_fwd(x, o, E, variant=jv.NO_RESCALE | jv.ZERO_FILL)
+    assert np.array_equal(y, np.concatenate([o, np.zeros((4, 2))], axis=1))
+    do, de, dE = junction_bwd(x, o, E, np.ones((4, 5)), variant=jv.NO_RESCALE | jv.ZERO_FILL)
+    assert np.all(do == 1.0) and np.all(de == 0.0) and np.all(dE == 0.0)
+
+
+def test_variant_stop_gradient():
+    x, o, E = _case(T=6, D=5, dl=3, V=4, seed=14)
+    y0, _ = junction_fwd(x, o, E)
+    y1, _ = junction_fwd(x, o, E, variant=jv.STOP_GRAD)
+    assert np.array_equal(y0, y1)                      # forward unchanged
+    R = np.random.default_rng(3).normal(size=(6, 8))
+    do, de, dE = _fd_check(x, o, E, R, jv.STOP_GRAD, wrt_o=False)   # embedding gradient = true derivative
+    assert np.all(do == 0.0)                           # nothing flows back into the block output
+    _, de0, _ = junction_bwd(x, o, E, R)
+    np.testing.assert_array_equal(de, de0)

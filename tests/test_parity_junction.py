@@ -145,3 +145,36 @@ def test_junction_full_size_sampled(name):
         do_e, de_e, _ = oracle.junction_bwd(d.x[rows], d.o[j][rows], d.E[j + 1], dy.cpu()[rows])
         assert_grad_close(do[sel], do_e, "do")
         assert_grad_close(de[sel], de_e, "de")
+
+
+VARIANTS = [1, 2, 4, 3, 5, 6, 7]   # no rescale, zero fill, stop-gradient and their combinations
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("name,j,small", [("main3", 1, dict(batch=1, seq=300, V=512)),
+                                          ("tiny3", 0, None)])
+def test_junction_variants_match_oracle(variant, name, j, small):
+    cfg = _cfg(name, small)
+    _, x, o, E, dy = _junction_case(cfg, j)
+    s = torch.empty(x.shape[0], dtype=torch.float32, device="cuda")
+    y = junction_fwd(x, o, E, scale_out=s, variant=variant)
+    y_e, s_e = oracle.junction_fwd(x.cpu().numpy(), o.cpu(), E.cpu(), variant=variant)
+    D = o.shape[1]
+    # the filled channels are an exact copy (or exact zeros)
+    assert torch.equal(y[:, D:].cpu(), torch.from_numpy(y_e[:, D:]).to(o.dtype))
+    np.testing.assert_allclose(f64(s), s_e, rtol=2e-6)
+    u = unit_roundoff(o.dtype)
+    got, exp = f64(y[:, :D]), y_e[:, :D]
+    assert np.all(np.abs(got - exp) <= u * np.abs(exp) * (1 + 1e-5) + 4e-6 * np.abs(exp) + 1e-30)
+    dE = torch.zeros(E.shape, dtype=torch.float32, device="cuda")
+    do, de, dE = junction_bwd(x, o, E, dy, dE=dE, variant=variant)
+    do_e, de_e, dE_e = oracle.junction_bwd(x.cpu().numpy(), o.cpu(), E.cpu(), dy.cpu(), variant=variant)
+    if variant & 4:
+        assert torch.all(do == 0)
+    else:
+        assert_grad_close(do, do_e, "do")
+    if (variant & 3) == 3:
+        assert torch.all(de == 0) and torch.all(dE == 0)
+    else:
+        assert_grad_close(de, de_e, "de")
+        assert_grad_close(dE, dE_e, "dE")
