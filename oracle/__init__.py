@@ -14,7 +14,8 @@ Parity is pinned for every function here; nothing in this package is
 """
 from .junction import junction_fwd, junction_bwd, JUNCTION_EPS
 from . import junction as junction_variants
-from .loss import multiexit_loss, multiexit_loss_vocab_rows, softmax_rows, logsumexp_rows
+from .loss import (exit_agreement, logsumexp_rows, multiexit_loss, multiexit_loss_vocab_rows,
+                   softmax_rows)
 
 __all__ = ["junction_fwd", "junction_bwd", "JUNCTION_EPS", "multiexit_loss", "multiexit_loss_vocab_rows",
-           "softmax_rows", "logsumexp_rows"]
+           "softmax_rows", "logsumexp_rows", "exit_agreement"]

@@ -164,3 +164,45 @@ def multiexit_loss_vocab_rows(y, h, W, alpha_d=0.3, grad_scale=1.0, vrows=None, 
     ce_kd /= T
     loss = float(np.sum((1.0 - alpha_d) * ce_lm[:M - 1]) + np.sum(alpha_d * ce_kd) + ce_lm[M - 1])
     return {"ce_lm": ce_lm, "ce_kd": ce_kd, "loss": loss, "dW_rows": dW_rows}
+
+
+def exit_agreement(h, W, rows=None, token_block=256):
+    """Agreement of every smaller exit m with the largest exit M, per token and
+    as means over the tokens.
+
+    Definitions followed:
+      * acceptance probability of a drafted token, beta = sum_v min(q_v, p_v)
+        (one minus the total-variation distance between draft q and verifier p;
+        "Is nesting the cheapest way to build a model suite?", section 4), with
+        the draft q = q_m and the verifier p = p_M;
+      * pairwise KL and top-1 next-token agreement between exits ("Matryoshka
+        Language Model Suites", agihunt.info summary, alignment paragraph),
+        read as KL(p_M || q_m) = sum_v p_M,v (log p_M,v - log q_m,v) and
+        [argmax_v q_m = argmax_v p_M], ties going to the lowest index.
+
+    Returns a dict with per-token beta, kl, agree [M-1, T'], top1 [M, T'] (int)
+    and their means beta_mean, kl_mean, agree_mean [M-1].
+    """
+    M = len(h)
+    Ws = [_f64(w) for w in W]
+    T = h[0].shape[0]
+    idx = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    Tn = idx.shape[0]
+    out = {"beta": np.zeros((M - 1, Tn)), "kl": np.zeros((M - 1, Tn)), "agree": np.zeros((M - 1, Tn)),
+           "top1": np.zeros((M, Tn), dtype=np.int64)}
+    for b0 in range(0, Tn, token_block):
+        sel = idx[b0:b0 + token_block]
+        n = sel.shape[0]
+        logits = [_f64(h[m][sel]) @ Ws[m].T for m in range(M)]
+        logp = [l - logsumexp_rows(l)[:, None] for l in logits]
+        pM = np.exp(logp[M - 1])
+        for m in range(M):
+            out["top1"][m, b0:b0 + n] = np.argmax(logits[m], axis=1)      # first maximum
+        for m in range(M - 1):
+            q = np.exp(logp[m])
+            out["beta"][m, b0:b0 + n] = np.sum(np.minimum(q, pM), axis=1)
+            out["kl"][m, b0:b0 + n] = np.sum(pM * (logp[M - 1] - logp[m]), axis=1)
+            out["agree"][m, b0:b0 + n] = (out["top1"][m, b0:b0 + n] == out["top1"][M - 1, b0:b0 + n])
+    for k in ("beta", "kl", "agree"):
+        out[k + "_mean"] = out[k].mean(axis=1)
+    return out
