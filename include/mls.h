@@ -257,6 +257,35 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   void* workspace, size_t ws_bytes,
                                   int32_t* dev_status, void* stream);
 
+/*
+ * mls_exit_agreement -- how well every smaller exit agrees with the largest
+ * one, per token, from the same logits (computed again, never stored) and the
+ * normalisers in `stats` from mls_multiexit_loss_fwd.  Measures named by the
+ * pages: the acceptance probability of a drafted token, beta = sum_v min(q, p)
+ * with draft q and verifier p ("Is nesting the cheapest way to build a model
+ * suite?", section 4), and pairwise KL and top-1 next-token agreement between
+ * exits ("Matryoshka Language Model Suites", alignment paragraph).  For each
+ * smaller exit m (draft q = q_m) against the largest exit (verifier p = p_M):
+ *   beta_m,t  = sum_v min(q_m,t,v, p_M,t,v)
+ *   KL_m,t    = sum_v p_M,t,v (log p_M,t,v - log q_m,t,v)
+ *   agree_m,t = [argmax_v l_m,t,v == argmax_v l_M,t,v], first maximum on ties
+ *
+ *   M >= 2; h, W, D, V, dt as for the loss; no targets are needed
+ *   stats      device f32 [3M-1, T] from mls_multiexit_loss_fwd (lse rows used)
+ *   metrics    device f32 [3(M-1)]: mean beta_m, mean KL_m, mean agree_m (m < M)
+ *   per_token  device f32 [3(M-1), T] or NULL: the per-token rows, same order
+ *   top1       device int32 [M, T] or NULL: argmax of every exit's logits
+ *   workspace  >= mls_exit_agreement_workspace(...) bytes
+ */
+mls_status mls_exit_agreement_workspace(int M, int64_t T, const int64_t* D, int64_t V,
+                                        mls_dtype dt, size_t* bytes);
+
+mls_status mls_exit_agreement(int M, int64_t T, int64_t V, const int64_t* D,
+                              const void* const* h, const void* const* W, mls_dtype dt,
+                              const float* stats, float* metrics, float* per_token,
+                              int32_t* top1, void* workspace, size_t ws_bytes,
+                              int32_t* dev_status, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Status                                                                    */
 /* ------------------------------------------------------------------------ */

@@ -54,6 +54,9 @@ PROTOTYPES = {
                                       ctypes.POINTER(_vp), ctypes.POINTER(_vp), _f32, _int,
                                       _vp, _f32, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int,
                                       _vp, _sz, _vp, _vp]),
+    "mls_exit_agreement_workspace": (_int, [_int, _i64, ctypes.POINTER(_i64), _i64, _int, ctypes.POINTER(_sz)]),
+    "mls_exit_agreement": (_int, [_int, _i64, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                  _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "mls_status_read": (_int, [_vp, _vp, ctypes.POINTER(_i32)]),
     "mls_status_string": (ctypes.c_char_p, [_int]),
     "mls_version": (_int, []),

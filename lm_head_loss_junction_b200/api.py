@@ -191,6 +191,39 @@ def multiexit_loss_bwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Ten
     return dh, dW
 
 
+def exit_agreement(h: List[torch.Tensor], W: List[torch.Tensor], stats: torch.Tensor, *, per_token=False,
+                   want_top1=False, workspace=None, status=None, stream=None):
+    """Agreement of every smaller exit with the largest (see mls_exit_agreement).
+
+    Returns (metrics [3(M-1)] = mean beta, mean KL, mean top-1 agreement per
+    smaller exit, per-token rows [3(M-1), T] or None, top-1 ids [M, T] or None).
+    """
+    M = len(h)
+    if len(W) != M or M < 2:
+        raise ValueError("need at least two exits")
+    T, V, dt = h[0].shape[0], W[0].shape[0], h[0].dtype
+    D = []
+    for m in range(M):
+        _need(h[m], f"h[{m}]", dt, 2)
+        _need(W[m], f"W[{m}]", dt, 2)
+        D.append(h[m].shape[1])
+    _need(stats, "stats", torch.float32, 2)
+    dev = h[0].device
+    metrics = torch.empty(3 * (M - 1), dtype=torch.float32, device=dev)
+    rows = torch.empty((3 * (M - 1), T), dtype=torch.float32, device=dev) if per_token else None
+    top1 = torch.empty((M, T), dtype=torch.int32, device=dev) if want_top1 else None
+    n = ctypes.c_size_t()
+    check("mls_exit_agreement_workspace",
+          lib().mls_exit_agreement_workspace(M, T, i64_array(D), V, _dtype_code(h[0]), ctypes.byref(n)))
+    workspace, ws_bytes = _workspace(workspace, n.value, dev)
+    code = lib().mls_exit_agreement(M, T, V, i64_array(D), ptr_array([t.data_ptr() for t in h]),
+                                    ptr_array([t.data_ptr() for t in W]), _dtype_code(h[0]), stats.data_ptr(),
+                                    metrics.data_ptr(), _ptr(rows), _ptr(top1), workspace.data_ptr(), ws_bytes,
+                                    _ptr(status), _stream_ptr(stream))
+    check("mls_exit_agreement", code)
+    return metrics, rows, top1
+
+
 def status_read(status: torch.Tensor, stream=None) -> Tuple[int, int]:
     """Synchronises, returns (status code, raw flag word) and clears the word."""
     out = ctypes.c_int32()

@@ -264,6 +264,48 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
   return from_cuda(mls::loss_simt_bwd(p, stats, grad_scale, dh, dW, accumulate_dW, workspace, s));
 }
 
+mls_status mls_exit_agreement_workspace(int M, int64_t T, const int64_t* D, int64_t V, mls_dtype dt,
+                                        size_t* bytes) {
+  if (bytes == nullptr) return MLS_ERR_INVALID_ARG;
+  size_t f = 0, b = 0;
+  mls_status st = mls_multiexit_loss_workspace(M, T, D, V, dt, &f, &b);
+  if (st != MLS_OK) return st;
+  if (M < 2) return MLS_ERR_INVALID_ARG;
+  const void* dummy[mls::kMaxExits];
+  alignas(16) static const char probe[16] = {0};
+  for (auto& d : dummy) d = probe;
+  LossProblem p{};
+  st = build_problem(M, T, V, D, reinterpret_cast<const int32_t*>(probe), dummy, dummy, 0.f, dt, nullptr, &p);
+  if (st != MLS_OK) return st;
+  *bytes = dt == MLS_BF16 ? mls::agree_tc_bytes(p) : mls::agree_simt_bytes(p);
+  return MLS_OK;
+}
+
+mls_status mls_exit_agreement(int M, int64_t T, int64_t V, const int64_t* D, const void* const* h,
+                              const void* const* W, mls_dtype dt, const float* stats, float* metrics,
+                              float* per_token, int32_t* top1, void* workspace, size_t ws_bytes,
+                              int32_t* dev_status, void* stream) {
+  if (M < 2) return MLS_ERR_INVALID_ARG;
+  alignas(16) static const int32_t no_targets[4] = {0, 0, 0, 0};
+  LossProblem p{};
+  mls_status st = build_problem(M, T, V, D, no_targets, h, W, 0.f, dt, dev_status, &p);
+  if (st != MLS_OK) return st;
+  if (stats == nullptr || metrics == nullptr) return MLS_ERR_INVALID_ARG;
+  if (!aligned16(stats) || (per_token != nullptr && !aligned16(per_token)) ||
+      (top1 != nullptr && !aligned16(top1)))
+    return MLS_ERR_UNSUPPORTED;
+  const size_t need = dt == MLS_BF16 ? mls::agree_tc_bytes(p) : mls::agree_simt_bytes(p);
+  if (workspace == nullptr || ws_bytes < need) return MLS_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
+  if ((st = device_ok()) != MLS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dt == MLS_BF16) {
+    if (!mls::tensor_map_encoder_available()) return MLS_ERR_CUDA;
+    return from_cuda(mls::agree_tc(p, stats, metrics, per_token, top1, workspace, s));
+  }
+  return from_cuda(mls::agree_simt(p, stats, metrics, per_token, top1, workspace, s));
+}
+
 mls_status mls_status_read(int32_t* dev_status, void* stream, int32_t* host_out) {
   if (dev_status == nullptr || host_out == nullptr) return MLS_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -83,6 +83,18 @@ cudaError_t loss_simt_fwd(const LossProblem& p, float* losses, float* stats, voi
 cudaError_t loss_simt_bwd(const LossProblem& p, const float* stats, float grad_scale, void* const* dh,
                           float* const* dW, int accumulate, void* ws, cudaStream_t st);
 
+// Agreement of every smaller exit with the largest: metrics [3(M-1)] = means of
+// beta, KL(p_M || q_m) and top-1 agreement; optional per-token rows and top-1 ids.
+size_t agree_tc_bytes(const LossProblem& p);
+size_t agree_simt_bytes(const LossProblem& p);
+cudaError_t agree_tc(const LossProblem& p, const float* stats, float* metrics, float* per_token, int32_t* top1,
+                     void* ws, cudaStream_t st);
+cudaError_t agree_simt(const LossProblem& p, const float* stats, float* metrics, float* per_token, int32_t* top1,
+                       void* ws, cudaStream_t st);
+
+// Shared: rows [Q][T] -> their means over T, fixed-order reduction.
+cudaError_t launch_row_means(const float* rows, int Q, int64_t T, float* out, cudaStream_t st);
+
 // Shared: per-token loss terms [2M-1][T] -> losses [2M], fixed-order reduction.
 cudaError_t launch_loss_reduce(const float* terms, int M, int64_t T, float alpha_d, float* losses,
                                cudaStream_t st);

@@ -238,6 +238,101 @@ __global__ void __launch_bounds__(1024) loss_reduce_kernel(const float* __restri
   }
 }
 
+// Mean over T of each of Q rows, fixed-order reduction; one block per row.
+__global__ void __launch_bounds__(1024) row_means_kernel(const float* __restrict__ rows, int64_t T,
+                                                         float* __restrict__ out) {
+  __shared__ float part[1024];
+  const int tid = threadIdx.x;
+  const float* r = rows + static_cast<int64_t>(blockIdx.x) * T;
+  float s = 0.f;
+  for (int64_t i = tid; i < T; i += 1024) s += r[i];
+  part[tid] = s;
+  __syncthreads();
+  for (int stride = 512; stride > 0; stride >>= 1) {
+    if (tid < stride) part[tid] += part[tid + stride];
+    __syncthreads();
+  }
+  if (tid == 0) out[blockIdx.x] = part[0] / static_cast<float>(T);
+}
+
+// Agreement of every smaller exit with the largest, one block per token, with
+// the normalisers from the forward statistics: sum_v min(q_m, p_T),
+// sum_v p_T l_m, sum_v p_T l_T and the first maximum of each exit's logits.
+__global__ void __launch_bounds__(kSimtThreads) simt_agree_kernel(const SimtDev p, const float* __restrict__ stats,
+                                                                  float* __restrict__ terms,
+                                                                  int32_t* __restrict__ top1) {
+  extern __shared__ float sm[];
+  const int M = p.M;
+  const int S = M - 1;
+  const int64_t t = blockIdx.x;
+  const int tid = threadIdx.x;
+  float* hrow = sm;
+  int64_t hsum = 0;
+  for (int m = 0; m < M; ++m) hsum += p.D[m];
+  float* red = sm + hsum;                     // [2S + 1 + M][kSimtThreads] floats
+  int* redi = reinterpret_cast<int*>(red + (2 * S + 1 + M) * kSimtThreads);   // [M][kSimtThreads]
+  for (int m = 0; m < M; ++m)
+    for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) hrow[p.Doff[m] + k] = p.h[m][t * p.D[m] + k];
+  __syncthreads();
+  float lse[kMaxExits];
+  for (int m = 0; m < M; ++m) lse[m] = stats[m * p.T + t];
+  float beta[kMaxExits - 1] = {0.f, 0.f, 0.f}, sl[kMaxExits - 1] = {0.f, 0.f, 0.f}, st = 0.f;
+  float mx[kMaxExits] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  int ix[kMaxExits] = {-1, -1, -1, -1};
+  for (int64_t v = tid; v < p.V; v += kSimtThreads) {
+    float l[kMaxExits];
+    for (int m = 0; m < M; ++m) {
+      const float* w = p.W[m] + v * p.D[m];
+      const float* hh = hrow + p.Doff[m];
+      float acc = 0.f;
+      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
+      l[m] = acc;
+      if (acc > mx[m]) { mx[m] = acc; ix[m] = static_cast<int>(v); }
+    }
+    const float pT = __expf(l[M - 1] - lse[M - 1]);
+    st = fmaf(pT, l[M - 1], st);
+    for (int s = 0; s < S; ++s) {
+      beta[s] += fminf(__expf(l[s] - lse[s]), pT);
+      sl[s] = fmaf(pT, l[s], sl[s]);
+    }
+  }
+  for (int s = 0; s < S; ++s) {
+    red[s * kSimtThreads + tid] = beta[s];
+    red[(S + s) * kSimtThreads + tid] = sl[s];
+  }
+  red[2 * S * kSimtThreads + tid] = st;
+  for (int m = 0; m < M; ++m) {
+    red[(2 * S + 1 + m) * kSimtThreads + tid] = mx[m];
+    redi[m * kSimtThreads + tid] = ix[m];
+  }
+  __syncthreads();
+  for (int stride = kSimtThreads / 2; stride > 0; stride >>= 1) {
+    if (tid < stride) {
+      const int o = tid + stride;
+      for (int q = 0; q < 2 * S + 1; ++q) red[q * kSimtThreads + tid] += red[q * kSimtThreads + o];
+      for (int m = 0; m < M; ++m) {
+        float* mv = red + (2 * S + 1 + m) * kSimtThreads;
+        int* iv = redi + m * kSimtThreads;
+        // larger value wins; on equal values the smaller vocabulary index
+        if (mv[o] > mv[tid] || (mv[o] == mv[tid] && iv[o] >= 0 && (iv[tid] < 0 || iv[o] < iv[tid]))) {
+          mv[tid] = mv[o];
+          iv[tid] = iv[o];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    for (int m = 0; m < M; ++m) top1[m * p.T + t] = redi[m * kSimtThreads];
+    const float stT = red[2 * S * kSimtThreads];
+    for (int s = 0; s < S; ++s) {
+      terms[s * p.T + t] = red[s * kSimtThreads];
+      terms[(S + s) * p.T + t] = (stT - red[(S + s) * kSimtThreads]) + (lse[s] - lse[M - 1]);
+      terms[(2 * S + s) * p.T + t] = (redi[s * kSimtThreads] == redi[(M - 1) * kSimtThreads]) ? 1.f : 0.f;
+    }
+  }
+}
+
 SimtDev make_dev(const LossProblem& p) {
   SimtDev d{};
   d.M = p.M;
@@ -276,6 +371,37 @@ size_t loss_simt_fwd_bytes(const LossProblem& p) {
 
 size_t loss_simt_bwd_bytes(const LossProblem& p) {
   return static_cast<size_t>(p.M) * p.T * p.V * sizeof(float);
+}
+
+cudaError_t launch_row_means(const float* rows, int Q, int64_t T, float* out, cudaStream_t st) {
+  row_means_kernel<<<Q, 1024, 0, st>>>(rows, T, out);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+size_t agree_simt_bytes(const LossProblem& p) {
+  const size_t terms = static_cast<size_t>(3 * (p.M - 1)) * p.T * sizeof(float);
+  const size_t top1 = static_cast<size_t>(p.M) * p.T * sizeof(int32_t);
+  return ((terms + 255) & ~size_t(255)) + top1;
+}
+
+cudaError_t agree_simt(const LossProblem& p, const float* stats, float* metrics, float* per_token, int32_t* top1,
+                       void* ws, cudaStream_t st) {
+  const SimtDev d = make_dev(p);
+  const size_t terms_b = static_cast<size_t>(3 * (p.M - 1)) * p.T * sizeof(float);
+  float* terms = per_token != nullptr ? per_token : static_cast<float*>(ws);
+  int32_t* top = top1 != nullptr ? top1
+                                 : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + ((terms_b + 255) & ~size_t(255)));
+  const int S = p.M - 1;
+  const size_t smem = (sum_d(p) + static_cast<size_t>(2 * S + 1 + p.M) * kSimtThreads) * sizeof(float) +
+                      static_cast<size_t>(p.M) * kSimtThreads * sizeof(int);
+  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(simt_agree_kernel), smem);
+  if (err != cudaSuccess) return err;
+  simt_agree_kernel<<<static_cast<unsigned>(p.T), kSimtThreads, smem, st>>>(d, stats, terms, top);
+  note_launches(1);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  return launch_row_means(terms, 3 * S, p.T, metrics, st);
 }
 
 cudaError_t launch_loss_reduce(const float* terms, int M, int64_t T, float alpha_d, float* losses,

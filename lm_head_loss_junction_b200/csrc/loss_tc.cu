@@ -84,7 +84,10 @@ struct __align__(1024) LossSmem {
   int abort;
 };
 
-enum LossMode { kModeStats = 0, kModeGrad = 1 };
+enum LossMode { kModeStats = 0, kModeGrad = 1, kModeAgree = 2 };
+
+// Partial rows per split in agreement mode: beta_s, S_s (students), S_T, max_m, argmax_m.
+__host__ __device__ constexpr int agree_rows(int M) { return 4 * M - 1; }
 
 __device__ __forceinline__ void loss_tile_coords(int i, const LossArgs& a, int& tt, int& vt) {
   const int per_group = a.group_tt * a.n_vt;
@@ -324,6 +327,50 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             a.partial[(static_cast<int64_t>(split) * Q + m) * a.T + t] = lse_part;
             if (j > 0) a.partial[(static_cast<int64_t>(split) * Q + M + m) * a.T + t] = abar;
           }
+        } else if (MODE == kModeAgree) {
+          // ---------------- agreement with the largest exit: sum_v min(q_m, p_T),
+          // sum_v p_T l_m (and p_T l_T), first maximum of the logits
+          float sum_min = 0.f, spl = 0.f, mxv = -INFINITY;
+          int mxi = -1;
+          if (live) {
+            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
+            const float ls = lse * kLog2e;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float r[32];
+              tmem_ld32(base + c * 32, r);
+#pragma unroll
+              for (int k = 0; k < 32; k += 2) {
+                const float e0 = exp2f(fmaf(r[k], kLog2e, -ls));
+                const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -ls));
+                if (r[k] > mxv) { mxv = r[k]; mxi = c0 + c * 32 + k; }
+                if (r[k + 1] > mxv) { mxv = r[k + 1]; mxi = c0 + c * 32 + k + 1; }
+                if (j == 0) {
+                  pt[c][k / 2] = pack_half2(e0, e1);
+                  spl = fmaf(e0, r[k], fmaf(e1, r[k + 1], spl));
+                } else {
+                  const float2 pp = unpack_half2(pt[c][k / 2]);
+                  sum_min += fminf(e0, pp.x) + fminf(e1, pp.y);
+                  spl = fmaf(pp.x, r[k], fmaf(pp.y, r[k + 1], spl));
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tempty[region]);
+          if (valid) {
+            const int QA = agree_rows(M);
+            float* prow = a.partial + static_cast<int64_t>(split) * QA * a.T + t;
+            if (j > 0) {
+              prow[static_cast<int64_t>(m) * a.T] = sum_min;
+              prow[static_cast<int64_t>(M - 1 + m) * a.T] = spl;
+            } else {
+              prow[static_cast<int64_t>(2 * (M - 1)) * a.T] = spl;
+            }
+            prow[static_cast<int64_t>(2 * M - 1 + m) * a.T] = mxv;
+            prow[static_cast<int64_t>(3 * M - 1 + m) * a.T] = __int_as_float(mxi);
+          }
         } else {
           // ---------------- backward: dense part of the logit gradient, bf16
           if (bad && j == 0 && vt == 0 && half == 0) set_flag(a.status, MLS_DEVFLAG_BAD_ID);
@@ -461,6 +508,63 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
     terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : lse - Sv;
   }
   if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
+}
+
+// ------------------------------------------------------------------ agreement merge
+// Per token: sums over the splits (plain sums: the agreement pass works with
+// the final normalisers), the first maximum over the splits in vocabulary
+// order, then beta, KL(p_T || q_m) = (S_T - S_m) + (lse_m - lse_T) and the
+// top-1 agreement.  Same 32-token x 8-row block layout as the loss merge.
+__global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const float* __restrict__ partial,
+                                                                      int n_splits, int M, int T,
+                                                                      const float* __restrict__ stats,
+                                                                      float* __restrict__ terms,
+                                                                      int32_t* __restrict__ top1) {
+  constexpr int S = kMaxExits - 1;
+  __shared__ float sh_b[kMergeRows][S][32], sh_s[kMergeRows][S][32], sh_st[kMergeRows][32];
+  __shared__ float sh_mx[kMergeRows][kMaxExits][32];
+  __shared__ int sh_ix[kMergeRows][kMaxExits][32];
+  const int lane = threadIdx.x, rowi = threadIdx.y;
+  const int t = blockIdx.x * 32 + lane;
+  const int QA = agree_rows(M);
+  const int per = (n_splits + kMergeRows - 1) / kMergeRows;
+  const int i0 = min(n_splits, rowi * per), i1 = min(n_splits, i0 + per);
+  float b[S] = {0.f, 0.f, 0.f}, sm[S] = {0.f, 0.f, 0.f}, st = 0.f;
+  float mx[kMaxExits] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  int ix[kMaxExits] = {-1, -1, -1, -1};
+  if (t < T) {
+    for (int i = i0; i < i1; ++i) {
+      const float* pi = partial + static_cast<int64_t>(i) * QA * T + t;
+      for (int s = 0; s < M - 1; ++s) {
+        b[s] += pi[static_cast<int64_t>(s) * T];
+        sm[s] += pi[static_cast<int64_t>(M - 1 + s) * T];
+      }
+      st += pi[static_cast<int64_t>(2 * (M - 1)) * T];
+      for (int m = 0; m < M; ++m) {
+        const float v = pi[static_cast<int64_t>(2 * M - 1 + m) * T];
+        if (v > mx[m]) { mx[m] = v; ix[m] = __float_as_int(pi[static_cast<int64_t>(3 * M - 1 + m) * T]); }
+      }
+    }
+  }
+  for (int s = 0; s < S; ++s) { sh_b[rowi][s][lane] = b[s]; sh_s[rowi][s][lane] = sm[s]; }
+  sh_st[rowi][lane] = st;
+  for (int m = 0; m < kMaxExits; ++m) { sh_mx[rowi][m][lane] = mx[m]; sh_ix[rowi][m][lane] = ix[m]; }
+  __syncthreads();
+  if (rowi != 0 || t >= T) return;
+  for (int r = 1; r < kMergeRows; ++r) {
+    for (int s = 0; s < M - 1; ++s) { b[s] += sh_b[r][s][lane]; sm[s] += sh_s[r][s][lane]; }
+    st += sh_st[r][lane];
+    for (int m = 0; m < M; ++m)
+      if (sh_mx[r][m][lane] > mx[m]) { mx[m] = sh_mx[r][m][lane]; ix[m] = sh_ix[r][m][lane]; }
+  }
+  const float lseT = stats[static_cast<int64_t>(M - 1) * T + t];
+  for (int m = 0; m < M; ++m) top1[static_cast<int64_t>(m) * T + t] = ix[m];
+  for (int s = 0; s < M - 1; ++s) {
+    const float lse = stats[static_cast<int64_t>(s) * T + t];
+    terms[static_cast<int64_t>(s) * T + t] = b[s];
+    terms[static_cast<int64_t>(M - 1 + s) * T + t] = (st - sm[s]) + (lse - lseT);
+    terms[static_cast<int64_t>(2 * (M - 1) + s) * T + t] = (ix[s] == ix[M - 1]) ? 1.f : 0.f;
+  }
 }
 
 // ------------------------------------------------------------------ grouped GEMM kernel (dh, dW)
@@ -893,6 +997,35 @@ size_t loss_tc_fwd_bytes(const LossProblem& p) {
   const size_t part = static_cast<size_t>(2 * loss_n_vt(p)) * (2 * p.M - 1) * p.T * sizeof(float);
   const size_t terms = static_cast<size_t>(2 * p.M - 1) * p.T * sizeof(float);
   return align_up(part) + align_up(terms);
+}
+
+size_t agree_tc_bytes(const LossProblem& p) {
+  const size_t part = static_cast<size_t>(2 * loss_n_vt(p)) * agree_rows(p.M) * p.T * sizeof(float);
+  const size_t terms = static_cast<size_t>(3 * (p.M - 1)) * p.T * sizeof(float);
+  const size_t top1 = static_cast<size_t>(p.M) * p.T * sizeof(int32_t);
+  return align_up(part) + align_up(terms) + align_up(top1);
+}
+
+cudaError_t agree_tc(const LossProblem& p, const float* stats, float* metrics, float* per_token, int32_t* top1,
+                     void* ws, cudaStream_t st) {
+  const size_t part = static_cast<size_t>(2 * loss_n_vt(p)) * agree_rows(p.M) * p.T * sizeof(float);
+  const size_t terms_b = static_cast<size_t>(3 * (p.M - 1)) * p.T * sizeof(float);
+  char* base = static_cast<char*>(ws);
+  float* partial = reinterpret_cast<float*>(base);
+  float* terms = per_token != nullptr ? per_token : reinterpret_cast<float*>(base + align_up(part));
+  int32_t* top = top1 != nullptr ? top1 : reinterpret_cast<int32_t*>(base + align_up(part) + align_up(terms_b));
+  LossArgs a = base_args(p);
+  a.partial = partial;
+  a.stats = const_cast<float*>(stats);
+  cudaError_t err = run_loss_tiles<kModeAgree>(p, a, st);
+  if (err != cudaSuccess) return err;
+  const int T = static_cast<int>(p.T);
+  agree_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(partial, 2 * a.n_vt, p.M, T, stats, terms,
+                                                                      top);
+  note_launches(1);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  return launch_row_means(terms, 3 * (p.M - 1), p.T, metrics, st);
 }
 
 size_t loss_tc_bwd_bytes(const LossProblem& p) {

@@ -88,6 +88,17 @@ def test_junction_argument_errors():
              None) == 3
 
 
+def test_agreement_argument_errors():
+    lib = _lib.lib()
+    one = lib.mls_exit_agreement(1, 16, 256, _lib.i64_array([64]), _lib.ptr_array([FAKE]), _lib.ptr_array([FAKE]),
+                                 _lib.MLS_BF16, FAKE, FAKE, None, None, FAKE, 1 << 30, None, None)
+    assert one == 1                                                  # needs a smaller exit
+    nostats = lib.mls_exit_agreement(2, 16, 256, _lib.i64_array([64, 128]), _lib.ptr_array([FAKE, FAKE]),
+                                     _lib.ptr_array([FAKE, FAKE]), _lib.MLS_BF16, None, FAKE, None, None, FAKE,
+                                     1 << 30, None, None)
+    assert nostats == 1
+
+
 def test_workspace_queries():
     import torch
     from lm_head_loss_junction_b200 import junction_bwd_workspace, multiexit_loss_workspace
