@@ -25,7 +25,6 @@
 // suite?" (section 4, the 0.7/0.3 mix), "Editing the methods of sub-models are
 // made of blocks" (Modeling paragraph: one LM head W^m in R^{V x D_m} per exit).
 #include <cuda.h>
-#include <cuda_fp16.h>
 #include <mutex>
 
 #include "kernels.h"
@@ -111,13 +110,14 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32
   (void)mbar_wait(bar, parity, &dummy, status);
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
+// Teacher probabilities are kept in registers as bf16 pairs: fp32's exponent
+// range (full-vocabulary probabilities reach 1e-9 and below, under fp16's
+// smallest subnormal) with round-to-nearest-even, so sums over the vocabulary
+// stay unbiased.
+__device__ __forceinline__ uint32_t pack_p2(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
-__device__ __forceinline__ float2 unpack_half2(uint32_t u) {
-  return __half22float2(*reinterpret_cast<__half2*>(&u));
+__device__ __forceinline__ float2 unpack_p2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
 // ------------------------------------------------------------------ loss tile kernel
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     const int Q = 2 * M - 1;
     const float al = a.alpha;
     uint32_t job = 0;
-    // teacher probabilities of this thread's row and split, packed fp16 pairs
+    // teacher probabilities of this thread's row and split, packed bf16 pairs
     uint32_t pt[4][16];
     float inv_z = 0.f;
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           float lse_part = -INFINITY, abar = 0.f;
           if (live) {
             if (j == 0) {
-              // teacher: split max, then p~ = exp(l - max) (fp16 in registers) and their sum
+              // teacher: split max, then p~ = exp(l - max) (bf16 in registers) and their sum
               float mx = -INFINITY;
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                   const float e0 = exp2f(fmaf(r[k], kLog2e, -mxs));
                   const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -mxs));
                   z += e0 + e1;
-                  pt[c][k / 2] = pack_half2(e0, e1);
+                  pt[c][k / 2] = pack_p2(e0, e1);
                 }
               }
               inv_z = 1.f / z;
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
                   zc += exp2f(fmaf(r[k], kLog2e, -mns)) + exp2f(fmaf(r[k + 1], kLog2e, -mns));
-                  const float2 pp = unpack_half2(pt[c][k / 2]);
+                  const float2 pp = unpack_p2(pt[c][k / 2]);
                   A = fmaf(pp.x, r[k], A);
                   A = fmaf(pp.y, r[k + 1], A);
                 }
@@ -346,10 +346,10 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 if (r[k] > mxv) { mxv = r[k]; mxi = c0 + c * 32 + k; }
                 if (r[k + 1] > mxv) { mxv = r[k + 1]; mxi = c0 + c * 32 + k + 1; }
                 if (j == 0) {
-                  pt[c][k / 2] = pack_half2(e0, e1);
+                  pt[c][k / 2] = pack_p2(e0, e1);
                   spl = fmaf(e0, r[k], fmaf(e1, r[k + 1], spl));
                 } else {
-                  const float2 pp = unpack_half2(pt[c][k / 2]);
+                  const float2 pp = unpack_p2(pt[c][k / 2]);
                   sum_min += fminf(e0, pp.x) + fminf(e1, pp.y);
                   spl = fmaf(pp.x, r[k], fmaf(pp.y, r[k + 1], spl));
                 }
@@ -389,11 +389,11 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -ls));
                 float g0, g1;
                 if (j == 0) {                      // teacher: G' = p_T
-                  pt[c][k / 2] = pack_half2(e0, e1);
+                  pt[c][k / 2] = pack_p2(e0, e1);
                   g0 = e0;
                   g1 = e1;
                 } else {                           // student: G' = q - alpha_d p_T
-                  const float2 pp = unpack_half2(pt[c][k / 2]);
+                  const float2 pp = unpack_p2(pt[c][k / 2]);
                   g0 = fmaf(-al, pp.x, e0);
                   g1 = fmaf(-al, pp.y, e1);
                 }
