@@ -25,6 +25,7 @@
 // suite?" (section 4, the 0.7/0.3 mix), "Editing the methods of sub-models are
 // made of blocks" (Modeling paragraph: one LM head W^m in R^{V x D_m} per exit).
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <mutex>
 
 #include "kernels.h"
@@ -85,8 +86,8 @@ struct __align__(1024) LossSmem {
 
 enum LossMode { kModeStats = 0, kModeGrad = 1, kModeAgree = 2 };
 
-// Partial rows per split in agreement mode: beta_s, S_s (students), S_T, max_m, argmax_m.
-__host__ __device__ constexpr int agree_rows(int M) { return 4 * M - 1; }
+// Partial rows per split in agreement mode: beta_s, KL_s (students), max_m, argmax_m.
+__host__ __device__ constexpr int agree_rows(int M) { return 4 * M - 2; }
 
 __device__ __forceinline__ void loss_tile_coords(int i, const LossArgs& a, int& tt, int& vt) {
   const int per_group = a.group_tt * a.n_vt;
@@ -110,14 +111,33 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32
   (void)mbar_wait(bar, parity, &dummy, status);
 }
 
-// Teacher probabilities are kept in registers as bf16 pairs: fp32's exponent
-// range (full-vocabulary probabilities reach 1e-9 and below, under fp16's
-// smallest subnormal) with round-to-nearest-even, so sums over the vocabulary
-// stay unbiased.
-__device__ __forceinline__ uint32_t pack_p2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+// Teacher probabilities are kept in registers as fp16 pairs (11-bit
+// significand) for the students of the same tile.  Values below fp16's range
+// (under about 6e-8 relative to the split maximum or the normaliser) carry
+// negligible weight in the statistics and in G'; the agreement pass, whose
+// acceptance sums those tiny values, reads the teacher's logits from TMEM
+// instead (see job_slot).
+__device__ __forceinline__ uint32_t pack_p2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 
-__device__ __forceinline__ float2 unpack_p2(uint32_t u) {
-  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+__device__ __forceinline__ float2 unpack_p2(uint32_t u) { return __half22float2(*reinterpret_cast<__half2*>(&u)); }
+
+// TMEM region and use count of job j (exit M-1-j) of the tile_iter-th tile of a CTA.
+// Statistics and gradient modes alternate the two regions between consecutive
+// jobs.  The agreement mode keeps the teacher in region 0 for the whole tile
+// and runs the students one after another in region 1, so the epilogue can
+// read both exits' logits of the same element.
+__device__ __forceinline__ void job_slot(int mode, int M, uint32_t tile_iter, int j, uint32_t job,
+                                         uint32_t& region, uint32_t& use) {
+  if (mode == 2) {
+    region = (j == 0) ? 0u : 1u;
+    use = (j == 0) ? tile_iter : tile_iter * static_cast<uint32_t>(M - 1) + static_cast<uint32_t>(j - 1);
+  } else {
+    region = job & 1u;
+    use = job >> 1;
+  }
 }
 
 // ------------------------------------------------------------------ loss tile kernel
@@ -193,13 +213,14 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kBM, kLossBN, false, false);
-      uint32_t stage = 0, phase = 0, job = 0;
+      uint32_t stage = 0, phase = 0, job = 0, tile_iter = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x, ++tile_iter) {
         for (int j = 0; j < M && ok; ++j, ++job) {
           const int m = M - 1 - j;
-          const uint32_t region = job & 1;
-          if (!mbar_wait(&s.tempty[region], ((job >> 1) & 1) ^ 1, abort, a.status)) { ok = false; break; }
+          uint32_t region, use;
+          job_slot(MODE, M, tile_iter, j, job, region, use);
+          if (!mbar_wait(&s.tempty[region], (use & 1) ^ 1, abort, a.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + region * kLossBN;
           for (int kb = 0; kb < a.kblocks[m]; ++kb) {
@@ -231,11 +252,11 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * kSplitCols;
     const int Q = 2 * M - 1;
     const float al = a.alpha;
-    uint32_t job = 0;
-    // teacher probabilities of this thread's row and split, packed bf16 pairs
+    uint32_t job = 0, tile_iter = 0;
+    // teacher probabilities of this thread's row and split, packed fp16 pairs
     uint32_t pt[4][16];
     float inv_z = 0.f;
-    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x, ++tile_iter) {
       int tt, vt;
       loss_tile_coords(tile, a, tt, vt);
       const int t = tt * kBM + row;
@@ -250,9 +271,10 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
       bool stop = false;
       for (int j = 0; j < M; ++j, ++job) {
         const int m = M - 1 - j;
-        const uint32_t region = job & 1;
+        uint32_t region, use;
+        job_slot(MODE, M, tile_iter, j, job, region, use);
         const uint32_t base = lane_base + region * kLossBN;
-        if (!warp_wait(&s.tfull[region], (job >> 1) & 1, abort, a.status)) { stop = true; break; }
+        if (!warp_wait(&s.tfull[region], use & 1, abort, a.status)) { stop = true; break; }
         tc_fence_after();
         if (MODE == kModeStats) {
           float lse_part = -INFINITY, abar = 0.f;
@@ -328,48 +350,53 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             if (j > 0) a.partial[(static_cast<int64_t>(split) * Q + M + m) * a.T + t] = abar;
           }
         } else if (MODE == kModeAgree) {
-          // ---------------- agreement with the largest exit: sum_v min(q_m, p_T),
-          // sum_v p_T l_m (and p_T l_T), first maximum of the logits
-          float sum_min = 0.f, spl = 0.f, mxv = -INFINITY;
+          // ---------------- agreement with the largest exit.  The teacher's tile stays in
+          // region 0 while each student's tile arrives in region 1: per element
+          // p = exp(l_T - lse_T), q = exp(l_m - lse_m); sum min(q, p) and
+          // sum p (log p - log q); first maximum of each exit's logits.
+          float mxv = -INFINITY, sum_min = 0.f, kl = 0.f;
           int mxi = -1;
           if (live) {
             const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
-            const float ls = lse * kLog2e;
-#pragma unroll
+            const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
+            const uint32_t tbase = lane_base;          // region 0: the teacher
+#pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float r[32];
               tmem_ld32(base + c * 32, r);
 #pragma unroll
-              for (int k = 0; k < 32; k += 2) {
-                const float e0 = exp2f(fmaf(r[k], kLog2e, -ls));
-                const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -ls));
+              for (int k = 0; k < 32; ++k)
                 if (r[k] > mxv) { mxv = r[k]; mxi = c0 + c * 32 + k; }
-                if (r[k + 1] > mxv) { mxv = r[k + 1]; mxi = c0 + c * 32 + k + 1; }
-                if (j == 0) {
-                  pt[c][k / 2] = pack_p2(e0, e1);
-                  spl = fmaf(e0, r[k], fmaf(e1, r[k + 1], spl));
-                } else {
-                  const float2 pp = unpack_p2(pt[c][k / 2]);
-                  sum_min += fminf(e0, pp.x) + fminf(e1, pp.y);
-                  spl = fmaf(pp.x, r[k], fmaf(pp.y, r[k + 1], spl));
+              if (j > 0) {
+                float lt[32];
+                tmem_ld32(tbase + c * 32, lt);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                  const float la = lt[k] - lseT;            // log p
+                  const float lb = r[k] - lse;              // log q
+                  const float pv = exp2f(la * kLog2e);
+                  const float qv = exp2f(lb * kLog2e);
+                  sum_min += fminf(pv, qv);
+                  kl = fmaf(pv, la - lb, kl);
                 }
               }
             }
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[region]);
+          if (lane == 0) {
+            if (j > 0) mbar_arrive(&s.tempty[1]);         // this student's region
+            if (j == M - 1) mbar_arrive(&s.tempty[0]);    // the teacher's, after the last student
+          }
           if (valid) {
             const int QA = agree_rows(M);
             float* prow = a.partial + static_cast<int64_t>(split) * QA * a.T + t;
             if (j > 0) {
               prow[static_cast<int64_t>(m) * a.T] = sum_min;
-              prow[static_cast<int64_t>(M - 1 + m) * a.T] = spl;
-            } else {
-              prow[static_cast<int64_t>(2 * (M - 1)) * a.T] = spl;
+              prow[static_cast<int64_t>(M - 1 + m) * a.T] = kl;
             }
-            prow[static_cast<int64_t>(2 * M - 1 + m) * a.T] = mxv;
-            prow[static_cast<int64_t>(3 * M - 1 + m) * a.T] = __int_as_float(mxi);
+            prow[static_cast<int64_t>(2 * (M - 1) + m) * a.T] = mxv;
+            prow[static_cast<int64_t>(3 * M - 2 + m) * a.T] = __int_as_float(mxi);
           }
         } else {
           // ---------------- backward: dense part of the logit gradient, bf16
@@ -511,17 +538,16 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
 }
 
 // ------------------------------------------------------------------ agreement merge
-// Per token: sums over the splits (plain sums: the agreement pass works with
-// the final normalisers), the first maximum over the splits in vocabulary
-// order, then beta, KL(p_T || q_m) = (S_T - S_m) + (lse_m - lse_T) and the
-// top-1 agreement.  Same 32-token x 8-row block layout as the loss merge.
+// Per token: sums over the splits of beta and KL (plain sums: the agreement
+// pass uses the final normalisers), the first maximum over the splits in
+// vocabulary order, and the top-1 agreement.  Same 32-token x 8-row block
+// layout as the loss merge.
 __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const float* __restrict__ partial,
                                                                       int n_splits, int M, int T,
-                                                                      const float* __restrict__ stats,
                                                                       float* __restrict__ terms,
                                                                       int32_t* __restrict__ top1) {
   constexpr int S = kMaxExits - 1;
-  __shared__ float sh_b[kMergeRows][S][32], sh_s[kMergeRows][S][32], sh_st[kMergeRows][32];
+  __shared__ float sh_b[kMergeRows][S][32], sh_k[kMergeRows][S][32];
   __shared__ float sh_mx[kMergeRows][kMaxExits][32];
   __shared__ int sh_ix[kMergeRows][kMaxExits][32];
   const int lane = threadIdx.x, rowi = threadIdx.y;
@@ -529,7 +555,7 @@ __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const floa
   const int QA = agree_rows(M);
   const int per = (n_splits + kMergeRows - 1) / kMergeRows;
   const int i0 = min(n_splits, rowi * per), i1 = min(n_splits, i0 + per);
-  float b[S] = {0.f, 0.f, 0.f}, sm[S] = {0.f, 0.f, 0.f}, st = 0.f;
+  float b[S] = {0.f, 0.f, 0.f}, kl[S] = {0.f, 0.f, 0.f};
   float mx[kMaxExits] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   int ix[kMaxExits] = {-1, -1, -1, -1};
   if (t < T) {
@@ -537,32 +563,27 @@ __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const floa
       const float* pi = partial + static_cast<int64_t>(i) * QA * T + t;
       for (int s = 0; s < M - 1; ++s) {
         b[s] += pi[static_cast<int64_t>(s) * T];
-        sm[s] += pi[static_cast<int64_t>(M - 1 + s) * T];
+        kl[s] += pi[static_cast<int64_t>(M - 1 + s) * T];
       }
-      st += pi[static_cast<int64_t>(2 * (M - 1)) * T];
       for (int m = 0; m < M; ++m) {
-        const float v = pi[static_cast<int64_t>(2 * M - 1 + m) * T];
-        if (v > mx[m]) { mx[m] = v; ix[m] = __float_as_int(pi[static_cast<int64_t>(3 * M - 1 + m) * T]); }
+        const float v = pi[static_cast<int64_t>(2 * (M - 1) + m) * T];
+        if (v > mx[m]) { mx[m] = v; ix[m] = __float_as_int(pi[static_cast<int64_t>(3 * M - 2 + m) * T]); }
       }
     }
   }
-  for (int s = 0; s < S; ++s) { sh_b[rowi][s][lane] = b[s]; sh_s[rowi][s][lane] = sm[s]; }
-  sh_st[rowi][lane] = st;
+  for (int s = 0; s < S; ++s) { sh_b[rowi][s][lane] = b[s]; sh_k[rowi][s][lane] = kl[s]; }
   for (int m = 0; m < kMaxExits; ++m) { sh_mx[rowi][m][lane] = mx[m]; sh_ix[rowi][m][lane] = ix[m]; }
   __syncthreads();
   if (rowi != 0 || t >= T) return;
   for (int r = 1; r < kMergeRows; ++r) {
-    for (int s = 0; s < M - 1; ++s) { b[s] += sh_b[r][s][lane]; sm[s] += sh_s[r][s][lane]; }
-    st += sh_st[r][lane];
+    for (int s = 0; s < M - 1; ++s) { b[s] += sh_b[r][s][lane]; kl[s] += sh_k[r][s][lane]; }
     for (int m = 0; m < M; ++m)
       if (sh_mx[r][m][lane] > mx[m]) { mx[m] = sh_mx[r][m][lane]; ix[m] = sh_ix[r][m][lane]; }
   }
-  const float lseT = stats[static_cast<int64_t>(M - 1) * T + t];
   for (int m = 0; m < M; ++m) top1[static_cast<int64_t>(m) * T + t] = ix[m];
   for (int s = 0; s < M - 1; ++s) {
-    const float lse = stats[static_cast<int64_t>(s) * T + t];
     terms[static_cast<int64_t>(s) * T + t] = b[s];
-    terms[static_cast<int64_t>(M - 1 + s) * T + t] = (st - sm[s]) + (lse - lseT);
+    terms[static_cast<int64_t>(M - 1 + s) * T + t] = kl[s];
     terms[static_cast<int64_t>(2 * (M - 1) + s) * T + t] = (ix[s] == ix[M - 1]) ? 1.f : 0.f;
   }
 }
@@ -1020,8 +1041,7 @@ cudaError_t agree_tc(const LossProblem& p, const float* stats, float* metrics, f
   cudaError_t err = run_loss_tiles<kModeAgree>(p, a, st);
   if (err != cudaSuccess) return err;
   const int T = static_cast<int>(p.T);
-  agree_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(partial, 2 * a.n_vt, p.M, T, stats, terms,
-                                                                      top);
+  agree_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(partial, 2 * a.n_vt, p.M, T, terms, top);
   note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
