@@ -258,6 +258,41 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   int32_t* dev_status, void* stream);
 
 /*
+ * Options of the _opts variants of the loss entry points (NULL = defaults).
+ *   exit_weights  HOST float [M] or NULL: per-exit loss weights lambda_m,
+ *                 L = sum_{m<M} lambda_m [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m]
+ *                     + lambda_M CE_LM,M,
+ *                 and every exit's gradient is scaled by its lambda_m.  NULL
+ *                 means 1 for every exit, the pages' equal weights; the same
+ *                 summary's limitations paragraph ("Matryoshka Language Model
+ *                 Suites") reports that reweighting closes much of the gap.
+ *                 Non-finite weights return MLS_ERR_INVALID_ARG.
+ * The per-exit CE_LM and CE_KD in `losses` are unweighted; L is weighted.
+ */
+typedef struct {
+  const float* exit_weights;
+} mls_loss_options;
+
+mls_status mls_multiexit_loss_fwd_opts(int M, int64_t T, int64_t V, const int64_t* D,
+                                       const int32_t* y_targets,
+                                       const void* const* h, const void* const* W,
+                                       float alpha_d, mls_dtype dt,
+                                       float* losses, float* stats,
+                                       void* workspace, size_t ws_bytes,
+                                       const mls_loss_options* opts,
+                                       int32_t* dev_status, void* stream);
+
+mls_status mls_multiexit_loss_bwd_opts(int M, int64_t T, int64_t V, const int64_t* D,
+                                       const int32_t* y_targets,
+                                       const void* const* h, const void* const* W,
+                                       float alpha_d, mls_dtype dt,
+                                       const float* stats, float grad_scale,
+                                       void* const* dh, float* const* dW, int accumulate_dW,
+                                       void* workspace, size_t ws_bytes,
+                                       const mls_loss_options* opts,
+                                       int32_t* dev_status, void* stream);
+
+/*
  * mls_exit_agreement -- how well every smaller exit agrees with the largest
  * one, per token, from the same logits (computed again, never stored) and the
  * normalisers in `stats` from mls_multiexit_loss_fwd.  Measures named by the

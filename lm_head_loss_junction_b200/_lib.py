@@ -34,6 +34,11 @@ _f32 = ctypes.c_float
 _sz = ctypes.c_size_t
 _u32 = ctypes.c_uint32
 
+class LossOptions(ctypes.Structure):
+    """mls_loss_options"""
+    _fields_ = [("exit_weights", ctypes.POINTER(ctypes.c_float))]
+
+
 # name -> (restype, argtypes), in the order of include/mls.h
 PROTOTYPES = {
     "mls_junction_fwd": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _int, _vp, _vp]),
@@ -54,6 +59,13 @@ PROTOTYPES = {
                                       ctypes.POINTER(_vp), ctypes.POINTER(_vp), _f32, _int,
                                       _vp, _f32, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int,
                                       _vp, _sz, _vp, _vp]),
+    "mls_multiexit_loss_fwd_opts": (_int, [_int, _i64, _i64, ctypes.POINTER(_i64), _vp,
+                                           ctypes.POINTER(_vp), ctypes.POINTER(_vp), _f32, _int,
+                                           _vp, _vp, _vp, _sz, ctypes.POINTER(LossOptions), _vp, _vp]),
+    "mls_multiexit_loss_bwd_opts": (_int, [_int, _i64, _i64, ctypes.POINTER(_i64), _vp,
+                                           ctypes.POINTER(_vp), ctypes.POINTER(_vp), _f32, _int,
+                                           _vp, _f32, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int,
+                                           _vp, _sz, ctypes.POINTER(LossOptions), _vp, _vp]),
     "mls_exit_agreement_workspace": (_int, [_int, _i64, ctypes.POINTER(_i64), _i64, _int, ctypes.POINTER(_sz)]),
     "mls_exit_agreement": (_int, [_int, _i64, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                   _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
@@ -106,3 +118,13 @@ def i64_array(vals):
     for i, v in enumerate(vals):
         arr[i] = int(v)
     return arr
+
+
+def loss_options(exit_weights=None):
+    """ctypes options struct (and the buffer it points to), or None for defaults."""
+    if exit_weights is None:
+        return None
+    buf = (ctypes.c_float * len(exit_weights))(*[float(w) for w in exit_weights])
+    opts = LossOptions(ctypes.cast(buf, ctypes.POINTER(ctypes.c_float)))
+    opts._buf = buf          # keep the weights alive with the struct
+    return opts

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <climits>
 #include <cstdint>
 
@@ -87,7 +88,20 @@ mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const in
   }
   p->y = y;
   p->alpha_d = alpha_d;
+  for (int m = 0; m < mls::kMaxExits; ++m) p->exit_w[m] = 1.f;
   p->status = status;
+  return MLS_OK;
+}
+
+mls_status apply_options(const mls_loss_options* opts, LossProblem* p) {
+  if (opts == nullptr) return MLS_OK;
+  if (opts->exit_weights != nullptr) {
+    for (int m = 0; m < p->M; ++m) {
+      const float w = opts->exit_weights[m];
+      if (!(w == w) || w == INFINITY || w == -INFINITY) return MLS_ERR_INVALID_ARG;
+      p->exit_w[m] = w;
+    }
+  }
   return MLS_OK;
 }
 
@@ -221,9 +235,18 @@ mls_status mls_multiexit_loss_fwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   const void* const* h, const void* const* W, float alpha_d, mls_dtype dt,
                                   float* losses, float* stats, void* workspace, size_t ws_bytes,
                                   int32_t* dev_status, void* stream) {
+  return mls_multiexit_loss_fwd_opts(M, T, V, D, y_targets, h, W, alpha_d, dt, losses, stats, workspace, ws_bytes,
+                                     nullptr, dev_status, stream);
+}
+
+mls_status mls_multiexit_loss_fwd_opts(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y_targets,
+                                       const void* const* h, const void* const* W, float alpha_d, mls_dtype dt,
+                                       float* losses, float* stats, void* workspace, size_t ws_bytes,
+                                       const mls_loss_options* opts, int32_t* dev_status, void* stream) {
   LossProblem p{};
   mls_status st = build_problem(M, T, V, D, y_targets, h, W, alpha_d, dt, dev_status, &p);
   if (st != MLS_OK) return st;
+  if ((st = apply_options(opts, &p)) != MLS_OK) return st;
   if (losses == nullptr || stats == nullptr) return MLS_ERR_INVALID_ARG;
   if (!aligned16(stats)) return MLS_ERR_UNSUPPORTED;
   const size_t need = dt == MLS_BF16 ? mls::loss_tc_fwd_bytes(p) : mls::loss_simt_fwd_bytes(p);
@@ -243,9 +266,19 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   const float* stats, float grad_scale, void* const* dh, float* const* dW,
                                   int accumulate_dW, void* workspace, size_t ws_bytes, int32_t* dev_status,
                                   void* stream) {
+  return mls_multiexit_loss_bwd_opts(M, T, V, D, y_targets, h, W, alpha_d, dt, stats, grad_scale, dh, dW,
+                                     accumulate_dW, workspace, ws_bytes, nullptr, dev_status, stream);
+}
+
+mls_status mls_multiexit_loss_bwd_opts(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y_targets,
+                                       const void* const* h, const void* const* W, float alpha_d, mls_dtype dt,
+                                       const float* stats, float grad_scale, void* const* dh, float* const* dW,
+                                       int accumulate_dW, void* workspace, size_t ws_bytes,
+                                       const mls_loss_options* opts, int32_t* dev_status, void* stream) {
   LossProblem p{};
   mls_status st = build_problem(M, T, V, D, y_targets, h, W, alpha_d, dt, dev_status, &p);
   if (st != MLS_OK) return st;
+  if ((st = apply_options(opts, &p)) != MLS_OK) return st;
   if (stats == nullptr || dh == nullptr || dW == nullptr) return MLS_ERR_INVALID_ARG;
   for (int m = 0; m < M; ++m) {
     if (dh[m] == nullptr || dW[m] == nullptr) return MLS_ERR_INVALID_ARG;

@@ -64,6 +64,7 @@ struct LossProblem {
   const void* h[kMaxExits];
   const void* W[kMaxExits];
   float alpha_d;
+  float exit_w[kMaxExits];   // per-exit loss weights (1 = equal weights)
   int32_t* status;
 };
 
@@ -96,8 +97,7 @@ cudaError_t agree_simt(const LossProblem& p, const float* stats, float* metrics,
 cudaError_t launch_row_means(const float* rows, int Q, int64_t T, float* out, cudaStream_t st);
 
 // Shared: per-token loss terms [2M-1][T] -> losses [2M], fixed-order reduction.
-cudaError_t launch_loss_reduce(const float* terms, int M, int64_t T, float alpha_d, float* losses,
-                               cudaStream_t st);
+cudaError_t launch_loss_reduce(const float* terms, const LossProblem& p, float* losses, cudaStream_t st);
 
 // Counts kernel launches issued by the library (diagnostics).
 void note_launches(int n);

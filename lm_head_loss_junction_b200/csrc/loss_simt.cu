@@ -26,6 +26,7 @@ struct SimtDev {
   const float* h[kMaxExits];
   const float* W[kMaxExits];
   float alpha_d;
+  float exit_w[kMaxExits];
   int32_t* status;
   float* dh[kMaxExits];
   float* dW[kMaxExits];
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
       float g;
       if (m == M - 1) g = pT - hot;
       else g = __expf(l[m] - lse[m]) - a * pT - (1.f - a) * hot;
-      G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : g;
+      G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : p.exit_w[m] * g;
     }
   }
   __syncthreads();
@@ -209,8 +210,12 @@ __global__ void __launch_bounds__(kSimtThreads) simt_dw_kernel(const SimtDev p, 
 }
 
 // Fixed-order sum of the per-token loss terms; one block.
+struct ExitWeights {
+  float w[kMaxExits];
+};
+
 __global__ void __launch_bounds__(1024) loss_reduce_kernel(const float* __restrict__ terms, int M, int64_t T,
-                                                           float alpha_d, float* __restrict__ losses) {
+                                                           float alpha_d, ExitWeights ew, float* __restrict__ losses) {
   __shared__ float part[1024];
   __shared__ float tot[2 * kMaxExits];
   const int tid = threadIdx.x;
@@ -228,11 +233,11 @@ __global__ void __launch_bounds__(1024) loss_reduce_kernel(const float* __restri
     __syncthreads();
   }
   if (tid == 0) {
-    float L = tot[M - 1];
+    float L = ew.w[M - 1] * tot[M - 1];
     for (int m = 0; m < M; ++m) losses[m] = tot[m];
     for (int s = 0; s < M - 1; ++s) {
       losses[M + s] = tot[M + s];
-      L += (1.f - alpha_d) * tot[s] + alpha_d * tot[M + s];
+      L += ew.w[s] * ((1.f - alpha_d) * tot[s] + alpha_d * tot[M + s]);
     }
     losses[2 * M - 1] = L;
   }
@@ -348,6 +353,7 @@ SimtDev make_dev(const LossProblem& p) {
   }
   d.y = p.y;
   d.alpha_d = p.alpha_d;
+  for (int m = 0; m < kMaxExits; ++m) d.exit_w[m] = p.exit_w[m];
   d.status = p.status;
   return d;
 }
@@ -404,9 +410,10 @@ cudaError_t agree_simt(const LossProblem& p, const float* stats, float* metrics,
   return launch_row_means(terms, 3 * S, p.T, metrics, st);
 }
 
-cudaError_t launch_loss_reduce(const float* terms, int M, int64_t T, float alpha_d, float* losses,
-                               cudaStream_t st) {
-  loss_reduce_kernel<<<1, 1024, 0, st>>>(terms, M, T, alpha_d, losses);
+cudaError_t launch_loss_reduce(const float* terms, const LossProblem& p, float* losses, cudaStream_t st) {
+  ExitWeights ew;
+  for (int m = 0; m < kMaxExits; ++m) ew.w[m] = p.exit_w[m];
+  loss_reduce_kernel<<<1, 1024, 0, st>>>(terms, p.M, p.T, p.alpha_d, ew, losses);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -423,7 +430,7 @@ cudaError_t loss_simt_fwd(const LossProblem& p, float* losses, float* stats, voi
   note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  return launch_loss_reduce(terms, p.M, p.T, p.alpha_d, losses, st);
+  return launch_loss_reduce(terms, p, losses, st);
 }
 
 cudaError_t loss_simt_bwd(const LossProblem& p, const float* stats, float grad_scale, void* const* dh,

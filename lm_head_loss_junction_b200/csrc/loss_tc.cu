@@ -612,7 +612,7 @@ struct GemmArgs {
   int Ndim[kMaxExits];
   int n_nt[kMaxExits];
   void* out[kMaxExits];
-  float alpha;
+  float alpha[kMaxExits];          // output scale of each problem
   int accumulate;
   int32_t* status;
   // Optional exact one-hot term (bf16 output only): row r of problem p also gets
@@ -782,7 +782,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const int32_t k = __ldg(g.onehot_idx + row);
         if (k >= 0 && k < g.onehot_limit) onehot_row = k;
       }
-      const float oh_scale = g.alpha * g.onehot_coef[p];
+      const float alpha = g.alpha[p];
+      const float oh_scale = alpha * g.onehot_coef[p];
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float r[32];
@@ -803,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           for (int u = 0; u < 4; ++u) {
             float f[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = r[8 * u + e] * g.alpha;
+            for (int e = 0; e < 8; ++e) f[e] = r[8 * u + e] * alpha;
             if (oh != nullptr) {
               float w[8];
               bf16x8_to_f32(__ldg(oh + u), w);
@@ -816,8 +817,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out[p]) + off);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            float4 v = make_float4(r[4 * u] * g.alpha, r[4 * u + 1] * g.alpha, r[4 * u + 2] * g.alpha,
-                                   r[4 * u + 3] * g.alpha);
+            float4 v = make_float4(r[4 * u] * alpha, r[4 * u + 1] * alpha, r[4 * u + 2] * alpha,
+                                   r[4 * u + 3] * alpha);
             if (g.accumulate) {
               const float4 o = dst[u];
               v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
@@ -971,7 +972,7 @@ cudaError_t run_dh_all(const LossProblem& p, const __nv_bfloat16* G, void* const
   g.nprob = p.M;
   g.Mdim = static_cast<int>(p.T);
   g.Kdim = static_cast<int>(p.V);
-  g.alpha = alpha;
+  for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
   g.status = p.status;
   g.onehot_idx = p.y;
   g.onehot_limit = static_cast<int>(p.V);
@@ -997,7 +998,7 @@ cudaError_t run_dw_all(const LossProblem& p, const __nv_bfloat16* G, float* cons
   g.nprob = p.M;
   g.Mdim = static_cast<int>(p.V);
   g.Kdim = static_cast<int>(p.T);
-  g.alpha = alpha;
+  for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
   g.accumulate = accumulate;
   g.status = p.status;
   for (int m = 0; m < p.M; ++m) {
@@ -1066,7 +1067,7 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  return launch_loss_reduce(w.terms, p.M, p.T, p.alpha_d, losses, st);
+  return launch_loss_reduce(w.terms, p, losses, st);
 }
 
 cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_scale, void* const* dh,
@@ -1097,7 +1098,7 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   // one-hot part of dW: (1 - alpha_d) for students, 1 for the teacher
   for (int m = 0; m < p.M; ++m) {
     const float c = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
-    err = scatter_target_rows(ix, p.h[m], static_cast<int>(p.D[m] / 8), dW[m], alpha * c, st);
+    err = scatter_target_rows(ix, p.h[m], static_cast<int>(p.D[m] / 8), dW[m], alpha * p.exit_w[m] * c, st);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;

@@ -57,13 +57,18 @@ def softmax_rows(l: np.ndarray) -> np.ndarray:
 
 
 def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
-                   rows=None, token_block=256):
+                   rows=None, token_block=256, exit_weights=None):
     """Multi-exit loss, per-token statistics and (optionally) gradients, fp64.
 
     y: int [T] targets; h: list of M arrays [T, D_m]; W: list of M arrays [V, D_m].
     rows: optional int array of token indices; when given, only those tokens are
     evaluated (their per-token statistics and dh rows; the means and dW are then
     over the selected tokens, normalised by the full T).
+    exit_weights: optional per-exit weights lambda_m (default 1 each: "summed
+    with equal weight"; "Matryoshka Language Model Suites", limitations
+    paragraph, notes that reweighting the exits closes much of the gap):
+    L = sum_{m<M} lambda_m [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m] + lambda_M CE_LM,M,
+    and each exit's gradient is scaled by its lambda_m.
 
     Returns a dict with
       ce_lm [M], ce_kd [M-1], loss (scalar)         -- means over the tokens
@@ -85,6 +90,7 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     if need_grad:
         out["dh"] = [np.zeros((Tn, w.shape[1])) for w in Ws]
         out["dW"] = [np.zeros_like(w) for w in Ws]
+    lam = np.ones(M) if exit_weights is None else np.asarray(exit_weights, dtype=np.float64)
     g = grad_scale / T
     for b0 in range(0, Tn, token_block):
         sel = idx[b0:b0 + token_block]
@@ -109,15 +115,15 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             for m in range(M):
                 q = np.exp(logq[m])
                 if m < M - 1:
-                    G = g * (q - (1.0 - alpha_d) * onehot - alpha_d * pM)
+                    G = lam[m] * g * (q - (1.0 - alpha_d) * onehot - alpha_d * pM)
                 else:
-                    G = g * (q - onehot)
+                    G = lam[m] * g * (q - onehot)
                 out["dh"][m][b0:b0 + n] = G @ Ws[m]
                 out["dW"][m] += G.T @ hb[m]
     out["ce_lm"] = out["ce_lm_sum"] / T
     out["ce_kd"] = out["ce_kd_sum"] / T
-    out["loss"] = float(np.sum((1.0 - alpha_d) * out["ce_lm"][:M - 1])
-                        + np.sum(alpha_d * out["ce_kd"]) + out["ce_lm"][M - 1])
+    out["loss"] = float(np.sum(lam[:M - 1] * ((1.0 - alpha_d) * out["ce_lm"][:M - 1] + alpha_d * out["ce_kd"]))
+                        + lam[M - 1] * out["ce_lm"][M - 1])
     return out
 
 

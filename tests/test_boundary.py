@@ -88,6 +88,15 @@ def test_junction_argument_errors():
              None) == 3
 
 
+def test_loss_options_reject_nonfinite_weights():
+    lib = _lib.lib()
+    opts = _lib.loss_options([1.0, float("nan")])
+    code = lib.mls_multiexit_loss_fwd_opts(2, 256, 1024, _lib.i64_array([512, 1024]), FAKE,
+                                           _lib.ptr_array([FAKE, FAKE]), _lib.ptr_array([FAKE, FAKE]), 0.3,
+                                           _lib.MLS_BF16, FAKE, FAKE, FAKE, 1 << 40, ctypes.byref(opts), None, None)
+    assert code == 1
+
+
 def test_agreement_argument_errors():
     lib = _lib.lib()
     one = lib.mls_exit_agreement(1, 16, 256, _lib.i64_array([64]), _lib.ptr_array([FAKE]), _lib.ptr_array([FAKE]),

@@ -242,3 +242,38 @@ def test_vocab_row_restriction_matches_full_gradient():
     np.testing.assert_allclose(r["ce_kd"], full["ce_kd"], rtol=1e-13)
     for m in range(3):
         np.testing.assert_allclose(r["dW_rows"][m], full["dW"][m][rows], rtol=1e-12, atol=1e-15)
+
+
+def test_exit_weights_are_linear_in_each_exit():
+    # L(lambda) = sum_m lambda_m L_m and each gradient scales with its own lambda
+    y, h, W = _rand_suite(M=3, T=6, D=(3, 5, 8), V=11, seed=21)
+    lam = np.array([0.5, 2.0, 1.25])
+    base = multiexit_loss(y, h, W, alpha_d=0.3)
+    r = multiexit_loss(y, h, W, alpha_d=0.3, exit_weights=lam)
+    Lm = [0.7 * base["ce_lm"][0] + 0.3 * base["ce_kd"][0], 0.7 * base["ce_lm"][1] + 0.3 * base["ce_kd"][1],
+          base["ce_lm"][2]]
+    np.testing.assert_allclose(r["loss"], float(np.dot(lam, Lm)), rtol=1e-14)
+    for m in range(3):
+        np.testing.assert_allclose(r["dh"][m], lam[m] * base["dh"][m], rtol=1e-13, atol=1e-16)
+        np.testing.assert_allclose(r["dW"][m], lam[m] * base["dW"][m], rtol=1e-13, atol=1e-16)
+    ones = multiexit_loss(y, h, W, alpha_d=0.3, exit_weights=[1.0, 1.0, 1.0])
+    np.testing.assert_allclose(ones["loss"], base["loss"], rtol=1e-15)
+
+
+def test_exit_weights_finite_differences():
+    M, T, D, V, alpha = 2, 3, (2, 4), 5, 0.3
+    y, h, W = _rand_suite(M=M, T=T, D=D, V=V, seed=22)
+    lam = [1.7, 0.4]
+    r = multiexit_loss(y, h, W, alpha_d=alpha, exit_weights=lam)
+    eps = 1e-6
+    # student: its whole loss term moves; teacher held fixed inside CE_KD (stop-gradient)
+    num = np.zeros_like(h[0])
+    for idx in np.ndindex(h[0].shape):
+        b = h[0][idx]
+        h[0][idx] = b + eps
+        lp = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False, exit_weights=lam)["loss"]
+        h[0][idx] = b - eps
+        lm = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False, exit_weights=lam)["loss"]
+        h[0][idx] = b
+        num[idx] = (lp - lm) / (2 * eps)
+    np.testing.assert_allclose(r["dh"][0], num, rtol=1e-6, atol=1e-9)

@@ -22,24 +22,24 @@ def _gpu_inputs(d):
     return y, h, W
 
 
-def _oracle(d, alpha, grad_scale=1.0, rows=None, need_grad=True):
+def _oracle(d, alpha, grad_scale=1.0, rows=None, need_grad=True, exit_weights=None):
     return oracle.multiexit_loss(d.y, d.o, d.W, alpha_d=alpha, grad_scale=grad_scale, rows=rows,
-                                 need_grad=need_grad)
+                                 need_grad=need_grad, exit_weights=exit_weights)
 
 
 def _losses_expected(r, M):
     return np.concatenate([r["ce_lm"], r["ce_kd"], [r["loss"]]])
 
 
-def _check_all(d, alpha, grad_scale=1.0):
+def _check_all(d, alpha, grad_scale=1.0, exit_weights=None):
     cfg = d.cfg
     M = cfg.M
     y, h, W = _gpu_inputs(d)
     st = new_status()
-    losses, stats = multiexit_loss_fwd(y, h, W, alpha, status=st)
-    dh, dW = multiexit_loss_bwd(y, h, W, stats, alpha, grad_scale, status=st)
+    losses, stats = multiexit_loss_fwd(y, h, W, alpha, status=st, exit_weights=exit_weights)
+    dh, dW = multiexit_loss_bwd(y, h, W, stats, alpha, grad_scale, status=st, exit_weights=exit_weights)
     assert status_read(st) == (0, 0)
-    r = _oracle(d, alpha, grad_scale)
+    r = _oracle(d, alpha, grad_scale, exit_weights=exit_weights)
     assert_loss_close(losses, _losses_expected(r, M), "losses")
     s = f64(stats)
     assert_stats_close(s[:M], r["lse"], "lse")
@@ -76,6 +76,13 @@ def test_alpha_and_grad_scale_are_runtime_arguments():
     d = wl.make_inputs(cfg, with_tables=False)
     for alpha, gs in ((0.0, 1.0), (0.7, 3.5)):
         _check_all(d, alpha, gs)
+
+
+@pytest.mark.parametrize("name,small", [("tiny3", None), ("main3", dict(batch=1, seq=200, V=512))])
+def test_exit_weights(name, small):
+    cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
+    d = wl.make_inputs(cfg, with_tables=False)
+    _check_all(d, 0.3, 1.0, exit_weights=[0.5, 2.0, 1.25])
 
 
 def test_single_exit_and_accumulate():
