@@ -426,6 +426,38 @@ def main():
         e2e = {"value": tokens_all * K / (ms_e2e / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 
+    # ---------------- inter-exit agreement pass (a measurement, outside the step)
+    extras = {}
+    if c.M > 1:
+        def agree_run(s):
+            return step.api.exit_agreement(step.o, step.W, step.stats, workspace=step.ws_loss, stream=s)[0]
+        am = agree_run(stream)
+        if args.eager:
+            arun = lambda: agree_run(stream)  # noqa: E731
+        else:
+            ga = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga, capture_error_mode="relaxed"):
+                am = agree_run(None)
+            arun = ga.replay
+        for _ in range(2):
+            arun()
+        barrier()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        ka = max(3, K // 5)
+        a0.record(stream)
+        for _ in range(ka):
+            arun()
+        a1.record(stream)
+        barrier()
+        ms_a = a0.elapsed_time(a1) / ka
+        vals = am.float().cpu().tolist()
+        S = c.M - 1
+        extras["exit_agreement"] = {
+            "ms": ms_a, "tflops": 2.0 * c.T * c.V * sum(c.D) / (ms_a / 1000.0) / 1e12,
+            "beta_mean": vals[:S], "kl_mean": vals[S:2 * S], "top1_agree_mean": vals[2 * S:],
+            "what": "each smaller exit vs the largest: acceptance sum_v min(q,p), KL(p||q), top-1 agreement"}
+
     # ---------------- roofline of the dominant kernel and phase rates
     ms_fwd, ms_bwd = phase_ms[1], phase_ms[2]
     flops_fwd = 2.0 * c.T * c.V * sum(c.D)
@@ -468,7 +500,7 @@ def main():
                        "l2": f"no flush; per-step working set {step.working_set_gb():.2f} GB > 126 MB L2"},
             "e2e": e2e, "gpu_launches": int(launches), "launch_mode": "eager" if args.eager else "cuda_graph",
             "roofline": roofline, "cpu_baseline": cpu,
-            "phases": phases, "clocks": clocks.summary(),
+            "phases": phases, "extras": extras, "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
     if ws > 1:
