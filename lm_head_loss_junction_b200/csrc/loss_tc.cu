@@ -793,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           __syncwarp();
           if (lane == 0) mbar_arrive(&s.tempty[buf]);
         }
-        if (!valid) continue;
+        if (!valid || col0 + c * 32 >= Ndim) continue;   // rows past M, columns past a ragged N
         const int64_t off = row * Ndim + col0 + c * 32;
         if (OUT_BF16) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out[p]) + off);
@@ -938,7 +938,7 @@ cudaError_t run_gemm(const GemmMaps& maps, GemmArgs g, cudaStream_t st) {
   g.group_m = 16;
   g.tile_start[0] = 0;
   for (int p = 0; p < g.nprob; ++p) {
-    g.n_nt[p] = g.Ndim[p] / BN;
+    g.n_nt[p] = (g.Ndim[p] + BN - 1) / BN;     // the last N tile may be ragged (zero-filled by TMA)
     g.tile_start[p + 1] = g.tile_start[p] + g.n_mt * g.n_nt[p];
   }
   const size_t smem = sizeof(GemmSmem<BN>) + 1024;
@@ -952,14 +952,12 @@ cudaError_t run_gemm(const GemmMaps& maps, GemmArgs g, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// Largest N tile that divides every exit's width.
+// N tile of the grouped GEMMs: 256 unless every exit is narrower (widths are
+// multiples of 64; a ragged last tile is zero-filled and not stored).
 int pick_bn(const LossProblem& p) {
-  bool d256 = true, d128 = true;
-  for (int m = 0; m < p.M; ++m) {
-    d256 = d256 && (p.D[m] % 256 == 0);
-    d128 = d128 && (p.D[m] % 128 == 0);
-  }
-  return d256 ? 256 : d128 ? 128 : 64;
+  int64_t dmax = 0;
+  for (int m = 0; m < p.M; ++m) dmax = p.D[m] > dmax ? p.D[m] : dmax;
+  return dmax >= 256 ? 256 : dmax >= 128 ? 128 : 64;
 }
 
 // dh_m[T x D_m] = a (G'_m[T x V] W^m[V x D_m] - c_m W^m[y_t]) for every exit in one launch:
