@@ -72,9 +72,14 @@ struct LossArgs {
   int32_t* status;
 };
 
+// Per-warp staging of one 32-row x 32-column bf16 chunk of G' (rows padded
+// to 80 bytes so the 16-byte writes of a warp hit every bank once per pass).
+constexpr int kStageRowBytes = 80;
+
 struct __align__(1024) LossSmem {
   uint8_t a[kLossStages][kBM * kBK * 2];
   uint8_t b[kLossStages][kLossBN * kBK * 2];
+  uint8_t gstage[kLossEpiWarps][32 * kStageRowBytes];
   uint64_t full[kLossStages];
   uint64_t empty[kLossStages];
   uint64_t tfull[2];
@@ -404,7 +409,6 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           if (live) {
             const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
             const float ls = lse * kLog2e;
-            __nv_bfloat16* grow = a.G + (static_cast<int64_t>(m) * a.T + t) * a.V + c0;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               float r[32];
@@ -426,12 +430,25 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 }
                 packed[k / 2] = bad ? 0u : pack_bf16x2(g0, g1);
               }
-              if (valid) {
-                uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+              // transpose through shared memory so that each store instruction
+              // writes 8 rows x 64 contiguous bytes (full sectors)
+              uint8_t* stage = s.gstage[warp - 2];
+              uint4* mine = reinterpret_cast<uint4*>(stage + lane * kStageRowBytes);
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+              for (int u = 0; u < 4; ++u)
+                mine[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+              __syncwarp();
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int piece = i * 32 + lane;
+                const int r = piece >> 2, ch = piece & 3;
+                const int tr = tt * kBM + q * 32 + r;
+                const uint4 v = *reinterpret_cast<const uint4*>(stage + r * kStageRowBytes + ch * 16);
+                if (tr < a.T)
+                  *reinterpret_cast<uint4*>(a.G + (static_cast<int64_t>(m) * a.T + tr) * a.V + c0 + c * 32 +
+                                            ch * 8) = v;
               }
+              __syncwarp();
             }
           }
           tc_fence_before();
