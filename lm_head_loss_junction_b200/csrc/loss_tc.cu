@@ -855,6 +855,229 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   }
 }
 
+// ------------------------------------------------------------------ grouped GEMM on CTA pairs
+// Same problem as gemm_kernel with 256 x 256 output tiles computed by a pair
+// of CTAs (a 2-CTA cluster) with tcgen05.mma.cta_group::2: each CTA loads its
+// 128 rows of A and 128 of the 256 rows of B, so every CTA reads half of B per
+// MMA and the B traffic through shared memory and L2 halves.  CTA rank 0 (the
+// leader) issues the MMAs; each CTA's TMEM holds its 128 rows of the two
+// accumulator buffers and its own epilogue drains them.
+constexpr int kPairStages = 6;
+
+struct __align__(1024) PairSmem {
+  uint8_t a[kPairStages][kBM * kBK * 2];
+  uint8_t b[kPairStages][128 * kBK * 2];
+  uint64_t full[kPairStages];      // leader: counts both CTAs' TMA bytes
+  uint64_t empty[kPairStages];     // each CTA: its stage may be refilled
+  uint64_t tfull[2];               // each CTA: accumulator buffer ready
+  uint64_t tempty[2];              // leader: both CTAs drained the buffer (8 warps)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void pair_tile(const GemmArgs& g, int i, int& p, int& mt, int& nt) {
+  gemm_tile(g, i, p, mt, nt);        // mt indexes 256-row blocks (g.n_mt counts them)
+}
+
+template <bool A_MN, bool B_MN, bool OUT_BF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs g) {
+  constexpr int BN = 256;
+  extern __shared__ uint8_t smem_raw[];
+  PairSmem& s = *reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile int* abort = &s.abort;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const int num_tiles = g.tile_start[g.nprob];
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPairStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 8);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int p = 0; p < g.nprob; ++p) {
+      tma_prefetch_desc(&maps.a[p]);
+      tma_prefetch_desc(&maps.b[p]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&s.tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();        // every barrier of both CTAs exists before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < num_tiles && ok; tile += nclusters) {
+        int p, mt, nt;
+        pair_tile(g, tile, p, mt, nt);
+        const CUtensorMap* ma = &maps.a[p];
+        const CUtensorMap* mb = &maps.b[p];
+        const int row0 = mt * 2 * kBM + static_cast<int>(rank) * kBM;   // this CTA's 128 rows of A
+        const int n0 = nt * BN + static_cast<int>(rank) * 128;           // this CTA's 128 rows of B
+        for (int kb = 0; kb < g.kblocks; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, g.status)) { ok = false; break; }
+          const uint32_t lfull = mapa_shared(smem_u32(&s.full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * (kBM + 128) * kBK * 2);
+          if (A_MN) {
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              tma_load_2d_pair(ma, lfull, s.a[stage] + j * (64 * kBK * 2), row0 + j * 64, kb * kBK);
+          } else {
+            tma_load_2d_pair(ma, lfull, s.a[stage], kb * kBK, row0);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_2d_pair(mb, lfull, s.b[stage] + j * (64 * kBK * 2), n0 + j * 64, kb * kBK);
+          } else {
+            tma_load_2d_pair(mb, lfull, s.b[stage], kb * kBK, n0);
+          }
+          ++issued;
+          if (++stage == kPairStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        // The loads of this CTA complete on the leader's barrier; give them time to land.
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16(2 * kBM, BN, A_MN, B_MN);
+      constexpr uint32_t a_step = A_MN ? (kUK * 128) >> 4 : (kUK * 2) >> 4;
+      constexpr uint32_t b_step = B_MN ? (kUK * 128) >> 4 : (kUK * 2) >> 4;
+      constexpr uint32_t a_lbo = A_MN ? 64 * kBK * 2 : 16;
+      constexpr uint32_t b_lbo = B_MN ? 64 * kBK * 2 : 16;
+      uint32_t stage = 0, phase = 0, iter = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < num_tiles && ok; tile += nclusters, ++iter) {
+        const uint32_t buf = iter & 1;
+        if (!mbar_wait(&s.tempty[buf], ((iter >> 1) & 1) ^ 1, abort, g.status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * BN;
+        for (int kb = 0; kb < g.kblocks; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort, g.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(smem_u32(s.a[stage]), a_lbo, 1024);
+          const uint64_t db = smem_desc_sw128(smem_u32(s.b[stage]), b_lbo, 1024);
+#pragma unroll
+          for (int k = 0; k < kBK / kUK; ++k)
+            umma_bf16_pair(d, da + static_cast<uint64_t>(k * a_step), db + static_cast<uint64_t>(k * b_step), idesc,
+                           (kb | k) != 0);
+          const uint32_t e = smem_u32(&s.empty[stage]);
+          umma_commit_pair(mapa_shared(e, 0));
+          umma_commit_pair(mapa_shared(e, 1));
+          if (++stage == kPairStages) { stage = 0; phase ^= 1; }
+        }
+        if (ok) {
+          const uint32_t f = smem_u32(&s.tfull[buf]);
+          umma_commit_pair(mapa_shared(f, 0));
+          umma_commit_pair(mapa_shared(f, 1));
+        }
+      }
+      umma_commit_pair(mapa_shared(smem_u32(&s.drain), 0));
+      drain_wait(&s.drain, 0, g.status);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t iter = 0;
+    for (int tile = cluster; tile < num_tiles; tile += nclusters, ++iter) {
+      int p, mt, nt;
+      pair_tile(g, tile, p, mt, nt);
+      const uint32_t buf = iter & 1;
+      if (!warp_wait(&s.tfull[buf], (iter >> 1) & 1, abort, g.status)) break;
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(mt) * 2 * kBM + rank * kBM + row_in_tile;
+      const bool valid = row < g.Mdim;
+      const int Ndim = g.Ndim[p];
+      const int64_t col0 = static_cast<int64_t>(nt) * BN;
+      int64_t onehot_row = -1;
+      if (OUT_BF16 && valid && g.onehot_idx != nullptr) {
+        const int32_t k = __ldg(g.onehot_idx + row);
+        if (k >= 0 && k < g.onehot_limit) onehot_row = k;
+      }
+      const float alpha = g.alpha[p];
+      const float oh_scale = alpha * g.onehot_coef[p];
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float r[32];
+        tmem_ld32(lane_base + buf * BN + c * 32, r);
+        if (c == BN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[buf]), 0));
+        }
+        if (!valid || col0 + c * 32 >= Ndim) continue;
+        const int64_t off = row * Ndim + col0 + c * 32;
+        if (OUT_BF16) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out[p]) + off);
+          const uint4* oh = (onehot_row >= 0)
+                                ? reinterpret_cast<const uint4*>(g.onehot_rows[p] + onehot_row * Ndim + col0 + c * 32)
+                                : nullptr;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = r[8 * u + e] * alpha;
+            if (oh != nullptr) {
+              float w[8];
+              bf16x8_to_f32(__ldg(oh + u), w);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = fmaf(-oh_scale, w[e], f[e]);
+            }
+            dst[u] = f32_to_bf16x8(f);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out[p]) + off);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float4 v = make_float4(r[4 * u] * alpha, r[4 * u + 1] * alpha, r[4 * u + 2] * alpha,
+                                   r[4 * u + 3] * alpha);
+            if (g.accumulate) {
+              const float4 o = dst[u];
+              v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+            }
+            dst[u] = v;
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync_all();        // no CTA leaves while its pair may still touch its memory
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -950,21 +1173,34 @@ LossArgs base_args(const LossProblem& p) {
 
 template <bool A_MN, bool B_MN, int BN, bool OUT_BF16>
 cudaError_t run_gemm(const GemmMaps& maps, GemmArgs g, cudaStream_t st) {
-  g.n_mt = (g.Mdim + kBM - 1) / kBM;
+  // 256-wide N tiles run on CTA pairs (256 x 256 output tiles), narrower ones on single CTAs.
+  constexpr bool kPair = (BN == 256);
+  const int rows_per_tile = kPair ? 2 * kBM : kBM;
+  g.n_mt = (g.Mdim + rows_per_tile - 1) / rows_per_tile;
   g.kblocks = (g.Kdim + kBK - 1) / kBK;
-  g.group_m = 16;
+  g.group_m = kPair ? 8 : 16;
   g.tile_start[0] = 0;
   for (int p = 0; p < g.nprob; ++p) {
     g.n_nt[p] = (g.Ndim[p] + BN - 1) / BN;     // the last N tile may be ragged (zero-filled by TMA)
     g.tile_start[p + 1] = g.tile_start[p] + g.n_mt * g.n_nt[p];
   }
-  const size_t smem = sizeof(GemmSmem<BN>) + 1024;
-  auto fn = gemm_kernel<A_MN, B_MN, BN, OUT_BF16>;
-  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
   const int tiles = g.tile_start[g.nprob];
-  const int grid = tiles < num_sms() ? tiles : num_sms();
-  fn<<<grid, kThreads, smem, st>>>(maps, g);
+  cudaError_t err;
+  if (kPair) {
+    const size_t smem = sizeof(PairSmem) + 1024;
+    auto fn = gemm_pair_kernel<A_MN, B_MN, OUT_BF16>;
+    err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+    fn<<<2 * pairs, kThreads, smem, st>>>(maps, g);
+  } else {
+    const size_t smem = sizeof(GemmSmem<BN>) + 1024;
+    auto fn = gemm_kernel<A_MN, B_MN, BN, OUT_BF16>;
+    err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    fn<<<grid, kThreads, smem, st>>>(maps, g);
+  }
   note_launches(1);
   return cudaGetLastError();
 }
