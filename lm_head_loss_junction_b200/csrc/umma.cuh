@@ -1,7 +1,7 @@
 // Thin inline-PTX wrappers for the sm_100a pieces the tensor-core kernels use:
 // mbarriers (with bounded waits), TMA tiled loads, tcgen05 TMEM allocation,
 // tcgen05.mma (kind::f16, bf16 in, fp32 accumulate), tcgen05.commit and
-// tcgen05.ld.  No multicast form of any load is used anywhere.
+// tcgen05.ld.  Every load writes only the issuing CTA's own shared memory.
 #pragma once
 #include <cstdint>
 #include <cuda.h>   // CUtensorMap (type only; the driver is reached at run time)
@@ -172,7 +172,7 @@ namespace mls {
 // ---------------------------------------------------------------- CTA pairs (cta_group::2)
 // A cluster of two CTAs shares one 256-row MMA: CTA rank 0 ("leader") issues
 // it, each CTA holds its 128 rows of A, half of B and its half of the
-// accumulator in its own TMEM.  No load here uses cluster multicast.
+// accumulator in its own TMEM.  Each CTA loads only into its own shared memory.
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
