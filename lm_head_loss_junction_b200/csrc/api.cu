@@ -58,18 +58,15 @@ mls_status check_junction_shape(const int32_t* x, int64_t T, const void* o_m, in
   return MLS_OK;
 }
 
-mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y, const void* const* h,
-                         const void* const* W, float alpha_d, mls_dtype dt, int32_t* status, LossProblem* p) {
+// Shape checks shared by every loss entry point (no pointers involved).
+mls_status check_loss_shape(int M, int64_t T, int64_t V, const int64_t* D, mls_dtype dt) {
   if (M < 1 || M > mls::kMaxExits) return M < 1 ? MLS_ERR_INVALID_ARG : MLS_ERR_UNSUPPORTED;
-  if (D == nullptr || h == nullptr || W == nullptr || y == nullptr) return MLS_ERR_INVALID_ARG;
+  if (D == nullptr) return MLS_ERR_INVALID_ARG;
   if (T <= 0 || V <= 0) return MLS_ERR_INVALID_ARG;
   if (dt != MLS_F32 && dt != MLS_BF16) return MLS_ERR_INVALID_ARG;
-  if (!(alpha_d == alpha_d)) return MLS_ERR_INVALID_ARG;   // NaN
   for (int m = 0; m < M; ++m) {
     if (D[m] <= 0) return MLS_ERR_INVALID_ARG;
     if (m > 0 && D[m] <= D[m - 1]) return MLS_ERR_INVALID_ARG;   // widths strictly increase
-    if (h[m] == nullptr || W[m] == nullptr) return MLS_ERR_INVALID_ARG;
-    if (!aligned16(h[m]) || !aligned16(W[m])) return MLS_ERR_UNSUPPORTED;
   }
   if (T > INT_MAX || V > INT_MAX) return MLS_ERR_UNSUPPORTED;
   if (dt == MLS_BF16) {
@@ -78,17 +75,37 @@ mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const in
       if (D[m] % 64 != 0 || D[m] > 65536) return MLS_ERR_UNSUPPORTED;
     if (static_cast<double>(V) * static_cast<double>(T) >= 9.0e15) return MLS_ERR_UNSUPPORTED;
   }
-  p->M = M;
-  p->T = T;
-  p->V = V;
+  return MLS_OK;
+}
+
+// Shape-only problem description, for the workspace queries.
+LossProblem shape_problem(int M, int64_t T, int64_t V, const int64_t* D) {
+  LossProblem p{};
+  p.M = M;
+  p.T = T;
+  p.V = V;
+  for (int m = 0; m < M; ++m) p.D[m] = D[m];
+  for (int m = 0; m < mls::kMaxExits; ++m) p.exit_w[m] = 1.f;
+  return p;
+}
+
+mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y, const void* const* h,
+                         const void* const* W, float alpha_d, mls_dtype dt, int32_t* status, LossProblem* p) {
+  mls_status st = check_loss_shape(M, T, V, D, dt);
+  if (st != MLS_OK) return st;
+  if (h == nullptr || W == nullptr || y == nullptr) return MLS_ERR_INVALID_ARG;
+  if (!(alpha_d == alpha_d)) return MLS_ERR_INVALID_ARG;   // NaN
   for (int m = 0; m < M; ++m) {
-    p->D[m] = D[m];
+    if (h[m] == nullptr || W[m] == nullptr) return MLS_ERR_INVALID_ARG;
+    if (!aligned16(h[m]) || !aligned16(W[m])) return MLS_ERR_UNSUPPORTED;
+  }
+  *p = shape_problem(M, T, V, D);
+  for (int m = 0; m < M; ++m) {
     p->h[m] = h[m];
     p->W[m] = W[m];
   }
   p->y = y;
   p->alpha_d = alpha_d;
-  for (int m = 0; m < mls::kMaxExits; ++m) p->exit_w[m] = 1.f;
   p->status = status;
   return MLS_OK;
 }
@@ -213,14 +230,9 @@ mls_status mls_junction_bwd_variant(const int32_t* x, int64_t T, const void* o_m
 mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int64_t V, mls_dtype dt,
                                         size_t* fwd_bytes, size_t* bwd_bytes) {
   if (fwd_bytes == nullptr || bwd_bytes == nullptr) return MLS_ERR_INVALID_ARG;
-  const void* dummy[mls::kMaxExits] = {&fwd_bytes, &fwd_bytes, &fwd_bytes, &fwd_bytes};
-  // The pointer arrays only need to be non-null and aligned for the shape check.
-  alignas(16) static const char probe[16] = {0};
-  for (auto& d : dummy) d = probe;
-  LossProblem p{};
-  mls_status st = build_problem(M, T, V, D, reinterpret_cast<const int32_t*>(probe), dummy, dummy, 0.f, dt,
-                                nullptr, &p);
+  const mls_status st = check_loss_shape(M, T, V, D, dt);
   if (st != MLS_OK) return st;
+  const LossProblem p = shape_problem(M, T, V, D);
   if (dt == MLS_BF16) {
     *fwd_bytes = mls::loss_tc_fwd_bytes(p);
     *bwd_bytes = mls::loss_tc_bwd_bytes(p);
@@ -299,17 +311,10 @@ mls_status mls_multiexit_loss_bwd_opts(int M, int64_t T, int64_t V, const int64_
 
 mls_status mls_exit_agreement_workspace(int M, int64_t T, const int64_t* D, int64_t V, mls_dtype dt,
                                         size_t* bytes) {
-  if (bytes == nullptr) return MLS_ERR_INVALID_ARG;
-  size_t f = 0, b = 0;
-  mls_status st = mls_multiexit_loss_workspace(M, T, D, V, dt, &f, &b);
+  if (bytes == nullptr || M < 2) return MLS_ERR_INVALID_ARG;
+  const mls_status st = check_loss_shape(M, T, V, D, dt);
   if (st != MLS_OK) return st;
-  if (M < 2) return MLS_ERR_INVALID_ARG;
-  const void* dummy[mls::kMaxExits];
-  alignas(16) static const char probe[16] = {0};
-  for (auto& d : dummy) d = probe;
-  LossProblem p{};
-  st = build_problem(M, T, V, D, reinterpret_cast<const int32_t*>(probe), dummy, dummy, 0.f, dt, nullptr, &p);
-  if (st != MLS_OK) return st;
+  const LossProblem p = shape_problem(M, T, V, D);
   *bytes = dt == MLS_BF16 ? mls::agree_tc_bytes(p) : mls::agree_simt_bytes(p);
   return MLS_OK;
 }
