@@ -57,7 +57,7 @@ def softmax_rows(l: np.ndarray) -> np.ndarray:
 
 
 def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
-                   rows=None, token_block=256, exit_weights=None):
+                   rows=None, token_block=256, exit_weights=None, distill="ce"):
     """Multi-exit loss, per-token statistics and (optionally) gradients, fp64.
 
     y: int [T] targets; h: list of M arrays [T, D_m]; W: list of M arrays [V, D_m].
@@ -69,6 +69,13 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     paragraph, notes that reweighting the exits closes much of the gap):
     L = sum_{m<M} lambda_m [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m] + lambda_M CE_LM,M,
     and each exit's gradient is scaled by its lambda_m.
+    distill: "ce" (the pages' token-level cross-entropy to the largest exit) or
+    "reverse_kl", the alternative distillation term the follow-ups propose to
+    swap in ("Is nesting the cheapest way to build a model suite?", section 4):
+    KD_m = mean_t KL(q_m || p_M) = mean_t sum_v q_m,v (log q_m,v - log p_M,v).
+    Its student gradient (teacher still stop-gradient) is
+    G_m = lambda_m grad_scale/T ((1 - alpha_d)(q_m - onehot) + alpha_d q_m (log q_m - log p_M - KL_t)),
+    and the per-token statistic returned in "R" is sum_v q_m,v (l_m,v - l_M,v).
 
     Returns a dict with
       ce_lm [M], ce_kd [M-1], loss (scalar)         -- means over the tokens
@@ -83,8 +90,11 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     Tn = idx.shape[0]
     Ws = [_f64(w) for w in W]
     V = Ws[0].shape[0]
+    if distill not in ("ce", "reverse_kl"):
+        raise ValueError(distill)
     out = {
         "lse": np.zeros((M, Tn)), "tgt": np.zeros((M, Tn)), "S": np.zeros((max(M - 1, 0), Tn)),
+        "R": np.zeros((max(M - 1, 0), Tn)),
         "ce_lm_sum": np.zeros(M), "ce_kd_sum": np.zeros(max(M - 1, 0)),
     }
     if need_grad:
@@ -106,16 +116,26 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             out["lse"][m, b0:b0 + n] = lse[m]
             out["tgt"][m, b0:b0 + n] = logits[m][ar, yb]
             out["ce_lm_sum"][m] += np.sum(lse[m] - logits[m][ar, yb])
+        rkl = []
         for m in range(M - 1):
             out["S"][m, b0:b0 + n] = np.sum(pM * logits[m], axis=1)
-            out["ce_kd_sum"][m] += np.sum(-np.sum(pM * logq[m], axis=1))
+            q = np.exp(logq[m])
+            out["R"][m, b0:b0 + n] = np.sum(q * (logits[m] - logits[M - 1]), axis=1)
+            rkl.append(np.sum(q * (logq[m] - logq[M - 1]), axis=1))
+            if distill == "ce":
+                out["ce_kd_sum"][m] += np.sum(-np.sum(pM * logq[m], axis=1))
+            else:
+                out["ce_kd_sum"][m] += np.sum(rkl[m])
         if need_grad:
             onehot = np.zeros((n, V))
             onehot[ar, yb] = 1.0
             for m in range(M):
                 q = np.exp(logq[m])
-                if m < M - 1:
+                if m < M - 1 and distill == "ce":
                     G = lam[m] * g * (q - (1.0 - alpha_d) * onehot - alpha_d * pM)
+                elif m < M - 1:
+                    kd = q * (logq[m] - logq[M - 1] - rkl[m][:, None])
+                    G = lam[m] * g * ((1.0 - alpha_d) * (q - onehot) + alpha_d * kd)
                 else:
                     G = lam[m] * g * (q - onehot)
                 out["dh"][m][b0:b0 + n] = G @ Ws[m]

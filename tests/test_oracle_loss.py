@@ -277,3 +277,54 @@ def test_exit_weights_finite_differences():
         h[0][idx] = b
         num[idx] = (lp - lm) / (2 * eps)
     np.testing.assert_allclose(r["dh"][0], num, rtol=1e-6, atol=1e-9)
+
+
+# ------------------------------------------------------------------ reverse KL distillation
+def test_reverse_kl_two_class_closed_form():
+    # student (b, 0), teacher (a, 0): KL(q || p) = s(b) log(s(b)/s(a)) + s(-b) log(s(-b)/s(-a))
+    a, b = 2.0, -1.0
+    y = np.array([0])
+    h = [np.array([[b]]), np.array([[a]])]
+    W = [np.array([[1.0], [0.0]]), np.array([[1.0], [0.0]])]
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="reverse_kl")
+    rkl = _sig(b) * math.log(_sig(b) / _sig(a)) + _sig(-b) * math.log(_sig(-b) / _sig(-a))
+    np.testing.assert_allclose(r["ce_kd"][0], rkl, rtol=1e-13)
+    np.testing.assert_allclose(r["loss"], 0.7 * _softplus(-b) + 0.3 * rkl + _softplus(-a), rtol=1e-13)
+
+
+def test_reverse_kl_vanishes_for_identical_exits_and_is_nonnegative():
+    y, h, W = _rand_suite(M=2, T=6, D=(5, 5), V=12, seed=31)
+    h[0], W[0] = h[1].copy(), W[1].copy()
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="reverse_kl")
+    np.testing.assert_allclose(r["ce_kd"], 0.0, atol=1e-13)
+    y, h, W = _rand_suite(M=3, T=6, seed=32)
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="reverse_kl")
+    assert np.all(r["ce_kd"] >= 0)
+    # per token KL(q||p) = R - lse_m + lse_M
+    base = multiexit_loss(y, h, W, alpha_d=0.3)
+    for m in range(2):
+        kl_t = r["R"][m] - r["lse"][m] + r["lse"][2]
+        np.testing.assert_allclose(kl_t.mean(), r["ce_kd"][m], rtol=1e-12)
+    np.testing.assert_allclose(r["ce_lm"], base["ce_lm"], rtol=1e-15)
+
+
+def test_reverse_kl_gradients_match_finite_differences():
+    M, T, D, V, alpha = 2, 3, (3, 4), 6, 0.4
+    y, h, W = _rand_suite(M=M, T=T, D=D, V=V, seed=33)
+    r = multiexit_loss(y, h, W, alpha_d=alpha, grad_scale=1.3, distill="reverse_kl")
+    eps = 1e-6
+    for arr, grad in ((h, r["dh"][0]), (W, r["dW"][0])):
+        num = np.zeros_like(arr[0])
+        for idx in np.ndindex(arr[0].shape):
+            b = arr[0][idx]
+            arr[0][idx] = b + eps
+            lp = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False, distill="reverse_kl")["loss"]
+            arr[0][idx] = b - eps
+            lm = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False, distill="reverse_kl")["loss"]
+            arr[0][idx] = b
+            num[idx] = 1.3 * (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-9)
+    # alpha_d = 0 gives the same gradients as the cross-entropy form
+    a = multiexit_loss(y, h, W, alpha_d=0.0, distill="reverse_kl")
+    c = multiexit_loss(y, h, W, alpha_d=0.0)
+    np.testing.assert_allclose(a["dh"][0], c["dh"][0], rtol=1e-13, atol=1e-16)
