@@ -257,8 +257,25 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   void* workspace, size_t ws_bytes,
                                   int32_t* dev_status, void* stream);
 
+/* Distillation term of the smaller exits. */
+typedef enum {
+  MLS_DISTILL_CE = 0,          /* token-level cross-entropy to the largest exit's softmax (default) */
+  MLS_DISTILL_REVERSE_KL = 1   /* KL(q_m || p_M), an alternative the pages' follow-ups propose   */
+} mls_distill;
+
 /*
  * Options of the _opts variants of the loss entry points (NULL = defaults).
+ *   distill       MLS_DISTILL_CE (the pages' method) or MLS_DISTILL_REVERSE_KL
+ *                 ("Is nesting the cheapest way to build a model suite?",
+ *                 section 4, proposes swapping in reverse KL):
+ *                   KD_m = mean_t sum_v q_m,v (log q_m,v - log p_M,v),
+ *                   student gradient (teacher still stop-gradient)
+ *                   G_m = grad_scale/T ((1 - alpha_d)(q_m - onehot(y))
+ *                                       + alpha_d q_m (log q_m - log p_M - KL_t)).
+ *                 With it, losses[M..2M-2] hold the mean KL and stats rows
+ *                 2M..3M-2 hold R_m,t = sum_v q_m,t,v (l_m,t,v - l_M,t,v), so
+ *                 KL_t = R_m,t - lse_m,t + lse_M,t; the backward call must get
+ *                 the same option.  Other values return MLS_ERR_INVALID_ARG.
  *   exit_weights  HOST float [M] or NULL: per-exit loss weights lambda_m,
  *                 L = sum_{m<M} lambda_m [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m]
  *                     + lambda_M CE_LM,M,
@@ -271,6 +288,7 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
  */
 typedef struct {
   const float* exit_weights;
+  int distill;                 /* mls_distill */
 } mls_loss_options;
 
 mls_status mls_multiexit_loss_fwd_opts(int M, int64_t T, int64_t V, const int64_t* D,

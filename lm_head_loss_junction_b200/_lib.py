@@ -36,7 +36,7 @@ _u32 = ctypes.c_uint32
 
 class LossOptions(ctypes.Structure):
     """mls_loss_options"""
-    _fields_ = [("exit_weights", ctypes.POINTER(ctypes.c_float))]
+    _fields_ = [("exit_weights", ctypes.POINTER(ctypes.c_float)), ("distill", ctypes.c_int)]
 
 
 # name -> (restype, argtypes), in the order of include/mls.h
@@ -120,11 +120,18 @@ def i64_array(vals):
     return arr
 
 
-def loss_options(exit_weights=None):
+MLS_DISTILL = {"ce": 0, "reverse_kl": 1}
+
+
+def loss_options(exit_weights=None, distill="ce"):
     """ctypes options struct (and the buffer it points to), or None for defaults."""
-    if exit_weights is None:
+    if exit_weights is None and distill == "ce":
         return None
+    if exit_weights is None:
+        opts = LossOptions(None, MLS_DISTILL[distill])
+        opts._buf = None
+        return opts
     buf = (ctypes.c_float * len(exit_weights))(*[float(w) for w in exit_weights])
-    opts = LossOptions(ctypes.cast(buf, ctypes.POINTER(ctypes.c_float)))
+    opts = LossOptions(ctypes.cast(buf, ctypes.POINTER(ctypes.c_float)), MLS_DISTILL[distill])
     opts._buf = buf          # keep the weights alive with the struct
     return opts

@@ -151,7 +151,8 @@ def _workspace(ws, nbytes, device):
 
 
 def multiexit_loss_fwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Tensor], alpha_d: float = 0.3, *,
-                       losses=None, stats=None, workspace=None, exit_weights=None, status=None, stream=None):
+                       losses=None, stats=None, workspace=None, exit_weights=None, distill="ce", status=None,
+                       stream=None):
     """Returns (losses [2M], stats [3M-1, T]) (see mls_multiexit_loss_fwd; `exit_weights`
     uses mls_multiexit_loss_fwd_opts)."""
     M, T, V, D, dt = _loss_common(y, h, W)
@@ -165,10 +166,10 @@ def multiexit_loss_fwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Ten
     args = (M, T, V, i64_array(D), y.data_ptr(), ptr_array([t.data_ptr() for t in h]),
             ptr_array([t.data_ptr() for t in W]), float(alpha_d), _dtype_code(h[0]), losses.data_ptr(),
             stats.data_ptr(), workspace.data_ptr(), ws_bytes)
-    if exit_weights is None:
+    opts = _lib.loss_options(exit_weights, distill)
+    if opts is None:
         code = lib().mls_multiexit_loss_fwd(*args, _ptr(status), _stream_ptr(stream))
     else:
-        opts = _lib.loss_options(exit_weights)
         code = lib().mls_multiexit_loss_fwd_opts(*args, ctypes.byref(opts), _ptr(status), _stream_ptr(stream))
     check("mls_multiexit_loss_fwd", code)
     return losses, stats
@@ -176,7 +177,8 @@ def multiexit_loss_fwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Ten
 
 def multiexit_loss_bwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Tensor], stats: torch.Tensor,
                        alpha_d: float = 0.3, grad_scale: float = 1.0, *, dh=None, dW=None,
-                       accumulate_dW: bool = False, workspace=None, exit_weights=None, status=None, stream=None):
+                       accumulate_dW: bool = False, workspace=None, exit_weights=None, distill="ce", status=None,
+                       stream=None):
     """Returns (dh list, dW list) (see mls_multiexit_loss_bwd)."""
     M, T, V, D, dt = _loss_common(y, h, W)
     dev = y.device
@@ -191,10 +193,10 @@ def multiexit_loss_bwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Ten
             ptr_array([t.data_ptr() for t in W]), float(alpha_d), _dtype_code(h[0]), stats.data_ptr(),
             float(grad_scale), ptr_array([t.data_ptr() for t in dh]), ptr_array([t.data_ptr() for t in dW]),
             int(bool(accumulate_dW)), workspace.data_ptr(), ws_bytes)
-    if exit_weights is None:
+    opts = _lib.loss_options(exit_weights, distill)
+    if opts is None:
         code = lib().mls_multiexit_loss_bwd(*args, _ptr(status), _stream_ptr(stream))
     else:
-        opts = _lib.loss_options(exit_weights)
         code = lib().mls_multiexit_loss_bwd_opts(*args, ctypes.byref(opts), _ptr(status), _stream_ptr(stream))
     check("mls_multiexit_loss_bwd", code)
     return dh, dW

@@ -65,6 +65,7 @@ struct LossProblem {
   const void* W[kMaxExits];
   float alpha_d;
   float exit_w[kMaxExits];   // per-exit loss weights (1 = equal weights)
+  int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M)
   int32_t* status;
 };
 

@@ -27,6 +27,7 @@ struct SimtDev {
   const float* W[kMaxExits];
   float alpha_d;
   float exit_w[kMaxExits];
+  int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M)
   int32_t* status;
   float* dh[kMaxExits];
   float* dW[kMaxExits];
@@ -76,15 +77,23 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
     if (lT > mT) {
       const float r = __expf(mT - lT);
       zT *= r;
-      for (int s = 0; s < S; ++s) A[s] *= r;
+      if (p.distill == 0)
+        for (int s = 0; s < S; ++s) A[s] *= r;
       mT = lT;
     }
     const float pt = __expf(lT - mT);
     zT += pt;
     for (int s = 0; s < S; ++s) {
-      A[s] = fmaf(pt, l[s], A[s]);
-      if (l[s] > ms[s]) { zs[s] = zs[s] * __expf(ms[s] - l[s]); ms[s] = l[s]; }
-      zs[s] += __expf(l[s] - ms[s]);
+      if (p.distill == 0) A[s] = fmaf(pt, l[s], A[s]);
+      if (l[s] > ms[s]) {
+        const float r = __expf(ms[s] - l[s]);
+        zs[s] *= r;
+        if (p.distill == 1) A[s] *= r;   // reverse KL: sum q~ (l_m - l_T) follows the student's max
+        ms[s] = l[s];
+      }
+      const float qs = __expf(l[s] - ms[s]);
+      zs[s] += qs;
+      if (p.distill == 1) A[s] = fmaf(qs, l[s] - lT, A[s]);
     }
     if (v == yt)
       for (int m = 0; m < M; ++m) tgt[m] = l[m];
@@ -112,9 +121,16 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       red[kSimtThreads + tid] = z1 * r1 + z2 * r2;
       for (int s = 0; s < S; ++s) {
         float* a = red + (2 + s) * kSimtThreads;
-        a[tid] = a[tid] * r1 + a[o] * r2;
         float* msp = red + (2 + S + 2 * s) * kSimtThreads;
         float* zsp = msp + kSimtThreads;
+        if (p.distill == 0) {
+          a[tid] = a[tid] * r1 + a[o] * r2;
+        } else {
+          const float sm = fmaxf(msp[tid], msp[o]);
+          const float s1 = (msp[tid] == -INFINITY) ? 0.f : __expf(msp[tid] - sm);
+          const float s2 = (msp[o] == -INFINITY) ? 0.f : __expf(msp[o] - sm);
+          a[tid] = a[tid] * s1 + a[o] * s2;
+        }
         float mA = msp[tid], zA = zsp[tid];
         merge_max_sum(mA, zA, msp[o], zsp[o]);
         msp[tid] = mA;
@@ -139,10 +155,12 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       terms[m * p.T + t] = bad ? 0.f : lse - tg;
     }
     for (int s = 0; s < S; ++s) {
-      const float Sv = red[(2 + s) * kSimtThreads] / red[kSimtThreads];
-      const float lse = red[(2 + S + 2 * s) * kSimtThreads] + logf(red[(2 + S + 2 * s + 1) * kSimtThreads]);
+      const float zsum = red[(2 + S + 2 * s + 1) * kSimtThreads];
+      const float lse = red[(2 + S + 2 * s) * kSimtThreads] + logf(zsum);
+      // cross-entropy: S = sum p_T l_m; reverse KL: R = sum q_m (l_m - l_T)
+      const float Sv = red[(2 + s) * kSimtThreads] / (p.distill == 0 ? red[kSimtThreads] : zsum);
       stats[(2 * M + s) * p.T + t] = Sv;
-      terms[(M + s) * p.T + t] = bad ? 0.f : lse - Sv;
+      terms[(M + s) * p.T + t] = bad ? 0.f : (p.distill == 0 ? lse - Sv : Sv - lse + lseT);
     }
     if (bad) set_flag(p.status, MLS_DEVFLAG_BAD_ID);
   }
@@ -162,8 +180,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
   __syncthreads();
   const int32_t yt = p.y[t];
   const bool bad = yt < 0 || yt >= p.V;
-  float lse[kMaxExits];
+  float lse[kMaxExits], kl[kMaxExits];
   for (int m = 0; m < M; ++m) lse[m] = stats[m * p.T + t];
+  for (int m = 0; m < M - 1; ++m) kl[m] = stats[(2 * M + m) * p.T + t] - lse[m] + lse[M - 1];
   const float a = p.alpha_d;
   for (int64_t v = tid; v < p.V; v += kSimtThreads) {
     float l[kMaxExits];
@@ -178,8 +197,15 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
     const float hot = (v == yt) ? 1.f : 0.f;
     for (int m = 0; m < M; ++m) {
       float g;
-      if (m == M - 1) g = pT - hot;
-      else g = __expf(l[m] - lse[m]) - a * pT - (1.f - a) * hot;
+      if (m == M - 1) {
+        g = pT - hot;
+      } else if (p.distill == 0) {
+        g = __expf(l[m] - lse[m]) - a * pT - (1.f - a) * hot;
+      } else {
+        const float q = __expf(l[m] - lse[m]);
+        const float d = (l[m] - lse[m]) - (l[M - 1] - lse[M - 1]) - kl[m];
+        g = (1.f - a) * (q - hot) + a * q * d;
+      }
       G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : p.exit_w[m] * g;
     }
   }
@@ -353,6 +379,7 @@ SimtDev make_dev(const LossProblem& p) {
   }
   d.y = p.y;
   d.alpha_d = p.alpha_d;
+  d.distill = p.distill;
   for (int m = 0; m < kMaxExits; ++m) d.exit_w[m] = p.exit_w[m];
   d.status = p.status;
   return d;

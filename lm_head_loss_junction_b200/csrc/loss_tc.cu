@@ -66,6 +66,7 @@ struct LossArgs {
   int n_tt, n_vt, num_tiles, group_tt;
   const int32_t* y;
   float alpha;                 // alpha_d
+  int distill;                 // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M)
   float* partial;              // forward: [2 n_vt][2M-1][T]
   float* stats;                // forward: target rows written; backward: lse read
   __nv_bfloat16* G;            // backward: [M][T][V]
@@ -130,13 +131,14 @@ __device__ __forceinline__ uint32_t pack_p2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_p2(uint32_t u) { return __half22float2(*reinterpret_cast<__half2*>(&u)); }
 
 // TMEM region and use count of job j (exit M-1-j) of the tile_iter-th tile of a CTA.
-// Statistics and gradient modes alternate the two regions between consecutive
-// jobs.  The agreement mode keeps the teacher in region 0 for the whole tile
-// and runs the students one after another in region 1, so the epilogue can
-// read both exits' logits of the same element.
-__device__ __forceinline__ void job_slot(int mode, int M, uint32_t tile_iter, int j, uint32_t job,
+// By default consecutive jobs alternate the two regions.  When the epilogue
+// needs the teacher's logits at every element of a student's tile (the
+// agreement mode, and the reverse-KL distillation), the teacher stays in
+// region 0 for the whole tile and the students run one after another in
+// region 1.
+__device__ __forceinline__ void job_slot(bool hold_teacher, int M, uint32_t tile_iter, int j, uint32_t job,
                                          uint32_t& region, uint32_t& use) {
-  if (mode == 2) {
+  if (hold_teacher) {
     region = (j == 0) ? 0u : 1u;
     use = (j == 0) ? tile_iter : tile_iter * static_cast<uint32_t>(M - 1) + static_cast<uint32_t>(j - 1);
   } else {
@@ -155,6 +157,8 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort;
   const int M = a.M;
+  const bool hold = (MODE == kModeAgree) || (a.distill == 1);
+  const bool rkl = (a.distill == 1);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kLossStages; ++i) {
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
         for (int j = 0; j < M && ok; ++j, ++job) {
           const int m = M - 1 - j;
           uint32_t region, use;
-          job_slot(MODE, M, tile_iter, j, job, region, use);
+          job_slot(hold, M, tile_iter, j, job, region, use);
           if (!mbar_wait(&s.tempty[region], (use & 1) ^ 1, abort, a.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + region * kLossBN;
@@ -277,8 +281,9 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
       for (int j = 0; j < M; ++j, ++job) {
         const int m = M - 1 - j;
         uint32_t region, use;
-        job_slot(MODE, M, tile_iter, j, job, region, use);
+        job_slot(hold, M, tile_iter, j, job, region, use);
         const uint32_t base = lane_base + region * kLossBN;
+        const uint32_t tbase = lane_base;                   // region 0: the teacher, when held
         if (!warp_wait(&s.tfull[region], use & 1, abort, a.status)) { stop = true; break; }
         tc_fence_after();
         if (MODE == kModeStats) {
@@ -315,6 +320,39 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
               }
               inv_z = 1.f / z;
               lse_part = mx + logf(z);
+            } else if (rkl) {
+              // student, reverse KL: online max/sum over the split and the
+              // student-weighted sum of (l_m - l_T), the teacher read from region 0
+              float ms = -INFINITY, zs = 0.f, B = 0.f;
+#pragma unroll 1
+              for (int c = 0; c < 4; ++c) {
+                float r[32], lt[32];
+                tmem_ld32(base + c * 32, r);
+                tmem_ld32(tbase + c * 32, lt);
+                float cm = r[0];
+#pragma unroll
+                for (int k = 1; k < 32; ++k) cm = fmaxf(cm, r[k]);
+                const float mn = fmaxf(ms, cm);
+                const float mns = mn * kLog2e;
+                float zc = 0.f, bc = 0.f;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                  const float e = exp2f(fmaf(r[k], kLog2e, -mns));
+                  zc += e;
+                  bc = fmaf(e, r[k] - lt[k], bc);
+                }
+                const float rs = exp2f((ms - mn) * kLog2e);
+                zs = zs * rs + zc;
+                B = B * rs + bc;
+                ms = mn;
+                if (has_tgt && (yl >> 5) == c) {
+#pragma unroll
+                  for (int k = 0; k < 32; ++k)
+                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.T + t] = r[k];
+                }
+              }
+              lse_part = ms + logf(zs);
+              abar = B / zs;
             } else {
               // student: online max/sum over the split and the teacher-weighted sum of its logits
               float ms = -INFINITY, zs = 0.f, A = 0.f;
@@ -349,7 +387,14 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[region]);
+          if (lane == 0) {
+            if (!hold) {
+              mbar_arrive(&s.tempty[region]);
+            } else {
+              if (j > 0) mbar_arrive(&s.tempty[1]);         // this student's region
+              if (j == M - 1) mbar_arrive(&s.tempty[0]);    // the teacher's, after the last student
+            }
+          }
           if (valid) {
             a.partial[(static_cast<int64_t>(split) * Q + m) * a.T + t] = lse_part;
             if (j > 0) a.partial[(static_cast<int64_t>(split) * Q + M + m) * a.T + t] = abar;
@@ -364,7 +409,6 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           if (live) {
             const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
             const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
-            const uint32_t tbase = lane_base;          // region 0: the teacher
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float r[32];
@@ -409,10 +453,23 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           if (live) {
             const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
             const float ls = lse * kLog2e;
-#pragma unroll
+            // reverse KL: per-token KL(q_m || p_T) = R_m - lse_m + lse_T (R from the forward pass)
+            float lseT = 0.f, klt = 0.f;
+            if (rkl && j > 0 && valid) {
+              lseT = a.stats[static_cast<int64_t>(M - 1) * a.T + t];
+              klt = a.stats[static_cast<int64_t>(2 * M + m) * a.T + t] - lse + lseT;
+            }
+#pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float r[32];
               tmem_ld32(base + c * 32, r);
+              float lt[32];
+              if (rkl && j > 0) {
+                tmem_ld32(tbase + c * 32, lt);
+              } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) lt[k] = 0.f;
+              }
               uint32_t packed[16];
 #pragma unroll
               for (int k = 0; k < 32; k += 2) {
@@ -420,9 +477,14 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -ls));
                 float g0, g1;
                 if (j == 0) {                      // teacher: G' = p_T
-                  pt[c][k / 2] = pack_p2(e0, e1);
+                  if (!rkl) pt[c][k / 2] = pack_p2(e0, e1);
                   g0 = e0;
                   g1 = e1;
+                } else if (rkl) {                  // student: G' = q ((1 - a) + a (log q - log p - KL))
+                  const float d0 = (r[k] - lse) - (lt[k] - lseT) - klt;
+                  const float d1 = (r[k + 1] - lse) - (lt[k + 1] - lseT) - klt;
+                  g0 = e0 * fmaf(al, d0, 1.f - al);
+                  g1 = e1 * fmaf(al, d1, 1.f - al);
                 } else {                           // student: G' = q - alpha_d p_T
                   const float2 pp = unpack_p2(pt[c][k / 2]);
                   g0 = fmaf(-al, pp.x, e0);
@@ -453,7 +515,14 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[region]);
+          if (lane == 0) {
+            if (!hold) {
+              mbar_arrive(&s.tempty[region]);
+            } else {
+              if (j > 0) mbar_arrive(&s.tempty[1]);
+              if (j == M - 1) mbar_arrive(&s.tempty[0]);
+            }
+          }
         }
       }
       if (stop || *abort) break;
@@ -476,7 +545,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
 constexpr int kMergeRows = 8;
 
 __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float* __restrict__ partial, int n_splits,
-                                                                     int M, int T, int V,
+                                                                     int M, int T, int V, int distill,
                                                                      const int32_t* __restrict__ y,
                                                                      float* __restrict__ stats,
                                                                      float* __restrict__ terms, int32_t* status) {
@@ -497,16 +566,27 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
       if (l > mT) {
         const float r = __expf(mT - l);
         zT *= r;
-        for (int s = 0; s < M - 1; ++s) A[s] *= r;
+        if (distill == 0)
+          for (int s = 0; s < M - 1; ++s) A[s] *= r;   // teacher-weighted sums follow the teacher's max
         mT = l;
       }
       const float w = (l == -INFINITY) ? 0.f : __expf(l - mT);
       zT += w;
       for (int s = 0; s < M - 1; ++s) {
-        A[s] = fmaf(w, pi[static_cast<int64_t>(M + s) * T], A[s]);
         const float ls = pi[static_cast<int64_t>(s) * T];
-        if (ls > ms[s]) { zs[s] *= __expf(ms[s] - ls); ms[s] = ls; }
-        if (ls != -INFINITY) zs[s] += __expf(ls - ms[s]);
+        const float ab = pi[static_cast<int64_t>(M + s) * T];
+        if (distill == 0) A[s] = fmaf(w, ab, A[s]);
+        if (ls > ms[s]) {
+          const float r = __expf(ms[s] - ls);
+          zs[s] *= r;
+          if (distill == 1) A[s] *= r;          // reverse KL: weights are the student's own
+          ms[s] = ls;
+        }
+        if (ls != -INFINITY) {
+          const float ws = __expf(ls - ms[s]);
+          zs[s] += ws;
+          if (distill == 1) A[s] = fmaf(ws, ab, A[s]);
+        }
       }
     }
   }
@@ -526,11 +606,12 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
     const float r2 = (m2 == -INFINITY) ? 0.f : __expf(m2 - mm);
     zT = zT * r1 + z2 * r2;
     for (int s = 0; s < M - 1; ++s) {
-      A[s] = A[s] * r1 + st_A[r][s][lane] * r2;
       const float n2 = st_ms[r][s][lane], y2 = st_zs[r][s][lane];
       const float mn = fmaxf(ms[s], n2);
       const float q1 = (ms[s] == -INFINITY) ? 0.f : __expf(ms[s] - mn);
       const float q2 = (n2 == -INFINITY) ? 0.f : __expf(n2 - mn);
+      if (distill == 0) A[s] = A[s] * r1 + st_A[r][s][lane] * r2;
+      else A[s] = A[s] * q1 + st_A[r][s][lane] * q2;
       zs[s] = zs[s] * q1 + y2 * q2;
       ms[s] = mn;
     }
@@ -544,12 +625,14 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
   terms[static_cast<int64_t>(M - 1) * T + t] = bad ? 0.f : lseT - stats[static_cast<int64_t>(2 * M - 1) * T + t];
   for (int s = 0; s < M - 1; ++s) {
     const float lse = ms[s] + logf(zs[s]);
-    const float Sv = A[s] / zT;
+    // cross-entropy: S = sum p_T l_m (teacher-weighted); reverse KL: R = sum q_m (l_m - l_T)
+    const float Sv = (distill == 0) ? A[s] / zT : A[s] / zs[s];
+    const float kd = (distill == 0) ? lse - Sv : Sv - lse + lseT;
     stats[static_cast<int64_t>(s) * T + t] = lse;
     stats[static_cast<int64_t>(2 * M + s) * T + t] = Sv;
     if (bad) stats[static_cast<int64_t>(M + s) * T + t] = 0.f;
     terms[static_cast<int64_t>(s) * T + t] = bad ? 0.f : lse - stats[static_cast<int64_t>(M + s) * T + t];
-    terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : lse - Sv;
+    terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : kd;
   }
   if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
 }
@@ -1167,6 +1250,7 @@ LossArgs base_args(const LossProblem& p) {
   a.group_tt = 16;
   a.y = p.y;
   a.alpha = p.alpha_d;
+  a.distill = p.distill;
   a.status = p.status;
   return a;
 }
@@ -1313,8 +1397,8 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   if (err != cudaSuccess) return err;
   const int T = static_cast<int>(p.T);
   loss_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
-                                                                     static_cast<int>(p.V), p.y, stats, w.terms,
-                                                                     p.status);
+                                                                     static_cast<int>(p.V), p.distill, p.y, stats,
+                                                                     w.terms, p.status);
   note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;

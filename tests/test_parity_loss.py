@@ -22,30 +22,31 @@ def _gpu_inputs(d):
     return y, h, W
 
 
-def _oracle(d, alpha, grad_scale=1.0, rows=None, need_grad=True, exit_weights=None):
+def _oracle(d, alpha, grad_scale=1.0, rows=None, need_grad=True, exit_weights=None, distill="ce"):
     return oracle.multiexit_loss(d.y, d.o, d.W, alpha_d=alpha, grad_scale=grad_scale, rows=rows,
-                                 need_grad=need_grad, exit_weights=exit_weights)
+                                 need_grad=need_grad, exit_weights=exit_weights, distill=distill)
 
 
 def _losses_expected(r, M):
     return np.concatenate([r["ce_lm"], r["ce_kd"], [r["loss"]]])
 
 
-def _check_all(d, alpha, grad_scale=1.0, exit_weights=None):
+def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce"):
     cfg = d.cfg
     M = cfg.M
     y, h, W = _gpu_inputs(d)
     st = new_status()
-    losses, stats = multiexit_loss_fwd(y, h, W, alpha, status=st, exit_weights=exit_weights)
-    dh, dW = multiexit_loss_bwd(y, h, W, stats, alpha, grad_scale, status=st, exit_weights=exit_weights)
+    losses, stats = multiexit_loss_fwd(y, h, W, alpha, status=st, exit_weights=exit_weights, distill=distill)
+    dh, dW = multiexit_loss_bwd(y, h, W, stats, alpha, grad_scale, status=st, exit_weights=exit_weights,
+                                distill=distill)
     assert status_read(st) == (0, 0)
-    r = _oracle(d, alpha, grad_scale, exit_weights=exit_weights)
+    r = _oracle(d, alpha, grad_scale, exit_weights=exit_weights, distill=distill)
     assert_loss_close(losses, _losses_expected(r, M), "losses")
     s = f64(stats)
     assert_stats_close(s[:M], r["lse"], "lse")
     assert_stats_close(s[M:2 * M], r["tgt"], "target logits")
     if M > 1:
-        assert_stats_close(s[2 * M:], r["S"], "teacher-weighted logits")
+        assert_stats_close(s[2 * M:], r["S"] if distill == "ce" else r["R"], "distillation statistic")
     for m in range(M):
         assert_grad_close(dh[m], r["dh"][m], f"dh[{m}]")
         assert_grad_close(dW[m], r["dW"][m], f"dW[{m}]")
@@ -83,6 +84,16 @@ def test_exit_weights(name, small):
     cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
     d = wl.make_inputs(cfg, with_tables=False)
     _check_all(d, 0.3, 1.0, exit_weights=[0.5, 2.0, 1.25])
+
+
+@pytest.mark.parametrize("name,small", [("tiny3", None), ("main3", dict(batch=1, seq=200, V=512)),
+                                        ("suite4", dict(batch=1, seq=130, V=384)),
+                                        ("main3_aligned", dict(batch=1, seq=256, V=768))])
+def test_reverse_kl_distillation(name, small):
+    cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
+    d = wl.make_inputs(cfg, with_tables=False)
+    _check_all(d, 0.3, 1.0, distill="reverse_kl")
+    _check_all(d, 0.6, 2.0, exit_weights=[1.5, 0.5] + [1.0] * (cfg.M - 2), distill="reverse_kl")
 
 
 def test_single_exit_and_accumulate():
