@@ -76,11 +76,19 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     Its student gradient (teacher still stop-gradient) is
     G_m = lambda_m grad_scale/T ((1 - alpha_d)(q_m - onehot) + alpha_d q_m (log q_m - log p_M - KL_t)),
     and the per-token statistic returned in "R" is sum_v q_m,v (l_m,v - l_M,v).
+    distill="js" takes the Jensen-Shannon divergence, the other alternative the
+    same section names:  with the mixture mu = (q_m + p_M) / 2,
+    KD_m = mean_t [ KL(q_m || mu) + KL(p_M || mu) ] / 2   (natural log, <= log 2).
+    Since d JS / d q_v = log(q_v / mu_v) / 2 (the other terms cancel), the
+    student gradient through the softmax is
+    G_m = lambda_m grad_scale/T ((1 - alpha_d)(q_m - onehot) + alpha_d q_m (g - K_t)),
+    g_v = log(q_v / mu_v) / 2,  K_t = sum_v q_v g_v = KL(q_m || mu) / 2,
+    and K_t is returned per token in "J".
 
     Returns a dict with
       ce_lm [M], ce_kd [M-1], loss (scalar)         -- means over the tokens
       lse [M, T'], tgt [M, T'], S [M-1, T']          -- per-token statistics,
-          S_m,t = sum_v p_{M,t,v} l_{m,t,v}
+          S_m,t = sum_v p_{M,t,v} l_{m,t,v}  (R and J as above, for every distill)
       dh (list of [T', D_m]) and dW (list of [V, D_m]) when need_grad.
     """
     y = np.asarray(y, dtype=np.int64)
@@ -90,11 +98,11 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     Tn = idx.shape[0]
     Ws = [_f64(w) for w in W]
     V = Ws[0].shape[0]
-    if distill not in ("ce", "reverse_kl"):
+    if distill not in ("ce", "reverse_kl", "js"):
         raise ValueError(distill)
     out = {
         "lse": np.zeros((M, Tn)), "tgt": np.zeros((M, Tn)), "S": np.zeros((max(M - 1, 0), Tn)),
-        "R": np.zeros((max(M - 1, 0), Tn)),
+        "R": np.zeros((max(M - 1, 0), Tn)), "J": np.zeros((max(M - 1, 0), Tn)),
         "ce_lm_sum": np.zeros(M), "ce_kd_sum": np.zeros(max(M - 1, 0)),
     }
     if need_grad:
@@ -116,16 +124,23 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             out["lse"][m, b0:b0 + n] = lse[m]
             out["tgt"][m, b0:b0 + n] = logits[m][ar, yb]
             out["ce_lm_sum"][m] += np.sum(lse[m] - logits[m][ar, yb])
-        rkl = []
+        rkl, logmix, jq = [], [], []
         for m in range(M - 1):
             out["S"][m, b0:b0 + n] = np.sum(pM * logits[m], axis=1)
             q = np.exp(logq[m])
             out["R"][m, b0:b0 + n] = np.sum(q * (logits[m] - logits[M - 1]), axis=1)
             rkl.append(np.sum(q * (logq[m] - logq[M - 1]), axis=1))
+            # Jensen-Shannon: log of the mixture (q + p)/2, and KL of each side against it
+            logmix.append(np.logaddexp(logq[m], logq[M - 1]) - np.log(2.0))
+            jq.append(np.sum(q * (logq[m] - logmix[m]), axis=1))
+            jp = np.sum(pM * (logq[M - 1] - logmix[m]), axis=1)
+            out["J"][m, b0:b0 + n] = 0.5 * jq[m]
             if distill == "ce":
                 out["ce_kd_sum"][m] += np.sum(-np.sum(pM * logq[m], axis=1))
-            else:
+            elif distill == "reverse_kl":
                 out["ce_kd_sum"][m] += np.sum(rkl[m])
+            else:
+                out["ce_kd_sum"][m] += np.sum(0.5 * (jq[m] + jp))
         if need_grad:
             onehot = np.zeros((n, V))
             onehot[ar, yb] = 1.0
@@ -133,8 +148,11 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
                 q = np.exp(logq[m])
                 if m < M - 1 and distill == "ce":
                     G = lam[m] * g * (q - (1.0 - alpha_d) * onehot - alpha_d * pM)
-                elif m < M - 1:
+                elif m < M - 1 and distill == "reverse_kl":
                     kd = q * (logq[m] - logq[M - 1] - rkl[m][:, None])
+                    G = lam[m] * g * ((1.0 - alpha_d) * (q - onehot) + alpha_d * kd)
+                elif m < M - 1:
+                    kd = q * (0.5 * (logq[m] - logmix[m]) - 0.5 * jq[m][:, None])
                     G = lam[m] * g * ((1.0 - alpha_d) * (q - onehot) + alpha_d * kd)
                 else:
                     G = lam[m] * g * (q - onehot)

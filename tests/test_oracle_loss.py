@@ -328,3 +328,83 @@ def test_reverse_kl_gradients_match_finite_differences():
     a = multiexit_loss(y, h, W, alpha_d=0.0, distill="reverse_kl")
     c = multiexit_loss(y, h, W, alpha_d=0.0)
     np.testing.assert_allclose(a["dh"][0], c["dh"][0], rtol=1e-13, atol=1e-16)
+
+
+# ------------------------------------------------------------------ Jensen-Shannon distillation
+def test_js_matches_scipy_distance_by_enumeration():
+    # scipy's jensenshannon returns the square root of the divergence (natural log by default)
+    from scipy.spatial.distance import jensenshannon
+    y, h, W = _rand_suite(M=3, T=5, D=(3, 5, 8), V=9, seed=41, scale=3.0)
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="js")
+    pM = softmax_rows(h[2] @ W[2].T)
+    for m in range(2):
+        q = softmax_rows(h[m] @ W[m].T)
+        js = np.array([jensenshannon(q[t], pM[t]) ** 2 for t in range(5)])
+        np.testing.assert_allclose(r["ce_kd"][m], js.mean(), rtol=1e-10)
+        # J = KL(q || mixture) / 2, written out per token and per vocabulary entry
+        mix = 0.5 * (q + pM)
+        kq = np.array([sum(q[t, v] * math.log(q[t, v] / mix[t, v]) for v in range(9)) for t in range(5)])
+        np.testing.assert_allclose(r["J"][m], 0.5 * kq, rtol=1e-12)
+    assert np.all(r["ce_kd"] >= 0) and np.all(r["ce_kd"] <= math.log(2.0))
+
+
+def test_js_is_symmetric_in_student_and_teacher():
+    y, h, W = _rand_suite(M=2, T=7, D=(6, 6), V=13, seed=42)
+    a = multiexit_loss(y, h, W, alpha_d=0.3, distill="js")
+    b = multiexit_loss(y, h[::-1], W[::-1], alpha_d=0.3, distill="js")
+    np.testing.assert_allclose(a["ce_kd"], b["ce_kd"], rtol=1e-13)
+    assert abs(a["J"][0].mean() - b["J"][0].mean()) > 1e-6    # each half is one-sided
+
+
+def test_js_limits():
+    # identical exits: zero divergence and no distillation gradient
+    y, h, W = _rand_suite(M=2, T=6, D=(5, 5), V=12, seed=43)
+    h[0], W[0] = h[1].copy(), W[1].copy()
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="js")
+    np.testing.assert_allclose(r["ce_kd"], 0.0, atol=1e-14)
+    c = multiexit_loss(y, h, W, alpha_d=0.0, distill="js")
+    np.testing.assert_allclose(r["dh"][0], 0.7 * c["dh"][0], rtol=1e-12, atol=1e-15)
+    # disjoint peaks: the divergence tends to log 2
+    y = np.array([0])
+    h = [np.array([[60.0]]), np.array([[60.0]])]
+    W = [np.array([[1.0], [0.0]]), np.array([[0.0], [1.0]])]
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="js")
+    np.testing.assert_allclose(r["ce_kd"][0], math.log(2.0), rtol=1e-12)
+
+
+def test_js_two_class_closed_form():
+    # student (b, 0), teacher (a, 0); mixture probabilities m1 = (s(a) + s(b)) / 2
+    a, b = 1.5, -0.5
+    y = np.array([1])
+    h = [np.array([[b]]), np.array([[a]])]
+    W = [np.array([[1.0], [0.0]]), np.array([[1.0], [0.0]])]
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="js")
+    qa, qb = _sig(a), _sig(b)
+    m1, m0 = 0.5 * (qa + qb), 0.5 * (2.0 - qa - qb)
+    js = 0.5 * (qb * math.log(qb / m1) + (1 - qb) * math.log((1 - qb) / m0)
+                + qa * math.log(qa / m1) + (1 - qa) * math.log((1 - qa) / m0))
+    np.testing.assert_allclose(r["ce_kd"][0], js, rtol=1e-13)
+    np.testing.assert_allclose(r["loss"], 0.7 * _softplus(b) + 0.3 * js + _softplus(a), rtol=1e-13)
+
+
+def test_js_gradients_match_finite_differences():
+    M, T, D, V, alpha = 3, 3, (3, 4, 5), 7, 0.45
+    y, h, W = _rand_suite(M=M, T=T, D=D, V=V, seed=44, scale=2.0)
+    lam = [1.4, 0.6, 0.9]
+    r = multiexit_loss(y, h, W, alpha_d=alpha, grad_scale=0.8, distill="js", exit_weights=lam)
+    eps = 1e-6
+    for s in range(2):
+        for arr, grad in ((h, r["dh"][s]), (W, r["dW"][s])):
+            num = np.zeros_like(arr[s])
+            for idx in np.ndindex(arr[s].shape):
+                b = arr[s][idx]
+                arr[s][idx] = b + eps
+                lp = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False, distill="js", exit_weights=lam)["loss"]
+                arr[s][idx] = b - eps
+                lm = multiexit_loss(y, h, W, alpha_d=alpha, need_grad=False, distill="js", exit_weights=lam)["loss"]
+                arr[s][idx] = b
+                num[idx] = 0.8 * (lp - lm) / (2 * eps)
+            np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-9)
+    # the teacher is stop-gradient: its gradient is the plain cross-entropy one
+    c = multiexit_loss(y, h, W, alpha_d=alpha, grad_scale=0.8, exit_weights=lam)
+    np.testing.assert_allclose(r["dh"][2], c["dh"][2], rtol=1e-14, atol=1e-16)
