@@ -260,7 +260,8 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
 /* Distillation term of the smaller exits. */
 typedef enum {
   MLS_DISTILL_CE = 0,          /* token-level cross-entropy to the largest exit's softmax (default) */
-  MLS_DISTILL_REVERSE_KL = 1   /* KL(q_m || p_M), an alternative the pages' follow-ups propose   */
+  MLS_DISTILL_REVERSE_KL = 1,  /* KL(q_m || p_M), an alternative the pages' follow-ups propose   */
+  MLS_DISTILL_JS = 2           /* Jensen-Shannon divergence of q_m and p_M, the other one          */
 } mls_distill;
 
 /*
@@ -275,7 +276,16 @@ typedef enum {
  *                 With it, losses[M..2M-2] hold the mean KL and stats rows
  *                 2M..3M-2 hold R_m,t = sum_v q_m,t,v (l_m,t,v - l_M,t,v), so
  *                 KL_t = R_m,t - lse_m,t + lse_M,t; the backward call must get
- *                 the same option.  Other values return MLS_ERR_INVALID_ARG.
+ *                 the same option.
+ *                 MLS_DISTILL_JS (same section): with mu = (q_m + p_M)/2,
+ *                   KD_m = mean_t (KL(q_m || mu) + KL(p_M || mu)) / 2  (<= ln 2),
+ *                   G_m = grad_scale/T ((1 - alpha_d)(q_m - onehot(y))
+ *                                       + alpha_d q_m (log(q_m/mu)/2 - K_t)),
+ *                 K_t = KL(q_m || mu)/2, stored by the forward call in stats
+ *                 rows 2M..3M-2.  Its forward takes a second pass over the
+ *                 logits (the divergence needs the final normalisers); the
+ *                 backward call must get the same option.
+ *                 Other values return MLS_ERR_INVALID_ARG.
  *   exit_weights  HOST float [M] or NULL: per-exit loss weights lambda_m,
  *                 L = sum_{m<M} lambda_m [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m]
  *                     + lambda_M CE_LM,M,

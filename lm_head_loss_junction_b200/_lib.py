@@ -120,7 +120,7 @@ def i64_array(vals):
     return arr
 
 
-MLS_DISTILL = {"ce": 0, "reverse_kl": 1}
+MLS_DISTILL = {"ce": 0, "reverse_kl": 1, "js": 2}
 
 
 def loss_options(exit_weights=None, distill="ce"):

@@ -112,7 +112,8 @@ mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const in
 
 mls_status apply_options(const mls_loss_options* opts, LossProblem* p) {
   if (opts == nullptr) return MLS_OK;
-  if (opts->distill != MLS_DISTILL_CE && opts->distill != MLS_DISTILL_REVERSE_KL) return MLS_ERR_INVALID_ARG;
+  if (opts->distill != MLS_DISTILL_CE && opts->distill != MLS_DISTILL_REVERSE_KL && opts->distill != MLS_DISTILL_JS)
+    return MLS_ERR_INVALID_ARG;
   p->distill = opts->distill;
   if (opts->exit_weights != nullptr) {
     for (int m = 0; m < p->M; ++m) {

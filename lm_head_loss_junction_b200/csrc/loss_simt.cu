@@ -27,7 +27,7 @@ struct SimtDev {
   const float* W[kMaxExits];
   float alpha_d;
   float exit_w[kMaxExits];
-  int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M)
+  int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
   int32_t* status;
   float* dh[kMaxExits];
   float* dW[kMaxExits];
@@ -40,11 +40,17 @@ __device__ __forceinline__ void merge_max_sum(float& m1, float& z1, float m2, fl
   m1 = m;
 }
 
+constexpr float kLn2 = 0.6931471805599453f;
+
+// log(1 + e^x), without overflow for large x.
+__device__ __forceinline__ float softplus(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
+
 // Quantities per thread, in shared memory for the tree merge:
 //   [0] m_T  [1] z_T  [2..2+M-2] A_s  then per student (m_s, z_s), then tgt[M]
 __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev p, float* __restrict__ stats,
                                                                   float* __restrict__ terms) {
   extern __shared__ float sm[];
+  __shared__ float lse_sh[kMaxExits];
   const int M = p.M;
   const int S = M - 1;
   const int64_t t = blockIdx.x;
@@ -77,14 +83,14 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
     if (lT > mT) {
       const float r = __expf(mT - lT);
       zT *= r;
-      if (p.distill == 0)
+      if (p.distill != 1)
         for (int s = 0; s < S; ++s) A[s] *= r;
       mT = lT;
     }
     const float pt = __expf(lT - mT);
     zT += pt;
     for (int s = 0; s < S; ++s) {
-      if (p.distill == 0) A[s] = fmaf(pt, l[s], A[s]);
+      if (p.distill != 1) A[s] = fmaf(pt, l[s], A[s]);
       if (l[s] > ms[s]) {
         const float r = __expf(ms[s] - l[s]);
         zs[s] *= r;
@@ -123,7 +129,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
         float* a = red + (2 + s) * kSimtThreads;
         float* msp = red + (2 + S + 2 * s) * kSimtThreads;
         float* zsp = msp + kSimtThreads;
-        if (p.distill == 0) {
+        if (p.distill != 1) {
           a[tid] = a[tid] * r1 + a[o] * r2;
         } else {
           const float sm = fmaxf(msp[tid], msp[o]);
@@ -158,11 +164,55 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       const float zsum = red[(2 + S + 2 * s + 1) * kSimtThreads];
       const float lse = red[(2 + S + 2 * s) * kSimtThreads] + logf(zsum);
       // cross-entropy: S = sum p_T l_m; reverse KL: R = sum q_m (l_m - l_T)
-      const float Sv = red[(2 + s) * kSimtThreads] / (p.distill == 0 ? red[kSimtThreads] : zsum);
+      const float Sv = red[(2 + s) * kSimtThreads] / (p.distill != 1 ? red[kSimtThreads] : zsum);
       stats[(2 * M + s) * p.T + t] = Sv;
-      terms[(M + s) * p.T + t] = bad ? 0.f : (p.distill == 0 ? lse - Sv : Sv - lse + lseT);
+      terms[(M + s) * p.T + t] = bad ? 0.f : (p.distill != 1 ? lse - Sv : Sv - lse + lseT);
     }
     if (bad) set_flag(p.status, MLS_DEVFLAG_BAD_ID);
+    for (int m = 0; m < M; ++m) lse_sh[m] = stats[m * p.T + t];
+  }
+  if (p.distill != 2 || S == 0) return;
+  // Jensen-Shannon: second walk over the vocabulary with the final normalisers,
+  // sum q log(q/mu) and sum p log(p/mu) per student (mu = (q + p)/2).
+  __syncthreads();
+  float lse[kMaxExits];
+  for (int m = 0; m < M; ++m) lse[m] = lse_sh[m];
+  float jq[kMaxExits - 1], jp[kMaxExits - 1];
+  for (int s = 0; s < kMaxExits - 1; ++s) { jq[s] = 0.f; jp[s] = 0.f; }
+  for (int64_t v = tid; v < p.V; v += kSimtThreads) {
+    float l[kMaxExits];
+    for (int m = 0; m < M; ++m) {
+      const float* w = p.W[m] + v * p.D[m];
+      const float* hh = hrow + p.Doff[m];
+      float acc = 0.f;
+      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
+      l[m] = acc;
+    }
+    const float lp = l[M - 1] - lse[M - 1];
+    const float pv = expf(lp);
+    for (int s = 0; s < S; ++s) {
+      const float lq = l[s] - lse[s];
+      const float d = lp - lq;
+      jq[s] = fmaf(expf(lq), kLn2 - softplus(d), jq[s]);
+      jp[s] = fmaf(pv, kLn2 - softplus(-d), jp[s]);
+    }
+  }
+  for (int s = 0; s < S; ++s) {
+    red[(2 * s) * kSimtThreads + tid] = jq[s];
+    red[(2 * s + 1) * kSimtThreads + tid] = jp[s];
+  }
+  __syncthreads();
+  for (int stride = kSimtThreads / 2; stride > 0; stride >>= 1) {
+    if (tid < stride)
+      for (int r = 0; r < 2 * S; ++r) red[r * kSimtThreads + tid] += red[r * kSimtThreads + tid + stride];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      const float a = red[(2 * s) * kSimtThreads], b = red[(2 * s + 1) * kSimtThreads];
+      stats[(2 * M + s) * p.T + t] = 0.5f * a;
+      terms[(M + s) * p.T + t] = bad ? 0.f : 0.5f * (a + b);
+    }
   }
 }
 
@@ -182,7 +232,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
   const bool bad = yt < 0 || yt >= p.V;
   float lse[kMaxExits], kl[kMaxExits];
   for (int m = 0; m < M; ++m) lse[m] = stats[m * p.T + t];
-  for (int m = 0; m < M - 1; ++m) kl[m] = stats[(2 * M + m) * p.T + t] - lse[m] + lse[M - 1];
+  // reverse KL: KL(q_m || p_T) = R - lse_m + lse_T; Jensen-Shannon: K = KL(q_m || mu)/2 as stored
+  for (int m = 0; m < M - 1; ++m)
+    kl[m] = (p.distill == 2) ? stats[(2 * M + m) * p.T + t] : stats[(2 * M + m) * p.T + t] - lse[m] + lse[M - 1];
   const float a = p.alpha_d;
   for (int64_t v = tid; v < p.V; v += kSimtThreads) {
     float l[kMaxExits];
@@ -201,9 +253,13 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
         g = pT - hot;
       } else if (p.distill == 0) {
         g = __expf(l[m] - lse[m]) - a * pT - (1.f - a) * hot;
-      } else {
+      } else if (p.distill == 1) {
         const float q = __expf(l[m] - lse[m]);
         const float d = (l[m] - lse[m]) - (l[M - 1] - lse[M - 1]) - kl[m];
+        g = (1.f - a) * (q - hot) + a * q * d;
+      } else {
+        const float q = __expf(l[m] - lse[m]);
+        const float d = 0.5f * (kLn2 - softplus((l[M - 1] - lse[M - 1]) - (l[m] - lse[m]))) - kl[m];
         g = (1.f - a) * (q - hot) + a * q * d;
       }
       G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : p.exit_w[m] * g;

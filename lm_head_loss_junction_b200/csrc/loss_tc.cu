@@ -66,7 +66,7 @@ struct LossArgs {
   int n_tt, n_vt, num_tiles, group_tt;
   const int32_t* y;
   float alpha;                 // alpha_d
-  int distill;                 // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M)
+  int distill;                 // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
   float* partial;              // forward: [2 n_vt][2M-1][T]
   float* stats;                // forward: target rows written; backward: lse read
   __nv_bfloat16* G;            // backward: [M][T][V]
@@ -90,10 +90,19 @@ struct __align__(1024) LossSmem {
   int abort;
 };
 
-enum LossMode { kModeStats = 0, kModeGrad = 1, kModeAgree = 2 };
+enum LossMode { kModeStats = 0, kModeGrad = 1, kModeAgree = 2, kModeJS = 3 };
 
 // Partial rows per split in agreement mode: beta_s, KL_s (students), max_m, argmax_m.
 __host__ __device__ constexpr int agree_rows(int M) { return 4 * M - 2; }
+
+// Partial rows per split of the Jensen-Shannon pass: sum q log(q/mu) and
+// sum p log(p/mu) of every student (mu the mixture (q + p)/2).
+__host__ __device__ constexpr int js_rows(int M) { return 2 * (M - 1); }
+
+constexpr float kLn2 = 0.6931471805599453f;
+
+// log(1 + e^x), without overflow for large x.
+__device__ __forceinline__ float softplus(float x) { return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))); }
 
 __device__ __forceinline__ void loss_tile_coords(int i, const LossArgs& a, int& tt, int& vt) {
   const int per_group = a.group_tt * a.n_vt;
@@ -148,7 +157,9 @@ __device__ __forceinline__ void job_slot(bool hold_teacher, int M, uint32_t tile
 }
 
 // ------------------------------------------------------------------ loss tile kernel
-template <int MODE>
+// DISTILL (0 cross-entropy, 1 reverse KL, 2 Jensen-Shannon) is a template
+// parameter so that each form gets its own register allocation.
+template <int MODE, int DISTILL>
 __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid_constant__ LossMaps maps,
                                                                     const LossArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -157,8 +168,11 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort;
   const int M = a.M;
-  const bool hold = (MODE == kModeAgree) || (a.distill == 1);
-  const bool rkl = (a.distill == 1);
+  constexpr bool rkl = (DISTILL == 1);
+  constexpr bool jsd = (DISTILL == 2);
+  // The statistics of the Jensen-Shannon form are the cross-entropy ones (it
+  // needs the final normalisers, so its divergence has a pass of its own).
+  constexpr bool hold = (MODE == kModeAgree) || (MODE == kModeJS) || rkl || (MODE == kModeGrad && jsd);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kLossStages; ++i) {
@@ -447,24 +461,64 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             prow[static_cast<int64_t>(2 * (M - 1) + m) * a.T] = mxv;
             prow[static_cast<int64_t>(3 * M - 2 + m) * a.T] = __int_as_float(mxi);
           }
+        } else if (MODE == kModeJS) {
+          // ---------------- Jensen-Shannon divergence to the largest exit, with the final
+          // normalisers: per element, with d = log p - log q,
+          //   log(q/mu) = ln 2 - softplus(d),  log(p/mu) = ln 2 - softplus(-d).
+          float jq = 0.f, jp = 0.f;
+          if (live && j > 0) {
+            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
+            const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              float r[32], lt[32];
+              tmem_ld32(base + c * 32, r);
+              tmem_ld32(tbase + c * 32, lt);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                const float lq = r[k] - lse;
+                const float lp = lt[k] - lseT;
+                const float d = lp - lq;
+                const float sp = __logf(1.f + __expf(-fabsf(d)));
+                jq = fmaf(exp2f(lq * kLog2e), kLn2 - fmaxf(d, 0.f) - sp, jq);
+                jp = fmaf(exp2f(lp * kLog2e), kLn2 - fmaxf(-d, 0.f) - sp, jp);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (j > 0) mbar_arrive(&s.tempty[1]);
+            if (j == M - 1) mbar_arrive(&s.tempty[0]);
+          }
+          if (valid && j > 0) {
+            float* prow = a.partial + static_cast<int64_t>(split) * js_rows(M) * a.T + t;
+            prow[static_cast<int64_t>(m) * a.T] = jq;
+            prow[static_cast<int64_t>(M - 1 + m) * a.T] = jp;
+          }
         } else {
           // ---------------- backward: dense part of the logit gradient, bf16
           if (bad && j == 0 && vt == 0 && half == 0) set_flag(a.status, MLS_DEVFLAG_BAD_ID);
           if (live) {
             const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
             const float ls = lse * kLog2e;
-            // reverse KL: per-token KL(q_m || p_T) = R_m - lse_m + lse_T (R from the forward pass)
+            // reverse KL: per-token KL(q_m || p_T) = R_m - lse_m + lse_T (R from the forward pass);
+            // Jensen-Shannon: per-token K = KL(q_m || mu) / 2, stored by the forward pass
             float lseT = 0.f, klt = 0.f;
-            if (rkl && j > 0 && valid) {
+            if ((rkl || jsd) && j > 0 && valid) {
               lseT = a.stats[static_cast<int64_t>(M - 1) * a.T + t];
-              klt = a.stats[static_cast<int64_t>(2 * M + m) * a.T + t] - lse + lseT;
+              const float st2 = a.stats[static_cast<int64_t>(2 * M + m) * a.T + t];
+              klt = rkl ? st2 - lse + lseT : st2;
             }
-#pragma unroll 1
+            // unrolled in the cross-entropy form so that the teacher's packed
+            // probabilities stay in registers (indexed by c)
+            constexpr int kUnrollC = hold ? 1 : 4;
+#pragma unroll kUnrollC
             for (int c = 0; c < 4; ++c) {
               float r[32];
               tmem_ld32(base + c * 32, r);
               float lt[32];
-              if (rkl && j > 0) {
+              if ((rkl || jsd) && j > 0) {
                 tmem_ld32(tbase + c * 32, lt);
               } else {
 #pragma unroll
@@ -477,12 +531,17 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -ls));
                 float g0, g1;
                 if (j == 0) {                      // teacher: G' = p_T
-                  if (!rkl) pt[c][k / 2] = pack_p2(e0, e1);
+                  if (!hold) pt[c][k / 2] = pack_p2(e0, e1);
                   g0 = e0;
                   g1 = e1;
                 } else if (rkl) {                  // student: G' = q ((1 - a) + a (log q - log p - KL))
                   const float d0 = (r[k] - lse) - (lt[k] - lseT) - klt;
                   const float d1 = (r[k + 1] - lse) - (lt[k + 1] - lseT) - klt;
+                  g0 = e0 * fmaf(al, d0, 1.f - al);
+                  g1 = e1 * fmaf(al, d1, 1.f - al);
+                } else if (jsd) {                  // student: G' = q ((1 - a) + a (log(q/mu)/2 - K))
+                  const float d0 = fmaf(-0.5f, softplus((lt[k] - lseT) - (r[k] - lse)), 0.5f * kLn2) - klt;
+                  const float d1 = fmaf(-0.5f, softplus((lt[k + 1] - lseT) - (r[k + 1] - lse)), 0.5f * kLn2) - klt;
                   g0 = e0 * fmaf(al, d0, 1.f - al);
                   g1 = e1 * fmaf(al, d1, 1.f - al);
                 } else {                           // student: G' = q - alpha_d p_T
@@ -566,7 +625,7 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
       if (l > mT) {
         const float r = __expf(mT - l);
         zT *= r;
-        if (distill == 0)
+        if (distill != 1)
           for (int s = 0; s < M - 1; ++s) A[s] *= r;   // teacher-weighted sums follow the teacher's max
         mT = l;
       }
@@ -575,7 +634,7 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
       for (int s = 0; s < M - 1; ++s) {
         const float ls = pi[static_cast<int64_t>(s) * T];
         const float ab = pi[static_cast<int64_t>(M + s) * T];
-        if (distill == 0) A[s] = fmaf(w, ab, A[s]);
+        if (distill != 1) A[s] = fmaf(w, ab, A[s]);
         if (ls > ms[s]) {
           const float r = __expf(ms[s] - ls);
           zs[s] *= r;
@@ -610,7 +669,7 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
       const float mn = fmaxf(ms[s], n2);
       const float q1 = (ms[s] == -INFINITY) ? 0.f : __expf(ms[s] - mn);
       const float q2 = (n2 == -INFINITY) ? 0.f : __expf(n2 - mn);
-      if (distill == 0) A[s] = A[s] * r1 + st_A[r][s][lane] * r2;
+      if (distill != 1) A[s] = A[s] * r1 + st_A[r][s][lane] * r2;
       else A[s] = A[s] * q1 + st_A[r][s][lane] * q2;
       zs[s] = zs[s] * q1 + y2 * q2;
       ms[s] = mn;
@@ -625,9 +684,10 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
   terms[static_cast<int64_t>(M - 1) * T + t] = bad ? 0.f : lseT - stats[static_cast<int64_t>(2 * M - 1) * T + t];
   for (int s = 0; s < M - 1; ++s) {
     const float lse = ms[s] + logf(zs[s]);
-    // cross-entropy: S = sum p_T l_m (teacher-weighted); reverse KL: R = sum q_m (l_m - l_T)
-    const float Sv = (distill == 0) ? A[s] / zT : A[s] / zs[s];
-    const float kd = (distill == 0) ? lse - Sv : Sv - lse + lseT;
+    // cross-entropy: S = sum p_T l_m (teacher-weighted); reverse KL: R = sum q_m (l_m - l_T).
+    // (Jensen-Shannon: S and the cross-entropy term here; its own pass overwrites both.)
+    const float Sv = (distill != 1) ? A[s] / zT : A[s] / zs[s];
+    const float kd = (distill != 1) ? lse - Sv : Sv - lse + lseT;
     stats[static_cast<int64_t>(s) * T + t] = lse;
     stats[static_cast<int64_t>(2 * M + s) * T + t] = Sv;
     if (bad) stats[static_cast<int64_t>(M + s) * T + t] = 0.f;
@@ -685,6 +745,46 @@ __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const floa
     terms[static_cast<int64_t>(s) * T + t] = b[s];
     terms[static_cast<int64_t>(M - 1 + s) * T + t] = kl[s];
     terms[static_cast<int64_t>(2 * (M - 1) + s) * T + t] = (ix[s] == ix[M - 1]) ? 1.f : 0.f;
+  }
+}
+
+// ------------------------------------------------------------------ Jensen-Shannon merge
+// Per token: plain sums over the splits (the pass used the final normalisers) of
+// sum q log(q/mu) and sum p log(p/mu); writes K = KL(q || mu)/2 into the
+// statistics row the backward pass reads and JS = (KL(q || mu) + KL(p || mu))/2
+// as the distillation term.
+__global__ void __launch_bounds__(32 * kMergeRows) js_merge_kernel(const float* __restrict__ partial, int n_splits,
+                                                                   int M, int T, int V,
+                                                                   const int32_t* __restrict__ y,
+                                                                   float* __restrict__ stats,
+                                                                   float* __restrict__ terms) {
+  constexpr int S = kMaxExits - 1;
+  __shared__ float sh_q[kMergeRows][S][32], sh_p[kMergeRows][S][32];
+  const int lane = threadIdx.x, rowi = threadIdx.y;
+  const int t = blockIdx.x * 32 + lane;
+  const int QJ = js_rows(M);
+  const int per = (n_splits + kMergeRows - 1) / kMergeRows;
+  const int i0 = min(n_splits, rowi * per), i1 = min(n_splits, i0 + per);
+  float jq[S] = {0.f, 0.f, 0.f}, jp[S] = {0.f, 0.f, 0.f};
+  if (t < T) {
+    for (int i = i0; i < i1; ++i) {
+      const float* pi = partial + static_cast<int64_t>(i) * QJ * T + t;
+      for (int s = 0; s < M - 1; ++s) {
+        jq[s] += pi[static_cast<int64_t>(s) * T];
+        jp[s] += pi[static_cast<int64_t>(M - 1 + s) * T];
+      }
+    }
+  }
+  for (int s = 0; s < S; ++s) { sh_q[rowi][s][lane] = jq[s]; sh_p[rowi][s][lane] = jp[s]; }
+  __syncthreads();
+  if (rowi != 0 || t >= T) return;
+  for (int r = 1; r < kMergeRows; ++r)
+    for (int s = 0; s < M - 1; ++s) { jq[s] += sh_q[r][s][lane]; jp[s] += sh_p[r][s][lane]; }
+  const int yt = y[t];
+  const bool bad = yt < 0 || yt >= V;
+  for (int s = 0; s < M - 1; ++s) {
+    stats[static_cast<int64_t>(2 * M + s) * T + t] = 0.5f * jq[s];
+    terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : 0.5f * (jq[s] + jp[s]);
   }
 }
 
@@ -1220,7 +1320,7 @@ TcWs fwd_layout(const LossProblem& p, void* ws) {
   return w;
 }
 
-template <int MODE>
+template <int MODE, int DISTILL>
 cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaStream_t st) {
   LossMaps maps;
   for (int m = 0; m < p.M; ++m) {
@@ -1229,7 +1329,7 @@ cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaSt
   }
   LossArgs a = args_in;
   const size_t smem = sizeof(LossSmem) + 1024;
-  auto fn = loss_tile_kernel<MODE>;
+  auto fn = loss_tile_kernel<MODE, DISTILL>;
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
@@ -1374,7 +1474,7 @@ cudaError_t agree_tc(const LossProblem& p, const float* stats, float* metrics, f
   LossArgs a = base_args(p);
   a.partial = partial;
   a.stats = const_cast<float*>(stats);
-  cudaError_t err = run_loss_tiles<kModeAgree>(p, a, st);
+  cudaError_t err = run_loss_tiles<kModeAgree, 0>(p, a, st);
   if (err != cudaSuccess) return err;
   const int T = static_cast<int>(p.T);
   agree_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(partial, 2 * a.n_vt, p.M, T, terms, top);
@@ -1393,7 +1493,8 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   LossArgs a = base_args(p);
   a.partial = w.partial;
   a.stats = stats;
-  cudaError_t err = run_loss_tiles<kModeStats>(p, a, st);
+  // the Jensen-Shannon form starts from the cross-entropy statistics
+  cudaError_t err = p.distill == 1 ? run_loss_tiles<kModeStats, 1>(p, a, st) : run_loss_tiles<kModeStats, 0>(p, a, st);
   if (err != cudaSuccess) return err;
   const int T = static_cast<int>(p.T);
   loss_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
@@ -1402,6 +1503,17 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
+  if (p.distill == 2 && p.M > 1) {
+    // Jensen-Shannon: a second pass over the logits with the final normalisers
+    // (its partials, 2(M-1) rows per split, reuse the statistics partial buffer).
+    err = run_loss_tiles<kModeJS, 0>(p, a, st);
+    if (err != cudaSuccess) return err;
+    js_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
+                                                                     static_cast<int>(p.V), p.y, stats, w.terms);
+    note_launches(1);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   return launch_loss_reduce(w.terms, p, losses, st);
 }
 
@@ -1411,7 +1523,9 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   LossArgs a = base_args(p);
   a.stats = const_cast<float*>(stats);
   a.G = G;
-  cudaError_t err = run_loss_tiles<kModeGrad>(p, a, st);
+  cudaError_t err = p.distill == 1   ? run_loss_tiles<kModeGrad, 1>(p, a, st)
+                    : p.distill == 2 ? run_loss_tiles<kModeGrad, 2>(p, a, st)
+                                     : run_loss_tiles<kModeGrad, 0>(p, a, st);
   if (err != cudaSuccess) return err;
   // Tokens grouped by target, for the exact one-hot part of dW.
   SegIndexDev ix;

@@ -46,7 +46,8 @@ def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce"):
     assert_stats_close(s[:M], r["lse"], "lse")
     assert_stats_close(s[M:2 * M], r["tgt"], "target logits")
     if M > 1:
-        assert_stats_close(s[2 * M:], r["S"] if distill == "ce" else r["R"], "distillation statistic")
+        assert_stats_close(s[2 * M:], {"ce": r["S"], "reverse_kl": r["R"], "js": r["J"]}[distill],
+                           "distillation statistic")
     for m in range(M):
         assert_grad_close(dh[m], r["dh"][m], f"dh[{m}]")
         assert_grad_close(dW[m], r["dW"][m], f"dW[{m}]")
@@ -89,11 +90,12 @@ def test_exit_weights(name, small):
 @pytest.mark.parametrize("name,small", [("tiny3", None), ("main3", dict(batch=1, seq=200, V=512)),
                                         ("suite4", dict(batch=1, seq=130, V=384)),
                                         ("main3_aligned", dict(batch=1, seq=256, V=768))])
-def test_reverse_kl_distillation(name, small):
+@pytest.mark.parametrize("distill", ["reverse_kl", "js"])
+def test_alternative_distillation(name, small, distill):
     cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
     d = wl.make_inputs(cfg, with_tables=False)
-    _check_all(d, 0.3, 1.0, distill="reverse_kl")
-    _check_all(d, 0.6, 2.0, exit_weights=[1.5, 0.5] + [1.0] * (cfg.M - 2), distill="reverse_kl")
+    _check_all(d, 0.3, 1.0, distill=distill)
+    _check_all(d, 0.6, 2.0, exit_weights=[1.5, 0.5] + [1.0] * (cfg.M - 2), distill=distill)
 
 
 def test_single_exit_and_accumulate():
