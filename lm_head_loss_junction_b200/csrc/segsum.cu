@@ -236,10 +236,16 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
     float acc[N];
 #pragma unroll
     for (int k = 0; k < N; ++k) acc[k] = 0.f;
-    for (int p = 0; p < cnt; ++p) {
-      const int64_t t = ix.toks[off + p];
-      Vec8<BF16>::add(acc, __ldg(src + t * src_ld + src_off + vi));
+    // four rows in flight per lane, added in token order
+    int p = 0;
+    for (; p + 4 <= cnt; p += 4) {
+      uint4 u[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) u[b] = __ldg(src + static_cast<int64_t>(ix.toks[off + p + b]) * src_ld + src_off + vi);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) Vec8<BF16>::add(acc, u[b]);
     }
+    for (; p < cnt; ++p) Vec8<BF16>::add(acc, __ldg(src + static_cast<int64_t>(ix.toks[off + p]) * src_ld + src_off + vi));
     emit<BF16, TABLE>(out_row, vi, acc, cs, E_row, scale, accumulate != 0);
   }
 }
@@ -265,7 +271,22 @@ __global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(
 #pragma unroll
   for (int k = 0; k < N; ++k) acc[k] = 0.f;
   float cs = 0.f;
-  for (int p = warp; p < cnt; p += kHeavyWarps) {
+  // this warp's tokens p = warp, warp + 16, ...; four rows in flight, added in order
+  int p = warp;
+  for (; p + 3 * kHeavyWarps < cnt; p += 4 * kHeavyWarps) {
+    int64_t t[4];
+    uint4 u[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) t[b] = ix.toks[off + p + b * kHeavyWarps];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) u[b] = active ? __ldg(src + t[b] * src_ld + src_off + vi) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      if (TABLE) cs += coef[t[b]];
+      if (active) Vec8<BF16>::add(acc, u[b]);
+    }
+  }
+  for (; p < cnt; p += kHeavyWarps) {
     const int64_t t = ix.toks[off + p];
     if (TABLE) cs += coef[t];
     if (active) Vec8<BF16>::add(acc, __ldg(src + t * src_ld + src_off + vi));
