@@ -57,7 +57,7 @@ def softmax_rows(l: np.ndarray) -> np.ndarray:
 
 
 def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
-                   rows=None, token_block=256, exit_weights=None, distill="ce"):
+                   rows=None, token_block=256, exit_weights=None, distill="ce", teacher_grad=False):
     """Multi-exit loss, per-token statistics and (optionally) gradients, fp64.
 
     y: int [T] targets; h: list of M arrays [T, D_m]; W: list of M arrays [V, D_m].
@@ -84,6 +84,13 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     G_m = lambda_m grad_scale/T ((1 - alpha_d)(q_m - onehot) + alpha_d q_m (g - K_t)),
     g_v = log(q_v / mu_v) / 2,  K_t = sum_v q_v g_v = KL(q_m || mu) / 2,
     and K_t is returned per token in "J".
+    teacher_grad: the largest exit also receives the gradient of every
+    distillation term (no stop-gradient; the pages leave this open).  With
+    T_m = d KD_m / d l_M, the teacher's logit gradient gains
+    lambda_m alpha_d T_m per smaller exit m, where
+      cross-entropy:  T_m = -p_M (l_m - S_m)           (S_m = sum_v p_M l_m)
+      reverse KL:     T_m = p_M - q_m
+      Jensen-Shannon: T_m = p_M (log(p_M / mu) / 2 - KL(p_M || mu) / 2).
 
     Returns a dict with
       ce_lm [M], ce_kd [M-1], loss (scalar)         -- means over the tokens
@@ -124,7 +131,7 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             out["lse"][m, b0:b0 + n] = lse[m]
             out["tgt"][m, b0:b0 + n] = logits[m][ar, yb]
             out["ce_lm_sum"][m] += np.sum(lse[m] - logits[m][ar, yb])
-        rkl, logmix, jq = [], [], []
+        rkl, logmix, jq, jps = [], [], [], []
         for m in range(M - 1):
             out["S"][m, b0:b0 + n] = np.sum(pM * logits[m], axis=1)
             q = np.exp(logq[m])
@@ -134,6 +141,7 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             logmix.append(np.logaddexp(logq[m], logq[M - 1]) - np.log(2.0))
             jq.append(np.sum(q * (logq[m] - logmix[m]), axis=1))
             jp = np.sum(pM * (logq[M - 1] - logmix[m]), axis=1)
+            jps.append(jp)
             out["J"][m, b0:b0 + n] = 0.5 * jq[m]
             if distill == "ce":
                 out["ce_kd_sum"][m] += np.sum(-np.sum(pM * logq[m], axis=1))
@@ -156,6 +164,15 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
                     G = lam[m] * g * ((1.0 - alpha_d) * (q - onehot) + alpha_d * kd)
                 else:
                     G = lam[m] * g * (q - onehot)
+                    if teacher_grad:
+                        for s in range(M - 1):
+                            if distill == "ce":
+                                Ts = -pM * (logits[s] - np.sum(pM * logits[s], axis=1)[:, None])
+                            elif distill == "reverse_kl":
+                                Ts = pM - np.exp(logq[s])
+                            else:
+                                Ts = pM * (0.5 * (logq[M - 1] - logmix[s]) - 0.5 * jps[s][:, None])
+                            G = G + lam[s] * g * alpha_d * Ts
                 out["dh"][m][b0:b0 + n] = G @ Ws[m]
                 out["dW"][m] += G.T @ hb[m]
     out["ce_lm"] = out["ce_lm_sum"] / T

@@ -408,3 +408,51 @@ def test_js_gradients_match_finite_differences():
     # the teacher is stop-gradient: its gradient is the plain cross-entropy one
     c = multiexit_loss(y, h, W, alpha_d=alpha, grad_scale=0.8, exit_weights=lam)
     np.testing.assert_allclose(r["dh"][2], c["dh"][2], rtol=1e-14, atol=1e-16)
+
+
+# ------------------------------------------------------------------ teacher gradient (no stop-gradient)
+@pytest.mark.parametrize("distill", ["ce", "reverse_kl", "js"])
+def test_teacher_gradient_matches_finite_differences_of_the_whole_loss(distill):
+    # Without the stop-gradient every parameter's gradient, the largest exit's
+    # included, is the plain derivative of the total loss.
+    M, T, D, V, alpha = 3, 3, (3, 4, 5), 7, 0.35
+    y, h, W = _rand_suite(M=M, T=T, D=D, V=V, seed=51, scale=2.0)
+    lam = [1.2, 0.7, 0.9]
+    kw = dict(alpha_d=alpha, distill=distill, exit_weights=lam)
+    r = multiexit_loss(y, h, W, grad_scale=1.1, teacher_grad=True, **kw)
+    eps = 1e-6
+    for m in range(M):
+        for arr, grad in ((h, r["dh"][m]), (W, r["dW"][m])):
+            num = np.zeros_like(arr[m])
+            for idx in np.ndindex(arr[m].shape):
+                b = arr[m][idx]
+                arr[m][idx] = b + eps
+                lp = multiexit_loss(y, h, W, need_grad=False, **kw)["loss"]
+                arr[m][idx] = b - eps
+                lm = multiexit_loss(y, h, W, need_grad=False, **kw)["loss"]
+                arr[m][idx] = b
+                num[idx] = 1.1 * (lp - lm) / (2 * eps)
+            # central differences at eps = 1e-6 on a loss of order 10 carry about
+            # 1e-16 * 10 / 1e-6 ~ 1e-9 of rounding error
+            np.testing.assert_allclose(grad, num, rtol=1e-6, atol=5e-9)
+    # the students' gradients do not depend on the option
+    s = multiexit_loss(y, h, W, grad_scale=1.1, **kw)
+    for m in range(M - 1):
+        np.testing.assert_allclose(r["dh"][m], s["dh"][m], rtol=1e-14, atol=1e-16)
+    # and at alpha_d = 0 the teacher's does not either
+    a = multiexit_loss(y, h, W, alpha_d=0.0, distill=distill, exit_weights=lam, teacher_grad=True)
+    b = multiexit_loss(y, h, W, alpha_d=0.0, distill=distill, exit_weights=lam)
+    np.testing.assert_allclose(a["dh"][M - 1], b["dh"][M - 1], rtol=1e-14, atol=1e-16)
+
+
+def test_teacher_gradient_of_identical_exits_ce():
+    # Student equal to the teacher, cross-entropy form: KD = H(p), whose
+    # derivative in l is -p (log p + H); the extra teacher term must equal it.
+    y, h, W = _rand_suite(M=2, T=5, D=(6, 6), V=10, seed=52)
+    h[0], W[0] = h[1].copy(), W[1].copy()
+    a = multiexit_loss(y, h, W, alpha_d=0.4, teacher_grad=True)
+    b = multiexit_loss(y, h, W, alpha_d=0.4)
+    p = softmax_rows(h[1] @ W[1].T)
+    H = -np.sum(p * np.log(p), axis=1)
+    extra = 0.4 / 5 * (-p * (np.log(p) + H[:, None]))
+    np.testing.assert_allclose(a["dh"][1] - b["dh"][1], extra @ W[1], rtol=1e-10, atol=1e-15)
