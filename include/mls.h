@@ -286,6 +286,17 @@ typedef enum {
  *                 logits (the divergence needs the final normalisers); the
  *                 backward call must get the same option.
  *                 Other values return MLS_ERR_INVALID_ARG.
+ *   teacher_grad  0 (default): the largest exit's softmax in the distillation
+ *                 terms is a constant (stop-gradient).  1: it is not, and the
+ *                 largest exit's logit gradient gains, for every smaller exit m,
+ *                 lambda_m alpha_d dKD_m/dl_M:
+ *                   MLS_DISTILL_CE:         -p_M (l_m - S_m),  S_m = sum_v p_M l_m
+ *                   MLS_DISTILL_REVERSE_KL:  p_M - q_m.
+ *                 Backward only (the forward is unchanged; pass the same
+ *                 options to both calls).  With MLS_DISTILL_JS it returns
+ *                 MLS_ERR_UNSUPPORTED: that gradient needs KL(p_M || mu) per
+ *                 token, which the statistics rows do not hold.  The pages
+ *                 leave the teacher's gradient open.
  *   exit_weights  HOST float [M] or NULL: per-exit loss weights lambda_m,
  *                 L = sum_{m<M} lambda_m [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m]
  *                     + lambda_M CE_LM,M,
@@ -299,6 +310,7 @@ typedef enum {
 typedef struct {
   const float* exit_weights;
   int distill;                 /* mls_distill */
+  int teacher_grad;            /* 0: teacher stop-gradient (default); 1: see above */
 } mls_loss_options;
 
 mls_status mls_multiexit_loss_fwd_opts(int M, int64_t T, int64_t V, const int64_t* D,

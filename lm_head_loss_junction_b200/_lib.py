@@ -36,7 +36,8 @@ _u32 = ctypes.c_uint32
 
 class LossOptions(ctypes.Structure):
     """mls_loss_options"""
-    _fields_ = [("exit_weights", ctypes.POINTER(ctypes.c_float)), ("distill", ctypes.c_int)]
+    _fields_ = [("exit_weights", ctypes.POINTER(ctypes.c_float)), ("distill", ctypes.c_int),
+                ("teacher_grad", ctypes.c_int)]
 
 
 # name -> (restype, argtypes), in the order of include/mls.h
@@ -123,15 +124,16 @@ def i64_array(vals):
 MLS_DISTILL = {"ce": 0, "reverse_kl": 1, "js": 2}
 
 
-def loss_options(exit_weights=None, distill="ce"):
+def loss_options(exit_weights=None, distill="ce", teacher_grad=False):
     """ctypes options struct (and the buffer it points to), or None for defaults."""
-    if exit_weights is None and distill == "ce":
+    if exit_weights is None and distill == "ce" and not teacher_grad:
         return None
     if exit_weights is None:
-        opts = LossOptions(None, MLS_DISTILL[distill])
+        opts = LossOptions(None, MLS_DISTILL[distill], int(bool(teacher_grad)))
         opts._buf = None
         return opts
     buf = (ctypes.c_float * len(exit_weights))(*[float(w) for w in exit_weights])
-    opts = LossOptions(ctypes.cast(buf, ctypes.POINTER(ctypes.c_float)), MLS_DISTILL[distill])
+    opts = LossOptions(ctypes.cast(buf, ctypes.POINTER(ctypes.c_float)), MLS_DISTILL[distill],
+                       int(bool(teacher_grad)))
     opts._buf = buf          # keep the weights alive with the struct
     return opts

@@ -177,8 +177,8 @@ def multiexit_loss_fwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Ten
 
 def multiexit_loss_bwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Tensor], stats: torch.Tensor,
                        alpha_d: float = 0.3, grad_scale: float = 1.0, *, dh=None, dW=None,
-                       accumulate_dW: bool = False, workspace=None, exit_weights=None, distill="ce", status=None,
-                       stream=None):
+                       accumulate_dW: bool = False, workspace=None, exit_weights=None, distill="ce",
+                       teacher_grad: bool = False, status=None, stream=None):
     """Returns (dh list, dW list) (see mls_multiexit_loss_bwd)."""
     M, T, V, D, dt = _loss_common(y, h, W)
     dev = y.device
@@ -193,7 +193,7 @@ def multiexit_loss_bwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Ten
             ptr_array([t.data_ptr() for t in W]), float(alpha_d), _dtype_code(h[0]), stats.data_ptr(),
             float(grad_scale), ptr_array([t.data_ptr() for t in dh]), ptr_array([t.data_ptr() for t in dW]),
             int(bool(accumulate_dW)), workspace.data_ptr(), ws_bytes)
-    opts = _lib.loss_options(exit_weights, distill)
+    opts = _lib.loss_options(exit_weights, distill, teacher_grad)
     if opts is None:
         code = lib().mls_multiexit_loss_bwd(*args, _ptr(status), _stream_ptr(stream))
     else:

@@ -65,7 +65,8 @@ struct LossProblem {
   const void* W[kMaxExits];
   float alpha_d;
   float exit_w[kMaxExits];   // per-exit loss weights (1 = equal weights)
-  int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M)
+  int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
+  int teacher_grad;          // 1: the largest exit also gets the distillation gradient (no stop-gradient)
   int32_t* status;
 };
 

@@ -28,6 +28,7 @@ struct SimtDev {
   float alpha_d;
   float exit_w[kMaxExits];
   int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
+  int teacher_grad;          // 1: no stop-gradient on the largest exit (cross-entropy and reverse KL)
   int32_t* status;
   float* dh[kMaxExits];
   float* dW[kMaxExits];
@@ -251,6 +252,18 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
       float g;
       if (m == M - 1) {
         g = pT - hot;
+        if (p.teacher_grad) {
+          // distillation gradient of every smaller exit s on the teacher's logits, relative to w_T:
+          //   cross-entropy -p_T (l_s - S_s);  reverse KL p_T - q_s
+          float extra = 0.f;
+          for (int s = 0; s < M - 1; ++s) {
+            const float ts = (p.distill == 1) ? pT - __expf(l[s] - lse[s])
+                                              : -pT * (l[s] - stats[(2 * M + s) * p.T + t]);
+            extra = fmaf(p.exit_w[s], ts, extra);
+          }
+          G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : fmaf(a, extra, p.exit_w[m] * g);
+          continue;
+        }
       } else if (p.distill == 0) {
         g = __expf(l[m] - lse[m]) - a * pT - (1.f - a) * hot;
       } else if (p.distill == 1) {
@@ -436,6 +449,7 @@ SimtDev make_dev(const LossProblem& p) {
   d.y = p.y;
   d.alpha_d = p.alpha_d;
   d.distill = p.distill;
+  d.teacher_grad = (p.teacher_grad != 0 && p.M > 1) ? 1 : 0;
   for (int m = 0; m < kMaxExits; ++m) d.exit_w[m] = p.exit_w[m];
   d.status = p.status;
   return d;

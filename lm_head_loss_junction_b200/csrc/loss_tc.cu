@@ -67,6 +67,8 @@ struct LossArgs {
   const int32_t* y;
   float alpha;                 // alpha_d
   int distill;                 // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
+  float exit_w[kMaxExits];     // per-exit weights (teacher-gradient backward only)
+  float student_wsum;          // sum of the smaller exits' weights
   float* partial;              // forward: [2 n_vt][2M-1][T]
   float* stats;                // forward: target rows written; backward: lse read
   __nv_bfloat16* G;            // backward: [M][T][V]
@@ -139,6 +141,13 @@ __device__ __forceinline__ uint32_t pack_p2(float lo, float hi) {
 
 __device__ __forceinline__ float2 unpack_p2(uint32_t u) { return __half22float2(*reinterpret_cast<__half2*>(&u)); }
 
+// acc + w * x on fp16 pairs (the teacher-gradient accumulator).
+__device__ __forceinline__ uint32_t hfma_p2(uint32_t w, uint32_t x, uint32_t acc) {
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&w), *reinterpret_cast<__half2*>(&x),
+                      *reinterpret_cast<__half2*>(&acc));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
 // TMEM region and use count of job j (exit M-1-j) of the tile_iter-th tile of a CTA.
 // By default consecutive jobs alternate the two regions.  When the epilogue
 // needs the teacher's logits at every element of a student's tile (the
@@ -156,10 +165,34 @@ __device__ __forceinline__ void job_slot(bool hold_teacher, int M, uint32_t tile
   }
 }
 
+// One 32-column chunk of G' (this lane's row: 16 packed bf16 pairs) through the
+// warp's staging rows, so that each store instruction writes 8 rows x 64
+// contiguous bytes (full sectors).  Rows at or past T are not stored.
+__device__ __forceinline__ void store_g_chunk(uint8_t* stage, int lane, const uint32_t (&packed)[16],
+                                              __nv_bfloat16* G, int row0, int T, int V, int col) {
+  uint4* mine = reinterpret_cast<uint4*>(stage + lane * kStageRowBytes);
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    mine[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int piece = i * 32 + lane;
+    const int rr = piece >> 2, ch = piece & 3;
+    const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * kStageRowBytes + ch * 16);
+    if (row0 + rr < T) *reinterpret_cast<uint4*>(G + static_cast<int64_t>(row0 + rr) * V + col + ch * 8) = v;
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ loss tile kernel
 // DISTILL (0 cross-entropy, 1 reverse KL, 2 Jensen-Shannon) is a template
-// parameter so that each form gets its own register allocation.
-template <int MODE, int DISTILL>
+// parameter so that each form gets its own register allocation.  TGRAD (the
+// backward without the teacher's stop-gradient) holds the teacher's logits in
+// region 0 while the students pass through region 1, accumulates each
+// student's contribution to the teacher's logit gradient in registers (fp16
+// pairs), and writes the teacher's G' after the last student.
+template <int MODE, int DISTILL, bool TGRAD = false>
 __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid_constant__ LossMaps maps,
                                                                     const LossArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -172,7 +205,8 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   constexpr bool jsd = (DISTILL == 2);
   // The statistics of the Jensen-Shannon form are the cross-entropy ones (it
   // needs the final normalisers, so its divergence has a pass of its own).
-  constexpr bool hold = (MODE == kModeAgree) || (MODE == kModeJS) || rkl || (MODE == kModeGrad && jsd);
+  constexpr bool hold = (MODE == kModeAgree) || (MODE == kModeJS) || rkl || (MODE == kModeGrad && (jsd || TGRAD));
+  static_assert(!TGRAD || (MODE == kModeGrad && DISTILL != 2), "teacher gradient: backward, CE or reverse KL");
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kLossStages; ++i) {
@@ -499,77 +533,118 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
         } else {
           // ---------------- backward: dense part of the logit gradient, bf16
           if (bad && j == 0 && vt == 0 && half == 0) set_flag(a.status, MLS_DEVFLAG_BAD_ID);
-          if (live) {
+          uint8_t* const stage = s.gstage[warp - 2];
+          const int row0 = tt * kBM + q * 32;               // first token row of this warp
+          if (TGRAD && j == 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int k = 0; k < 16; ++k) pt[c][k] = 0u;   // the teacher-gradient accumulator
+          }
+          const float lseT = (hold && valid) ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
+          const float lsT = lseT * kLog2e;
+          if (live && !(TGRAD && j == 0)) {
             const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
             const float ls = lse * kLog2e;
-            // reverse KL: per-token KL(q_m || p_T) = R_m - lse_m + lse_T (R from the forward pass);
-            // Jensen-Shannon: per-token K = KL(q_m || mu) / 2, stored by the forward pass
-            float lseT = 0.f, klt = 0.f;
-            if ((rkl || jsd) && j > 0 && valid) {
-              lseT = a.stats[static_cast<int64_t>(M - 1) * a.T + t];
-              const float st2 = a.stats[static_cast<int64_t>(2 * M + m) * a.T + t];
-              klt = rkl ? st2 - lse + lseT : st2;
-            }
-            // unrolled in the cross-entropy form so that the teacher's packed
-            // probabilities stay in registers (indexed by c)
-            constexpr int kUnrollC = hold ? 1 : 4;
+            // per-token statistic of the student from the forward pass:
+            //   cross-entropy S_m = sum p_T l_m; reverse KL R_m = sum q_m (l_m - l_T), so that
+            //   log q - log p - KL(q_m || p_T) = l_m - l_T - R_m;  Jensen-Shannon: K = KL(q_m || mu) / 2
+            const float klt = (hold && j > 0 && valid) ? a.stats[static_cast<int64_t>(2 * M + m) * a.T + t] : 0.f;
+            const uint32_t wm2 = TGRAD ? pack_p2(a.exit_w[m], a.exit_w[m]) : 0u;
+            // unrolled where a register array is indexed by c (the teacher's
+            // packed probabilities, or the teacher-gradient accumulator)
+            constexpr int kUnrollC = (hold && !TGRAD) ? 1 : 4;
+            // TMEM is read 16 columns at a time when the accumulator is live
+            constexpr int kW = TGRAD ? 16 : 32;
 #pragma unroll kUnrollC
             for (int c = 0; c < 4; ++c) {
-              float r[32];
-              tmem_ld32(base + c * 32, r);
-              float lt[32];
-              if ((rkl || jsd) && j > 0) {
-                tmem_ld32(tbase + c * 32, lt);
-              } else {
-#pragma unroll
-                for (int k = 0; k < 32; ++k) lt[k] = 0.f;
-              }
               uint32_t packed[16];
 #pragma unroll
-              for (int k = 0; k < 32; k += 2) {
-                const float e0 = exp2f(fmaf(r[k], kLog2e, -ls));
-                const float e1 = exp2f(fmaf(r[k + 1], kLog2e, -ls));
+              for (int sub = 0; sub < 32 / kW; ++sub) {
+              float r[kW];
+              tmem_ld<kW>(base + c * 32 + sub * kW, r);
+              float lt[kW];
+              if (hold && j > 0) {
+                tmem_ld<kW>(tbase + c * 32 + sub * kW, lt);
+              } else {
+#pragma unroll
+                for (int k = 0; k < kW; ++k) lt[k] = 0.f;
+              }
+#pragma unroll
+              for (int kk = 0; kk < kW; kk += 2) {
+                const int k = sub * kW + kk;       // column inside the 32-column chunk (pair index k / 2)
+                const float e0 = exp2f(fmaf(r[kk], kLog2e, -ls));
+                const float e1 = exp2f(fmaf(r[kk + 1], kLog2e, -ls));
                 float g0, g1;
                 if (j == 0) {                      // teacher: G' = p_T
                   if (!hold) pt[c][k / 2] = pack_p2(e0, e1);
                   g0 = e0;
                   g1 = e1;
                 } else if (rkl) {                  // student: G' = q ((1 - a) + a (log q - log p - KL))
-                  const float d0 = (r[k] - lse) - (lt[k] - lseT) - klt;
-                  const float d1 = (r[k + 1] - lse) - (lt[k + 1] - lseT) - klt;
+                  const float d0 = (r[kk] - lt[kk]) - klt;
+                  const float d1 = (r[kk + 1] - lt[kk + 1]) - klt;
                   g0 = e0 * fmaf(al, d0, 1.f - al);
                   g1 = e1 * fmaf(al, d1, 1.f - al);
+                  if (TGRAD) pt[c][k / 2] = hfma_p2(wm2, pack_p2(e0, e1), pt[c][k / 2]);   // sum_m w_m q_m
                 } else if (jsd) {                  // student: G' = q ((1 - a) + a (log(q/mu)/2 - K))
-                  const float d0 = fmaf(-0.5f, softplus((lt[k] - lseT) - (r[k] - lse)), 0.5f * kLn2) - klt;
-                  const float d1 = fmaf(-0.5f, softplus((lt[k + 1] - lseT) - (r[k + 1] - lse)), 0.5f * kLn2) - klt;
+                  const float d0 = fmaf(-0.5f, softplus((lt[kk] - lseT) - (r[kk] - lse)), 0.5f * kLn2) - klt;
+                  const float d1 = fmaf(-0.5f, softplus((lt[kk + 1] - lseT) - (r[kk + 1] - lse)), 0.5f * kLn2) - klt;
                   g0 = e0 * fmaf(al, d0, 1.f - al);
                   g1 = e1 * fmaf(al, d1, 1.f - al);
                 } else {                           // student: G' = q - alpha_d p_T
-                  const float2 pp = unpack_p2(pt[c][k / 2]);
-                  g0 = fmaf(-al, pp.x, e0);
-                  g1 = fmaf(-al, pp.y, e1);
+                  float p0, p1;
+                  if (hold) {
+                    p0 = exp2f(fmaf(lt[kk], kLog2e, -lsT));
+                    p1 = exp2f(fmaf(lt[kk + 1], kLog2e, -lsT));
+                  } else {
+                    const float2 pp = unpack_p2(pt[c][k / 2]);
+                    p0 = pp.x;
+                    p1 = pp.y;
+                  }
+                  g0 = fmaf(-al, p0, e0);
+                  g1 = fmaf(-al, p1, e1);
+                  if (TGRAD)                       // sum_m w_m (l_m - S_m)
+                    pt[c][k / 2] = hfma_p2(wm2, pack_p2(r[kk] - klt, r[kk + 1] - klt), pt[c][k / 2]);
                 }
                 packed[k / 2] = bad ? 0u : pack_bf16x2(g0, g1);
               }
-              // transpose through shared memory so that each store instruction
-              // writes 8 rows x 64 contiguous bytes (full sectors)
-              uint8_t* stage = s.gstage[warp - 2];
-              uint4* mine = reinterpret_cast<uint4*>(stage + lane * kStageRowBytes);
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                mine[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
-              __syncwarp();
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int piece = i * 32 + lane;
-                const int r = piece >> 2, ch = piece & 3;
-                const int tr = tt * kBM + q * 32 + r;
-                const uint4 v = *reinterpret_cast<const uint4*>(stage + r * kStageRowBytes + ch * 16);
-                if (tr < a.T)
-                  *reinterpret_cast<uint4*>(a.G + (static_cast<int64_t>(m) * a.T + tr) * a.V + c0 + c * 32 +
-                                            ch * 8) = v;
               }
-              __syncwarp();
+              store_g_chunk(stage, lane, packed, a.G + static_cast<int64_t>(m) * a.T * a.V, row0, a.T, a.V,
+                            c0 + c * 32);
+            }
+          }
+          if (TGRAD && j == M - 1 && j > 0 && live) {
+            // the teacher's G' with every student's distillation gradient:
+            //   cross-entropy: w_T p - a p sum_m w_m (l_m - S_m)
+            //   reverse KL:    (w_T + a sum_m w_m) p - a sum_m w_m q_m
+            const float wT = a.exit_w[M - 1];
+            const float cp = rkl ? fmaf(al, a.student_wsum, wT) : wT;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t packed[16];
+#pragma unroll
+              for (int sub = 0; sub < 2; ++sub) {
+                float lt[16];
+                tmem_ld16(tbase + c * 32 + sub * 16, lt);
+#pragma unroll
+                for (int kk = 0; kk < 16; kk += 2) {
+                  const int k = sub * 16 + kk;
+                  const float p0 = exp2f(fmaf(lt[kk], kLog2e, -lsT));
+                  const float p1 = exp2f(fmaf(lt[kk + 1], kLog2e, -lsT));
+                  const float2 acc = unpack_p2(pt[c][k / 2]);
+                  float g0, g1;
+                  if (rkl) {
+                    g0 = fmaf(-al, acc.x, cp * p0);
+                    g1 = fmaf(-al, acc.y, cp * p1);
+                  } else {
+                    g0 = p0 * fmaf(-al, acc.x, cp);
+                    g1 = p1 * fmaf(-al, acc.y, cp);
+                  }
+                  packed[k / 2] = bad ? 0u : pack_bf16x2(g0, g1);
+                }
+              }
+              store_g_chunk(stage, lane, packed, a.G + static_cast<int64_t>(M - 1) * a.T * a.V, row0, a.T, a.V,
+                            c0 + c * 32);
             }
           }
           tc_fence_before();
@@ -1320,7 +1395,7 @@ TcWs fwd_layout(const LossProblem& p, void* ws) {
   return w;
 }
 
-template <int MODE, int DISTILL>
+template <int MODE, int DISTILL, bool TGRAD = false>
 cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaStream_t st) {
   LossMaps maps;
   for (int m = 0; m < p.M; ++m) {
@@ -1329,7 +1404,7 @@ cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaSt
   }
   LossArgs a = args_in;
   const size_t smem = sizeof(LossSmem) + 1024;
-  auto fn = loss_tile_kernel<MODE, DISTILL>;
+  auto fn = loss_tile_kernel<MODE, DISTILL, TGRAD>;
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
@@ -1351,6 +1426,9 @@ LossArgs base_args(const LossProblem& p) {
   a.y = p.y;
   a.alpha = p.alpha_d;
   a.distill = p.distill;
+  for (int m = 0; m < p.M; ++m) a.exit_w[m] = p.exit_w[m];
+  a.student_wsum = 0.f;
+  for (int m = 0; m + 1 < p.M; ++m) a.student_wsum += p.exit_w[m];
   a.status = p.status;
   return a;
 }
@@ -1408,6 +1486,8 @@ cudaError_t run_dh_all(const LossProblem& p, const __nv_bfloat16* G, void* const
   g.Mdim = static_cast<int>(p.T);
   g.Kdim = static_cast<int>(p.V);
   for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
+  const bool tgrad = p.teacher_grad != 0 && p.M > 1;
+  if (tgrad) g.alpha[p.M - 1] = alpha;             // the teacher's G' already carries w_T
   g.status = p.status;
   g.onehot_idx = p.y;
   g.onehot_limit = static_cast<int>(p.V);
@@ -1418,7 +1498,7 @@ cudaError_t run_dh_all(const LossProblem& p, const __nv_bfloat16* G, void* const
     g.Ndim[m] = static_cast<int>(p.D[m]);
     g.out[m] = dh[m];
     g.onehot_rows[m] = static_cast<const __nv_bfloat16*>(p.W[m]);
-    g.onehot_coef[m] = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
+    g.onehot_coef[m] = (m == p.M - 1) ? (tgrad ? p.exit_w[m] : 1.f) : 1.f - p.alpha_d;
   }
   return run_gemm<false, true, BN, true>(maps, g, st);
 }
@@ -1434,6 +1514,7 @@ cudaError_t run_dw_all(const LossProblem& p, const __nv_bfloat16* G, float* cons
   g.Mdim = static_cast<int>(p.V);
   g.Kdim = static_cast<int>(p.T);
   for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
+  if (p.teacher_grad != 0 && p.M > 1) g.alpha[p.M - 1] = alpha;   // the teacher's G' already carries w_T
   g.accumulate = accumulate;
   g.status = p.status;
   for (int m = 0; m < p.M; ++m) {
@@ -1523,7 +1604,10 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   LossArgs a = base_args(p);
   a.stats = const_cast<float*>(stats);
   a.G = G;
-  cudaError_t err = p.distill == 1   ? run_loss_tiles<kModeGrad, 1>(p, a, st)
+  const bool tgrad = p.teacher_grad != 0 && p.M > 1;
+  cudaError_t err = tgrad ? (p.distill == 1 ? run_loss_tiles<kModeGrad, 1, true>(p, a, st)
+                                            : run_loss_tiles<kModeGrad, 0, true>(p, a, st))
+                    : p.distill == 1 ? run_loss_tiles<kModeGrad, 1>(p, a, st)
                     : p.distill == 2 ? run_loss_tiles<kModeGrad, 2>(p, a, st)
                                      : run_loss_tiles<kModeGrad, 0>(p, a, st);
   if (err != cudaSuccess) return err;

@@ -22,25 +22,27 @@ def _gpu_inputs(d):
     return y, h, W
 
 
-def _oracle(d, alpha, grad_scale=1.0, rows=None, need_grad=True, exit_weights=None, distill="ce"):
+def _oracle(d, alpha, grad_scale=1.0, rows=None, need_grad=True, exit_weights=None, distill="ce",
+            teacher_grad=False):
     return oracle.multiexit_loss(d.y, d.o, d.W, alpha_d=alpha, grad_scale=grad_scale, rows=rows,
-                                 need_grad=need_grad, exit_weights=exit_weights, distill=distill)
+                                 need_grad=need_grad, exit_weights=exit_weights, distill=distill,
+                                 teacher_grad=teacher_grad)
 
 
 def _losses_expected(r, M):
     return np.concatenate([r["ce_lm"], r["ce_kd"], [r["loss"]]])
 
 
-def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce"):
+def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce", teacher_grad=False):
     cfg = d.cfg
     M = cfg.M
     y, h, W = _gpu_inputs(d)
     st = new_status()
     losses, stats = multiexit_loss_fwd(y, h, W, alpha, status=st, exit_weights=exit_weights, distill=distill)
     dh, dW = multiexit_loss_bwd(y, h, W, stats, alpha, grad_scale, status=st, exit_weights=exit_weights,
-                                distill=distill)
+                                distill=distill, teacher_grad=teacher_grad)
     assert status_read(st) == (0, 0)
-    r = _oracle(d, alpha, grad_scale, exit_weights=exit_weights, distill=distill)
+    r = _oracle(d, alpha, grad_scale, exit_weights=exit_weights, distill=distill, teacher_grad=teacher_grad)
     assert_loss_close(losses, _losses_expected(r, M), "losses")
     s = f64(stats)
     assert_stats_close(s[:M], r["lse"], "lse")
@@ -96,6 +98,28 @@ def test_alternative_distillation(name, small, distill):
     d = wl.make_inputs(cfg, with_tables=False)
     _check_all(d, 0.3, 1.0, distill=distill)
     _check_all(d, 0.6, 2.0, exit_weights=[1.5, 0.5] + [1.0] * (cfg.M - 2), distill=distill)
+
+
+@pytest.mark.parametrize("name,small", [("tiny3", None), ("main3", dict(batch=1, seq=200, V=512)),
+                                        ("suite4", dict(batch=1, seq=130, V=384)),
+                                        ("main3_aligned", dict(batch=1, seq=256, V=768))])
+@pytest.mark.parametrize("distill", ["ce", "reverse_kl"])
+def test_teacher_gradient(name, small, distill):
+    cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
+    d = wl.make_inputs(cfg, with_tables=False)
+    _check_all(d, 0.3, 1.0, distill=distill, teacher_grad=True)
+    _check_all(d, 0.6, 2.0, exit_weights=[1.5, 0.5] + [1.0] * (cfg.M - 3) + [0.8], distill=distill,
+               teacher_grad=True)
+
+
+def test_teacher_gradient_rejected_with_js():
+    from lm_head_loss_junction_b200._lib import MLSError
+    cfg = wl.small_variant(wl.CONFIGS["main3"], batch=1, seq=128, V=256)
+    d = wl.make_inputs(cfg, with_tables=False)
+    y, h, W = _gpu_inputs(d)
+    _, stats = multiexit_loss_fwd(y, h, W, 0.3, distill="js")
+    with pytest.raises(MLSError):
+        multiexit_loss_bwd(y, h, W, stats, 0.3, distill="js", teacher_grad=True)
 
 
 def test_single_exit_and_accumulate():
