@@ -43,6 +43,9 @@ struct SegIndexDev {
   const int32_t* heavy;      // ids with many tokens
   const int32_t* n_heavy;
   int64_t max_heavy;
+  const int32_t* light;      // ids with 1..kHeavy tokens (any order)
+  const int32_t* n_light;
+  int64_t max_light;
 };
 
 size_t segindex_bytes(int64_t T, int64_t V);

@@ -673,23 +673,24 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
 
 // ------------------------------------------------------------------ merge kernel
 // Per token: combine the per-split partials into lse_m and S_m, write the stats
-// rows and the per-token loss terms.  A block covers 32 tokens; its 8 thread
-// rows each merge a contiguous range of splits, and the 8 results are combined
-// in row order (deterministic).
-constexpr int kMergeRows = 8;
+// rows and the per-token loss terms.  A block covers 32 tokens; each of its
+// thread rows merges a contiguous range of splits, and the rows' results are
+// combined in row order (deterministic).
+constexpr int kLossMergeRows = 32;   // thread rows per 32-token block of the loss merge
+constexpr int kMergeRows = 16;       // ... of the agreement and Jensen-Shannon merges
 
-__global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float* __restrict__ partial, int n_splits,
+__global__ void __launch_bounds__(32 * kLossMergeRows) loss_merge_kernel(const float* __restrict__ partial, int n_splits,
                                                                      int M, int T, int V, int distill,
                                                                      const int32_t* __restrict__ y,
                                                                      float* __restrict__ stats,
                                                                      float* __restrict__ terms, int32_t* status) {
   constexpr int S = kMaxExits - 1;
-  __shared__ float st_mT[kMergeRows][32], st_zT[kMergeRows][32];
-  __shared__ float st_A[kMergeRows][S][32], st_ms[kMergeRows][S][32], st_zs[kMergeRows][S][32];
+  __shared__ float st_mT[kLossMergeRows][32], st_zT[kLossMergeRows][32];
+  __shared__ float st_A[kLossMergeRows][S][32], st_ms[kLossMergeRows][S][32], st_zs[kLossMergeRows][S][32];
   const int lane = threadIdx.x, rowi = threadIdx.y;
   const int t = blockIdx.x * 32 + lane;
   const int Q = 2 * M - 1;
-  const int per = (n_splits + kMergeRows - 1) / kMergeRows;
+  const int per = (n_splits + kLossMergeRows - 1) / kLossMergeRows;
   const int i0 = min(n_splits, rowi * per), i1 = min(n_splits, i0 + per);
   float mT = -INFINITY, zT = 0.f;
   float A[S] = {0.f, 0.f, 0.f}, ms[S] = {-INFINITY, -INFINITY, -INFINITY}, zs[S] = {0.f, 0.f, 0.f};
@@ -733,7 +734,7 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
   }
   __syncthreads();
   if (rowi != 0 || t >= T) return;
-  for (int r = 1; r < kMergeRows; ++r) {
+  for (int r = 1; r < kLossMergeRows; ++r) {
     const float m2 = st_mT[r][lane], z2 = st_zT[r][lane];
     const float mm = fmaxf(mT, m2);
     const float r1 = (mT == -INFINITY) ? 0.f : __expf(mT - mm);
@@ -775,8 +776,8 @@ __global__ void __launch_bounds__(32 * kMergeRows) loss_merge_kernel(const float
 // ------------------------------------------------------------------ agreement merge
 // Per token: sums over the splits of beta and KL (plain sums: the agreement
 // pass uses the final normalisers), the first maximum over the splits in
-// vocabulary order, and the top-1 agreement.  Same 32-token x 8-row block
-// layout as the loss merge.
+// vocabulary order, and the top-1 agreement.  Blocks of 32 tokens x 16 thread
+// rows.
 __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const float* __restrict__ partial,
                                                                       int n_splits, int M, int T,
                                                                       float* __restrict__ terms,
@@ -1578,7 +1579,7 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   cudaError_t err = p.distill == 1 ? run_loss_tiles<kModeStats, 1>(p, a, st) : run_loss_tiles<kModeStats, 0>(p, a, st);
   if (err != cudaSuccess) return err;
   const int T = static_cast<int>(p.T);
-  loss_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
+  loss_merge_kernel<<<(T + 31) / 32, dim3(32, kLossMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
                                                                      static_cast<int>(p.V), p.distill, p.y, stats,
                                                                      w.terms, p.status);
   note_launches(1);

@@ -7,7 +7,11 @@
 // fixed order: results are bitwise reproducible, with no floating-point
 // atomics.  Rows with few tokens are reduced by one warp; rows with many
 // (Zipf-frequent ids) by a whole block whose warps split the tokens and are
-// combined in warp order.
+// combined in warp order.  The ids present are listed (light and heavy) so
+// that no warp is spent on absent ids; each row slice is still summed by one
+// warp in token order, so the list order does not change any result.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -130,18 +134,21 @@ __global__ void __launch_bounds__(kSortBlock) sort_scatter_kernel(
 
 // Segment bounds from the sorted keys: offsets[v] = first position of id v,
 // ends[v] = one past its last (both 0 for absent ids, preset by a memset).
-// Ids with more than kHeavy tokens are appended to the heavy list; its order
-// does not matter, every row is reduced independently in a fixed order.
+// Ids with more than kHeavy tokens are appended to the heavy list, the others
+// present to the light list; list order does not matter, every row is reduced
+// independently in a fixed order.  counts[0] = heavy ids, counts[1] = light ids.
 __global__ void segment_bounds_kernel(const int32_t* __restrict__ keys, int64_t n, int64_t V,
                                       int32_t* __restrict__ offsets, int32_t* __restrict__ ends,
-                                      int32_t* __restrict__ heavy, int32_t* __restrict__ n_heavy) {
+                                      int32_t* __restrict__ heavy, int32_t* __restrict__ light,
+                                      int32_t* __restrict__ counts) {
   const int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (p >= n) return;
   const int32_t k = keys[p];
   if (k >= V) return;                                    // invalid ids sort last
   if (p == 0 || keys[p - 1] != k) {
     offsets[k] = static_cast<int32_t>(p);
-    if (p + kHeavy < n && keys[p + kHeavy] == k) heavy[atomicAdd(n_heavy, 1)] = k;
+    if (p + kHeavy < n && keys[p + kHeavy] == k) heavy[atomicAdd(counts, 1)] = k;
+    else light[atomicAdd(counts + 1, 1)] = k;
   }
   if (p == n - 1 || keys[p + 1] != k) ends[k] = static_cast<int32_t>(p + 1);
 }
@@ -205,7 +212,8 @@ __device__ __forceinline__ void emit(float* out_row, int vi, const float (&acc)[
   }
 }
 
-// One warp per id row (light rows, and the zero rows of table mode).
+// Light rows: warp w of block (x, y) takes light ids x*8 + w, x*8 + w + 8*gridDim.x, ...
+// and their slice y of 32 vectors (one 16-byte vector per lane).
 //   src row of token t: src + t*src_ld + src_off (16-byte vectors)
 template <bool BF16, bool TABLE>
 __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix, const uint4* __restrict__ src,
@@ -215,24 +223,18 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
                                                            float scale, int accumulate) {
   constexpr int N = Vec8<BF16>::N;
   const int lane = threadIdx.x & 31;
-  const int64_t v = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (v >= ix.V) return;
-  const int32_t off = ix.offsets[v];
-  const int32_t cnt = ix.ends[v] - off;
-  if (cnt > kHeavy) return;                   // handled by the heavy kernel
-  if (cnt == 0 && (!TABLE || accumulate)) return;   // nothing to add
-  float* out_row = out + v * static_cast<int64_t>(n_vec) * N;
-  if (cnt == 0) {                             // overwrite mode: the row of an unused id is zero
-    float4* o4 = reinterpret_cast<float4*>(out_row);
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = lane; i < n_vec * (N / 4); i += 32) o4[i] = z;
-    return;
-  }
-  const uint4* E_row = TABLE ? E + v * static_cast<int64_t>(n_vec) : nullptr;
-  float cs = 0.f;
-  if (TABLE)
-    for (int p = 0; p < cnt; ++p) cs += coef[ix.toks[off + p]];
-  for (int vi = lane; vi < n_vec; vi += 32) {
+  const int warp = threadIdx.x >> 5;
+  const int vi = static_cast<int>(blockIdx.y) * 32 + lane;
+  const bool active = vi < n_vec;
+  const int n_light = *ix.n_light;
+  for (int i = static_cast<int>(blockIdx.x) * 8 + warp; i < n_light; i += static_cast<int>(gridDim.x) * 8) {
+    const int64_t v = ix.light[i];
+    const int32_t off = ix.offsets[v];
+    const int32_t cnt = ix.ends[v] - off;
+    float cs = 0.f;
+    if (TABLE)
+      for (int p = 0; p < cnt; ++p) cs += coef[ix.toks[off + p]];
+    if (!active) continue;
     float acc[N];
 #pragma unroll
     for (int k = 0; k < N; ++k) acc[k] = 0.f;
@@ -246,8 +248,22 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
       for (int b = 0; b < 4; ++b) Vec8<BF16>::add(acc, u[b]);
     }
     for (; p < cnt; ++p) Vec8<BF16>::add(acc, __ldg(src + static_cast<int64_t>(ix.toks[off + p]) * src_ld + src_off + vi));
+    float* out_row = out + v * static_cast<int64_t>(n_vec) * N;
+    const uint4* E_row = TABLE ? E + v * static_cast<int64_t>(n_vec) : nullptr;
     emit<BF16, TABLE>(out_row, vi, acc, cs, E_row, scale, accumulate != 0);
   }
+}
+
+// Overwrite mode of the table gradient: the rows of absent ids are zero.  One
+// warp per row; rows of present ids are left to the light and heavy kernels.
+__global__ void __launch_bounds__(256) zero_absent_rows_kernel(const SegIndexDev ix, float4* __restrict__ out,
+                                                               int f4_per_row) {
+  const int lane = threadIdx.x & 31;
+  const int64_t v = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (v >= ix.V || ix.ends[v] != 0) return;               // present ids have ends > 0
+  float4* o = out + v * f4_per_row;
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = lane; i < f4_per_row; i += 32) o[i] = z;
 }
 
 // One block per (heavy row, slice of 32 vectors); warps split the row's tokens
@@ -317,10 +333,23 @@ template <bool BF16, bool TABLE>
 cudaError_t launch_segsum(const SegIndexDev& ix, const uint4* src, int64_t src_ld, int src_off, int n_vec,
                           const float* coef, const uint4* E, float* out, float scale, int accumulate,
                           cudaStream_t st) {
-  const int64_t blocks = (ix.V * 32 + 255) / 256;
-  segsum_light_kernel<BF16, TABLE><<<static_cast<unsigned>(blocks), 256, 0, st>>>(ix, src, src_ld, src_off, n_vec,
-                                                                                 coef, E, out, scale, accumulate);
-  dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>((n_vec + 31) / 32));
+  constexpr int N = Vec8<BF16>::N;
+  if (TABLE && !accumulate) {
+    const int64_t blocks = (ix.V * 32 + 255) / 256;
+    zero_absent_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(ix, reinterpret_cast<float4*>(out),
+                                                                          n_vec * N / 4);
+    note_launches(1);
+  }
+  // light rows: about one full wave of 8-warp blocks over (light ids) x (32-vector slices)
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int slices = (n_vec + 31) / 32;
+  const int64_t want = (static_cast<int64_t>(sms) * 8 + slices - 1) / slices;
+  const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(want, (ix.max_light + 7) / 8));
+  segsum_light_kernel<BF16, TABLE><<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices)), 256, 0, st>>>(
+      ix, src, src_ld, src_off, n_vec, coef, E, out, scale, accumulate);
+  dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>(slices));
   segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, src, src_ld, src_off, n_vec, coef, E,
                                                                       out, scale, accumulate);
   note_launches(2);
@@ -333,8 +362,9 @@ size_t segindex_bytes(int64_t T, int64_t V) {
   const int64_t nblk = (T + kSortBlock - 1) / kSortBlock;
   const size_t t4 = static_cast<size_t>(T) * 4;
   const int64_t max_heavy = T / (kHeavy + 1) + 1;
+  const int64_t max_light = T < V ? T : V;
   return up256(t4) * 4 + up256(static_cast<size_t>(256) * nblk * 4) + up256(static_cast<size_t>(V) * 4) * 2 +
-         up256(static_cast<size_t>(max_heavy) * 4) + 256;
+         up256(static_cast<size_t>(max_heavy) * 4) + up256(static_cast<size_t>(max_light) * 4) + 256;
 }
 
 cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, SegIndexDev* out, cudaStream_t st) {
@@ -349,8 +379,10 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
   int32_t* offsets = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V) * 4);
   int32_t* ends = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(V) * 4);
   const int64_t max_heavy = T / (kHeavy + 1) + 1;
+  const int64_t max_light = T < V ? T : V;
   int32_t* heavy = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(max_heavy) * 4);
-  int32_t* n_heavy = reinterpret_cast<int32_t*>(p);
+  int32_t* light = reinterpret_cast<int32_t*>(p); p += up256(static_cast<size_t>(max_light) * 4);
+  int32_t* counts = reinterpret_cast<int32_t*>(p);        // [0] heavy ids, [1] light ids
 
   // stable radix sort of the ids carrying token indices
   int bits = 1;
@@ -373,18 +405,21 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
   // per-id segment bounds in sorted order, and the heavy ids
   cudaError_t err = cudaMemsetAsync(offsets, 0, static_cast<size_t>(V) * 4, st);
   if (err == cudaSuccess) err = cudaMemsetAsync(ends, 0, static_cast<size_t>(V) * 4, st);
-  if (err == cudaSuccess) err = cudaMemsetAsync(n_heavy, 0, 4, st);
+  if (err == cudaSuccess) err = cudaMemsetAsync(counts, 0, 8, st);
   if (err != cudaSuccess) return err;
   segment_bounds_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(kin, T, V, offsets, ends, heavy,
-                                                                                n_heavy);
+                                                                                light, counts);
   note_launches(1);
   out->V = V;
   out->ends = ends;
   out->offsets = offsets;
   out->toks = vin;
   out->heavy = heavy;
-  out->n_heavy = n_heavy;
+  out->n_heavy = counts;
   out->max_heavy = max_heavy;
+  out->light = light;
+  out->n_light = counts + 1;
+  out->max_light = max_light;
   return cudaGetLastError();
 }
 
