@@ -223,6 +223,30 @@ def _dist_env():
     return ws, rank, local
 
 
+def grad_sync(tensors, mode: str, ws: int, shards=None):
+    """Data-parallel exchange of the step's parameter gradients (dW^m of every
+    head, dE of every residual table) over the process group: "allreduce" sums
+    them on every rank; "reduce_scatter" leaves rank r the sum of its 1/ws
+    slice of each flattened gradient (a sharded optimizer's input) in
+    shards[i].  Every rank issues the same collectives in the same order."""
+    if ws == 1 or mode == "none":
+        return
+    import torch.distributed as dist
+    for i, t in enumerate(tensors):
+        if mode == "allreduce":
+            dist.all_reduce(t)
+        else:
+            dist.reduce_scatter_tensor(shards[i], t.view(-1))
+
+
+def grad_shards(tensors, ws: int):
+    """Output buffers of the reduce-scatter (each flattened gradient must split evenly)."""
+    for t in tensors:
+        if t.numel() % ws:
+            raise ValueError(f"gradient of {t.numel()} elements does not split over {ws} ranks")
+    return [torch.empty(t.numel() // ws, dtype=t.dtype, device=t.device) for t in tensors]
+
+
 def _max_over_ranks(v: float, ws: int, device) -> float:
     if ws == 1:
         return v
@@ -303,6 +327,8 @@ def main():
                     help="run the workload with this many tokens per GPU instead of its own batch")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step from Python instead of replaying a captured CUDA graph")
+    ap.add_argument("--grad-sync", default="none", choices=["none", "allreduce", "reduce_scatter"],
+                    help="with more than one rank, exchange dW and dE over NCCL inside every step")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = wl.CONFIGS[args.workload]
@@ -357,14 +383,21 @@ def main():
                 f(None)
             graphs.append(g)
         runners = [g.replay for g in graphs]
-        for _ in range(2):
-            for r in runners:
-                r()
+    # the data-parallel gradient exchange (eager NCCL calls), when asked for
+    sync_on = ws > 1 and args.grad_sync != "none"
+    grads = step.dW + step.dE
+    shards = grad_shards(grads, ws) if sync_on and args.grad_sync == "reduce_scatter" else None
+    if sync_on:
+        runners.append(lambda: grad_sync(grads, args.grad_sync, ws, shards))
+    for _ in range(2):
+        for r in runners:
+            r()
     barrier()
 
     # ---------------- timed region: K steps, events between phases
     K = args.steps
-    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    NP = len(runners)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(NP + 1)] for _ in range(K)]
     barrier()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -374,14 +407,14 @@ def main():
             for i, r in enumerate(runners):
                 marks[k][i].record(stream)
                 r()
-            marks[k][4].record(stream)
+            marks[k][NP].record(stream)
         end.record(stream)
         barrier()
     launches = launches_per_step * K
     ms_total = start.elapsed_time(end)
     ms_total = _max_over_ranks(ms_total, ws, device)
     ms_step = ms_total / K
-    phase_ms = [statistics.mean(marks[k][i].elapsed_time(marks[k][i + 1]) for k in range(K)) for i in range(4)]
+    phase_ms = [statistics.mean(marks[k][i].elapsed_time(marks[k][i + 1]) for k in range(K)) for i in range(NP)]
     code, word = step.api.status_read(step.status, stream)
     if code != 0:
         raise RuntimeError(f"device status after timing: {code} ({word})")
@@ -405,7 +438,11 @@ def main():
             step.run(s)
             host_out.copy_(step.losses, non_blocking=True)
 
-        if args.eager:
+        if sync_on:                      # the collective stays outside the graph
+            def e2e_run():
+                e2e_step(stream)
+                grad_sync(grads, args.grad_sync, ws, shards)
+        elif args.eager:
             e2e_run = lambda: e2e_step(stream)  # noqa: E731
         else:
             ge = torch.cuda.CUDAGraph()
@@ -475,6 +512,10 @@ def main():
         "junction_fwd_frac_of_hbm": jf_bytes / (phase_ms[0] / 1000.0) / 1e9 / hbm if c.M > 1 else None,
         "junction_bwd_gbs_incl_scatter": jb_bytes / (phase_ms[3] / 1000.0) / 1e9 if c.M > 1 else None,
     }
+    if sync_on:
+        gbytes = sum(t.numel() * t.element_size() for t in grads)
+        phases["grad_sync_ms"] = phase_ms[4]
+        phases["grad_sync_bytes"] = gbytes
     roofline = {"bound": "tensor", "achieved": ach_fwd, "peak": peak_tc, "unit": "TFLOP/s",
                 "frac": ach_fwd / peak_tc, "traffic": measured_traffic(c),
                 "kernel": "loss_tile_kernel<stats> (mls_multiexit_loss_fwd call: tile kernel + merge + reduce)",
@@ -496,7 +537,8 @@ def main():
             "dtype": "bf16" if c.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": c.name, "global_batch": c.batch * ws, "seq_len": c.seq, "tokens_per_gpu": c.T,
                        "M": c.M, "D": list(c.D), "V": c.V, "alpha_d": c.alpha_d,
-                       "parallelism": f"dp{ws} (independent batches)",
+                       "parallelism": f"dp{ws} (independent batches)" if not sync_on else
+                                      f"dp{ws} (dW and dE {args.grad_sync} over NCCL every step)",
                        "l2": f"no flush; per-step working set {step.working_set_gb():.2f} GB > 126 MB L2"},
             "e2e": e2e, "gpu_launches": int(launches), "launch_mode": "eager" if args.eager else "cuda_graph",
             "roofline": roofline, "cpu_baseline": cpu,
