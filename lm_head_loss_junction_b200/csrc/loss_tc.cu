@@ -48,7 +48,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // TMEM lane quadrant, each owning one 128-column half ("split") of the tile.
 constexpr int kLossBN = 256;
 constexpr int kSplitCols = 128;
-constexpr int kLossStages = 4;
+constexpr int kLossStages = 4;        // single CTA: 48 KB per stage
+constexpr int kLossPairStages = 6;    // CTA pair: 32 KB per stage and CTA
 constexpr int kLossEpiWarps = 8;
 constexpr int kLossThreads = 64 + 32 * kLossEpiWarps;
 
@@ -79,12 +80,17 @@ struct LossArgs {
 // to 80 bytes so the 16-byte writes of a warp hit every bank once per pass).
 constexpr int kStageRowBytes = 80;
 
+// PAIR: two CTAs share each 256-token x 256-vocabulary MMA (cta_group::2);
+// each loads its own 128 token rows and half (128 rows) of the W tile.
+template <bool PAIR>
 struct __align__(1024) LossSmem {
-  uint8_t a[kLossStages][kBM * kBK * 2];
-  uint8_t b[kLossStages][kLossBN * kBK * 2];
+  static constexpr int kStages = PAIR ? kLossPairStages : kLossStages;
+  static constexpr int kBRows = PAIR ? kLossBN / 2 : kLossBN;
+  uint8_t a[kStages][kBM * kBK * 2];
+  uint8_t b[kStages][kBRows * kBK * 2];
   uint8_t gstage[kLossEpiWarps][32 * kStageRowBytes];
-  uint64_t full[kLossStages];
-  uint64_t empty[kLossStages];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -192,15 +198,31 @@ __device__ __forceinline__ void store_g_chunk(uint8_t* stage, int lane, const ui
 // region 0 while the students pass through region 1, accumulates each
 // student's contribution to the teacher's logit gradient in registers (fp16
 // pairs), and writes the teacher's G' after the last student.
-template <int MODE, int DISTILL, bool TGRAD = false>
+//
+// PAIR (launched as clusters of two CTAs): the pair's tile is 256 tokens x 256
+// vocabulary columns; CTA rank r owns tokens [128 r, 128 r + 128) of it in its
+// TMEM and shared memory, loads half of the W tile, and runs the same
+// epilogue on its rows.  The leader (rank 0) issues the MMAs (M = 256) and
+// commits to both CTAs' barriers; both CTAs' loads complete on the leader's
+// stage barriers, and both CTAs' epilogue warps release the leader's TMEM
+// regions.  Halving each SM's share of the W tile cuts its shared-memory and
+// L2 operand traffic per flop by a third.
+template <int MODE, int DISTILL, bool TGRAD = false, bool PAIR = false>
 __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid_constant__ LossMaps maps,
                                                                     const LossArgs a) {
+  using Smem = LossSmem<PAIR>;
+  constexpr int kStages = Smem::kStages;
+  constexpr int kTileRows = PAIR ? 2 * kBM : kBM;      // tokens per tile
   extern __shared__ uint8_t smem_raw[];
-  LossSmem& s = *reinterpret_cast<LossSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort;
   const int M = a.M;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int slot = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nslots = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   constexpr bool rkl = (DISTILL == 1);
   constexpr bool jsd = (DISTILL == 2);
   // The statistics of the Jensen-Shannon form are the cross-entropy ones (it
@@ -209,13 +231,13 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   static_assert(!TGRAD || (MODE == kModeGrad && DISTILL != 2), "teacher gradient: backward, CE or reverse KL");
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kLossStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
     for (int r = 0; r < 2; ++r) {
       mbar_init(&s.tfull[r], 1);
-      mbar_init(&s.tempty[r], kLossEpiWarps);
+      mbar_init(&s.tempty[r], PAIR ? 2 * kLossEpiWarps : kLossEpiWarps);
     }
     mbar_init(&s.drain, 1);
     s.abort = 0;
@@ -228,51 +250,84 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     }
   }
   if (warp == 1) {
-    tmem_alloc(&s.tmem_base, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(&s.tmem_base, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&s.tmem_base, 512);
+      tmem_relinquish();
+    }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  if constexpr (PAIR) {
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();        // every barrier of both CTAs exists before any remote arrive
+    tc_fence_after();
+  } else {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
   const uint32_t tmem = s.tmem_base;
+  // an epilogue warp is done with TMEM region r (the leader's barrier counts both CTAs)
+  auto release_region = [&](uint32_t r) {
+    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[r]), 0));
+    else mbar_arrive(&s.tempty[r]);
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x) {
+      for (int tile = slot; tile < a.num_tiles && ok; tile += nslots) {
         int tt, vt;
         loss_tile_coords(tile, a, tt, vt);
+        const int row0 = tt * kTileRows + static_cast<int>(rank) * kBM;                // this CTA's tokens
+        const int v0 = vt * kLossBN + static_cast<int>(rank) * Smem::kBRows;           // this CTA's W rows
         for (int j = 0; j < M && ok; ++j) {
           const int m = M - 1 - j;                // teacher first, then students
           for (int kb = 0; kb < a.kblocks[m]; ++kb) {
             if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, a.status)) { ok = false; break; }
-            mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
-            tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, tt * kBM);
-            tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, vt * kLossBN);
+            if constexpr (PAIR) {
+              const uint32_t lfull = mapa_shared(smem_u32(&s.full[stage]), 0);
+              if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * (kBM + Smem::kBRows) * kBK * 2);
+              tma_load_2d_pair(&maps.h[m], lfull, s.a[stage], kb * kBK, row0);
+              tma_load_2d_pair(&maps.w[m], lfull, s.b[stage], kb * kBK, v0);
+            } else {
+              mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
+              tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0);
+              tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0);
+            }
             ++issued;
-            if (++stage == kLossStages) { stage = 0; phase ^= 1; }
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
           }
         }
       }
       if (!ok) {
-        // Let every load already issued land before the CTA can exit.
-        const uint32_t n = issued < kLossStages ? issued : kLossStages;
-        uint32_t st = stage, ph = phase;
-        for (uint32_t i = 0; i < n; ++i) {
-          if (st == 0) { st = kLossStages - 1; ph ^= 1; } else { --st; }
-          drain_wait(&s.full[st], ph, a.status);
+        if constexpr (PAIR) {
+          // This CTA's loads complete on the leader's barriers; give them time to land.
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 2000000ull) {
+          }
+        } else {
+          // Let every load already issued land before the CTA can exit.
+          const uint32_t n = issued < kStages ? issued : kStages;
+          uint32_t st = stage, ph = phase;
+          for (uint32_t i = 0; i < n; ++i) {
+            if (st == 0) { st = kStages - 1; ph ^= 1; } else { --st; }
+            drain_wait(&s.full[st], ph, a.status);
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, kLossBN, false, false);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16(kTileRows, kLossBN, false, false);
       uint32_t stage = 0, phase = 0, job = 0, tile_iter = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < a.num_tiles && ok; tile += gridDim.x, ++tile_iter) {
+      for (int tile = slot; tile < a.num_tiles && ok; tile += nslots, ++tile_iter) {
         for (int j = 0; j < M && ok; ++j, ++job) {
           const int m = M - 1 - j;
           uint32_t region, use;
@@ -288,17 +343,36 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
 #pragma unroll
             for (int k = 0; k < kBK / kUK; ++k) {
               // +32 bytes along K inside the 128-byte swizzled row
-              umma_bf16(d, da + static_cast<uint64_t>(k * 2), db + static_cast<uint64_t>(k * 2), idesc,
-                        (kb | k) != 0);
+              if constexpr (PAIR)
+                umma_bf16_pair(d, da + static_cast<uint64_t>(k * 2), db + static_cast<uint64_t>(k * 2), idesc,
+                               (kb | k) != 0);
+              else
+                umma_bf16(d, da + static_cast<uint64_t>(k * 2), db + static_cast<uint64_t>(k * 2), idesc,
+                          (kb | k) != 0);
             }
-            umma_commit(&s.empty[stage]);
-            if (++stage == kLossStages) { stage = 0; phase ^= 1; }
+            if constexpr (PAIR) {
+              const uint32_t e = smem_u32(&s.empty[stage]);
+              umma_commit_pair(mapa_shared(e, 0));
+              umma_commit_pair(mapa_shared(e, 1));
+            } else {
+              umma_commit(&s.empty[stage]);
+            }
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
           }
-          if (ok) umma_commit(&s.tfull[region]);
+          if (ok) {
+            if constexpr (PAIR) {
+              const uint32_t f = smem_u32(&s.tfull[region]);
+              umma_commit_pair(mapa_shared(f, 0));
+              umma_commit_pair(mapa_shared(f, 1));
+            } else {
+              umma_commit(&s.tfull[region]);
+            }
+          }
         }
       }
       // Make sure every MMA issued has finished before TMEM is released.
-      umma_commit(&s.drain);
+      if constexpr (PAIR) umma_commit_pair(mapa_shared(smem_u32(&s.drain), 0));
+      else umma_commit(&s.drain);
       drain_wait(&s.drain, 0, a.status);
     }
   } else {
@@ -313,10 +387,11 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     // teacher probabilities of this thread's row and split, packed fp16 pairs
     uint32_t pt[4][16];
     float inv_z = 0.f;
-    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x, ++tile_iter) {
+    for (int tile = slot; tile < a.num_tiles; tile += nslots, ++tile_iter) {
       int tt, vt;
       loss_tile_coords(tile, a, tt, vt);
-      const int t = tt * kBM + row;
+      const int rbase = tt * kTileRows + static_cast<int>(rank) * kBM;   // first token of this CTA's rows
+      const int t = rbase + row;
       const bool valid = t < a.T;
       const int c0 = vt * kLossBN + half * kSplitCols;     // first vocabulary column of the split
       const bool live = c0 < a.V;                           // the last tile may be half outside V
@@ -437,10 +512,10 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           __syncwarp();
           if (lane == 0) {
             if (!hold) {
-              mbar_arrive(&s.tempty[region]);
+              release_region(region);
             } else {
-              if (j > 0) mbar_arrive(&s.tempty[1]);         // this student's region
-              if (j == M - 1) mbar_arrive(&s.tempty[0]);    // the teacher's, after the last student
+              if (j > 0) release_region(1);         // this student's region
+              if (j == M - 1) release_region(0);    // the teacher's, after the last student
             }
           }
           if (valid) {
@@ -482,8 +557,8 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
-            if (j > 0) mbar_arrive(&s.tempty[1]);         // this student's region
-            if (j == M - 1) mbar_arrive(&s.tempty[0]);    // the teacher's, after the last student
+            if (j > 0) release_region(1);         // this student's region
+            if (j == M - 1) release_region(0);    // the teacher's, after the last student
           }
           if (valid) {
             const int QA = agree_rows(M);
@@ -522,8 +597,8 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
-            if (j > 0) mbar_arrive(&s.tempty[1]);
-            if (j == M - 1) mbar_arrive(&s.tempty[0]);
+            if (j > 0) release_region(1);
+            if (j == M - 1) release_region(0);
           }
           if (valid && j > 0) {
             float* prow = a.partial + static_cast<int64_t>(split) * js_rows(M) * a.T + t;
@@ -534,7 +609,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           // ---------------- backward: dense part of the logit gradient, bf16
           if (bad && j == 0 && vt == 0 && half == 0) set_flag(a.status, MLS_DEVFLAG_BAD_ID);
           uint8_t* const stage = s.gstage[warp - 2];
-          const int row0 = tt * kBM + q * 32;               // first token row of this warp
+          const int row0 = rbase + q * 32;                   // first token row of this warp
           if (TGRAD && j == 0) {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -651,10 +726,10 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           __syncwarp();
           if (lane == 0) {
             if (!hold) {
-              mbar_arrive(&s.tempty[region]);
+              release_region(region);
             } else {
-              if (j > 0) mbar_arrive(&s.tempty[1]);
-              if (j == M - 1) mbar_arrive(&s.tempty[0]);
+              if (j > 0) release_region(1);
+              if (j == M - 1) release_region(0);
             }
           }
         }
@@ -664,10 +739,20 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   }
 
   __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
+  if constexpr (PAIR) {
+    tc_fence_before();
+    cluster_sync_all();        // no CTA leaves while its pair may still touch its memory
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if (warp == 1) {
+      __syncwarp();
+      tmem_dealloc_pair(tmem, 512);
+    }
+  } else {
+    if (warp == 1) {
+      __syncwarp();
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
   }
 }
 
@@ -1396,20 +1481,51 @@ TcWs fwd_layout(const LossProblem& p, void* ws) {
   return w;
 }
 
+// The loss tile kernels run on single CTAs.  The CTA-pair form (256-token
+// tiles, half of the W tile per SM) passes the same parity tests but measured
+// slower on the 3-exit suite at T = 8192: 5.6-5.7 ms per forward launch
+// instead of 5.2 ms, with 8-10 GB of DRAM reads per launch instead of 3.6 GB
+// at the same 2048-token tile grouping, and lower clocks under the power cap.
+constexpr bool kLossPair = false;
+
 template <int MODE, int DISTILL, bool TGRAD = false>
 cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaStream_t st) {
+  constexpr bool PAIR = kLossPair;
   LossMaps maps;
   for (int m = 0; m < p.M; ++m) {
     if (!make_map(&maps.h[m], p.h[m], p.D[m], p.T, kBK, kBM)) return cudaErrorInvalidValue;
-    if (!make_map(&maps.w[m], p.W[m], p.D[m], p.V, kBK, kLossBN)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.w[m], p.W[m], p.D[m], p.V, kBK, LossSmem<PAIR>::kBRows)) return cudaErrorInvalidValue;
   }
   LossArgs a = args_in;
-  const size_t smem = sizeof(LossSmem) + 1024;
-  auto fn = loss_tile_kernel<MODE, DISTILL, TGRAD>;
+  if (PAIR) {
+    a.n_tt = static_cast<int>((p.T + 2 * kBM - 1) / (2 * kBM));
+    a.num_tiles = a.n_tt * a.n_vt;
+    a.group_tt = 8;                 // 2048 tokens per group, as with 128-token tiles
+  }
+  const size_t smem = sizeof(LossSmem<PAIR>) + 1024;
+  auto fn = loss_tile_kernel<MODE, DISTILL, TGRAD, PAIR>;
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-  fn<<<grid, kLossThreads, smem, st>>>(maps, a);
+  if (PAIR) {
+    const int pairs = a.num_tiles < num_sms() / 2 ? a.num_tiles : num_sms() / 2;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(kLossThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, fn, maps, a);
+    if (err != cudaSuccess) return err;
+  } else {
+    const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+    fn<<<grid, kLossThreads, smem, st>>>(maps, a);
+  }
   note_launches(1);
   return cudaGetLastError();
 }
