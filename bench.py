@@ -495,6 +495,41 @@ def main():
             "beta_mean": vals[:S], "kl_mean": vals[S:2 * S], "top1_agree_mean": vals[2 * S:],
             "what": "each smaller exit vs the largest: acceptance sum_v min(q,p), KL(p||q), top-1 agreement"}
 
+    # ---------------- each junction kernel alone (L2 flushed before every call)
+    if c.M > 1:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)     # 2x the 126 MB L2
+        b = 2 if c.dtype == "bf16" else 4
+        alone = []
+        for j in range(c.M - 1):
+            D, dl, Dn = c.D[j], c.deltas[j + 1], c.D[j + 1]
+            calls = {
+                "fwd": (lambda j=j: step.api.junction_fwd(step.x, step.o[j], step.E[j + 1], out=step.jy[j],
+                                                          scale_out=step.jscale[j], status=step.status,
+                                                          stream=stream),
+                        c.T * ((D + dl + Dn) * b + 8)),
+                "bwd_rows": (lambda j=j: step.api.junction_bwd(step.x, step.o[j], step.E[j + 1], step.dh[j + 1],
+                                                               do_out=step.do[j], de_out=step.de[j], dE=None,
+                                                               workspace=step.ws_j, status=step.status,
+                                                               stream=stream),
+                             c.T * ((Dn + 2 * D + 2 * dl) * b + 4)),
+            }
+            for kind, (fn, nbytes) in calls.items():
+                ts = []
+                for _ in range(12):
+                    flush.zero_()
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                    e1.synchronize()
+                    ts.append(e0.elapsed_time(e1))
+                us = statistics.median(ts[2:]) * 1000.0
+                alone.append({"junction": f"{D}->{Dn}", "pass": kind, "us": us, "bytes": nbytes,
+                              "gbs": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / peaks.get("hbm_gbs")})
+        del flush
+        extras["junction_alone"] = alone
+
     # ---------------- roofline of the dominant kernel and phase rates
     ms_fwd, ms_bwd = phase_ms[1], phase_ms[2]
     flops_fwd = 2.0 * c.T * c.V * sum(c.D)

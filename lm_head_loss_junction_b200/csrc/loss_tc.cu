@@ -1461,6 +1461,30 @@ int num_sms() {
   return n;
 }
 
+// Pairs of CTAs (2-CTA clusters) that can be resident at once for kernel fn with
+// this block size and shared memory: a persistent grid larger than that would
+// leave whole clusters waiting for a second wave.  Falls back to SMs / 2.
+template <typename Kernel>
+int resident_pairs(Kernel fn, int threads, size_t smem) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms()));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = num_sms() / 2;
+  }
+  return n;
+}
+
 size_t align_up(size_t b) { return (b + 255) & ~size_t(255); }
 
 // bf16 G' of every exit: [M][T][V]
@@ -1507,7 +1531,8 @@ cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaSt
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   if (PAIR) {
-    const int pairs = a.num_tiles < num_sms() / 2 ? a.num_tiles : num_sms() / 2;
+    const int resident = resident_pairs(fn, kLossThreads, smem);
+    const int pairs = a.num_tiles < resident ? a.num_tiles : resident;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     cfg.blockDim = dim3(kLossThreads);
@@ -1570,7 +1595,8 @@ cudaError_t run_gemm(const GemmMaps& maps, GemmArgs g, cudaStream_t st) {
     auto fn = gemm_pair_kernel<A_MN, B_MN, OUT_BF16>;
     err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+    const int resident = resident_pairs(fn, kThreads, smem);
+    const int pairs = tiles < resident ? tiles : resident;
     fn<<<2 * pairs, kThreads, smem, st>>>(maps, g);
   } else {
     const size_t smem = sizeof(GemmSmem<BN>) + 1024;
