@@ -495,39 +495,56 @@ def main():
             "beta_mean": vals[:S], "kl_mean": vals[S:2 * S], "top1_agree_mean": vals[2 * S:],
             "what": "each smaller exit vs the largest: acceptance sum_v min(q,p), KL(p||q), top-1 agreement"}
 
-    # ---------------- each junction kernel alone (L2 flushed before every call)
+    # ---------------- each junction kernel alone: 24 back-to-back launches rotating
+    # over enough copies of the streamed rows (o, dy in; y, do, de out) that they
+    # span at least 3x the 126 MB L2, captured as one CUDA graph, CUDA events
+    # around its replay
     if c.M > 1:
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)     # 2x the 126 MB L2
         b = 2 if c.dtype == "bf16" else 4
         alone = []
         for j in range(c.M - 1):
             D, dl, Dn = c.D[j], c.deltas[j + 1], c.D[j + 1]
+            fwd_bytes = c.T * ((D + dl + Dn) * b + 8)
+            bwd_bytes = c.T * ((Dn + 2 * D + 2 * dl) * b + 4)
+            copies = max(2, -(-3 * (126 << 20) // fwd_bytes))
+            o_c = [step.o[j]] + [step.o[j].clone() for _ in range(copies - 1)]
+            y_c = [torch.empty_like(step.jy[j]) for _ in range(copies)]
+            dy_c = [step.dh[j + 1]] + [step.dh[j + 1].clone() for _ in range(copies - 1)]
+            do_c = [torch.empty_like(step.do[j]) for _ in range(copies)]
+            de_c = [torch.empty_like(step.de[j]) for _ in range(copies)]
             calls = {
-                "fwd": (lambda j=j: step.api.junction_fwd(step.x, step.o[j], step.E[j + 1], out=step.jy[j],
-                                                          scale_out=step.jscale[j], status=step.status,
-                                                          stream=stream),
-                        c.T * ((D + dl + Dn) * b + 8)),
-                "bwd_rows": (lambda j=j: step.api.junction_bwd(step.x, step.o[j], step.E[j + 1], step.dh[j + 1],
-                                                               do_out=step.do[j], de_out=step.de[j], dE=None,
-                                                               workspace=step.ws_j, status=step.status,
-                                                               stream=stream),
-                             c.T * ((Dn + 2 * D + 2 * dl) * b + 4)),
+                "fwd": (lambda i, s, j=j: step.api.junction_fwd(step.x, o_c[i], step.E[j + 1], out=y_c[i],
+                                                                scale_out=step.jscale[j], status=step.status,
+                                                                stream=s), fwd_bytes),
+                "bwd_rows": (lambda i, s, j=j: step.api.junction_bwd(step.x, o_c[i], step.E[j + 1], dy_c[i],
+                                                                     do_out=do_c[i], de_out=de_c[i], dE=None,
+                                                                     workspace=step.ws_j, status=step.status,
+                                                                     stream=s), bwd_bytes),
             }
             for kind, (fn, nbytes) in calls.items():
-                ts = []
-                for _ in range(12):
-                    flush.zero_()
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    fn()
-                    e1.record(stream)
-                    e1.synchronize()
-                    ts.append(e0.elapsed_time(e1))
-                us = statistics.median(ts[2:]) * 1000.0
+                n = 24
+                for i in range(copies):
+                    fn(i, stream)
+                if args.eager:
+                    batch = lambda fn=fn: [fn(i % copies, stream) for i in range(n)]  # noqa: E731
+                else:
+                    gj = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gj, capture_error_mode="relaxed"):
+                        for i in range(n):
+                            fn(i % copies, None)
+                    batch = gj.replay
+                batch()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                batch()
+                e1.record(stream)
+                e1.synchronize()
+                us = e0.elapsed_time(e1) * 1000.0 / n
                 alone.append({"junction": f"{D}->{Dn}", "pass": kind, "us": us, "bytes": nbytes,
-                              "gbs": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / peaks.get("hbm_gbs")})
-        del flush
+                              "gbs": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / peaks.get("hbm_gbs"),
+                              "copies": copies})
+            del o_c, y_c, dy_c, do_c, de_c
         extras["junction_alone"] = alone
 
     # ---------------- roofline of the dominant kernel and phase rates
