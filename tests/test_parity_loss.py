@@ -102,13 +102,14 @@ def test_alternative_distillation(name, small, distill):
 
 @pytest.mark.parametrize("name,small", [("tiny3", None), ("main3", dict(batch=1, seq=200, V=512)),
                                         ("suite4", dict(batch=1, seq=130, V=384)),
-                                        ("main3_aligned", dict(batch=1, seq=256, V=768))])
+                                        ("main3_aligned", dict(batch=1, seq=256, V=768)),
+                                        ("proxy2", dict(batch=1, seq=160, V=512))])
 @pytest.mark.parametrize("distill", ["ce", "reverse_kl"])
 def test_teacher_gradient(name, small, distill):
     cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
     d = wl.make_inputs(cfg, with_tables=False)
     _check_all(d, 0.3, 1.0, distill=distill, teacher_grad=True)
-    _check_all(d, 0.6, 2.0, exit_weights=[1.5, 0.5] + [1.0] * (cfg.M - 3) + [0.8], distill=distill,
+    _check_all(d, 0.6, 2.0, exit_weights=[1.5] + [0.7] * (cfg.M - 2) + [0.8], distill=distill,
                teacher_grad=True)
 
 
