@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           float lse_part = -INFINITY, abar = 0.f;
           if (live) {
             if (j == 0) {
-              // teacher: split max, then p~ = exp(l - max) (bf16 in registers) and their sum
+              // teacher: split max, then p~ = exp(l - max) (fp16 pairs in registers) and their sum
               float mx = -INFINITY;
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
