@@ -229,7 +229,10 @@ mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int6
  * mls_multiexit_loss_fwd
  *   losses  device f32 [2M]: CE_LM[0..M-1], CE_KD[0..M-2], L
  *   stats   device f32 [3M-1, T]: rows 0..M-1 lse_m, rows M..2M-1 the target
- *           logits l_m,y, rows 2M..3M-2 S_m.  Kept for the backward pass.
+ *           logits l_m,y, rows 2M..3M-2 S_m (the _opts form: the statistic of
+ *           the chosen distillation, and for Jensen-Shannon with the teacher
+ *           gradient 4M-2 rows, see mls_loss_options).  Kept for the
+ *           backward pass.
  */
 mls_status mls_multiexit_loss_fwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   const int32_t* y_targets,
@@ -291,12 +294,13 @@ typedef enum {
  *                 largest exit's logit gradient gains, for every smaller exit m,
  *                 lambda_m alpha_d dKD_m/dl_M:
  *                   MLS_DISTILL_CE:         -p_M (l_m - S_m),  S_m = sum_v p_M l_m
- *                   MLS_DISTILL_REVERSE_KL:  p_M - q_m.
- *                 Backward only (the forward is unchanged; pass the same
- *                 options to both calls).  With MLS_DISTILL_JS it returns
- *                 MLS_ERR_UNSUPPORTED: that gradient needs KL(p_M || mu) per
- *                 token, which the statistics rows do not hold.  The pages
- *                 leave the teacher's gradient open.
+ *                   MLS_DISTILL_REVERSE_KL:  p_M - q_m
+ *                   MLS_DISTILL_JS:          p_M (log(p_M/mu)/2 - KL(p_M || mu)/2).
+ *                 Pass the same options to both calls.  With MLS_DISTILL_JS
+ *                 the forward call then also writes KL(p_M || mu)/2 per token
+ *                 into stats rows 3M-1 .. 4M-3, so stats must have 4M-2 rows
+ *                 (otherwise 3M-1).  The pages leave the teacher's gradient
+ *                 open.
  *   exit_weights  HOST float [M] or NULL: per-exit loss weights lambda_m,
  *                 L = sum_{m<M} lambda_m [(1 - alpha_d) CE_LM,m + alpha_d CE_KD,m]
  *                     + lambda_M CE_LM,M,

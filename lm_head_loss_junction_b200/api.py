@@ -151,22 +151,25 @@ def _workspace(ws, nbytes, device):
 
 
 def multiexit_loss_fwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Tensor], alpha_d: float = 0.3, *,
-                       losses=None, stats=None, workspace=None, exit_weights=None, distill="ce", status=None,
-                       stream=None):
-    """Returns (losses [2M], stats [3M-1, T]) (see mls_multiexit_loss_fwd; `exit_weights`
-    uses mls_multiexit_loss_fwd_opts)."""
+                       losses=None, stats=None, workspace=None, exit_weights=None, distill="ce",
+                       teacher_grad: bool = False, status=None, stream=None):
+    """Returns (losses [2M], stats [3M-1, T], or [4M-2, T] for Jensen-Shannon with the
+    teacher gradient) (see mls_multiexit_loss_fwd; any option uses mls_multiexit_loss_fwd_opts)."""
     M, T, V, D, dt = _loss_common(y, h, W)
     dev = y.device
     if losses is None:
         losses = torch.empty(2 * M, dtype=torch.float32, device=dev)
+    rows = 4 * M - 2 if (distill == "js" and teacher_grad and M > 1) else 3 * M - 1
     if stats is None:
-        stats = torch.empty((3 * M - 1, T), dtype=torch.float32, device=dev)
+        stats = torch.empty((rows, T), dtype=torch.float32, device=dev)
+    elif stats.shape[0] < rows:
+        raise ValueError(f"stats needs {rows} rows")
     fwd_b, _ = multiexit_loss_workspace(T, D, V, dt)
     workspace, ws_bytes = _workspace(workspace, fwd_b, dev)
     args = (M, T, V, i64_array(D), y.data_ptr(), ptr_array([t.data_ptr() for t in h]),
             ptr_array([t.data_ptr() for t in W]), float(alpha_d), _dtype_code(h[0]), losses.data_ptr(),
             stats.data_ptr(), workspace.data_ptr(), ws_bytes)
-    opts = _lib.loss_options(exit_weights, distill)
+    opts = _lib.loss_options(exit_weights, distill, teacher_grad)
     if opts is None:
         code = lib().mls_multiexit_loss_fwd(*args, _ptr(status), _stream_ptr(stream))
     else:

@@ -116,7 +116,6 @@ mls_status apply_options(const mls_loss_options* opts, LossProblem* p) {
     return MLS_ERR_INVALID_ARG;
   p->distill = opts->distill;
   if (opts->teacher_grad != 0 && opts->teacher_grad != 1) return MLS_ERR_INVALID_ARG;
-  if (opts->teacher_grad != 0 && opts->distill == MLS_DISTILL_JS) return MLS_ERR_UNSUPPORTED;
   p->teacher_grad = opts->teacher_grad;
   if (opts->exit_weights != nullptr) {
     for (int m = 0; m < p->M; ++m) {

@@ -28,7 +28,7 @@ struct SimtDev {
   float alpha_d;
   float exit_w[kMaxExits];
   int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
-  int teacher_grad;          // 1: no stop-gradient on the largest exit (cross-entropy and reverse KL)
+  int teacher_grad;          // 1: no stop-gradient on the largest exit
   int32_t* status;
   float* dh[kMaxExits];
   float* dW[kMaxExits];
@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
     for (int s = 0; s < S; ++s) {
       const float a = red[(2 * s) * kSimtThreads], b = red[(2 * s + 1) * kSimtThreads];
       stats[(2 * M + s) * p.T + t] = 0.5f * a;
+      if (p.teacher_grad) stats[(3 * M - 1 + s) * p.T + t] = 0.5f * b;   // KL(p_T || mu)/2
       terms[(M + s) * p.T + t] = bad ? 0.f : 0.5f * (a + b);
     }
   }
@@ -253,12 +254,20 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
       if (m == M - 1) {
         g = pT - hot;
         if (p.teacher_grad) {
-          // distillation gradient of every smaller exit s on the teacher's logits, relative to w_T:
-          //   cross-entropy -p_T (l_s - S_s);  reverse KL p_T - q_s
+          // distillation gradient of every smaller exit s on the teacher's logits:
+          //   cross-entropy -p_T (l_s - S_s);  reverse KL p_T - q_s;
+          //   Jensen-Shannon p_T (log(p_T/mu_s)/2 - K^p_s), log(p/mu) = ln 2 - softplus(log q - log p)
           float extra = 0.f;
           for (int s = 0; s < M - 1; ++s) {
-            const float ts = (p.distill == 1) ? pT - __expf(l[s] - lse[s])
-                                              : -pT * (l[s] - stats[(2 * M + s) * p.T + t]);
+            float ts;
+            if (p.distill == 1) {
+              ts = pT - __expf(l[s] - lse[s]);
+            } else if (p.distill == 2) {
+              const float lq = l[s] - lse[s], lp = l[M - 1] - lse[M - 1];
+              ts = pT * (0.5f * (kLn2 - softplus(lq - lp)) - stats[(3 * M - 1 + s) * p.T + t]);
+            } else {
+              ts = -pT * (l[s] - stats[(2 * M + s) * p.T + t]);
+            }
             extra = fmaf(p.exit_w[s], ts, extra);
           }
           G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : fmaf(a, extra, p.exit_w[m] * g);

@@ -48,6 +48,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // TMEM lane quadrant, each owning one 128-column half ("split") of the tile.
 constexpr int kLossBN = 256;
 constexpr int kSplitCols = 128;
+constexpr bool kLossL2Hints = false;  // L2 eviction hints on the operand loads (h evict-last, W evict-first)
 constexpr int kLossStages = 4;        // single CTA: 48 KB per stage
 constexpr int kLossPairStages = 6;    // CTA pair: 32 KB per stage and CTA
 constexpr int kLossEpiWarps = 8;
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   // The statistics of the Jensen-Shannon form are the cross-entropy ones (it
   // needs the final normalisers, so its divergence has a pass of its own).
   constexpr bool hold = (MODE == kModeAgree) || (MODE == kModeJS) || rkl || (MODE == kModeGrad && (jsd || TGRAD));
-  static_assert(!TGRAD || (MODE == kModeGrad && DISTILL != 2), "teacher gradient: backward, CE or reverse KL");
+  static_assert(!TGRAD || MODE == kModeGrad, "teacher gradient: backward only");
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -280,6 +281,9 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
+      // h panels are reused across the vocabulary tiles of a token group; W streams
+      [[maybe_unused]] const uint64_t pol_h = kLossL2Hints ? l2_policy_evict_last() : 0;
+      [[maybe_unused]] const uint64_t pol_w = kLossL2Hints ? l2_policy_evict_first() : 0;
       for (int tile = slot; tile < a.num_tiles && ok; tile += nslots) {
         int tt, vt;
         loss_tile_coords(tile, a, tt, vt);
@@ -292,12 +296,22 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             if constexpr (PAIR) {
               const uint32_t lfull = mapa_shared(smem_u32(&s.full[stage]), 0);
               if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * (kBM + Smem::kBRows) * kBK * 2);
-              tma_load_2d_pair(&maps.h[m], lfull, s.a[stage], kb * kBK, row0);
-              tma_load_2d_pair(&maps.w[m], lfull, s.b[stage], kb * kBK, v0);
+              if constexpr (kLossL2Hints) {
+                tma_load_2d_pair_hint(&maps.h[m], lfull, s.a[stage], kb * kBK, row0, pol_h);
+                tma_load_2d_pair_hint(&maps.w[m], lfull, s.b[stage], kb * kBK, v0, pol_w);
+              } else {
+                tma_load_2d_pair(&maps.h[m], lfull, s.a[stage], kb * kBK, row0);
+                tma_load_2d_pair(&maps.w[m], lfull, s.b[stage], kb * kBK, v0);
+              }
             } else {
               mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
-              tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0);
-              tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0);
+              if constexpr (kLossL2Hints) {
+                tma_load_2d_hint(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0, pol_h);
+                tma_load_2d_hint(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0, pol_w);
+              } else {
+                tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0);
+                tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0);
+              }
             }
             ++issued;
             if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -625,6 +639,9 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             //   cross-entropy S_m = sum p_T l_m; reverse KL R_m = sum q_m (l_m - l_T), so that
             //   log q - log p - KL(q_m || p_T) = l_m - l_T - R_m;  Jensen-Shannon: K = KL(q_m || mu) / 2
             const float klt = (hold && j > 0 && valid) ? a.stats[static_cast<int64_t>(2 * M + m) * a.T + t] : 0.f;
+            // Jensen-Shannon with the teacher gradient: K^p = KL(p_T || mu)/2, stored by the forward pass
+            const float kpt = (TGRAD && jsd && j > 0 && valid) ? a.stats[static_cast<int64_t>(3 * M - 1 + m) * a.T + t]
+                                                               : 0.f;
             const uint32_t wm2 = TGRAD ? pack_p2(a.exit_w[m], a.exit_w[m]) : 0u;
             // unrolled where a register array is indexed by c (the teacher's
             // packed probabilities, or the teacher-gradient accumulator)
@@ -662,10 +679,17 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                   g1 = e1 * fmaf(al, d1, 1.f - al);
                   if (TGRAD) pt[c][k / 2] = hfma_p2(wm2, pack_p2(e0, e1), pt[c][k / 2]);   // sum_m w_m q_m
                 } else if (jsd) {                  // student: G' = q ((1 - a) + a (log(q/mu)/2 - K))
-                  const float d0 = fmaf(-0.5f, softplus((lt[kk] - lseT) - (r[kk] - lse)), 0.5f * kLn2) - klt;
-                  const float d1 = fmaf(-0.5f, softplus((lt[kk + 1] - lseT) - (r[kk + 1] - lse)), 0.5f * kLn2) - klt;
+                  // x = log p - log q; log(q/mu) = ln 2 - softplus(x), log(p/mu) = ln 2 - softplus(x) + x
+                  const float x0 = (lt[kk] - lseT) - (r[kk] - lse);
+                  const float x1 = (lt[kk + 1] - lseT) - (r[kk + 1] - lse);
+                  const float sp0 = softplus(x0), sp1 = softplus(x1);
+                  const float d0 = fmaf(-0.5f, sp0, 0.5f * kLn2) - klt;
+                  const float d1 = fmaf(-0.5f, sp1, 0.5f * kLn2) - klt;
                   g0 = e0 * fmaf(al, d0, 1.f - al);
                   g1 = e1 * fmaf(al, d1, 1.f - al);
+                  if (TGRAD)                       // sum_m w_m (log(p/mu_m)/2 - K^p_m)
+                    pt[c][k / 2] = hfma_p2(wm2, pack_p2(0.5f * (kLn2 - sp0 + x0) - kpt, 0.5f * (kLn2 - sp1 + x1) - kpt),
+                                           pt[c][k / 2]);
                 } else {                           // student: G' = q - alpha_d p_T
                   float p0, p1;
                   if (hold) {
@@ -690,8 +714,9 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           }
           if (TGRAD && j == M - 1 && j > 0 && live) {
             // the teacher's G' with every student's distillation gradient:
-            //   cross-entropy: w_T p - a p sum_m w_m (l_m - S_m)
-            //   reverse KL:    (w_T + a sum_m w_m) p - a sum_m w_m q_m
+            //   cross-entropy:  w_T p - a p sum_m w_m (l_m - S_m)
+            //   reverse KL:     (w_T + a sum_m w_m) p - a sum_m w_m q_m
+            //   Jensen-Shannon: w_T p + a p sum_m w_m (log(p/mu_m)/2 - K^p_m)
             const float wT = a.exit_w[M - 1];
             const float cp = rkl ? fmaf(al, a.student_wsum, wT) : wT;
 #pragma unroll
@@ -711,6 +736,9 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                   if (rkl) {
                     g0 = fmaf(-al, acc.x, cp * p0);
                     g1 = fmaf(-al, acc.y, cp * p1);
+                  } else if (jsd) {
+                    g0 = p0 * fmaf(al, acc.x, cp);
+                    g1 = p1 * fmaf(al, acc.y, cp);
                   } else {
                     g0 = p0 * fmaf(-al, acc.x, cp);
                     g1 = p1 * fmaf(-al, acc.y, cp);
@@ -915,7 +943,7 @@ __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const floa
 // statistics row the backward pass reads and JS = (KL(q || mu) + KL(p || mu))/2
 // as the distillation term.
 __global__ void __launch_bounds__(32 * kMergeRows) js_merge_kernel(const float* __restrict__ partial, int n_splits,
-                                                                   int M, int T, int V,
+                                                                   int M, int T, int V, int teacher_rows,
                                                                    const int32_t* __restrict__ y,
                                                                    float* __restrict__ stats,
                                                                    float* __restrict__ terms) {
@@ -945,6 +973,8 @@ __global__ void __launch_bounds__(32 * kMergeRows) js_merge_kernel(const float* 
   const bool bad = yt < 0 || yt >= V;
   for (int s = 0; s < M - 1; ++s) {
     stats[static_cast<int64_t>(2 * M + s) * T + t] = 0.5f * jq[s];
+    // with the teacher gradient: KL(p || mu)/2 in rows 3M-1 .. 4M-3
+    if (teacher_rows) stats[static_cast<int64_t>(3 * M - 1 + s) * T + t] = 0.5f * jp[s];
     terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : 0.5f * (jq[s] + jp[s]);
   }
 }
@@ -1733,7 +1763,8 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
     err = run_loss_tiles<kModeJS, 0>(p, a, st);
     if (err != cudaSuccess) return err;
     js_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
-                                                                     static_cast<int>(p.V), p.y, stats, w.terms);
+                                                                     static_cast<int>(p.V), p.teacher_grad, p.y,
+                                                                     stats, w.terms);
     note_launches(1);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -1748,8 +1779,9 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   a.stats = const_cast<float*>(stats);
   a.G = G;
   const bool tgrad = p.teacher_grad != 0 && p.M > 1;
-  cudaError_t err = tgrad ? (p.distill == 1 ? run_loss_tiles<kModeGrad, 1, true>(p, a, st)
-                                            : run_loss_tiles<kModeGrad, 0, true>(p, a, st))
+  cudaError_t err = tgrad ? (p.distill == 1   ? run_loss_tiles<kModeGrad, 1, true>(p, a, st)
+                             : p.distill == 2 ? run_loss_tiles<kModeGrad, 2, true>(p, a, st)
+                                              : run_loss_tiles<kModeGrad, 0, true>(p, a, st))
                     : p.distill == 1 ? run_loss_tiles<kModeGrad, 1>(p, a, st)
                     : p.distill == 2 ? run_loss_tiles<kModeGrad, 2>(p, a, st)
                                      : run_loss_tiles<kModeGrad, 0>(p, a, st);

@@ -83,7 +83,7 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     student gradient through the softmax is
     G_m = lambda_m grad_scale/T ((1 - alpha_d)(q_m - onehot) + alpha_d q_m (g - K_t)),
     g_v = log(q_v / mu_v) / 2,  K_t = sum_v q_v g_v = KL(q_m || mu) / 2,
-    and K_t is returned per token in "J".
+    and K_t is returned per token in "J" (KL(p_M || mu)/2 in "Jp").
     teacher_grad: the largest exit also receives the gradient of every
     distillation term (no stop-gradient; the pages leave this open).  With
     T_m = d KD_m / d l_M, the teacher's logit gradient gains
@@ -110,6 +110,7 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     out = {
         "lse": np.zeros((M, Tn)), "tgt": np.zeros((M, Tn)), "S": np.zeros((max(M - 1, 0), Tn)),
         "R": np.zeros((max(M - 1, 0), Tn)), "J": np.zeros((max(M - 1, 0), Tn)),
+        "Jp": np.zeros((max(M - 1, 0), Tn)),
         "ce_lm_sum": np.zeros(M), "ce_kd_sum": np.zeros(max(M - 1, 0)),
     }
     if need_grad:
@@ -143,6 +144,7 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             jp = np.sum(pM * (logq[M - 1] - logmix[m]), axis=1)
             jps.append(jp)
             out["J"][m, b0:b0 + n] = 0.5 * jq[m]
+            out["Jp"][m, b0:b0 + n] = 0.5 * jp
             if distill == "ce":
                 out["ce_kd_sum"][m] += np.sum(-np.sum(pM * logq[m], axis=1))
             elif distill == "reverse_kl":

@@ -105,11 +105,6 @@ def test_loss_options_reject_nonfinite_weights():
                                            _lib.ptr_array([FAKE, FAKE]), _lib.ptr_array([FAKE, FAKE]), 0.3,
                                            _lib.MLS_BF16, FAKE, FAKE, FAKE, 1 << 40, ctypes.byref(bad), None, None)
     assert code == 1                                                 # teacher_grad must be 0 or 1
-    js_t = _lib.LossOptions(None, 2, 1)
-    code = lib.mls_multiexit_loss_fwd_opts(2, 256, 1024, _lib.i64_array([512, 1024]), FAKE,
-                                           _lib.ptr_array([FAKE, FAKE]), _lib.ptr_array([FAKE, FAKE]), 0.3,
-                                           _lib.MLS_BF16, FAKE, FAKE, FAKE, 1 << 40, ctypes.byref(js_t), None, None)
-    assert code == 2                                                 # no teacher gradient for Jensen-Shannon
 
 
 def test_agreement_argument_errors():

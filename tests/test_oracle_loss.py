@@ -345,6 +345,9 @@ def test_js_matches_scipy_distance_by_enumeration():
         mix = 0.5 * (q + pM)
         kq = np.array([sum(q[t, v] * math.log(q[t, v] / mix[t, v]) for v in range(9)) for t in range(5)])
         np.testing.assert_allclose(r["J"][m], 0.5 * kq, rtol=1e-12)
+        kp = np.array([sum(pM[t, v] * math.log(pM[t, v] / mix[t, v]) for v in range(9)) for t in range(5)])
+        np.testing.assert_allclose(r["Jp"][m], 0.5 * kp, rtol=1e-12)
+        np.testing.assert_allclose(np.mean(r["J"][m] + r["Jp"][m]), r["ce_kd"][m], rtol=1e-12)
     assert np.all(r["ce_kd"] >= 0) and np.all(r["ce_kd"] <= math.log(2.0))
 
 
