@@ -48,7 +48,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 // TMEM lane quadrant, each owning one 128-column half ("split") of the tile.
 constexpr int kLossBN = 256;
 constexpr int kSplitCols = 128;
-constexpr bool kLossL2Hints = false;  // L2 eviction hints on the operand loads (h evict-last, W evict-first)
 constexpr int kLossStages = 4;        // single CTA: 48 KB per stage
 constexpr int kLossPairStages = 6;    // CTA pair: 32 KB per stage and CTA
 constexpr int kLossEpiWarps = 8;
@@ -281,9 +280,6 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
-      // h panels are reused across the vocabulary tiles of a token group; W streams
-      [[maybe_unused]] const uint64_t pol_h = kLossL2Hints ? l2_policy_evict_last() : 0;
-      [[maybe_unused]] const uint64_t pol_w = kLossL2Hints ? l2_policy_evict_first() : 0;
       for (int tile = slot; tile < a.num_tiles && ok; tile += nslots) {
         int tt, vt;
         loss_tile_coords(tile, a, tt, vt);
@@ -296,22 +292,12 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             if constexpr (PAIR) {
               const uint32_t lfull = mapa_shared(smem_u32(&s.full[stage]), 0);
               if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * (kBM + Smem::kBRows) * kBK * 2);
-              if constexpr (kLossL2Hints) {
-                tma_load_2d_pair_hint(&maps.h[m], lfull, s.a[stage], kb * kBK, row0, pol_h);
-                tma_load_2d_pair_hint(&maps.w[m], lfull, s.b[stage], kb * kBK, v0, pol_w);
-              } else {
-                tma_load_2d_pair(&maps.h[m], lfull, s.a[stage], kb * kBK, row0);
-                tma_load_2d_pair(&maps.w[m], lfull, s.b[stage], kb * kBK, v0);
-              }
+              tma_load_2d_pair(&maps.h[m], lfull, s.a[stage], kb * kBK, row0);
+              tma_load_2d_pair(&maps.w[m], lfull, s.b[stage], kb * kBK, v0);
             } else {
               mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
-              if constexpr (kLossL2Hints) {
-                tma_load_2d_hint(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0, pol_h);
-                tma_load_2d_hint(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0, pol_w);
-              } else {
-                tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0);
-                tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0);
-              }
+              tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0);
+              tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0);
             }
             ++issued;
             if (++stage == kStages) { stage = 0; phase ^= 1; }
