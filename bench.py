@@ -585,11 +585,20 @@ def main():
         gbytes = sum(t.numel() * t.element_size() for t in grads)
         phases["grad_sync_ms"] = phase_ms[4]
         phases["grad_sync_bytes"] = gbytes
-    roofline = {"bound": "tensor", "achieved": ach_fwd, "peak": peak_tc, "unit": "TFLOP/s",
-                "frac": ach_fwd / peak_tc, "traffic": measured_traffic(c),
-                "kernel": "loss_tile_kernel<stats> (mls_multiexit_loss_fwd call: tile kernel + merge + reduce)",
-                "algorithmic_per_launch": f"2*T*V*sum(D) = {flops_fwd:.4g} flop",
-                "peak_source": f"{peak_kind} bf16_tflops_sustained"}
+    if c.dtype == "bf16":
+        roofline = {"bound": "tensor", "achieved": ach_fwd, "peak": peak_tc, "unit": "TFLOP/s",
+                    "frac": ach_fwd / peak_tc, "traffic": measured_traffic(c),
+                    "kernel": "loss_tile_kernel<stats> (mls_multiexit_loss_fwd call: tile kernel + merge + reduce)",
+                    "algorithmic_per_launch": f"2*T*V*sum(D) = {flops_fwd:.4g} flop",
+                    "peak_source": f"{peak_kind} bf16_tflops_sustained"}
+    else:
+        # fp32 inputs take the CUDA-core path: 148 SMs x 128 fp32 FMA lanes x 2 flop x 1.965 GHz
+        peak_fma = 148 * 128 * 2 * 1.965e9 / 1e12
+        roofline = {"bound": "alu", "achieved": ach_fwd, "peak": peak_fma, "unit": "TFLOP/s",
+                    "frac": ach_fwd / peak_fma, "traffic": None,
+                    "kernel": "simt_stats_kernel (mls_multiexit_loss_fwd call, fp32 CUDA-core path)",
+                    "algorithmic_per_launch": f"2*T*V*sum(D) = {flops_fwd:.4g} flop",
+                    "peak_source": "nominal fp32 FMA rate at the maximum SM clock (no measured fp32 figure)"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
