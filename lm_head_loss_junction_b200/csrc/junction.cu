@@ -180,6 +180,84 @@ __global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __r
   }
 }
 
+// Short rows (at most CAP = 4 vectors of o and ECAP = 6 of e per lane): a
+// persistent grid of warps that each walk several tokens and load token
+// t + nwarps's id, block-output row and embedding row into registers while
+// token t is reduced and stored, so every warp keeps a row's worth of loads in
+// flight and the launch has no partial last wave.
+template <bool BF16, int CAP, int ECAP>
+__global__ void __launch_bounds__(256, 2) junction_fwd_pipe_kernel(const int32_t* __restrict__ x, int64_t T,
+                                                                  const uint4* __restrict__ o, int d_vec,
+                                                                  const uint4* __restrict__ E, int64_t V,
+                                                                  int dl_vec, uint4* __restrict__ y,
+                                                                  float* __restrict__ scale_out,
+                                                                  int32_t* __restrict__ status, uint32_t variant) {
+  const int lane = threadIdx.x & 31;
+  const bool zero_fill = (variant & kZeroFill) != 0;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const int dp_vec = d_vec + dl_vec;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  uint4 oc[CAP], ec[ECAP];
+  bool bad;
+  auto load_token = [&](int64_t tk, uint4 (&ov)[CAP], uint4 (&ev)[ECAP], bool& bd) {
+    const int32_t id = __ldg(x + tk);
+    bd = (id < 0) || (static_cast<int64_t>(id) >= V);
+    const uint4* orow = o + tk * d_vec;
+    const uint4* erow = E + static_cast<int64_t>(bd ? 0 : id) * dl_vec;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      ov[j] = (i < d_vec) ? __ldcs(orow + i) : zero;
+    }
+#pragma unroll
+    for (int j = 0; j < ECAP; ++j) {
+      const int i = j * 32 + lane;
+      ev[j] = (i < dl_vec) ? __ldg(erow + i) : zero;
+    }
+  };
+  load_token(t, oc, ec, bad);
+  while (true) {
+    const int64_t tn = t + nwarps;
+    const bool has_next = tn < T;
+    uint4 on[CAP], en[ECAP];
+    bool badn = false;
+    if (has_next) load_token(tn, on, en, badn);
+    float so = 0.f, se = 0.f;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) so += sumsq<BF16>(oc[j]);
+#pragma unroll
+    for (int j = 0; j < ECAP; ++j) se += sumsq<BF16>(ec[j]);
+    so = warp_sum(so);
+    se = warp_sum(se);
+    float s = (variant & kNoRescale) ? 1.f : sqrtf(se) / fmaxf(sqrtf(so), kJunctionEps);
+    if (bad) s = 0.f;
+    uint4* yrow = y + t * dp_vec;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < d_vec) yrow[i] = scale_vec<BF16>(oc[j], s);
+    }
+#pragma unroll
+    for (int j = 0; j < ECAP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < dl_vec) yrow[d_vec + i] = (bad || zero_fill) ? zero : ec[j];
+    }
+    if (lane == 0) {
+      if (scale_out != nullptr) scale_out[t] = s;
+      if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
+    }
+    if (!has_next) break;
+    t = tn;
+    bad = badn;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) oc[j] = on[j];
+#pragma unroll
+    for (int j = 0; j < ECAP; ++j) ec[j] = en[j];
+  }
+}
+
 // ---------------------------------------------------------------- backward
 // do = s (g_o - u (u.g_o)),  de = g_e + (u.g_o) e_hat, written as
 //   do = s g_o - (s ug / ||o||) o,   de = g_e + (ug / ||e||) e,   ug = o.g_o / ||o||.
@@ -295,10 +373,36 @@ cudaError_t launch_fwd_t(const JunctionArgs& a, cudaStream_t st) {
   constexpr int N = Elt<BF16>::kPerVec;
   const int d_vec = static_cast<int>(a.D / N), dl_vec = static_cast<int>(a.delta / N);
   const int cap = pick_cap(d_vec);
-  const int grid = grid_for(a.T, 8);
+  const int ecap = pick_cap(dl_vec);
   auto* o = static_cast<const uint4*>(a.o);
   auto* E = static_cast<const uint4*>(a.E);
   auto* y = static_cast<uint4*>(a.y);
+  if (cap <= 4 && ecap <= 6) {
+    // short rows: a persistent grid (two 8-warp blocks per SM) of prefetching warps
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t need = (a.T + 7) / 8;
+    const int pgrid = static_cast<int>(need < 2 * sms ? (need > 0 ? need : 1) : 2 * sms);
+#define MLS_JFP(C, EC) junction_fwd_pipe_kernel<BF16, C, EC><<<pgrid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, y, a.scale_out, a.status, a.variant)
+#define MLS_JFP_E(C)              \
+  switch (ecap) {                 \
+    case 1: MLS_JFP(C, 1); break; \
+    case 2: MLS_JFP(C, 2); break; \
+    case 4: MLS_JFP(C, 4); break; \
+    default: MLS_JFP(C, 6); break; \
+  }
+    switch (cap) {
+      case 1: MLS_JFP_E(1); break;
+      case 2: MLS_JFP_E(2); break;
+      default: MLS_JFP_E(4); break;
+    }
+#undef MLS_JFP_E
+#undef MLS_JFP
+    note_launches(1);
+    return cudaGetLastError();
+  }
+  const int grid = grid_for(a.T, 8);
 #define MLS_JF(C) junction_fwd_kernel<BF16, C><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, y, a.scale_out, a.status, a.variant)
   switch (cap) {
     case 1: MLS_JF(1); break;
