@@ -351,6 +351,107 @@ __global__ void __launch_bounds__(256, MINB) junction_bwd_kernel(
   }
 }
 
+// Short block-output rows (at most CAP = 4 vectors per lane): a persistent grid
+// of warps that each walk several tokens and load token t + nwarps's id, o row
+// and g_o row into registers while token t is reduced and stored; the
+// embedding row and g_e stream as in junction_bwd_kernel.
+template <bool BF16, int CAP>
+__global__ void __launch_bounds__(256, 2) junction_bwd_pipe_kernel(
+    const int32_t* __restrict__ x, int64_t T, const uint4* __restrict__ o, int d_vec,
+    const uint4* __restrict__ E, int64_t V, int dl_vec, const uint4* __restrict__ dy,
+    uint4* __restrict__ do_out, uint4* __restrict__ de_out, float* __restrict__ coef_out,
+    int32_t* __restrict__ status, uint32_t variant) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const int dp_vec = d_vec + dl_vec;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  uint4 oc[CAP], gc[CAP];
+  int32_t id;
+  auto load_og = [&](int64_t tk, uint4 (&ov)[CAP], uint4 (&gv)[CAP], int32_t& idk) {
+    idk = __ldg(x + tk);
+    const uint4* orow = o + tk * d_vec;
+    const uint4* grow = dy + tk * dp_vec;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      ov[j] = (i < d_vec) ? __ldcs(orow + i) : zero;
+      gv[j] = (i < d_vec) ? __ldcs(grow + i) : zero;
+    }
+  };
+  load_og(t, oc, gc, id);
+  while (true) {
+    const int64_t tn = t + nwarps;
+    const bool has_next = tn < T;
+    uint4 on[CAP], gn[CAP];
+    int32_t idn = 0;
+    if (has_next) load_og(tn, on, gn, idn);
+    const bool bad = (id < 0) || (static_cast<int64_t>(id) >= V);
+    const uint4* grow = dy + t * dp_vec;
+    const uint4* erow = E + static_cast<int64_t>(bad ? 0 : id) * dl_vec;
+    float so = 0.f, sog = 0.f, se = 0.f;
+#pragma unroll 2
+    for (int i = lane; i < dl_vec; i += 32) se += sumsq<BF16>(__ldg(erow + i));
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      so += sumsq<BF16>(oc[j]);
+      sog += dotv<BF16>(oc[j], gc[j]);
+    }
+    so = warp_sum(so);
+    sog = warp_sum(sog);
+    se = warp_sum(se);
+    const float n_o = fmaxf(sqrtf(so), kJunctionEps);
+    const float n_e = sqrtf(se);
+    const float s = n_e / n_o;
+    const float ug = sog / n_o;
+    float a = s, b = s * ug / n_o, c = (n_e > 0.f) ? ug / n_e : 0.f;
+    if (variant & kNoRescale) { a = 1.f; b = 0.f; c = 0.f; }   // y = [o ; .]
+    if (variant & kStopGrad) { a = 0.f; b = 0.f; }              // nothing flows into o
+    const float ge = (variant & kZeroFill) ? 0.f : 1.f;         // the fill does not carry g_e
+    if (bad) { a = 0.f; b = 0.f; c = 0.f; }
+    uint4* drow = do_out + t * d_vec;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < d_vec) drow[i] = axpby_vec<BF16>(a, gc[j], b, oc[j]);
+    }
+    if (de_out != nullptr) {
+      uint4* erow_out = de_out + t * dl_vec;
+      // groups of kDeGroup vectors per lane (smaller when the prefetched rows are long)
+      constexpr int kDeGroup = CAP >= 4 ? 2 : 4;
+      for (int i0 = lane; i0 < dl_vec; i0 += kDeGroup * 32) {
+        uint4 gv[kDeGroup], ev[kDeGroup];
+#pragma unroll
+        for (int u = 0; u < kDeGroup; ++u) {
+          const int i = i0 + u * 32;
+          if (i < dl_vec) {
+            gv[u] = __ldcs(grow + d_vec + i);
+            ev[u] = __ldg(erow + i);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kDeGroup; ++u) {
+          const int i = i0 + u * 32;
+          if (i < dl_vec) erow_out[i] = bad ? zero : lincomb_vec<BF16>(ge, gv[u], c, ev[u]);
+        }
+      }
+    }
+    if (lane == 0) {
+      if (coef_out != nullptr) coef_out[t] = c;
+      if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
+    }
+    if (!has_next) break;
+    t = tn;
+    id = idn;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      oc[j] = on[j];
+      gc[j] = gn[j];
+    }
+  }
+}
+
 int pick_cap(int nvec) {
   const int per_lane = (nvec + 31) / 32;
   static const int caps[] = {1, 2, 4, 6, 8, 9, 12, 16};
@@ -432,18 +533,29 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   auto* deo = static_cast<uint4*>(a.de_out);
   float* coef = nullptr;
   if (a.dE != nullptr) coef = static_cast<float*>(a.workspace);
+  if (cap <= 4) {
+    // short rows: a persistent grid (two 8-warp blocks per SM) of prefetching warps
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t need = (a.T + 7) / 8;
+    const int pgrid = static_cast<int>(need < 2 * sms ? (need > 0 ? need : 1) : 2 * sms);
+#define MLS_JBP(C) junction_bwd_pipe_kernel<BF16, C><<<pgrid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status, a.variant)
+    switch (cap) {
+      case 1: MLS_JBP(1); break;
+      case 2: MLS_JBP(2); break;
+      default: MLS_JBP(4); break;
+    }
+#undef MLS_JBP
+  } else {
 #define MLS_JB(C, B) junction_bwd_kernel<BF16, C, B><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status, a.variant)
-  // Rows of more than 4 vectors per lane: 4 blocks per SM with 2 vectors of o
-  // and g_o kept in registers (the rest re-read from L1) outrun 2 blocks per SM
-  // with the whole rows in registers (measured on the 2304 -> 4352 junction:
-  // 74-81% of the copy bandwidth against 60-68%); shorter rows keep them all.
-  switch (cap) {
-    case 1: MLS_JB(1, 2); break;
-    case 2: MLS_JB(2, 2); break;
-    case 4: MLS_JB(4, 2); break;
-    default: MLS_JB(2, 4); break;
-  }
+    // Rows of more than 4 vectors per lane: 4 blocks per SM with 2 vectors of o
+    // and g_o kept in registers (the rest re-read from L1) outrun 2 blocks per SM
+    // with the whole rows in registers (measured on the 2304 -> 4352 junction:
+    // 74-81% of the copy bandwidth against 60-68%).
+    MLS_JB(2, 4);
 #undef MLS_JB
+  }
   note_launches(1);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || a.dE == nullptr) return err;
