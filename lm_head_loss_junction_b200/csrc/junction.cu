@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(256, MINB) junction_bwd_kernel(
   }
 }
 
-// Short block-output rows (at most CAP = 4 vectors per lane): a persistent grid
+// Short block-output rows (at most CAP = 2 vectors per lane): a persistent grid
 // of warps that each walk several tokens and load token t + nwarps's id, o row
 // and g_o row into registers while token t is reduced and stored; the
 // embedding row and g_e stream as in junction_bwd_kernel.
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_pipe_kernel(
     const uint4* grow = dy + t * dp_vec;
     const uint4* erow = E + static_cast<int64_t>(bad ? 0 : id) * dl_vec;
     float so = 0.f, sog = 0.f, se = 0.f;
-#pragma unroll 2
+#pragma unroll 4
     for (int i = lane; i < dl_vec; i += 32) se += sumsq<BF16>(__ldg(erow + i));
 #pragma unroll
     for (int j = 0; j < CAP; ++j) {
@@ -418,8 +418,7 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_pipe_kernel(
     }
     if (de_out != nullptr) {
       uint4* erow_out = de_out + t * dl_vec;
-      // groups of kDeGroup vectors per lane (smaller when the prefetched rows are long)
-      constexpr int kDeGroup = CAP >= 4 ? 2 : 4;
+      constexpr int kDeGroup = 4;                      // vectors per lane in flight
       for (int i0 = lane; i0 < dl_vec; i0 += kDeGroup * 32) {
         uint4 gv[kDeGroup], ev[kDeGroup];
 #pragma unroll
@@ -533,27 +532,28 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   auto* deo = static_cast<uint4*>(a.de_out);
   float* coef = nullptr;
   if (a.dE != nullptr) coef = static_cast<float*>(a.workspace);
-  if (cap <= 4) {
-    // short rows: a persistent grid (two 8-warp blocks per SM) of prefetching warps
+  // Measured on the B200 (fraction of the copy bandwidth, T = 8192 .. 32768):
+  //  - rows of <= 2 vectors per lane: the prefetching persistent kernel
+  //    (512 -> 1024: 0.71 against 0.50-0.56);
+  //  - 4 vectors per lane: whole rows in registers, 2 blocks per SM (the
+  //    prefetching form, at 128 registers, was 0.49-0.68 against 0.60-0.80);
+  //  - longer rows: 4 blocks per SM with 2 vectors of o and g_o per lane in
+  //    registers and the rest re-read from L1 (2304 -> 4352: 0.74-0.84
+  //    against 0.60-0.68 with whole rows in registers at 2 blocks per SM).
+  if (cap <= 2) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t need = (a.T + 7) / 8;
     const int pgrid = static_cast<int>(need < 2 * sms ? (need > 0 ? need : 1) : 2 * sms);
 #define MLS_JBP(C) junction_bwd_pipe_kernel<BF16, C><<<pgrid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status, a.variant)
-    switch (cap) {
-      case 1: MLS_JBP(1); break;
-      case 2: MLS_JBP(2); break;
-      default: MLS_JBP(4); break;
-    }
+    if (cap == 1) MLS_JBP(1);
+    else MLS_JBP(2);
 #undef MLS_JBP
   } else {
 #define MLS_JB(C, B) junction_bwd_kernel<BF16, C, B><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status, a.variant)
-    // Rows of more than 4 vectors per lane: 4 blocks per SM with 2 vectors of o
-    // and g_o kept in registers (the rest re-read from L1) outrun 2 blocks per SM
-    // with the whole rows in registers (measured on the 2304 -> 4352 junction:
-    // 74-81% of the copy bandwidth against 60-68%).
-    MLS_JB(2, 4);
+    if (cap == 4) MLS_JB(4, 2);
+    else MLS_JB(2, 4);
 #undef MLS_JB
   }
   note_launches(1);
