@@ -54,9 +54,10 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
 cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
                                const float* coef, float ge, const void* E, float* dE, bool accumulate,
                                cudaStream_t st);
-// dW[v] -= scale * sum_t h_t (bf16 rows of d_vec 16-byte vectors).
-cudaError_t scatter_target_rows(const SegIndexDev& ix, const void* h, int d_vec, float* dW, float scale,
-                                cudaStream_t st);
+// For every job z < njobs (at most kMaxExits; one launch pair for all):
+//   dW[z][v] -= scale[z] * sum_{t: y_t = v} h[z]_t  (bf16 rows of d_vec[z] 16-byte vectors).
+cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,
+                                float* const* dW, const float* scale, cudaStream_t st);
 
 // ------------------------------------------------------------------ loss
 struct LossProblem {

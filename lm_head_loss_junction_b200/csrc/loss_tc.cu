@@ -1789,13 +1789,15 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
     default: err = run_dw_all<64>(p, G, dW, alpha, accumulate, st); break;
   }
   if (err != cudaSuccess) return err;
-  // one-hot part of dW: (1 - alpha_d) for students, 1 for the teacher
+  // one-hot part of dW: (1 - alpha_d) for students, 1 for the teacher; every exit in one launch pair
+  int d_vec[kMaxExits];
+  float scale[kMaxExits];
   for (int m = 0; m < p.M; ++m) {
     const float c = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
-    err = scatter_target_rows(ix, p.h[m], static_cast<int>(p.D[m] / 8), dW[m], alpha * p.exit_w[m] * c, st);
-    if (err != cudaSuccess) return err;
+    d_vec[m] = static_cast<int>(p.D[m] / 8);
+    scale[m] = alpha * p.exit_w[m] * c;
   }
-  return cudaSuccess;
+  return scatter_target_rows(ix, p.M, p.h, d_vec, dW, scale, st);
 }
 
 }  // namespace mls

@@ -212,16 +212,35 @@ __device__ __forceinline__ void emit(float* out_row, int vi, const float (&acc)[
   }
 }
 
-// Light rows: warp w of block (x, y) takes light ids x*8 + w, x*8 + w + 8*gridDim.x, ...
-// and their slice y of 32 vectors (one 16-byte vector per lane).
-//   src row of token t: src + t*src_ld + src_off (16-byte vectors)
+// One row-sum job: the rows of token t are src + t*src_ld + src_off (16-byte
+// vectors, n_vec per row); the sums go to out (fp32 rows of n_vec vectors).
+// Several jobs that share the id grouping (the exits of the loss, which share
+// the targets) run in one launch, one per blockIdx.z.
+struct SegJob {
+  const uint4* src;
+  int64_t src_ld;
+  int src_off;
+  int n_vec;
+  const uint4* E;
+  float* out;
+  float scale;
+};
+struct SegJobs {
+  SegJob j[kMaxExits];
+};
+
+// Light rows: warp w of block (x, y, z) takes light ids x*8 + w, x*8 + w + 8*gridDim.x, ...
+// and their slice y of 32 vectors (one 16-byte vector per lane) of job z.
 template <bool BF16, bool TABLE>
-__global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix, const uint4* __restrict__ src,
-                                                           int64_t src_ld, int src_off, int n_vec,
-                                                           const float* __restrict__ coef,
-                                                           const uint4* __restrict__ E, float* __restrict__ out,
-                                                           float scale, int accumulate) {
+__global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix, const SegJobs jobs,
+                                                           const float* __restrict__ coef, int accumulate) {
   constexpr int N = Vec8<BF16>::N;
+  const SegJob& jb = jobs.j[blockIdx.z];
+  const uint4* __restrict__ src = jb.src;
+  const int64_t src_ld = jb.src_ld;
+  const int src_off = jb.src_off;
+  const int n_vec = jb.n_vec;
+  if (static_cast<int>(blockIdx.y) * 32 >= n_vec) return;   // this job's rows are narrower
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int vi = static_cast<int>(blockIdx.y) * 32 + lane;
@@ -248,9 +267,9 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
       for (int b = 0; b < 4; ++b) Vec8<BF16>::add(acc, u[b]);
     }
     for (; p < cnt; ++p) Vec8<BF16>::add(acc, __ldg(src + static_cast<int64_t>(ix.toks[off + p]) * src_ld + src_off + vi));
-    float* out_row = out + v * static_cast<int64_t>(n_vec) * N;
-    const uint4* E_row = TABLE ? E + v * static_cast<int64_t>(n_vec) : nullptr;
-    emit<BF16, TABLE>(out_row, vi, acc, cs, E_row, scale, accumulate != 0);
+    float* out_row = jb.out + v * static_cast<int64_t>(n_vec) * N;
+    const uint4* E_row = TABLE ? jb.E + v * static_cast<int64_t>(n_vec) : nullptr;
+    emit<BF16, TABLE>(out_row, vi, acc, cs, E_row, jb.scale, accumulate != 0);
   }
 }
 
@@ -266,17 +285,21 @@ __global__ void __launch_bounds__(256) zero_absent_rows_kernel(const SegIndexDev
   for (int i = lane; i < f4_per_row; i += 32) o[i] = z;
 }
 
-// One block per (heavy row, slice of 32 vectors); warps split the row's tokens
-// round-robin and are combined in warp order.
+// One block per (heavy row, slice of 32 vectors, job); warps split the row's
+// tokens round-robin and are combined in warp order.
 template <bool BF16, bool TABLE>
-__global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(
-    const SegIndexDev ix, const uint4* __restrict__ src, int64_t src_ld, int src_off, int n_vec,
-    const float* __restrict__ coef, const uint4* __restrict__ E, float* __restrict__ out, float scale,
-    int accumulate) {
+__global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(const SegIndexDev ix, const SegJobs jobs,
+                                                                        const float* __restrict__ coef,
+                                                                        int accumulate) {
   constexpr int N = Vec8<BF16>::N;
   __shared__ float part[kHeavyWarps][32 * N];
   __shared__ float cpart[kHeavyWarps];
-  if (static_cast<int>(blockIdx.x) >= *ix.n_heavy) return;
+  const SegJob& jb = jobs.j[blockIdx.z];
+  const uint4* __restrict__ src = jb.src;
+  const int64_t src_ld = jb.src_ld;
+  const int src_off = jb.src_off;
+  const int n_vec = jb.n_vec;
+  if (static_cast<int>(blockIdx.x) >= *ix.n_heavy || static_cast<int>(blockIdx.y) * 32 >= n_vec) return;
   const int64_t v = ix.heavy[blockIdx.x];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vi = blockIdx.y * 32 + lane;
@@ -322,36 +345,40 @@ __global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(
       ctot += cpart[w];
     }
     if (active) {
-      float* out_row = out + v * static_cast<int64_t>(n_vec) * N;
-      const uint4* E_row = TABLE ? E + v * static_cast<int64_t>(n_vec) : nullptr;
-      emit<BF16, TABLE>(out_row, vi, tot, ctot, E_row, scale, accumulate != 0);
+      float* out_row = jb.out + v * static_cast<int64_t>(n_vec) * N;
+      const uint4* E_row = TABLE ? jb.E + v * static_cast<int64_t>(n_vec) : nullptr;
+      emit<BF16, TABLE>(out_row, vi, tot, ctot, E_row, jb.scale, accumulate != 0);
     }
   }
 }
 
 template <bool BF16, bool TABLE>
-cudaError_t launch_segsum(const SegIndexDev& ix, const uint4* src, int64_t src_ld, int src_off, int n_vec,
-                          const float* coef, const uint4* E, float* out, float scale, int accumulate,
-                          cudaStream_t st) {
+cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs, const float* coef,
+                          int accumulate, cudaStream_t st) {
   constexpr int N = Vec8<BF16>::N;
   if (TABLE && !accumulate) {
     const int64_t blocks = (ix.V * 32 + 255) / 256;
-    zero_absent_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(ix, reinterpret_cast<float4*>(out),
-                                                                          n_vec * N / 4);
+    zero_absent_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        ix, reinterpret_cast<float4*>(jobs.j[0].out), jobs.j[0].n_vec * N / 4);
     note_launches(1);
   }
-  // light rows: about one full wave of 8-warp blocks over (light ids) x (32-vector slices)
+  int slices = 0, total_slices = 0;
+  for (int z = 0; z < njobs; ++z) {
+    const int sz = (jobs.j[z].n_vec + 31) / 32;
+    slices = std::max(slices, sz);
+    total_slices += sz;
+  }
+  // light rows: about one full wave of 8-warp blocks over (light ids) x (32-vector slices of every job)
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int slices = (n_vec + 31) / 32;
-  const int64_t want = (static_cast<int64_t>(sms) * 8 + slices - 1) / slices;
+  const int64_t want = (static_cast<int64_t>(sms) * 8 + total_slices - 1) / total_slices;
   const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(want, (ix.max_light + 7) / 8));
-  segsum_light_kernel<BF16, TABLE><<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices)), 256, 0, st>>>(
-      ix, src, src_ld, src_off, n_vec, coef, E, out, scale, accumulate);
-  dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>(slices));
-  segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, src, src_ld, src_off, n_vec, coef, E,
-                                                                      out, scale, accumulate);
+  segsum_light_kernel<BF16, TABLE>
+      <<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices), static_cast<unsigned>(njobs)), 256, 0, st>>>(
+          ix, jobs, coef, accumulate);
+  dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>(slices), static_cast<unsigned>(njobs));
+  segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, jobs, coef, accumulate);
   note_launches(2);
   return cudaGetLastError();
 }
@@ -426,17 +453,18 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
 cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
                                const float* coef, float ge, const void* E, float* dE, bool accumulate,
                                cudaStream_t st) {
-  const uint4* src = static_cast<const uint4*>(dy);
-  const int64_t ld = d_vec + dl_vec;
-  const uint4* e = static_cast<const uint4*>(E);
-  return bf16 ? launch_segsum<true, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, ge, accumulate, st)
-              : launch_segsum<false, true>(ix, src, ld, d_vec, dl_vec, coef, e, dE, ge, accumulate, st);
+  SegJobs jobs{};
+  jobs.j[0] = SegJob{static_cast<const uint4*>(dy), d_vec + dl_vec, d_vec, dl_vec, static_cast<const uint4*>(E), dE, ge};
+  return bf16 ? launch_segsum<true, true>(ix, jobs, 1, coef, accumulate, st)
+              : launch_segsum<false, true>(ix, jobs, 1, coef, accumulate, st);
 }
 
-cudaError_t scatter_target_rows(const SegIndexDev& ix, const void* h, int d_vec, float* dW, float scale,
-                                cudaStream_t st) {
-  const uint4* src = static_cast<const uint4*>(h);
-  return launch_segsum<true, false>(ix, src, d_vec, 0, d_vec, nullptr, nullptr, dW, scale, 1, st);
+cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,
+                                float* const* dW, const float* scale, cudaStream_t st) {
+  SegJobs jobs{};
+  for (int z = 0; z < njobs; ++z)
+    jobs.j[z] = SegJob{static_cast<const uint4*>(h[z]), d_vec[z], 0, d_vec[z], nullptr, dW[z], scale[z]};
+  return launch_segsum<true, false>(ix, jobs, njobs, nullptr, 1, st);
 }
 
 }  // namespace mls
