@@ -151,7 +151,9 @@ VARIANTS = [1, 2, 4, 3, 5, 6, 7]   # no rescale, zero fill, stop-gradient and th
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
-@pytest.mark.parametrize("name,j,small", [("main3", 1, dict(batch=1, seq=300, V=512)),
+@pytest.mark.parametrize("name,j,small", [("main3", 1, dict(batch=1, seq=300, V=512)),    # long rows
+                                          ("main3", 0, dict(batch=1, seq=300, V=512)),    # prefetching forward
+                                          ("proxy2", 0, dict(batch=1, seq=300, V=256)),   # prefetching both ways
                                           ("tiny3", 0, None)])
 def test_junction_variants_match_oracle(variant, name, j, small):
     cfg = _cfg(name, small)
