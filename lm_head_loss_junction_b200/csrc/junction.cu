@@ -451,6 +451,81 @@ __global__ void __launch_bounds__(256, 2) junction_bwd_pipe_kernel(
   }
 }
 
+// Short rows (at most CAP = 4 vectors of o and ECAP = 5 of the embedding per
+// lane): every row of the token (o, g_o, e, g_e) is loaded into registers
+// before any reduction, so a token costs one round trip to memory; the
+// embedding row is read once.
+template <bool BF16, int CAP, int ECAP>
+__global__ void __launch_bounds__(256, 2) junction_bwd_rows_kernel(
+    const int32_t* __restrict__ x, int64_t T, const uint4* __restrict__ o, int d_vec,
+    const uint4* __restrict__ E, int64_t V, int dl_vec, const uint4* __restrict__ dy,
+    uint4* __restrict__ do_out, uint4* __restrict__ de_out, float* __restrict__ coef_out,
+    int32_t* __restrict__ status, uint32_t variant) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int dp_vec = d_vec + dl_vec;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  for (int64_t t = warp0; t < T; t += nwarps) {
+    const int32_t id = __ldg(x + t);
+    const bool bad = (id < 0) || (static_cast<int64_t>(id) >= V);
+    const uint4* orow = o + t * d_vec;
+    const uint4* grow = dy + t * dp_vec;
+    const uint4* erow = E + static_cast<int64_t>(bad ? 0 : id) * dl_vec;
+    uint4 oc[CAP], gc[CAP], ec[ECAP], gec[ECAP];
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      oc[j] = (i < d_vec) ? __ldcs(orow + i) : zero;
+      gc[j] = (i < d_vec) ? __ldcs(grow + i) : zero;
+    }
+#pragma unroll
+    for (int j = 0; j < ECAP; ++j) {
+      const int i = j * 32 + lane;
+      ec[j] = (i < dl_vec) ? __ldg(erow + i) : zero;
+      gec[j] = (i < dl_vec) ? __ldcs(grow + d_vec + i) : zero;
+    }
+    float so = 0.f, sog = 0.f, se = 0.f;
+#pragma unroll
+    for (int j = 0; j < ECAP; ++j) se += sumsq<BF16>(ec[j]);
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      so += sumsq<BF16>(oc[j]);
+      sog += dotv<BF16>(oc[j], gc[j]);
+    }
+    so = warp_sum(so);
+    sog = warp_sum(sog);
+    se = warp_sum(se);
+    const float n_o = fmaxf(sqrtf(so), kJunctionEps);
+    const float n_e = sqrtf(se);
+    const float s = n_e / n_o;
+    const float ug = sog / n_o;
+    float a = s, b = s * ug / n_o, c = (n_e > 0.f) ? ug / n_e : 0.f;
+    if (variant & kNoRescale) { a = 1.f; b = 0.f; c = 0.f; }   // y = [o ; .]
+    if (variant & kStopGrad) { a = 0.f; b = 0.f; }              // nothing flows into o
+    const float ge = (variant & kZeroFill) ? 0.f : 1.f;         // the fill does not carry g_e
+    if (bad) { a = 0.f; b = 0.f; c = 0.f; }
+    uint4* drow = do_out + t * d_vec;
+#pragma unroll
+    for (int j = 0; j < CAP; ++j) {
+      const int i = j * 32 + lane;
+      if (i < d_vec) drow[i] = axpby_vec<BF16>(a, gc[j], b, oc[j]);
+    }
+    if (de_out != nullptr) {
+      uint4* erow_out = de_out + t * dl_vec;
+#pragma unroll
+      for (int j = 0; j < ECAP; ++j) {
+        const int i = j * 32 + lane;
+        if (i < dl_vec) erow_out[i] = bad ? zero : lincomb_vec<BF16>(ge, gec[j], c, ec[j]);
+      }
+    }
+    if (lane == 0) {
+      if (coef_out != nullptr) coef_out[t] = c;
+      if (bad) set_flag(status, MLS_DEVFLAG_BAD_ID);
+    }
+  }
+}
+
 int pick_cap(int nvec) {
   const int per_lane = (nvec + 31) / 32;
   static const int caps[] = {1, 2, 4, 6, 8, 9, 12, 16};
@@ -552,8 +627,22 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
 #undef MLS_JBP
   } else {
 #define MLS_JB(C, B) junction_bwd_kernel<BF16, C, B><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status, a.variant)
-    if (cap == 4) MLS_JB(4, 2);
-    else MLS_JB(2, 4);
+#define MLS_JBR(C, EC) junction_bwd_rows_kernel<BF16, C, EC><<<grid, 256, 0, st>>>(a.x, a.T, o, d_vec, E, a.V, dl_vec, dy, dout, deo, coef, a.status, a.variant)
+    const int ecap = (dl_vec + 31) / 32;              // exact: every register row is used
+    if (cap == 4 && ecap <= 5) {
+      switch (ecap) {
+        case 1: MLS_JBR(4, 1); break;
+        case 2: MLS_JBR(4, 2); break;
+        case 3: MLS_JBR(4, 3); break;
+        case 4: MLS_JBR(4, 4); break;
+        default: MLS_JBR(4, 5); break;
+      }
+    } else if (cap == 4) {
+      MLS_JB(4, 2);
+    } else {
+      MLS_JB(2, 4);
+    }
+#undef MLS_JBR
 #undef MLS_JB
   }
   note_launches(1);
