@@ -84,13 +84,22 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     G_m = lambda_m grad_scale/T ((1 - alpha_d)(q_m - onehot) + alpha_d q_m (g - K_t)),
     g_v = log(q_v / mu_v) / 2,  K_t = sum_v q_v g_v = KL(q_m || mu) / 2,
     and K_t is returned per token in "J" (KL(p_M || mu)/2 in "Jp").
+    distill="accept" takes the acceptance loss the same section lists: train
+    the draft for the probability that its sampled token is accepted,
+    beta = sum_v min(q_v, p_v), i.e. KD_m = mean_t (1 - beta_t), the total
+    variation distance.  Its student (sub)gradient, with the indicator of
+    q_v < p_v taken strictly, is
+    G_m = lambda_m grad_scale/T ((1 - alpha_d)(q_m - onehot) + alpha_d q_m (A_t - [q < p])),
+    A_t = sum_{v: q_v < p_v} q_v, returned per token in "A" (and
+    B_t = beta_t - A_t = sum_{v: q_v >= p_v} p_v in "B").
     teacher_grad: the largest exit also receives the gradient of every
     distillation term (no stop-gradient; the pages leave this open).  With
     T_m = d KD_m / d l_M, the teacher's logit gradient gains
     lambda_m alpha_d T_m per smaller exit m, where
       cross-entropy:  T_m = -p_M (l_m - S_m)           (S_m = sum_v p_M l_m)
       reverse KL:     T_m = p_M - q_m
-      Jensen-Shannon: T_m = p_M (log(p_M / mu) / 2 - KL(p_M || mu) / 2).
+      Jensen-Shannon: T_m = p_M (log(p_M / mu) / 2 - KL(p_M || mu) / 2)
+      acceptance:     T_m = p_M (B_t - [q_m >= p_M]).
 
     Returns a dict with
       ce_lm [M], ce_kd [M-1], loss (scalar)         -- means over the tokens
@@ -105,12 +114,13 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
     Tn = idx.shape[0]
     Ws = [_f64(w) for w in W]
     V = Ws[0].shape[0]
-    if distill not in ("ce", "reverse_kl", "js"):
+    if distill not in ("ce", "reverse_kl", "js", "accept"):
         raise ValueError(distill)
     out = {
         "lse": np.zeros((M, Tn)), "tgt": np.zeros((M, Tn)), "S": np.zeros((max(M - 1, 0), Tn)),
         "R": np.zeros((max(M - 1, 0), Tn)), "J": np.zeros((max(M - 1, 0), Tn)),
-        "Jp": np.zeros((max(M - 1, 0), Tn)),
+        "Jp": np.zeros((max(M - 1, 0), Tn)), "A": np.zeros((max(M - 1, 0), Tn)),
+        "B": np.zeros((max(M - 1, 0), Tn)),
         "ce_lm_sum": np.zeros(M), "ce_kd_sum": np.zeros(max(M - 1, 0)),
     }
     if need_grad:
@@ -132,7 +142,7 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             out["lse"][m, b0:b0 + n] = lse[m]
             out["tgt"][m, b0:b0 + n] = logits[m][ar, yb]
             out["ce_lm_sum"][m] += np.sum(lse[m] - logits[m][ar, yb])
-        rkl, logmix, jq, jps = [], [], [], []
+        rkl, logmix, jq, jps, accA, accB = [], [], [], [], [], []
         for m in range(M - 1):
             out["S"][m, b0:b0 + n] = np.sum(pM * logits[m], axis=1)
             q = np.exp(logq[m])
@@ -145,12 +155,20 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
             jps.append(jp)
             out["J"][m, b0:b0 + n] = 0.5 * jq[m]
             out["Jp"][m, b0:b0 + n] = 0.5 * jp
+            # acceptance: beta = sum min(q, p) = A + B with A over q < p, B over q >= p
+            below = q < pM
+            accA.append(np.sum(np.where(below, q, 0.0), axis=1))
+            accB.append(np.sum(np.where(below, 0.0, pM), axis=1))
+            out["A"][m, b0:b0 + n] = accA[m]
+            out["B"][m, b0:b0 + n] = accB[m]
             if distill == "ce":
                 out["ce_kd_sum"][m] += np.sum(-np.sum(pM * logq[m], axis=1))
             elif distill == "reverse_kl":
                 out["ce_kd_sum"][m] += np.sum(rkl[m])
-            else:
+            elif distill == "js":
                 out["ce_kd_sum"][m] += np.sum(0.5 * (jq[m] + jp))
+            else:
+                out["ce_kd_sum"][m] += np.sum(1.0 - (accA[m] + accB[m]))
         if need_grad:
             onehot = np.zeros((n, V))
             onehot[ar, yb] = 1.0
@@ -161,8 +179,11 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
                 elif m < M - 1 and distill == "reverse_kl":
                     kd = q * (logq[m] - logq[M - 1] - rkl[m][:, None])
                     G = lam[m] * g * ((1.0 - alpha_d) * (q - onehot) + alpha_d * kd)
-                elif m < M - 1:
+                elif m < M - 1 and distill == "js":
                     kd = q * (0.5 * (logq[m] - logmix[m]) - 0.5 * jq[m][:, None])
+                    G = lam[m] * g * ((1.0 - alpha_d) * (q - onehot) + alpha_d * kd)
+                elif m < M - 1:
+                    kd = q * (accA[m][:, None] - (q < pM).astype(np.float64))
                     G = lam[m] * g * ((1.0 - alpha_d) * (q - onehot) + alpha_d * kd)
                 else:
                     G = lam[m] * g * (q - onehot)
@@ -172,8 +193,11 @@ def multiexit_loss(y, h, W, alpha_d=0.3, grad_scale=1.0, need_grad=True,
                                 Ts = -pM * (logits[s] - np.sum(pM * logits[s], axis=1)[:, None])
                             elif distill == "reverse_kl":
                                 Ts = pM - np.exp(logq[s])
-                            else:
+                            elif distill == "js":
                                 Ts = pM * (0.5 * (logq[M - 1] - logmix[s]) - 0.5 * jps[s][:, None])
+                            else:
+                                qs = np.exp(logq[s])
+                                Ts = pM * (accB[s][:, None] - (qs >= pM).astype(np.float64))
                             G = G + lam[s] * g * alpha_d * Ts
                 out["dh"][m][b0:b0 + n] = G @ Ws[m]
                 out["dW"][m] += G.T @ hb[m]

@@ -414,7 +414,7 @@ def test_js_gradients_match_finite_differences():
 
 
 # ------------------------------------------------------------------ teacher gradient (no stop-gradient)
-@pytest.mark.parametrize("distill", ["ce", "reverse_kl", "js"])
+@pytest.mark.parametrize("distill", ["ce", "reverse_kl", "js", "accept"])
 def test_teacher_gradient_matches_finite_differences_of_the_whole_loss(distill):
     # Without the stop-gradient every parameter's gradient, the largest exit's
     # included, is the plain derivative of the total loss.
@@ -459,3 +459,59 @@ def test_teacher_gradient_of_identical_exits_ce():
     H = -np.sum(p * np.log(p), axis=1)
     extra = 0.4 / 5 * (-p * (np.log(p) + H[:, None]))
     np.testing.assert_allclose(a["dh"][1] - b["dh"][1], extra @ W[1], rtol=1e-10, atol=1e-15)
+
+
+# ------------------------------------------------------------------ acceptance loss
+def test_acceptance_is_total_variation_written_out():
+    # 1 - sum min(q, p) = (1/2) sum |q - p| (total variation), token by token
+    y, h, W = _rand_suite(M=3, T=6, D=(3, 5, 8), V=11, seed=61, scale=2.5)
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="accept")
+    pM = softmax_rows(h[2] @ W[2].T)
+    for m in range(2):
+        q = softmax_rows(h[m] @ W[m].T)
+        tv = np.array([0.5 * sum(abs(q[t, v] - pM[t, v]) for v in range(11)) for t in range(6)])
+        np.testing.assert_allclose(r["ce_kd"][m], tv.mean(), rtol=1e-12)
+        # A = sum over q < p of q, B = sum over q >= p of p, beta = A + B
+        a = np.array([sum(q[t, v] for v in range(11) if q[t, v] < pM[t, v]) for t in range(6)])
+        np.testing.assert_allclose(r["A"][m], a, rtol=1e-12)
+        np.testing.assert_allclose(1.0 - (r["A"][m] + r["B"][m]), tv, rtol=1e-10, atol=1e-15)
+
+
+def test_acceptance_two_class_closed_form_and_limits():
+    # student (b, 0), teacher (a, 0): beta = 1 - |s(a) - s(b)|
+    a, b = 1.2, -0.7
+    y = np.array([0])
+    h = [np.array([[b]]), np.array([[a]])]
+    W = [np.array([[1.0], [0.0]]), np.array([[1.0], [0.0]])]
+    r = multiexit_loss(y, h, W, alpha_d=0.3, distill="accept")
+    kd = abs(_sig(a) - _sig(b))
+    np.testing.assert_allclose(r["ce_kd"][0], kd, rtol=1e-13)
+    np.testing.assert_allclose(r["loss"], 0.7 * _softplus(-b) + 0.3 * kd + _softplus(-a), rtol=1e-13)
+    # identical exits: beta = 1, no distillation gradient
+    y, h, W = _rand_suite(M=2, T=5, D=(4, 4), V=9, seed=62)
+    h[0], W[0] = h[1].copy(), W[1].copy()
+    r = multiexit_loss(y, h, W, alpha_d=0.4, distill="accept")
+    c = multiexit_loss(y, h, W, alpha_d=0.0, distill="accept")
+    np.testing.assert_allclose(r["ce_kd"], 0.0, atol=1e-14)
+    np.testing.assert_allclose(r["dh"][0], 0.6 * c["dh"][0], rtol=1e-12, atol=1e-15)
+
+
+def test_acceptance_gradients_match_finite_differences():
+    M, T, D, V, alpha = 3, 3, (3, 4, 5), 7, 0.45
+    y, h, W = _rand_suite(M=M, T=T, D=D, V=V, seed=63, scale=2.0)
+    lam = [1.3, 0.6, 0.9]
+    kw = dict(alpha_d=alpha, distill="accept", exit_weights=lam)
+    r = multiexit_loss(y, h, W, grad_scale=0.9, **kw)
+    eps = 1e-6
+    for s in range(2):
+        for arr, grad in ((h, r["dh"][s]), (W, r["dW"][s])):
+            num = np.zeros_like(arr[s])
+            for idx in np.ndindex(arr[s].shape):
+                b = arr[s][idx]
+                arr[s][idx] = b + eps
+                lp = multiexit_loss(y, h, W, need_grad=False, **kw)["loss"]
+                arr[s][idx] = b - eps
+                lm = multiexit_loss(y, h, W, need_grad=False, **kw)["loss"]
+                arr[s][idx] = b
+                num[idx] = 0.9 * (lp - lm) / (2 * eps)
+            np.testing.assert_allclose(grad, num, rtol=1e-6, atol=5e-9)
