@@ -230,8 +230,8 @@ mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int6
  *   losses  device f32 [2M]: CE_LM[0..M-1], CE_KD[0..M-2], L
  *   stats   device f32 [3M-1, T]: rows 0..M-1 lse_m, rows M..2M-1 the target
  *           logits l_m,y, rows 2M..3M-2 S_m (the _opts form: the statistic of
- *           the chosen distillation, and for Jensen-Shannon with the teacher
- *           gradient 4M-2 rows, see mls_loss_options).  Kept for the
+ *           the chosen distillation, and for Jensen-Shannon or acceptance with
+ *           the teacher gradient 4M-2 rows, see mls_loss_options).  Kept for the
  *           backward pass.
  */
 mls_status mls_multiexit_loss_fwd(int M, int64_t T, int64_t V, const int64_t* D,
@@ -264,7 +264,8 @@ mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
 typedef enum {
   MLS_DISTILL_CE = 0,          /* token-level cross-entropy to the largest exit's softmax (default) */
   MLS_DISTILL_REVERSE_KL = 1,  /* KL(q_m || p_M), an alternative the pages' follow-ups propose   */
-  MLS_DISTILL_JS = 2           /* Jensen-Shannon divergence of q_m and p_M, the other one          */
+  MLS_DISTILL_JS = 2,          /* Jensen-Shannon divergence of q_m and p_M                         */
+  MLS_DISTILL_ACCEPT = 3       /* 1 - sum_v min(q_m, p_M): acceptance of a drafted token           */
 } mls_distill;
 
 /*
@@ -288,6 +289,13 @@ typedef enum {
  *                 rows 2M..3M-2.  Its forward takes a second pass over the
  *                 logits (the divergence needs the final normalisers); the
  *                 backward call must get the same option.
+ *                 MLS_DISTILL_ACCEPT (same section: train the draft for
+ *                 acceptance): KD_m = mean_t (1 - beta_t), beta = sum_v
+ *                 min(q_m, p_M), the total variation distance; student
+ *                 (sub)gradient G_m = grad_scale/T ((1 - alpha_d)(q_m - onehot(y))
+ *                 + alpha_d q_m (A_t - [q_m < p_M])), A_t = sum over q < p of q,
+ *                 stored by the forward call in stats rows 2M..3M-2.  Its
+ *                 forward takes a second pass like Jensen-Shannon.
  *                 Other values return MLS_ERR_INVALID_ARG.
  *   teacher_grad  0 (default): the largest exit's softmax in the distillation
  *                 terms is a constant (stop-gradient).  1: it is not, and the
@@ -295,9 +303,11 @@ typedef enum {
  *                 lambda_m alpha_d dKD_m/dl_M:
  *                   MLS_DISTILL_CE:         -p_M (l_m - S_m),  S_m = sum_v p_M l_m
  *                   MLS_DISTILL_REVERSE_KL:  p_M - q_m
- *                   MLS_DISTILL_JS:          p_M (log(p_M/mu)/2 - KL(p_M || mu)/2).
+ *                   MLS_DISTILL_JS:          p_M (log(p_M/mu)/2 - KL(p_M || mu)/2)
+ *                   MLS_DISTILL_ACCEPT:      p_M (B_t - [q_m >= p_M]), B_t = sum over q >= p of p.
  *                 Pass the same options to both calls.  With MLS_DISTILL_JS
- *                 the forward call then also writes KL(p_M || mu)/2 per token
+ *                 or MLS_DISTILL_ACCEPT the forward call then also writes the
+ *                 teacher-side statistic (KL(p_M || mu)/2, or B_t) per token
  *                 into stats rows 3M-1 .. 4M-3, so stats must have 4M-2 rows
  *                 (otherwise 3M-1).  The pages leave the teacher's gradient
  *                 open.

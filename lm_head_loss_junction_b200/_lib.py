@@ -121,7 +121,7 @@ def i64_array(vals):
     return arr
 
 
-MLS_DISTILL = {"ce": 0, "reverse_kl": 1, "js": 2}
+MLS_DISTILL = {"ce": 0, "reverse_kl": 1, "js": 2, "accept": 3}
 
 
 def loss_options(exit_weights=None, distill="ce", teacher_grad=False):

@@ -153,13 +153,13 @@ def _workspace(ws, nbytes, device):
 def multiexit_loss_fwd(y: torch.Tensor, h: List[torch.Tensor], W: List[torch.Tensor], alpha_d: float = 0.3, *,
                        losses=None, stats=None, workspace=None, exit_weights=None, distill="ce",
                        teacher_grad: bool = False, status=None, stream=None):
-    """Returns (losses [2M], stats [3M-1, T], or [4M-2, T] for Jensen-Shannon with the
-    teacher gradient) (see mls_multiexit_loss_fwd; any option uses mls_multiexit_loss_fwd_opts)."""
+    """Returns (losses [2M], stats [3M-1, T], or [4M-2, T] for Jensen-Shannon or acceptance
+    with the teacher gradient) (see mls_multiexit_loss_fwd; any option uses mls_multiexit_loss_fwd_opts)."""
     M, T, V, D, dt = _loss_common(y, h, W)
     dev = y.device
     if losses is None:
         losses = torch.empty(2 * M, dtype=torch.float32, device=dev)
-    rows = 4 * M - 2 if (distill == "js" and teacher_grad and M > 1) else 3 * M - 1
+    rows = 4 * M - 2 if (distill in ("js", "accept") and teacher_grad and M > 1) else 3 * M - 1
     if stats is None:
         stats = torch.empty((rows, T), dtype=torch.float32, device=dev)
     elif stats.shape[0] < rows:

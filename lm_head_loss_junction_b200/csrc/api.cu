@@ -112,7 +112,8 @@ mls_status build_problem(int M, int64_t T, int64_t V, const int64_t* D, const in
 
 mls_status apply_options(const mls_loss_options* opts, LossProblem* p) {
   if (opts == nullptr) return MLS_OK;
-  if (opts->distill != MLS_DISTILL_CE && opts->distill != MLS_DISTILL_REVERSE_KL && opts->distill != MLS_DISTILL_JS)
+  if (opts->distill != MLS_DISTILL_CE && opts->distill != MLS_DISTILL_REVERSE_KL && opts->distill != MLS_DISTILL_JS &&
+      opts->distill != MLS_DISTILL_ACCEPT)
     return MLS_ERR_INVALID_ARG;
   p->distill = opts->distill;
   if (opts->teacher_grad != 0 && opts->teacher_grad != 1) return MLS_ERR_INVALID_ARG;

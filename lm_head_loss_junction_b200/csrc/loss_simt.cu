@@ -27,7 +27,7 @@ struct SimtDev {
   const float* W[kMaxExits];
   float alpha_d;
   float exit_w[kMaxExits];
-  int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
+  int distill;               // 0: cross-entropy, 1: KL(q_m || p_M), 2: Jensen-Shannon, 3: 1 - sum min(q, p)
   int teacher_grad;          // 1: no stop-gradient on the largest exit
   int32_t* status;
   float* dh[kMaxExits];
@@ -172,9 +172,10 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
     if (bad) set_flag(p.status, MLS_DEVFLAG_BAD_ID);
     for (int m = 0; m < M; ++m) lse_sh[m] = stats[m * p.T + t];
   }
-  if (p.distill != 2 || S == 0) return;
-  // Jensen-Shannon: second walk over the vocabulary with the final normalisers,
-  // sum q log(q/mu) and sum p log(p/mu) per student (mu = (q + p)/2).
+  if ((p.distill != 2 && p.distill != 3) || S == 0) return;
+  // Jensen-Shannon or acceptance: second walk over the vocabulary with the final
+  // normalisers; Jensen-Shannon sums q log(q/mu) and p log(p/mu) (mu = (q + p)/2),
+  // acceptance sums q where q < p (A) and p where q >= p (B).
   __syncthreads();
   float lse[kMaxExits];
   for (int m = 0; m < M; ++m) lse[m] = lse_sh[m];
@@ -193,9 +194,14 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
     const float pv = expf(lp);
     for (int s = 0; s < S; ++s) {
       const float lq = l[s] - lse[s];
-      const float d = lp - lq;
-      jq[s] = fmaf(expf(lq), kLn2 - softplus(d), jq[s]);
-      jp[s] = fmaf(pv, kLn2 - softplus(-d), jp[s]);
+      if (p.distill == 3) {
+        if (lq < lp) jq[s] += expf(lq);
+        else jp[s] += pv;
+      } else {
+        const float d = lp - lq;
+        jq[s] = fmaf(expf(lq), kLn2 - softplus(d), jq[s]);
+        jp[s] = fmaf(pv, kLn2 - softplus(-d), jp[s]);
+      }
     }
   }
   for (int s = 0; s < S; ++s) {
@@ -211,9 +217,15 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       const float a = red[(2 * s) * kSimtThreads], b = red[(2 * s + 1) * kSimtThreads];
-      stats[(2 * M + s) * p.T + t] = 0.5f * a;
-      if (p.teacher_grad) stats[(3 * M - 1 + s) * p.T + t] = 0.5f * b;   // KL(p_T || mu)/2
-      terms[(M + s) * p.T + t] = bad ? 0.f : 0.5f * (a + b);
+      if (p.distill == 3) {                 // A, then B for the teacher; the term is 1 - (A + B)
+        stats[(2 * M + s) * p.T + t] = a;
+        if (p.teacher_grad) stats[(3 * M - 1 + s) * p.T + t] = b;
+        terms[(M + s) * p.T + t] = bad ? 0.f : 1.f - (a + b);
+      } else {
+        stats[(2 * M + s) * p.T + t] = 0.5f * a;
+        if (p.teacher_grad) stats[(3 * M - 1 + s) * p.T + t] = 0.5f * b;   // KL(p_T || mu)/2
+        terms[(M + s) * p.T + t] = bad ? 0.f : 0.5f * (a + b);
+      }
     }
   }
 }
@@ -236,7 +248,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
   for (int m = 0; m < M; ++m) lse[m] = stats[m * p.T + t];
   // reverse KL: KL(q_m || p_T) = R - lse_m + lse_T; Jensen-Shannon: K = KL(q_m || mu)/2 as stored
   for (int m = 0; m < M - 1; ++m)
-    kl[m] = (p.distill == 2) ? stats[(2 * M + m) * p.T + t] : stats[(2 * M + m) * p.T + t] - lse[m] + lse[M - 1];
+    kl[m] = (p.distill >= 2) ? stats[(2 * M + m) * p.T + t] : stats[(2 * M + m) * p.T + t] - lse[m] + lse[M - 1];
   const float a = p.alpha_d;
   for (int64_t v = tid; v < p.V; v += kSimtThreads) {
     float l[kMaxExits];
@@ -256,7 +268,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
         if (p.teacher_grad) {
           // distillation gradient of every smaller exit s on the teacher's logits:
           //   cross-entropy -p_T (l_s - S_s);  reverse KL p_T - q_s;
-          //   Jensen-Shannon p_T (log(p_T/mu_s)/2 - K^p_s), log(p/mu) = ln 2 - softplus(log q - log p)
+          //   Jensen-Shannon p_T (log(p_T/mu_s)/2 - K^p_s), log(p/mu) = ln 2 - softplus(log q - log p);
+          //   acceptance p_T (B_s - [q_s >= p_T])
           float extra = 0.f;
           for (int s = 0; s < M - 1; ++s) {
             float ts;
@@ -265,6 +278,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
             } else if (p.distill == 2) {
               const float lq = l[s] - lse[s], lp = l[M - 1] - lse[M - 1];
               ts = pT * (0.5f * (kLn2 - softplus(lq - lp)) - stats[(3 * M - 1 + s) * p.T + t]);
+            } else if (p.distill == 3) {    // acceptance: p_T (B_s - [q_s >= p_T])
+              const float lq = l[s] - lse[s], lp = l[M - 1] - lse[M - 1];
+              ts = pT * (stats[(3 * M - 1 + s) * p.T + t] - ((lq < lp) ? 0.f : 1.f));
             } else {
               ts = -pT * (l[s] - stats[(2 * M + s) * p.T + t]);
             }
@@ -279,10 +295,14 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
         const float q = __expf(l[m] - lse[m]);
         const float d = (l[m] - lse[m]) - (l[M - 1] - lse[M - 1]) - kl[m];
         g = (1.f - a) * (q - hot) + a * q * d;
-      } else {
+      } else if (p.distill == 2) {
         const float q = __expf(l[m] - lse[m]);
         const float d = 0.5f * (kLn2 - softplus((l[M - 1] - lse[M - 1]) - (l[m] - lse[m]))) - kl[m];
         g = (1.f - a) * (q - hot) + a * q * d;
+      } else {                              // acceptance: q (A - [q < p])
+        const float q = __expf(l[m] - lse[m]);
+        const float ind = ((l[m] - lse[m]) < (l[M - 1] - lse[M - 1])) ? 1.f : 0.f;
+        g = (1.f - a) * (q - hot) + a * q * (kl[m] - ind);
       }
       G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : p.exit_w[m] * g;
     }

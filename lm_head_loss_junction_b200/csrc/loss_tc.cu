@@ -67,7 +67,7 @@ struct LossArgs {
   int n_tt, n_vt, num_tiles, group_tt;
   const int32_t* y;
   float alpha;                 // alpha_d
-  int distill;                 // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
+  int distill;                 // 0: cross-entropy, 1: KL(q_m || p_M), 2: Jensen-Shannon, 3: 1 - sum min(q, p)
   float exit_w[kMaxExits];     // per-exit weights (teacher-gradient backward only)
   float student_wsum;          // sum of the smaller exits' weights
   float* partial;              // forward: [2 n_vt][2M-1][T]
@@ -192,7 +192,7 @@ __device__ __forceinline__ void store_g_chunk(uint8_t* stage, int lane, const ui
 }
 
 // ------------------------------------------------------------------ loss tile kernel
-// DISTILL (0 cross-entropy, 1 reverse KL, 2 Jensen-Shannon) is a template
+// DISTILL (0 cross-entropy, 1 reverse KL, 2 Jensen-Shannon, 3 acceptance) is a template
 // parameter so that each form gets its own register allocation.  TGRAD (the
 // backward without the teacher's stop-gradient) holds the teacher's logits in
 // region 0 while the students pass through region 1, accumulates each
@@ -225,9 +225,11 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   const int nslots = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   constexpr bool rkl = (DISTILL == 1);
   constexpr bool jsd = (DISTILL == 2);
+  constexpr bool accd = (DISTILL == 3);
   // The statistics of the Jensen-Shannon form are the cross-entropy ones (it
   // needs the final normalisers, so its divergence has a pass of its own).
-  constexpr bool hold = (MODE == kModeAgree) || (MODE == kModeJS) || rkl || (MODE == kModeGrad && (jsd || TGRAD));
+  constexpr bool hold =
+      (MODE == kModeAgree) || (MODE == kModeJS) || rkl || (MODE == kModeGrad && (jsd || accd || TGRAD));
   static_assert(!TGRAD || MODE == kModeGrad, "teacher gradient: backward only");
 
   if (threadIdx.x == 0) {
@@ -571,8 +573,8 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             prow[static_cast<int64_t>(3 * M - 2 + m) * a.T] = __int_as_float(mxi);
           }
         } else if (MODE == kModeJS) {
-          // ---------------- Jensen-Shannon divergence to the largest exit, with the final
-          // normalisers: per element, with d = log p - log q,
+          // ---------------- second pass with the final normalisers, Jensen-Shannon or
+          // acceptance.  Jensen-Shannon, per element with d = log p - log q:
           //   log(q/mu) = ln 2 - softplus(d),  log(p/mu) = ln 2 - softplus(-d).
           float jq = 0.f, jp = 0.f;
           if (live && j > 0) {
@@ -587,10 +589,16 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
               for (int k = 0; k < 32; ++k) {
                 const float lq = r[k] - lse;
                 const float lp = lt[k] - lseT;
-                const float d = lp - lq;
-                const float sp = __logf(1.f + __expf(-fabsf(d)));
-                jq = fmaf(exp2f(lq * kLog2e), kLn2 - fmaxf(d, 0.f) - sp, jq);
-                jp = fmaf(exp2f(lp * kLog2e), kLn2 - fmaxf(-d, 0.f) - sp, jp);
+                if constexpr (accd) {
+                  // acceptance: A = sum of q where q < p, B = sum of p where q >= p (beta = A + B)
+                  if (lq < lp) jq += exp2f(lq * kLog2e);
+                  else jp += exp2f(lp * kLog2e);
+                } else {
+                  const float d = lp - lq;
+                  const float sp = __logf(1.f + __expf(-fabsf(d)));
+                  jq = fmaf(exp2f(lq * kLog2e), kLn2 - fmaxf(d, 0.f) - sp, jq);
+                  jp = fmaf(exp2f(lp * kLog2e), kLn2 - fmaxf(-d, 0.f) - sp, jp);
+                }
               }
             }
           }
@@ -626,8 +634,9 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             //   log q - log p - KL(q_m || p_T) = l_m - l_T - R_m;  Jensen-Shannon: K = KL(q_m || mu) / 2
             const float klt = (hold && j > 0 && valid) ? a.stats[static_cast<int64_t>(2 * M + m) * a.T + t] : 0.f;
             // Jensen-Shannon with the teacher gradient: K^p = KL(p_T || mu)/2, stored by the forward pass
-            const float kpt = (TGRAD && jsd && j > 0 && valid) ? a.stats[static_cast<int64_t>(3 * M - 1 + m) * a.T + t]
-                                                               : 0.f;
+            const float kpt = (TGRAD && (jsd || accd) && j > 0 && valid)
+                                  ? a.stats[static_cast<int64_t>(3 * M - 1 + m) * a.T + t]
+                                  : 0.f;
             const uint32_t wm2 = TGRAD ? pack_p2(a.exit_w[m], a.exit_w[m]) : 0u;
             // unrolled where a register array is indexed by c (the teacher's
             // packed probabilities, or the teacher-gradient accumulator)
@@ -676,6 +685,13 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                   if (TGRAD)                       // sum_m w_m (log(p/mu_m)/2 - K^p_m)
                     pt[c][k / 2] = hfma_p2(wm2, pack_p2(0.5f * (kLn2 - sp0 + x0) - kpt, 0.5f * (kLn2 - sp1 + x1) - kpt),
                                            pt[c][k / 2]);
+                } else if (accd) {                 // student: G' = q ((1 - a) + a (A - [q < p]))
+                  const float i0 = (r[kk] - lse < lt[kk] - lseT) ? 1.f : 0.f;
+                  const float i1 = (r[kk + 1] - lse < lt[kk + 1] - lseT) ? 1.f : 0.f;
+                  g0 = e0 * fmaf(al, klt - i0, 1.f - al);
+                  g1 = e1 * fmaf(al, klt - i1, 1.f - al);
+                  if (TGRAD)                       // sum_m w_m (B_m - [q_m >= p])
+                    pt[c][k / 2] = hfma_p2(wm2, pack_p2(kpt - (1.f - i0), kpt - (1.f - i1)), pt[c][k / 2]);
                 } else {                           // student: G' = q - alpha_d p_T
                   float p0, p1;
                   if (hold) {
@@ -703,6 +719,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
             //   cross-entropy:  w_T p - a p sum_m w_m (l_m - S_m)
             //   reverse KL:     (w_T + a sum_m w_m) p - a sum_m w_m q_m
             //   Jensen-Shannon: w_T p + a p sum_m w_m (log(p/mu_m)/2 - K^p_m)
+            //   acceptance:     w_T p + a p sum_m w_m (B_m - [q_m >= p])
             const float wT = a.exit_w[M - 1];
             const float cp = rkl ? fmaf(al, a.student_wsum, wT) : wT;
 #pragma unroll
@@ -722,7 +739,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                   if (rkl) {
                     g0 = fmaf(-al, acc.x, cp * p0);
                     g1 = fmaf(-al, acc.y, cp * p1);
-                  } else if (jsd) {
+                  } else if (jsd || accd) {
                     g0 = p0 * fmaf(al, acc.x, cp);
                     g1 = p1 * fmaf(al, acc.y, cp);
                   } else {
@@ -929,7 +946,7 @@ __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const floa
 // statistics row the backward pass reads and JS = (KL(q || mu) + KL(p || mu))/2
 // as the distillation term.
 __global__ void __launch_bounds__(32 * kMergeRows) js_merge_kernel(const float* __restrict__ partial, int n_splits,
-                                                                   int M, int T, int V, int teacher_rows,
+                                                                   int M, int T, int V, int kind, int teacher_rows,
                                                                    const int32_t* __restrict__ y,
                                                                    float* __restrict__ stats,
                                                                    float* __restrict__ terms) {
@@ -958,10 +975,17 @@ __global__ void __launch_bounds__(32 * kMergeRows) js_merge_kernel(const float* 
   const int yt = y[t];
   const bool bad = yt < 0 || yt >= V;
   for (int s = 0; s < M - 1; ++s) {
-    stats[static_cast<int64_t>(2 * M + s) * T + t] = 0.5f * jq[s];
-    // with the teacher gradient: KL(p || mu)/2 in rows 3M-1 .. 4M-3
-    if (teacher_rows) stats[static_cast<int64_t>(3 * M - 1 + s) * T + t] = 0.5f * jp[s];
-    terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : 0.5f * (jq[s] + jp[s]);
+    if (kind == 3) {
+      // acceptance: A into the statistics row, 1 - beta = 1 - (A + B) as the term, B for the teacher
+      stats[static_cast<int64_t>(2 * M + s) * T + t] = jq[s];
+      if (teacher_rows) stats[static_cast<int64_t>(3 * M - 1 + s) * T + t] = jp[s];
+      terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : 1.f - (jq[s] + jp[s]);
+    } else {
+      stats[static_cast<int64_t>(2 * M + s) * T + t] = 0.5f * jq[s];
+      // with the teacher gradient: KL(p || mu)/2 in rows 3M-1 .. 4M-3
+      if (teacher_rows) stats[static_cast<int64_t>(3 * M - 1 + s) * T + t] = 0.5f * jp[s];
+      terms[static_cast<int64_t>(M + s) * T + t] = bad ? 0.f : 0.5f * (jq[s] + jp[s]);
+    }
   }
 }
 
@@ -1743,14 +1767,14 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
   note_launches(1);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  if (p.distill == 2 && p.M > 1) {
-    // Jensen-Shannon: a second pass over the logits with the final normalisers
-    // (its partials, 2(M-1) rows per split, reuse the statistics partial buffer).
-    err = run_loss_tiles<kModeJS, 0>(p, a, st);
+  if ((p.distill == 2 || p.distill == 3) && p.M > 1) {
+    // Jensen-Shannon or acceptance: a second pass over the logits with the final
+    // normalisers (its partials, 2(M-1) rows per split, reuse the statistics partial buffer).
+    err = p.distill == 3 ? run_loss_tiles<kModeJS, 3>(p, a, st) : run_loss_tiles<kModeJS, 2>(p, a, st);
     if (err != cudaSuccess) return err;
     js_merge_kernel<<<(T + 31) / 32, dim3(32, kMergeRows), 0, st>>>(w.partial, 2 * a.n_vt, p.M, T,
-                                                                     static_cast<int>(p.V), p.teacher_grad, p.y,
-                                                                     stats, w.terms);
+                                                                     static_cast<int>(p.V), p.distill,
+                                                                     p.teacher_grad, p.y, stats, w.terms);
     note_launches(1);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -1767,9 +1791,11 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   const bool tgrad = p.teacher_grad != 0 && p.M > 1;
   cudaError_t err = tgrad ? (p.distill == 1   ? run_loss_tiles<kModeGrad, 1, true>(p, a, st)
                              : p.distill == 2 ? run_loss_tiles<kModeGrad, 2, true>(p, a, st)
+                             : p.distill == 3 ? run_loss_tiles<kModeGrad, 3, true>(p, a, st)
                                               : run_loss_tiles<kModeGrad, 0, true>(p, a, st))
                     : p.distill == 1 ? run_loss_tiles<kModeGrad, 1>(p, a, st)
                     : p.distill == 2 ? run_loss_tiles<kModeGrad, 2>(p, a, st)
+                    : p.distill == 3 ? run_loss_tiles<kModeGrad, 3>(p, a, st)
                                      : run_loss_tiles<kModeGrad, 0>(p, a, st);
   if (err != cudaSuccess) return err;
   // Tokens grouped by target, for the exact one-hot part of dW.

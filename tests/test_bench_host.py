@@ -3,7 +3,6 @@ parser, the validity check of the committed DRAM-traffic record, the peak
 fallback, and the algorithmic byte and flop counts."""
 import json
 import os
-import shutil
 import sys
 
 import pytest
@@ -33,25 +32,25 @@ def test_clock_summary_takes_the_median_and_collects_reasons():
 
 
 def test_traffic_record_is_used_only_for_the_captured_source(tmp_path, monkeypatch):
+    import hashlib
     cfg = wl.CONFIGS["main3"]
-    rec_path = os.path.join(ROOT, "profiles", "traffic_loss_tile_stats_main3_T8192.json")
-    rec = json.load(open(rec_path))
-    v = bench.measured_traffic(cfg)
-    # the committed record matches the committed kernel source
-    assert v == pytest.approx(rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"])
-    assert bench.measured_traffic(wl.CONFIGS["proxy2"]) is None          # another workload
-    # an edited kernel source invalidates the record
     fake_root = tmp_path / "repo"
     (fake_root / "profiles").mkdir(parents=True)
     src_dir = fake_root / "lm_head_loss_junction_b200" / "csrc"
     src_dir.mkdir(parents=True)
-    shutil.copy(rec_path, fake_root / "profiles")
-    text = open(os.path.join(ROOT, rec["source"])).read()
-    (src_dir / "loss_tc.cu").write_text(text + "\n// edited\n")
-    monkeypatch.setattr(bench, "ROOT", str(fake_root))
-    assert bench.measured_traffic(cfg) is None
+    text = "// a kernel source\n"
     (src_dir / "loss_tc.cu").write_text(text)
-    assert bench.measured_traffic(cfg) == pytest.approx(v)
+    rec = {"source": "lm_head_loss_junction_b200/csrc/loss_tc.cu",
+           "source_sha256_16": hashlib.sha256(text.encode()).hexdigest()[:16],
+           "dram_bytes_read_per_launch": 3.0e9, "dram_bytes_write_per_launch": 0.5e8}
+    (fake_root / "profiles" / "traffic_loss_tile_stats_main3_T8192.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(fake_root))
+    assert bench.measured_traffic(cfg) == pytest.approx(3.05e9)          # the captured source
+    assert bench.measured_traffic(wl.CONFIGS["proxy2"]) is None          # another workload
+    (src_dir / "loss_tc.cu").write_text(text + "// edited\n")
+    assert bench.measured_traffic(cfg) is None                            # the source changed since
+    (fake_root / "profiles" / "traffic_loss_tile_stats_main3_T8192.json").unlink()
+    assert bench.measured_traffic(cfg) is None                            # no record at all
 
 
 def test_peaks_fall_back_when_the_file_is_missing(monkeypatch, tmp_path):

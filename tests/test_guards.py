@@ -98,13 +98,13 @@ def test_junction_writes_stay_in_bounds(name, small):
 
 @pytest.mark.parametrize("name,small", CASES)
 @pytest.mark.parametrize("opts", [dict(), dict(distill="reverse_kl", teacher_grad=True),
-                                  dict(distill="js", teacher_grad=True)])
+                                  dict(distill="js", teacher_grad=True), dict(distill="accept", teacher_grad=True)])
 def test_loss_writes_stay_in_bounds(name, small, opts):
     cfg = _cfg(name, small)
     d, x, y, o, E, W = _inputs(cfg)
     M, T, V = cfg.M, cfg.T, cfg.V
     fb, bb = multiexit_loss_workspace(T, list(cfg.D), V, o[0].dtype)
-    rows = 4 * M - 2 if (opts.get("distill") == "js" and M > 1) else 3 * M - 1
+    rows = 4 * M - 2 if (opts.get("distill") in ("js", "accept") and M > 1) else 3 * M - 1
     ins = [y] + o + W
     snap = _snapshot(ins)
     losses = Guarded((2 * M,), torch.float32)

@@ -49,10 +49,12 @@ def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce", teache
     assert_stats_close(s[:M], r["lse"], "lse")
     assert_stats_close(s[M:2 * M], r["tgt"], "target logits")
     if M > 1:
-        assert_stats_close(s[2 * M:3 * M - 1], {"ce": r["S"], "reverse_kl": r["R"], "js": r["J"]}[distill],
+        assert_stats_close(s[2 * M:3 * M - 1],
+                           {"ce": r["S"], "reverse_kl": r["R"], "js": r["J"], "accept": r["A"]}[distill],
                            "distillation statistic")
-        if distill == "js" and teacher_grad:
-            assert_stats_close(s[3 * M - 1:], r["Jp"], "teacher-side Jensen-Shannon statistic")
+        if distill in ("js", "accept") and teacher_grad:
+            assert_stats_close(s[3 * M - 1:], {"js": r["Jp"], "accept": r["B"]}[distill],
+                               "teacher-side distillation statistic")
     for m in range(M):
         assert_grad_close(dh[m], r["dh"][m], f"dh[{m}]")
         assert_grad_close(dW[m], r["dW"][m], f"dW[{m}]")
@@ -95,7 +97,7 @@ def test_exit_weights(name, small):
 @pytest.mark.parametrize("name,small", [("tiny3", None), ("main3", dict(batch=1, seq=200, V=512)),
                                         ("suite4", dict(batch=1, seq=130, V=384)),
                                         ("main3_aligned", dict(batch=1, seq=256, V=768))])
-@pytest.mark.parametrize("distill", ["reverse_kl", "js"])
+@pytest.mark.parametrize("distill", ["reverse_kl", "js", "accept"])
 def test_alternative_distillation(name, small, distill):
     cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
     d = wl.make_inputs(cfg, with_tables=False)
@@ -107,7 +109,7 @@ def test_alternative_distillation(name, small, distill):
                                         ("suite4", dict(batch=1, seq=130, V=384)),
                                         ("main3_aligned", dict(batch=1, seq=256, V=768)),
                                         ("proxy2", dict(batch=1, seq=160, V=512))])
-@pytest.mark.parametrize("distill", ["ce", "reverse_kl", "js"])
+@pytest.mark.parametrize("distill", ["ce", "reverse_kl", "js", "accept"])
 def test_teacher_gradient(name, small, distill):
     cfg = wl.CONFIGS[name] if small is None else wl.small_variant(wl.CONFIGS[name], **small)
     d = wl.make_inputs(cfg, with_tables=False)
