@@ -289,8 +289,8 @@ typedef enum {
  *                 rows 2M..3M-2.  Its forward takes a second pass over the
  *                 logits (the divergence needs the final normalisers); the
  *                 backward call must get the same option.
- *                 MLS_DISTILL_ACCEPT (same section: train the draft for
- *                 acceptance): KD_m = mean_t (1 - beta_t), beta = sum_v
+ *                 MLS_DISTILL_ACCEPT (same section; the acceptance probability
+ *                 of a drafted token as the objective): KD_m = mean_t (1 - beta_t), beta = sum_v
  *                 min(q_m, p_M), the total variation distance; student
  *                 (sub)gradient G_m = grad_scale/T ((1 - alpha_d)(q_m - onehot(y))
  *                 + alpha_d q_m (A_t - [q_m < p_M])), A_t = sum over q < p of q,
