@@ -11,6 +11,13 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: long CPU work (full-size oracle)")
+    # The boundary tests load libmls.so; build it in-tree (nvcc cross-compiles
+    # without a GPU) when it is missing or older than its sources.
+    try:
+        from lm_head_loss_junction_b200 import build
+        build.build()
+    except Exception as exc:  # the tests that need the library then fail with its error
+        sys.stderr.write(f"libmls.so could not be built: {exc}\n")
 
 
 def pytest_collection_modifyitems(config, items):
