@@ -111,7 +111,7 @@ class ClockSampler:
 class Step:
     """Device-resident inputs, outputs and workspaces of one hot-path step."""
 
-    def __init__(self, cfg: wl.SuiteConfig, device, seed_offset: int = 0):
+    def __init__(self, cfg: wl.SuiteConfig, device, seed_offset: int = 0, bwd_ws_bytes: int = 0):
         import dataclasses
         from lm_head_loss_junction_b200 import api
         self.api = api
@@ -137,7 +137,9 @@ class Step:
         self.de = [torch.empty((T, c.deltas[j + 1]), dtype=dt, device=device) for j in range(M - 1)]
         self.dE = [torch.empty((V, c.deltas[j + 1]), dtype=torch.float32, device=device) for j in range(M - 1)]
         fb, bb = api.multiexit_loss_workspace(T, list(c.D), V, dt)
+        bb = bwd_ws_bytes or bb               # the query's bounded size unless asked otherwise
         self.ws_loss = torch.empty(max(fb, bb), dtype=torch.uint8, device=device)
+        self.bwd_plan = api.multiexit_loss_bwd_plan(T, list(c.D), V, dt, max(fb, bb))
         self.ws_j = torch.empty(api.junction_bwd_workspace(T, V), dtype=torch.uint8, device=device)
         self.status = api.new_status(device)
 
@@ -327,6 +329,9 @@ def main():
                     help="run the workload with this many tokens per GPU instead of its own batch")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step from Python instead of replaying a captured CUDA graph")
+    ap.add_argument("--bwd-ws-gb", type=float, default=0.0,
+                    help="workspace of the loss backward call in GB (default: the size the workspace query "
+                         "returns); a larger one lets the call use fewer token blocks and vocabulary chunks")
     ap.add_argument("--grad-sync", default="none", choices=["none", "allreduce", "reduce_scatter"],
                     help="with more than one rank, exchange dW and dE over NCCL inside every step")
     args = ap.parse_args()
@@ -349,7 +354,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
     from lm_head_loss_junction_b200 import _lib
-    step = Step(cfg, device, seed_offset=rank)
+    step = Step(cfg, device, seed_offset=rank, bwd_ws_bytes=int(args.bwd_ws_gb * 1e9))
     stream = torch.cuda.current_stream(device)
     peaks, peak_kind = load_peaks()
 
@@ -617,7 +622,9 @@ def main():
                        "M": c.M, "D": list(c.D), "V": c.V, "alpha_d": c.alpha_d,
                        "parallelism": f"dp{ws} (independent batches)" if not sync_on else
                                       f"dp{ws} (dW and dE {args.grad_sync} over NCCL every step)",
-                       "l2": f"no flush; per-step working set {step.working_set_gb():.2f} GB > 126 MB L2"},
+                       "l2": f"no flush; per-step working set {step.working_set_gb():.2f} GB > 126 MB L2",
+                       "loss_bwd_pieces": {"token_block": step.bwd_plan[0], "vocab_chunk": step.bwd_plan[1],
+                                           "workspace_bytes": step.ws_loss.numel()}},
             "e2e": e2e, "gpu_launches": int(launches), "launch_mode": "eager" if args.eager else "cuda_graph",
             "roofline": roofline, "cpu_baseline": cpu,
             "phases": phases, "extras": extras, "clocks": clocks.summary(),

@@ -164,22 +164,28 @@ mls_status mls_junction_bwd_workspace(int64_t T, int64_t V, size_t* bytes);
  * The paper has no counterpart: this is a convenience of this library.
  *
  * For callers that cannot allocate device memory where they call the junction
- * backward pass: code running while a stream is captured into a CUDA graph
- * (cudaMalloc cannot be captured), code that must not block on the device
- * (cudaMalloc/cudaFree may synchronise), or programs whose device memory is
- * all handed out by another allocator.  The table-gradient scratch comes from
- * a fixed 4 MiB array in the library's own device memory, held by every GPU
+ * backward pass: programs whose device memory is all handed out up front by
+ * another allocator (a framework's caching allocator, a fixed pool), and
+ * latency-critical code that must not call cudaMalloc/cudaFree, which can
+ * synchronise the whole device.  The table-gradient scratch comes from a
+ * fixed 4 MiB array in the library's own device memory, held by every GPU
  * that loads the library until the process exits; nothing is allocated.
  *
- * Arguments, results and errors are those of mls_junction_bwd.  Additionally:
+ * Arguments, results and errors are those of mls_junction_bwd, checked in the
+ * same order.  Additionally:
  *   - with dE_table non-NULL, (T, V) must satisfy
  *     mls_junction_bwd_workspace(T, V) <= 4 MiB (for example T <= 65536 with
- *     V <= 262144); larger sizes return MLS_ERR_UNSUPPORTED and launch nothing;
- *   - every call on a device shares the one array: calls whose work overlaps
- *     on the GPU (different streams, or different host threads, without
- *     ordering between them) race on it and give undefined results;
- *   - the first call on each device looks the array's address up (once) and
- *     must come before any stream capture on that device.
+ *     V <= 262144); larger sizes return MLS_ERR_UNSUPPORTED (after the
+ *     argument checks) and launch nothing;
+ *   - every call on a device shares the one array and leaves its contents
+ *     behind (each call re-initialises what it reads): calls whose work
+ *     overlaps on the GPU (different streams, or different host threads,
+ *     without ordering between them) race on it and give undefined results;
+ *   - the first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current) and must come before
+ *     any stream capture on that device.  The lookup is repeated on the first
+ *     call after the device's context has been destroyed and re-created
+ *     (cudaDeviceReset); that call must likewise come before any capture.
  */
 mls_status mls_junction_bwd_noalloc(const int32_t* x, int64_t T,
                                     const void* o_m, int64_t D_m,
@@ -221,9 +227,30 @@ mls_status mls_junction_bwd_noalloc(const int32_t* x, int64_t T,
  *   device pointers 16-byte aligned.
  */
 
-/* Workspace bytes for the forward and backward calls of this shape. */
+/*
+ * Workspace bytes for the forward and backward calls of this shape.
+ *
+ * MLS_BF16 backward: the dense logit gradient G' is formed and consumed one
+ * block of tokens x one chunk of the vocabulary at a time, so its workspace
+ * does not grow with T x V.  *bwd_bytes is the workspace of the split chosen
+ * for a 1 GiB budget (or of the whole problem in one piece, when that is
+ * smaller); mls_multiexit_loss_bwd accepts any workspace of at least
+ * mls_multiexit_loss_bwd_plan's minimum and splits the work to fit the size
+ * it is given (a larger workspace means fewer, larger pieces).
+ */
 mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int64_t V,
                                         mls_dtype dt, size_t* fwd_bytes, size_t* bwd_bytes);
+
+/*
+ * How mls_multiexit_loss_bwd (MLS_BF16) splits its work for a workspace of
+ * ws_bytes: token blocks of *Tb tokens and vocabulary chunks of *Vc columns
+ * (the last block and chunk may be shorter; *Tb = T and *Vc = V is one
+ * piece), and *min_bytes, the smallest workspace the call accepts.  With
+ * ws_bytes below *min_bytes, *Tb = *Vc = 0.  Host-only; no device is needed.
+ * MLS_F32 has no split: *Tb = T, *Vc = V, *min_bytes = its bwd_bytes.
+ */
+mls_status mls_multiexit_loss_bwd_plan(int M, int64_t T, const int64_t* D, int64_t V, mls_dtype dt,
+                                       size_t ws_bytes, int64_t* Tb, int64_t* Vc, size_t* min_bytes);
 
 /*
  * mls_multiexit_loss_fwd
@@ -250,6 +277,14 @@ mls_status mls_multiexit_loss_fwd(int M, int64_t T, int64_t V, const int64_t* D,
  *   dh[m] = G_m W^m           device dt [T, D[m]], overwritten
  *   dW[m] (+)= G_m^T h_m      device f32 [V, D[m]]; accumulate_dW != 0 adds
  *   stats is the forward call's output for the same inputs.
+ * MLS_BF16: the logits are computed again tile by tile (never stored) and
+ * the dense part of G (q_m - alpha_d p_M, or p_M for the largest exit) is
+ * written in bf16 for one token block x vocabulary chunk at a time into the
+ * workspace (see mls_multiexit_loss_bwd_plan), then multiplied out on the
+ * tensor cores; the one-hot part is applied exactly in fp32.  dh rows of a
+ * block are summed over the chunks in fp32 (fixed order), dW rows of a chunk
+ * over the blocks in fp32 (fixed order): results are deterministic for a
+ * given workspace size.
  */
 mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   const int32_t* y_targets,
@@ -385,6 +420,28 @@ mls_status mls_exit_agreement(int M, int64_t T, int64_t V, const int64_t* D,
  * flag was set (timeout wins), MLS_OK when the word was 0.
  */
 mls_status mls_status_read(int32_t* dev_status, void* stream, int32_t* host_out);
+
+/*
+ * mls_selftest_wait_timeout -- exercises the bounded device-side waits; not
+ * part of the method (the pages have no counterpart).  It launches the
+ * tensor-core statistics kernel of mls_multiexit_loss_fwd on the given
+ * problem (MLS_BF16 only, arguments as for that call) with two changes: the
+ * kernel's load warp issues no loads, so the barriers the other warps wait on
+ * never complete, and every wait gives up after wait_limit_ns nanoseconds
+ * (1e3 <= wait_limit_ns <= 4e9) instead of the library's 4 s.  The kernel
+ * then sets MLS_DEVFLAG_TIMEOUT in *dev_status (required, non-NULL) and
+ * returns with nothing in flight; the merge and reduction kernels that follow
+ * still run, so `losses` and `stats` hold meaningless values.  The stream
+ * stays usable: mls_status_read() reports MLS_ERR_DEVICE_TIMEOUT and clears
+ * the flag, and later calls on the same stream behave normally.
+ */
+mls_status mls_selftest_wait_timeout(int M, int64_t T, int64_t V, const int64_t* D,
+                                     const int32_t* y_targets,
+                                     const void* const* h, const void* const* W,
+                                     float* losses, float* stats,
+                                     void* workspace, size_t ws_bytes,
+                                     uint64_t wait_limit_ns,
+                                     int32_t* dev_status, void* stream);
 
 /* Static English text for a status code. */
 const char* mls_status_string(mls_status s);

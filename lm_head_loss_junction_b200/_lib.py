@@ -53,6 +53,8 @@ PROTOTYPES = {
                                         _int, _vp, _vp]),
     "mls_multiexit_loss_workspace": (_int, [_int, _i64, ctypes.POINTER(_i64), _i64, _int,
                                             ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
+    "mls_multiexit_loss_bwd_plan": (_int, [_int, _i64, ctypes.POINTER(_i64), _i64, _int, _sz,
+                                           ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_sz)]),
     "mls_multiexit_loss_fwd": (_int, [_int, _i64, _i64, ctypes.POINTER(_i64), _vp,
                                       ctypes.POINTER(_vp), ctypes.POINTER(_vp), _f32, _int,
                                       _vp, _vp, _vp, _sz, _vp, _vp]),
@@ -70,6 +72,8 @@ PROTOTYPES = {
     "mls_exit_agreement_workspace": (_int, [_int, _i64, ctypes.POINTER(_i64), _i64, _int, ctypes.POINTER(_sz)]),
     "mls_exit_agreement": (_int, [_int, _i64, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                   _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "mls_selftest_wait_timeout": (_int, [_int, _i64, _i64, ctypes.POINTER(_i64), _vp, ctypes.POINTER(_vp),
+                                         ctypes.POINTER(_vp), _vp, _vp, _vp, _sz, ctypes.c_uint64, _vp, _vp]),
     "mls_status_read": (_int, [_vp, _vp, ctypes.POINTER(_i32)]),
     "mls_status_string": (ctypes.c_char_p, [_int]),
     "mls_version": (_int, []),

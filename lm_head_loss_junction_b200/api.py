@@ -126,6 +126,19 @@ def multiexit_loss_workspace(T: int, D: Sequence[int], V: int, dtype: torch.dtyp
     return f.value, b.value
 
 
+def multiexit_loss_bwd_plan(T: int, D: Sequence[int], V: int, dtype: torch.dtype, ws_bytes: int):
+    """(Tb, Vc, min_bytes): how the backward call splits its work for a workspace of ws_bytes
+    (see mls_multiexit_loss_bwd_plan)."""
+    tb = ctypes.c_int64()
+    vc = ctypes.c_int64()
+    mn = ctypes.c_size_t()
+    code = lib().mls_multiexit_loss_bwd_plan(len(D), T, i64_array(D), V,
+                                             MLS_BF16 if dtype == torch.bfloat16 else MLS_F32, int(ws_bytes),
+                                             ctypes.byref(tb), ctypes.byref(vc), ctypes.byref(mn))
+    check("mls_multiexit_loss_bwd_plan", code)
+    return tb.value, vc.value, mn.value
+
+
 def _loss_common(y, h, W):
     M = len(h)
     if len(W) != M or M < 1:

@@ -7,6 +7,7 @@ The library links the CUDA runtime statically and reaches the driver API
 """
 from __future__ import annotations
 
+import hashlib
 import os
 import shutil
 import subprocess
@@ -28,15 +29,34 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
+HASH = LIB + ".srchash"
+
+
+def source_hash() -> str:
+    """SHA-256 over every source file, the public header and the compiler flags.
+
+    Content, not modification times: a copied tree (whose files all get new
+    times) keeps a valid library, and an edited source always rebuilds it.
+    """
+    h = hashlib.sha256()
+    deps = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC)) + [os.path.join(INCLUDE, "mls.h")]
+    for d in deps:
+        h.update(os.path.basename(d).encode())
+        with open(d, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(ARCH + SOURCES).encode())
+    return h.hexdigest()
+
+
 def _stale() -> bool:
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(HASH)):
         return True
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "mls.h")]
-    return any(os.path.getmtime(d) > t for d in deps)
+    with open(HASH) as f:
+        return f.read().strip() != source_hash()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compiles libmls.so unless the library on disk was built from the current sources."""
     if not force and not _stale():
         return LIB
     objdir = os.path.join(PKG, "_build")
@@ -54,6 +74,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = LIB + ".tmp"
     subprocess.run([nvcc(), *ARCH, "-shared", "--cudart", "static", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
+    with open(HASH, "w") as f:
+        f.write(source_hash() + "\n")
     return LIB
 
 

@@ -130,6 +130,24 @@ mls_status apply_options(const mls_loss_options* opts, LossProblem* p) {
 
 }  // namespace
 
+namespace mls {
+
+mls_status check_junction_bwd_args(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
+                                   int64_t V, int64_t delta, const void* dy, const void* do_m, const void* de_rows,
+                                   const float* dE_table, uint32_t variant, mls_dtype dt) {
+  if (variant & ~kKnownVariants) return MLS_ERR_INVALID_ARG;
+  mls_status st = check_junction_shape(x, T, o_m, D_m, e_next, V, delta, dt);
+  if (st != MLS_OK) return st;
+  if (dy == nullptr || do_m == nullptr) return MLS_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(do_m) || (de_rows != nullptr && !aligned16(de_rows)) ||
+      (dE_table != nullptr && !aligned16(dE_table)))
+    return MLS_ERR_UNSUPPORTED;
+  if (T > INT_MAX) return MLS_ERR_UNSUPPORTED;
+  return MLS_OK;
+}
+
+}  // namespace mls
+
 extern "C" {
 
 int mls_version(void) { return 100; }
@@ -200,14 +218,9 @@ mls_status mls_junction_bwd_variant(const int32_t* x, int64_t T, const void* o_m
                                     int64_t V, int64_t delta, const void* dy, void* do_m, void* de_rows,
                                     float* dE_table, int accumulate_dE, void* workspace, size_t ws_bytes,
                                     uint32_t variant, mls_dtype dt, int32_t* dev_status, void* stream) {
-  if (variant & ~kKnownVariants) return MLS_ERR_INVALID_ARG;
-  mls_status st = check_junction_shape(x, T, o_m, D_m, e_next, V, delta, dt);
+  mls_status st = mls::check_junction_bwd_args(x, T, o_m, D_m, e_next, V, delta, dy, do_m, de_rows, dE_table,
+                                               variant, dt);
   if (st != MLS_OK) return st;
-  if (dy == nullptr || do_m == nullptr) return MLS_ERR_INVALID_ARG;
-  if (!aligned16(dy) || !aligned16(do_m) || (de_rows != nullptr && !aligned16(de_rows)) ||
-      (dE_table != nullptr && !aligned16(dE_table)))
-    return MLS_ERR_UNSUPPORTED;
-  if (T > INT_MAX) return MLS_ERR_UNSUPPORTED;
   if (dE_table != nullptr) {
     if (workspace == nullptr || ws_bytes < mls::junction_scatter_bytes(T, V)) return MLS_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
@@ -246,6 +259,28 @@ mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int6
     *fwd_bytes = mls::loss_simt_fwd_bytes(p);
     *bwd_bytes = mls::loss_simt_bwd_bytes(p);
   }
+  return MLS_OK;
+}
+
+mls_status mls_multiexit_loss_bwd_plan(int M, int64_t T, const int64_t* D, int64_t V, mls_dtype dt,
+                                       size_t ws_bytes, int64_t* Tb, int64_t* Vc, size_t* min_bytes) {
+  if (Tb == nullptr || Vc == nullptr || min_bytes == nullptr) return MLS_ERR_INVALID_ARG;
+  const mls_status st = check_loss_shape(M, T, V, D, dt);
+  if (st != MLS_OK) return st;
+  const LossProblem p = shape_problem(M, T, V, D);
+  if (dt != MLS_BF16) {
+    *Tb = T;
+    *Vc = V;
+    *min_bytes = mls::loss_simt_bwd_bytes(p);
+    return MLS_OK;
+  }
+  *min_bytes = mls::loss_tc_bwd_min_bytes(p);
+  if (ws_bytes < *min_bytes) {
+    *Tb = 0;
+    *Vc = 0;
+    return MLS_OK;
+  }
+  mls::loss_tc_bwd_plan(p, ws_bytes, Tb, Vc);
   return MLS_OK;
 }
 
@@ -303,14 +338,14 @@ mls_status mls_multiexit_loss_bwd_opts(int M, int64_t T, int64_t V, const int64_
     if (!aligned16(dh[m]) || !aligned16(dW[m])) return MLS_ERR_UNSUPPORTED;
   }
   if (!(grad_scale == grad_scale)) return MLS_ERR_INVALID_ARG;
-  const size_t need = dt == MLS_BF16 ? mls::loss_tc_bwd_bytes(p) : mls::loss_simt_bwd_bytes(p);
+  const size_t need = dt == MLS_BF16 ? mls::loss_tc_bwd_min_bytes(p) : mls::loss_simt_bwd_bytes(p);
   if (workspace == nullptr || ws_bytes < need) return MLS_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
   if ((st = device_ok()) != MLS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dt == MLS_BF16) {
     if (!mls::tensor_map_encoder_available()) return MLS_ERR_CUDA;
-    return from_cuda(mls::loss_tc_bwd(p, stats, grad_scale, dh, dW, accumulate_dW, workspace, s));
+    return from_cuda(mls::loss_tc_bwd(p, stats, grad_scale, dh, dW, accumulate_dW, workspace, ws_bytes, s));
   }
   return from_cuda(mls::loss_simt_bwd(p, stats, grad_scale, dh, dW, accumulate_dW, workspace, s));
 }
@@ -348,6 +383,25 @@ mls_status mls_exit_agreement(int M, int64_t T, int64_t V, const int64_t* D, con
     return from_cuda(mls::agree_tc(p, stats, metrics, per_token, top1, workspace, s));
   }
   return from_cuda(mls::agree_simt(p, stats, metrics, per_token, top1, workspace, s));
+}
+
+mls_status mls_selftest_wait_timeout(int M, int64_t T, int64_t V, const int64_t* D, const int32_t* y_targets,
+                                     const void* const* h, const void* const* W, float* losses, float* stats,
+                                     void* workspace, size_t ws_bytes, uint64_t wait_limit_ns,
+                                     int32_t* dev_status, void* stream) {
+  LossProblem p{};
+  mls_status st = build_problem(M, T, V, D, y_targets, h, W, 0.3f, MLS_BF16, dev_status, &p);
+  if (st != MLS_OK) return st;
+  if (losses == nullptr || stats == nullptr || dev_status == nullptr) return MLS_ERR_INVALID_ARG;
+  if (wait_limit_ns < 1000ull || wait_limit_ns > 4000000000ull) return MLS_ERR_INVALID_ARG;
+  if (!aligned16(stats)) return MLS_ERR_UNSUPPORTED;
+  if (workspace == nullptr || ws_bytes < mls::loss_tc_fwd_bytes(p)) return MLS_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
+  if ((st = device_ok()) != MLS_OK) return st;
+  if (!mls::tensor_map_encoder_available()) return MLS_ERR_CUDA;
+  p.wait_ns = wait_limit_ns;
+  p.withhold_loads = 1;
+  return from_cuda(mls::loss_tc_fwd(p, losses, stats, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 mls_status mls_status_read(int32_t* dev_status, void* stream, int32_t* host_out) {

@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "mls.h"
+
 namespace mls {
 
 constexpr int kMaxExits = 4;
@@ -27,6 +29,11 @@ struct JunctionArgs {
   int32_t* status;
   uint32_t variant;   // junction variant bits (0 = the standard junction)
 };
+
+// Every argument check of mls_junction_bwd_variant except the workspace's.
+mls_status check_junction_bwd_args(const int32_t* x, int64_t T, const void* o_m, int64_t D_m, const void* e_next,
+                                   int64_t V, int64_t delta, const void* dy, const void* do_m, const void* de_rows,
+                                   const float* dE_table, uint32_t variant, mls_dtype dt);
 
 size_t junction_scatter_bytes(int64_t T, int64_t V);
 cudaError_t launch_junction_fwd(const JunctionArgs& a, cudaStream_t st);
@@ -72,6 +79,8 @@ struct LossProblem {
   int distill;               // 0: cross-entropy to the largest exit, 1: KL(q_m || p_M), 2: Jensen-Shannon
   int teacher_grad;          // 1: the largest exit also gets the distillation gradient (no stop-gradient)
   int32_t* status;
+  uint64_t wait_ns;          // limit of the tile kernels' barrier waits; 0 = the library default
+  int withhold_loads;        // test of the bounded waits only: the tile kernel's producer issues no loads
 };
 
 // Workspace sizes (bytes) of each path.
@@ -80,10 +89,15 @@ size_t loss_tc_bwd_bytes(const LossProblem& p);
 size_t loss_simt_fwd_bytes(const LossProblem& p);
 size_t loss_simt_bwd_bytes(const LossProblem& p);
 
-// Tensor-core (bf16) path.
+// Tensor-core (bf16) path.  The backward pass runs in (token block x vocabulary
+// chunk) pieces sized to the workspace it is given: loss_tc_bwd_bytes is the
+// size of the plan for a 1 GiB budget (or of the whole problem, when smaller),
+// loss_tc_bwd_min_bytes the smallest workspace any plan fits in.
+size_t loss_tc_bwd_min_bytes(const LossProblem& p);
+void loss_tc_bwd_plan(const LossProblem& p, size_t ws_bytes, int64_t* Tb, int64_t* Vc);
 cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void* ws, cudaStream_t st);
 cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_scale, void* const* dh,
-                        float* const* dW, int accumulate, void* ws, cudaStream_t st);
+                        float* const* dW, int accumulate, void* ws, size_t ws_bytes, cudaStream_t st);
 
 // CUDA-core (fp32) path.
 cudaError_t loss_simt_fwd(const LossProblem& p, float* losses, float* stats, void* ws, cudaStream_t st);

@@ -48,8 +48,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // TMEM lane quadrant, each owning one 128-column half ("split") of the tile.
 constexpr int kLossBN = 256;
 constexpr int kSplitCols = 128;
-constexpr int kLossStages = 4;        // single CTA: 48 KB per stage
-constexpr int kLossPairStages = 6;    // CTA pair: 32 KB per stage and CTA
+constexpr int kLossStages = 4;        // 48 KB per stage
 constexpr int kLossEpiWarps = 8;
 constexpr int kLossThreads = 64 + 32 * kLossEpiWarps;
 
@@ -61,8 +60,11 @@ struct LossMaps {
 
 struct LossArgs {
   int M;
-  int T;
-  int V;
+  int T;                       // tokens of this launch (a block of the call's tokens in the backward)
+  int V;                       // vocabulary columns of this launch (a chunk in the backward)
+  int v0;                      // first vocabulary id of the launch's columns
+  int Vtot;                    // the vocabulary size (targets outside [0, Vtot) are invalid)
+  int ldS;                     // row stride of stats (the call's token count)
   int kblocks[kMaxExits];      // D_m / kBK
   int n_tt, n_vt, num_tiles, group_tt;
   const int32_t* y;
@@ -72,22 +74,20 @@ struct LossArgs {
   float student_wsum;          // sum of the smaller exits' weights
   float* partial;              // forward: [2 n_vt][2M-1][T]
   float* stats;                // forward: target rows written; backward: lse read
-  __nv_bfloat16* G;            // backward: [M][T][V]
+  __nv_bfloat16* G;            // backward: [M][T][V] of the launch's tokens and columns
   int32_t* status;
+  uint64_t wait_ns;            // limit of every barrier wait (the library default, or a test's)
+  int withhold_loads;          // test of the bounded waits: the producer issues no loads
 };
 
 // Per-warp staging of one 32-row x 32-column bf16 chunk of G' (rows padded
 // to 80 bytes so the 16-byte writes of a warp hit every bank once per pass).
 constexpr int kStageRowBytes = 80;
 
-// PAIR: two CTAs share each 256-token x 256-vocabulary MMA (cta_group::2);
-// each loads its own 128 token rows and half (128 rows) of the W tile.
-template <bool PAIR>
 struct __align__(1024) LossSmem {
-  static constexpr int kStages = PAIR ? kLossPairStages : kLossStages;
-  static constexpr int kBRows = PAIR ? kLossBN / 2 : kLossBN;
+  static constexpr int kStages = kLossStages;
   uint8_t a[kStages][kBM * kBK * 2];
-  uint8_t b[kStages][kBRows * kBK * 2];
+  uint8_t b[kStages][kLossBN * kBK * 2];
   uint8_t gstage[kLossEpiWarps][32 * kStageRowBytes];
   uint64_t full[kStages];
   uint64_t empty[kStages];
@@ -123,8 +123,9 @@ __device__ __forceinline__ void loss_tile_coords(int i, const LossArgs& a, int& 
 }
 
 // All lanes of a warp wait; the warp agrees on the outcome.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status) {
-  const bool ok = mbar_wait(bar, parity, abort, status);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, abort, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -198,31 +199,19 @@ __device__ __forceinline__ void store_g_chunk(uint8_t* stage, int lane, const ui
 // region 0 while the students pass through region 1, accumulates each
 // student's contribution to the teacher's logit gradient in registers (fp16
 // pairs), and writes the teacher's G' after the last student.
-//
-// PAIR (launched as clusters of two CTAs): the pair's tile is 256 tokens x 256
-// vocabulary columns; CTA rank r owns tokens [128 r, 128 r + 128) of it in its
-// TMEM and shared memory, loads half of the W tile, and runs the same
-// epilogue on its rows.  The leader (rank 0) issues the MMAs (M = 256) and
-// commits to both CTAs' barriers; both CTAs' loads complete on the leader's
-// stage barriers, and both CTAs' epilogue warps release the leader's TMEM
-// regions.  Halving each SM's share of the W tile cuts its shared-memory and
-// L2 operand traffic per flop by a third.
-template <int MODE, int DISTILL, bool TGRAD = false, bool PAIR = false>
+template <int MODE, int DISTILL, bool TGRAD = false>
 __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid_constant__ LossMaps maps,
                                                                     const LossArgs a) {
-  using Smem = LossSmem<PAIR>;
+  using Smem = LossSmem;
   constexpr int kStages = Smem::kStages;
-  constexpr int kTileRows = PAIR ? 2 * kBM : kBM;      // tokens per tile
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort;
   const int M = a.M;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
-  const bool leader = rank == 0;
-  const int slot = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int nslots = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int slot = static_cast<int>(blockIdx.x);
+  const int nslots = static_cast<int>(gridDim.x);
   constexpr bool rkl = (DISTILL == 1);
   constexpr bool jsd = (DISTILL == 2);
   constexpr bool accd = (DISTILL == 3);
@@ -239,7 +228,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     }
     for (int r = 0; r < 2; ++r) {
       mbar_init(&s.tfull[r], 1);
-      mbar_init(&s.tempty[r], PAIR ? 2 * kLossEpiWarps : kLossEpiWarps);
+      mbar_init(&s.tempty[r], kLossEpiWarps);
     }
     mbar_init(&s.drain, 1);
     s.abort = 0;
@@ -252,81 +241,52 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     }
   }
   if (warp == 1) {
-    if constexpr (PAIR) {
-      tmem_alloc_pair(&s.tmem_base, 512);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(&s.tmem_base, 512);
-      tmem_relinquish();
-    }
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
   }
-  if constexpr (PAIR) {
-    __syncwarp();
-    tc_fence_before();
-    cluster_sync_all();        // every barrier of both CTAs exists before any remote arrive
-    tc_fence_after();
-  } else {
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  // an epilogue warp is done with TMEM region r (the leader's barrier counts both CTAs)
-  auto release_region = [&](uint32_t r) {
-    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[r]), 0));
-    else mbar_arrive(&s.tempty[r]);
-  };
+  // an epilogue warp is done with TMEM region r
+  auto release_region = [&](uint32_t r) { mbar_arrive(&s.tempty[r]); };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
+    if (lane == 0 && !a.withhold_loads) {
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
       for (int tile = slot; tile < a.num_tiles && ok; tile += nslots) {
         int tt, vt;
         loss_tile_coords(tile, a, tt, vt);
-        const int row0 = tt * kTileRows + static_cast<int>(rank) * kBM;                // this CTA's tokens
-        const int v0 = vt * kLossBN + static_cast<int>(rank) * Smem::kBRows;           // this CTA's W rows
+        const int row0 = tt * kBM;               // the tile's tokens
+        const int v0 = vt * kLossBN;             // the tile's W rows
         for (int j = 0; j < M && ok; ++j) {
           const int m = M - 1 - j;                // teacher first, then students
           for (int kb = 0; kb < a.kblocks[m]; ++kb) {
-            if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, a.status)) { ok = false; break; }
-            if constexpr (PAIR) {
-              const uint32_t lfull = mapa_shared(smem_u32(&s.full[stage]), 0);
-              if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * (kBM + Smem::kBRows) * kBK * 2);
-              tma_load_2d_pair(&maps.h[m], lfull, s.a[stage], kb * kBK, row0);
-              tma_load_2d_pair(&maps.w[m], lfull, s.b[stage], kb * kBK, v0);
-            } else {
-              mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
-              tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0);
-              tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0);
-            }
+            if (!mbar_wait(&s.empty[stage], phase ^ 1, abort, a.status, a.wait_ns)) { ok = false; break; }
+            mbar_arrive_expect_tx(&s.full[stage], (kBM + kLossBN) * kBK * 2);
+            tma_load_2d(&maps.h[m], &s.full[stage], s.a[stage], kb * kBK, row0);
+            tma_load_2d(&maps.w[m], &s.full[stage], s.b[stage], kb * kBK, v0);
             ++issued;
             if (++stage == kStages) { stage = 0; phase ^= 1; }
           }
         }
       }
       if (!ok) {
-        if constexpr (PAIR) {
-          // This CTA's loads complete on the leader's barriers; give them time to land.
-          const uint64_t t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 2000000ull) {
-          }
-        } else {
-          // Let every load already issued land before the CTA can exit.
-          const uint32_t n = issued < kStages ? issued : kStages;
-          uint32_t st = stage, ph = phase;
-          for (uint32_t i = 0; i < n; ++i) {
-            if (st == 0) { st = kStages - 1; ph ^= 1; } else { --st; }
-            drain_wait(&s.full[st], ph, a.status);
-          }
+        // Let every load already issued land before the CTA can exit.
+        const uint32_t n = issued < kStages ? issued : kStages;
+        uint32_t st = stage, ph = phase;
+        for (uint32_t i = 0; i < n; ++i) {
+          if (st == 0) { st = kStages - 1; ph ^= 1; } else { --st; }
+          drain_wait(&s.full[st], ph, a.status);
         }
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_bf16(kTileRows, kLossBN, false, false);
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kBM, kLossBN, false, false);
       uint32_t stage = 0, phase = 0, job = 0, tile_iter = 0;
       bool ok = true;
       for (int tile = slot; tile < a.num_tiles && ok; tile += nslots, ++tile_iter) {
@@ -334,47 +294,28 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           const int m = M - 1 - j;
           uint32_t region, use;
           job_slot(hold, M, tile_iter, j, job, region, use);
-          if (!mbar_wait(&s.tempty[region], (use & 1) ^ 1, abort, a.status)) { ok = false; break; }
+          if (!mbar_wait(&s.tempty[region], (use & 1) ^ 1, abort, a.status, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + region * kLossBN;
           for (int kb = 0; kb < a.kblocks[m]; ++kb) {
-            if (!mbar_wait(&s.full[stage], phase, abort, a.status)) { ok = false; break; }
+            if (!mbar_wait(&s.full[stage], phase, abort, a.status, a.wait_ns)) { ok = false; break; }
             tc_fence_after();
             const uint64_t da = smem_desc_sw128(smem_u32(s.a[stage]), 16, 1024);
             const uint64_t db = smem_desc_sw128(smem_u32(s.b[stage]), 16, 1024);
 #pragma unroll
             for (int k = 0; k < kBK / kUK; ++k) {
               // +32 bytes along K inside the 128-byte swizzled row
-              if constexpr (PAIR)
-                umma_bf16_pair(d, da + static_cast<uint64_t>(k * 2), db + static_cast<uint64_t>(k * 2), idesc,
-                               (kb | k) != 0);
-              else
-                umma_bf16(d, da + static_cast<uint64_t>(k * 2), db + static_cast<uint64_t>(k * 2), idesc,
-                          (kb | k) != 0);
+              umma_bf16(d, da + static_cast<uint64_t>(k * 2), db + static_cast<uint64_t>(k * 2), idesc,
+                        (kb | k) != 0);
             }
-            if constexpr (PAIR) {
-              const uint32_t e = smem_u32(&s.empty[stage]);
-              umma_commit_pair(mapa_shared(e, 0));
-              umma_commit_pair(mapa_shared(e, 1));
-            } else {
-              umma_commit(&s.empty[stage]);
-            }
+            umma_commit(&s.empty[stage]);
             if (++stage == kStages) { stage = 0; phase ^= 1; }
           }
-          if (ok) {
-            if constexpr (PAIR) {
-              const uint32_t f = smem_u32(&s.tfull[region]);
-              umma_commit_pair(mapa_shared(f, 0));
-              umma_commit_pair(mapa_shared(f, 1));
-            } else {
-              umma_commit(&s.tfull[region]);
-            }
-          }
+          if (ok) umma_commit(&s.tfull[region]);
         }
       }
       // Make sure every MMA issued has finished before TMEM is released.
-      if constexpr (PAIR) umma_commit_pair(mapa_shared(smem_u32(&s.drain), 0));
-      else umma_commit(&s.drain);
+      umma_commit(&s.drain);
       drain_wait(&s.drain, 0, a.status);
     }
   } else {
@@ -392,16 +333,16 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     for (int tile = slot; tile < a.num_tiles; tile += nslots, ++tile_iter) {
       int tt, vt;
       loss_tile_coords(tile, a, tt, vt);
-      const int rbase = tt * kTileRows + static_cast<int>(rank) * kBM;   // first token of this CTA's rows
+      const int rbase = tt * kBM;                           // first token of the tile
       const int t = rbase + row;
       const bool valid = t < a.T;
       const int c0 = vt * kLossBN + half * kSplitCols;     // first vocabulary column of the split
       const bool live = c0 < a.V;                           // the last tile may be half outside V
       const int split = vt * 2 + half;
       const int yt = valid ? __ldg(a.y + t) : -1;
-      const int yl = yt - c0;                               // target column inside this split, if any
+      const int yl = yt - a.v0 - c0;                        // target column inside this split, if any
       const bool has_tgt = valid && yl >= 0 && yl < kSplitCols;
-      const bool bad = valid && (yt < 0 || yt >= a.V);
+      const bool bad = valid && (yt < 0 || yt >= a.Vtot);
       bool stop = false;
       for (int j = 0; j < M; ++j, ++job) {
         const int m = M - 1 - j;
@@ -409,7 +350,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
         job_slot(hold, M, tile_iter, j, job, region, use);
         const uint32_t base = lane_base + region * kLossBN;
         const uint32_t tbase = lane_base;                   // region 0: the teacher, when held
-        if (!warp_wait(&s.tfull[region], use & 1, abort, a.status)) { stop = true; break; }
+        if (!warp_wait(&s.tfull[region], use & 1, abort, a.status, a.wait_ns)) { stop = true; break; }
         tc_fence_after();
         if (MODE == kModeStats) {
           float lse_part = -INFINITY, abar = 0.f;
@@ -426,7 +367,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 if (has_tgt && (yl >> 5) == c) {
 #pragma unroll
                   for (int k = 0; k < 32; ++k)
-                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.T + t] = r[k];
+                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = r[k];
                 }
               }
               const float mxs = mx * kLog2e;
@@ -473,7 +414,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 if (has_tgt && (yl >> 5) == c) {
 #pragma unroll
                   for (int k = 0; k < 32; ++k)
-                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.T + t] = r[k];
+                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = r[k];
                 }
               }
               lse_part = ms + logf(zs);
@@ -503,7 +444,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 if (has_tgt && (yl >> 5) == c) {
 #pragma unroll
                   for (int k = 0; k < 32; ++k)
-                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.T + t] = r[k];
+                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = r[k];
                 }
               }
               lse_part = ms + logf(zs);
@@ -532,8 +473,8 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           float mxv = -INFINITY, sum_min = 0.f, kl = 0.f;
           int mxi = -1;
           if (live) {
-            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
-            const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
+            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.ldS + t] : 0.f;
+            const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.ldS + t] : 0.f;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float r[32];
@@ -578,8 +519,8 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           //   log(q/mu) = ln 2 - softplus(d),  log(p/mu) = ln 2 - softplus(-d).
           float jq = 0.f, jp = 0.f;
           if (live && j > 0) {
-            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
-            const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
+            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.ldS + t] : 0.f;
+            const float lseT = valid ? a.stats[static_cast<int64_t>(M - 1) * a.ldS + t] : 0.f;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float r[32], lt[32];
@@ -615,7 +556,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           }
         } else {
           // ---------------- backward: dense part of the logit gradient, bf16
-          if (bad && j == 0 && vt == 0 && half == 0) set_flag(a.status, MLS_DEVFLAG_BAD_ID);
+          if (bad && j == 0 && vt == 0 && half == 0 && a.v0 == 0) set_flag(a.status, MLS_DEVFLAG_BAD_ID);
           uint8_t* const stage = s.gstage[warp - 2];
           const int row0 = rbase + q * 32;                   // first token row of this warp
           if (TGRAD && j == 0) {
@@ -624,18 +565,18 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
 #pragma unroll
               for (int k = 0; k < 16; ++k) pt[c][k] = 0u;   // the teacher-gradient accumulator
           }
-          const float lseT = (hold && valid) ? a.stats[static_cast<int64_t>(M - 1) * a.T + t] : 0.f;
+          const float lseT = (hold && valid) ? a.stats[static_cast<int64_t>(M - 1) * a.ldS + t] : 0.f;
           const float lsT = lseT * kLog2e;
           if (live && !(TGRAD && j == 0)) {
-            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.T + t] : 0.f;
+            const float lse = valid ? a.stats[static_cast<int64_t>(m) * a.ldS + t] : 0.f;
             const float ls = lse * kLog2e;
             // per-token statistic of the student from the forward pass:
             //   cross-entropy S_m = sum p_T l_m; reverse KL R_m = sum q_m (l_m - l_T), so that
             //   log q - log p - KL(q_m || p_T) = l_m - l_T - R_m;  Jensen-Shannon: K = KL(q_m || mu) / 2
-            const float klt = (hold && j > 0 && valid) ? a.stats[static_cast<int64_t>(2 * M + m) * a.T + t] : 0.f;
+            const float klt = (hold && j > 0 && valid) ? a.stats[static_cast<int64_t>(2 * M + m) * a.ldS + t] : 0.f;
             // Jensen-Shannon with the teacher gradient: K^p = KL(p_T || mu)/2, stored by the forward pass
             const float kpt = (TGRAD && (jsd || accd) && j > 0 && valid)
-                                  ? a.stats[static_cast<int64_t>(3 * M - 1 + m) * a.T + t]
+                                  ? a.stats[static_cast<int64_t>(3 * M - 1 + m) * a.ldS + t]
                                   : 0.f;
             const uint32_t wm2 = TGRAD ? pack_p2(a.exit_w[m], a.exit_w[m]) : 0u;
             // unrolled where a register array is indexed by c (the teacher's
@@ -770,20 +711,10 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
   }
 
   __syncthreads();
-  if constexpr (PAIR) {
-    tc_fence_before();
-    cluster_sync_all();        // no CTA leaves while its pair may still touch its memory
+  if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
-    if (warp == 1) {
-      __syncwarp();
-      tmem_dealloc_pair(tmem, 512);
-    }
-  } else {
-    if (warp == 1) {
-      __syncwarp();
-      tc_fence_after();
-      tmem_dealloc(tmem, 512);
-    }
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1022,6 +953,9 @@ struct GemmArgs {
   const __nv_bfloat16* onehot_rows[kMaxExits];
   float onehot_coef[kMaxExits];
   int onehot_limit;
+  // Optional fp32 partial sums (bf16 output only): out_p = alpha acc + addend_p (same layout as out_p)
+  // before the one-hot term and the rounding; the earlier vocabulary chunks of dh.
+  const float* addend[kMaxExits];
 };
 
 template <int BN>
@@ -1201,11 +1135,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           const uint4* oh = (onehot_row >= 0)
                                 ? reinterpret_cast<const uint4*>(g.onehot_rows[p] + onehot_row * Ndim + col0 + c * 32)
                                 : nullptr;
+          const float4* ad = (g.addend[p] != nullptr) ? reinterpret_cast<const float4*>(g.addend[p] + off) : nullptr;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = r[8 * u + e] * alpha;
+            if (ad != nullptr) {
+              const float4 a0 = ad[2 * u], a1 = ad[2 * u + 1];
+              f[0] += a0.x; f[1] += a0.y; f[2] += a0.z; f[3] += a0.w;
+              f[4] += a1.x; f[5] += a1.y; f[6] += a1.z; f[7] += a1.w;
+            }
             if (oh != nullptr) {
               float w[8];
               bf16x8_to_f32(__ldg(oh + u), w);
@@ -1422,11 +1362,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint4* oh = (onehot_row >= 0)
                                 ? reinterpret_cast<const uint4*>(g.onehot_rows[p] + onehot_row * Ndim + col0 + c * 32)
                                 : nullptr;
+          const float4* ad = (g.addend[p] != nullptr) ? reinterpret_cast<const float4*>(g.addend[p] + off) : nullptr;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = r[8 * u + e] * alpha;
+            if (ad != nullptr) {
+              const float4 a0 = ad[2 * u], a1 = ad[2 * u + 1];
+              f[0] += a0.x; f[1] += a0.y; f[2] += a0.z; f[3] += a0.w;
+              f[4] += a1.x; f[5] += a1.y; f[6] += a1.z; f[7] += a1.w;
+            }
             if (oh != nullptr) {
               float w[8];
               bf16x8_to_f32(__ldg(oh + u), w);
@@ -1527,8 +1473,89 @@ int resident_pairs(Kernel fn, int threads, size_t smem) {
 
 size_t align_up(size_t b) { return (b + 255) & ~size_t(255); }
 
-// bf16 G' of every exit: [M][T][V]
-size_t g_bytes(const LossProblem& p) { return static_cast<size_t>(p.M) * p.T * p.V * sizeof(__nv_bfloat16); }
+// ------------------------------------------------------------------ backward chunk plan
+// The backward pass writes the dense logit gradient G' of every exit for one
+// block of tokens x one chunk of the vocabulary at a time into the workspace,
+// then consumes it with the two GEMMs.  dW rows of a chunk are complete after
+// their chunk (K runs over the block's tokens; token blocks after the first
+// add into dW), dh rows of a block after the block's last chunk (K runs over
+// the chunk's columns; the chunks before the last leave fp32 partial sums in
+// the workspace).  Workspace: [G' chunk: M x Tb x Vc bf16][dh partials:
+// Tb x sum(D) f32, only with more than one chunk][targets grouped by id].
+struct BwdPlan {
+  int64_t Tb, Vc;          // tokens per block (last block shorter), columns per chunk (last chunk shorter)
+  int64_t nT, nV;
+  size_t g_bytes, acc_bytes, seg_bytes;
+  size_t total() const { return g_bytes + acc_bytes + seg_bytes; }
+};
+
+constexpr size_t kDefaultBwdBudget = size_t(1) << 30;   // 1 GiB
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+int64_t sum_d(const LossProblem& p) {
+  int64_t s = 0;
+  for (int m = 0; m < p.M; ++m) s += p.D[m];
+  return s;
+}
+
+BwdPlan plan_shape(const LossProblem& p, int64_t Tb, int64_t Vc) {
+  BwdPlan b{};
+  b.Tb = Tb;
+  b.Vc = Vc;
+  b.nT = ceil_div(p.T, Tb);
+  b.nV = ceil_div(p.V, Vc);
+  b.g_bytes = align_up(static_cast<size_t>(p.M) * Tb * Vc * sizeof(__nv_bfloat16));
+  b.acc_bytes = b.nV > 1 ? align_up(static_cast<size_t>(Tb) * sum_d(p) * sizeof(float)) : 0;
+  b.seg_bytes = align_up(segindex_bytes(p.T, p.V));
+  return b;
+}
+
+// Bytes the plan moves beyond one pass over G': the dW read-modify-write of
+// every token block after the first, the dh partials of every chunk but the
+// last, and a fixed charge per (block, chunk) for its three launches' ramps.
+double plan_cost(const LossProblem& p, const BwdPlan& b) {
+  const double sd = static_cast<double>(sum_d(p));
+  const double dw_rmw = static_cast<double>(b.nT - 1) * 8.0 * static_cast<double>(p.V) * sd;
+  const double dh_part = static_cast<double>(b.nT) * static_cast<double>(b.nV - 1) * 8.0 * static_cast<double>(b.Tb) * sd;
+  return dw_rmw + dh_part + 3.0e8 * static_cast<double>(b.nT * b.nV);
+}
+
+// The cheapest plan whose workspace fits in `budget` bytes (Tb = 0 when none fits).
+BwdPlan choose_plan(const LossProblem& p, size_t budget) {
+  BwdPlan best{};
+  double best_cost = 0.0;
+  for (int64_t nT = 1;; ++nT) {
+    const int64_t Tb = nT == 1 ? p.T : round_up(ceil_div(p.T, nT), kBM);
+    if (nT > 1 && Tb >= round_up(ceil_div(p.T, nT - 1), kBM)) {   // same block size as fewer blocks
+      if (Tb <= kBM) break;
+      continue;
+    }
+    BwdPlan b = plan_shape(p, Tb, p.V);
+    if (b.total() > budget) {
+      const BwdPlan probe = plan_shape(p, Tb, kLossBN);   // smallest chunk: does any chunk width fit?
+      if (probe.total() > budget) {
+        if (Tb <= kBM) break;
+        continue;
+      }
+      // widest chunk (a multiple of the tile width) that fits, then equal chunks of at most that width
+      const size_t fixed = probe.acc_bytes + probe.seg_bytes;
+      int64_t vmax = static_cast<int64_t>((budget - fixed) / (static_cast<size_t>(p.M) * Tb * 2)) / kLossBN * kLossBN;
+      while (vmax > kLossBN && plan_shape(p, Tb, vmax).total() > budget) vmax -= kLossBN;
+      if (vmax < kLossBN) vmax = kLossBN;
+      const int64_t nV = ceil_div(p.V, vmax);
+      b = plan_shape(p, Tb, round_up(ceil_div(p.V, nV), kLossBN));
+    }
+    const double c = plan_cost(p, b);
+    if (best.Tb == 0 || c < best_cost) {
+      best = b;
+      best_cost = c;
+    }
+    if (Tb <= kBM) break;
+  }
+  return best;
+}
 
 struct TcWs {
   float* partial;
@@ -1545,52 +1572,19 @@ TcWs fwd_layout(const LossProblem& p, void* ws) {
   return w;
 }
 
-// The loss tile kernels run on single CTAs.  The CTA-pair form (256-token
-// tiles, half of the W tile per SM) passes the same parity tests but measured
-// slower on the 3-exit suite at T = 8192: 5.6-5.7 ms per forward launch
-// instead of 5.2 ms, with 8-10 GB of DRAM reads per launch instead of 3.6 GB
-// at the same 2048-token tile grouping, and lower clocks under the power cap.
-constexpr bool kLossPair = false;
-
 template <int MODE, int DISTILL, bool TGRAD = false>
-cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& args_in, cudaStream_t st) {
-  constexpr bool PAIR = kLossPair;
+cudaError_t run_loss_tiles(const LossProblem& p, const LossArgs& a, cudaStream_t st) {
   LossMaps maps;
   for (int m = 0; m < p.M; ++m) {
     if (!make_map(&maps.h[m], p.h[m], p.D[m], p.T, kBK, kBM)) return cudaErrorInvalidValue;
-    if (!make_map(&maps.w[m], p.W[m], p.D[m], p.V, kBK, LossSmem<PAIR>::kBRows)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.w[m], p.W[m], p.D[m], p.V, kBK, kLossBN)) return cudaErrorInvalidValue;
   }
-  LossArgs a = args_in;
-  if (PAIR) {
-    a.n_tt = static_cast<int>((p.T + 2 * kBM - 1) / (2 * kBM));
-    a.num_tiles = a.n_tt * a.n_vt;
-    a.group_tt = 8;                 // 2048 tokens per group, as with 128-token tiles
-  }
-  const size_t smem = sizeof(LossSmem<PAIR>) + 1024;
-  auto fn = loss_tile_kernel<MODE, DISTILL, TGRAD, PAIR>;
+  const size_t smem = sizeof(LossSmem) + 1024;
+  auto fn = loss_tile_kernel<MODE, DISTILL, TGRAD>;
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  if (PAIR) {
-    const int resident = resident_pairs(fn, kLossThreads, smem);
-    const int pairs = a.num_tiles < resident ? a.num_tiles : resident;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    cfg.blockDim = dim3(kLossThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, fn, maps, a);
-    if (err != cudaSuccess) return err;
-  } else {
-    const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-    fn<<<grid, kLossThreads, smem, st>>>(maps, a);
-  }
+  const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+  fn<<<grid, kLossThreads, smem, st>>>(maps, a);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -1600,6 +1594,9 @@ LossArgs base_args(const LossProblem& p) {
   a.M = p.M;
   a.T = static_cast<int>(p.T);
   a.V = static_cast<int>(p.V);
+  a.v0 = 0;
+  a.Vtot = static_cast<int>(p.V);
+  a.ldS = static_cast<int>(p.T);
   for (int m = 0; m < p.M; ++m) a.kblocks[m] = static_cast<int>(p.D[m] / kBK);
   a.n_tt = static_cast<int>((p.T + kBM - 1) / kBM);
   a.n_vt = loss_n_vt(p);
@@ -1612,6 +1609,8 @@ LossArgs base_args(const LossProblem& p) {
   a.student_wsum = 0.f;
   for (int m = 0; m + 1 < p.M; ++m) a.student_wsum += p.exit_w[m];
   a.status = p.status;
+  a.wait_ns = p.wait_ns != 0 ? p.wait_ns : kWaitLimitNs;
+  a.withhold_loads = p.withhold_loads;
   return a;
 }
 
@@ -1658,56 +1657,109 @@ int pick_bn(const LossProblem& p) {
   return dmax >= 256 ? 256 : dmax >= 128 ? 128 : 64;
 }
 
-// dh_m[T x D_m] = a (G'_m[T x V] W^m[V x D_m] - c_m W^m[y_t]) for every exit in one launch:
-// A = G'_m (K = V contiguous), B = W^m (N = D_m contiguous); the one-hot row of
-// W^m is subtracted exactly in the epilogue.
+// One (token block, vocabulary chunk) of the backward pass: its tokens [t0, t0 + Tb)
+// and columns [v0, v0 + Vc), with G' = [M][Tb][Vc] bf16.
+struct BwdChunk {
+  int64_t t0, Tb, v0, Vc;
+  bool first_v, last_v;    // first / last chunk of the block
+  bool first_t;            // first block
+  const __nv_bfloat16* G;
+  float* acc;              // dh partial sums [Tb][sum D] (NULL with a single chunk)
+};
+
+// dh_m[Tb x D_m] (+)= a G'_m[Tb x Vc] W^m[v0 : v0 + Vc] for every exit in one launch:
+// A = G'_m (K = Vc contiguous), B = the chunk's rows of W^m (N = D_m contiguous).
+// The last chunk of a block adds the earlier chunks' fp32 partials, subtracts
+// the one-hot row a c_m W^m[y_t] exactly and writes bf16 dh; the others write
+// (first) or add to (later) the fp32 partials.
 template <int BN>
-cudaError_t run_dh_all(const LossProblem& p, const __nv_bfloat16* G, void* const* dh, float alpha, cudaStream_t st) {
+cudaError_t run_dh_chunk(const LossProblem& p, const BwdChunk& c, void* const* dh, float alpha, cudaStream_t st) {
   GemmMaps maps;
   GemmArgs g{};
   g.nprob = p.M;
-  g.Mdim = static_cast<int>(p.T);
-  g.Kdim = static_cast<int>(p.V);
+  g.Mdim = static_cast<int>(c.Tb);
+  g.Kdim = static_cast<int>(c.Vc);
   for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
   const bool tgrad = p.teacher_grad != 0 && p.M > 1;
   if (tgrad) g.alpha[p.M - 1] = alpha;             // the teacher's G' already carries w_T
   g.status = p.status;
-  g.onehot_idx = p.y;
+  g.onehot_idx = p.y + c.t0;
   g.onehot_limit = static_cast<int>(p.V);
+  g.accumulate = c.first_v ? 0 : 1;
+  int64_t acc_off = 0;
   for (int m = 0; m < p.M; ++m) {
-    const __nv_bfloat16* Gm = G + static_cast<int64_t>(m) * p.T * p.V;
-    if (!make_map(&maps.a[m], Gm, p.V, p.T, kBK, kBM)) return cudaErrorInvalidValue;
-    if (!make_map(&maps.b[m], p.W[m], p.D[m], p.V, 64, kBK)) return cudaErrorInvalidValue;
+    const __nv_bfloat16* Gm = c.G + static_cast<int64_t>(m) * c.Tb * c.Vc;
+    const __nv_bfloat16* Wc = static_cast<const __nv_bfloat16*>(p.W[m]) + c.v0 * p.D[m];
+    if (!make_map(&maps.a[m], Gm, c.Vc, c.Tb, kBK, kBM)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.b[m], Wc, p.D[m], c.Vc, 64, kBK)) return cudaErrorInvalidValue;
     g.Ndim[m] = static_cast<int>(p.D[m]);
-    g.out[m] = dh[m];
-    g.onehot_rows[m] = static_cast<const __nv_bfloat16*>(p.W[m]);
-    g.onehot_coef[m] = (m == p.M - 1) ? (tgrad ? p.exit_w[m] : 1.f) : 1.f - p.alpha_d;
+    float* acc_m = c.acc != nullptr ? c.acc + acc_off : nullptr;
+    acc_off += c.Tb * p.D[m];
+    if (c.last_v) {
+      g.out[m] = static_cast<__nv_bfloat16*>(dh[m]) + c.t0 * p.D[m];
+      g.onehot_rows[m] = static_cast<const __nv_bfloat16*>(p.W[m]);
+      g.onehot_coef[m] = (m == p.M - 1) ? (tgrad ? p.exit_w[m] : 1.f) : 1.f - p.alpha_d;
+      g.addend[m] = c.first_v ? nullptr : acc_m;
+    } else {
+      g.out[m] = acc_m;
+    }
   }
-  return run_gemm<false, true, BN, true>(maps, g, st);
+  if (c.last_v) return run_gemm<false, true, BN, true>(maps, g, st);
+  return run_gemm<false, true, BN, false>(maps, g, st);
 }
 
-// dW^m[V x D_m] (+)= a G'_m^T h_m for every exit in one launch: A = G'^T (M = V
-// contiguous), B = h_m (N = D_m contiguous), K = T.
+// dW^m[v0 : v0 + Vc] (+)= a G'_m^T h_m[t0 : t0 + Tb] for every exit in one launch:
+// A = G'^T (M = Vc contiguous), B = the block's rows of h_m (N = D_m contiguous),
+// K = Tb.  Blocks after the first (and every block with accumulate) add.
 template <int BN>
-cudaError_t run_dw_all(const LossProblem& p, const __nv_bfloat16* G, float* const* dW, float alpha, int accumulate,
-                       cudaStream_t st) {
+cudaError_t run_dw_chunk(const LossProblem& p, const BwdChunk& c, float* const* dW, float alpha, int accumulate,
+                         cudaStream_t st) {
   GemmMaps maps;
   GemmArgs g{};
   g.nprob = p.M;
-  g.Mdim = static_cast<int>(p.V);
-  g.Kdim = static_cast<int>(p.T);
+  g.Mdim = static_cast<int>(c.Vc);
+  g.Kdim = static_cast<int>(c.Tb);
   for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
   if (p.teacher_grad != 0 && p.M > 1) g.alpha[p.M - 1] = alpha;   // the teacher's G' already carries w_T
-  g.accumulate = accumulate;
+  g.accumulate = (accumulate || !c.first_t) ? 1 : 0;
   g.status = p.status;
   for (int m = 0; m < p.M; ++m) {
-    const __nv_bfloat16* Gm = G + static_cast<int64_t>(m) * p.T * p.V;
-    if (!make_map(&maps.a[m], Gm, p.V, p.T, 64, kBK)) return cudaErrorInvalidValue;
-    if (!make_map(&maps.b[m], p.h[m], p.D[m], p.T, 64, kBK)) return cudaErrorInvalidValue;
+    const __nv_bfloat16* Gm = c.G + static_cast<int64_t>(m) * c.Tb * c.Vc;
+    const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(p.h[m]) + c.t0 * p.D[m];
+    if (!make_map(&maps.a[m], Gm, c.Vc, c.Tb, 64, kBK)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.b[m], hb, p.D[m], c.Tb, 64, kBK)) return cudaErrorInvalidValue;
     g.Ndim[m] = static_cast<int>(p.D[m]);
-    g.out[m] = dW[m];
+    g.out[m] = dW[m] + c.v0 * p.D[m];
   }
   return run_gemm<true, true, BN, false>(maps, g, st);
+}
+
+// G' of one (token block, vocabulary chunk): the tile kernel on the block's
+// rows of h, y and stats and the chunk's rows of W.
+cudaError_t run_grad_chunk(const LossProblem& p, const BwdChunk& c, const float* stats, cudaStream_t st) {
+  LossProblem q = p;
+  q.T = c.Tb;
+  q.V = c.Vc;
+  q.y = p.y + c.t0;
+  for (int m = 0; m < p.M; ++m) {
+    q.h[m] = static_cast<const __nv_bfloat16*>(p.h[m]) + c.t0 * p.D[m];
+    q.W[m] = static_cast<const __nv_bfloat16*>(p.W[m]) + c.v0 * p.D[m];
+  }
+  LossArgs a = base_args(q);
+  a.v0 = static_cast<int>(c.v0);
+  a.Vtot = static_cast<int>(p.V);
+  a.ldS = static_cast<int>(p.T);
+  a.stats = const_cast<float*>(stats) + c.t0;
+  a.G = const_cast<__nv_bfloat16*>(c.G);
+  const bool tgrad = p.teacher_grad != 0 && p.M > 1;
+  return tgrad ? (p.distill == 1   ? run_loss_tiles<kModeGrad, 1, true>(q, a, st)
+                  : p.distill == 2 ? run_loss_tiles<kModeGrad, 2, true>(q, a, st)
+                  : p.distill == 3 ? run_loss_tiles<kModeGrad, 3, true>(q, a, st)
+                                   : run_loss_tiles<kModeGrad, 0, true>(q, a, st))
+         : p.distill == 1 ? run_loss_tiles<kModeGrad, 1>(q, a, st)
+         : p.distill == 2 ? run_loss_tiles<kModeGrad, 2>(q, a, st)
+         : p.distill == 3 ? run_loss_tiles<kModeGrad, 3>(q, a, st)
+                          : run_loss_tiles<kModeGrad, 0>(q, a, st);
 }
 
 }  // namespace
@@ -1749,7 +1801,23 @@ cudaError_t agree_tc(const LossProblem& p, const float* stats, float* metrics, f
 }
 
 size_t loss_tc_bwd_bytes(const LossProblem& p) {
-  return align_up(g_bytes(p)) + segindex_bytes(p.T, p.V);
+  const BwdPlan whole = plan_shape(p, p.T, p.V);
+  return whole.total() <= kDefaultBwdBudget ? whole.total() : choose_plan(p, kDefaultBwdBudget).total();
+}
+
+size_t loss_tc_bwd_min_bytes(const LossProblem& p) {
+  // one tile of tokens per block: either the whole vocabulary at once (no dh
+  // partials) or one tile of columns per chunk, whichever is smaller
+  const int64_t Tb = p.T < kBM ? p.T : kBM;
+  const size_t whole_v = plan_shape(p, Tb, p.V).total();
+  const size_t one_tile = plan_shape(p, Tb, p.V < kLossBN ? p.V : kLossBN).total();
+  return whole_v < one_tile ? whole_v : one_tile;
+}
+
+void loss_tc_bwd_plan(const LossProblem& p, size_t ws_bytes, int64_t* Tb, int64_t* Vc) {
+  const BwdPlan b = choose_plan(p, ws_bytes);
+  *Tb = b.Tb;
+  *Vc = b.Vc;
 }
 
 cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void* ws, cudaStream_t st) {
@@ -1783,45 +1851,55 @@ cudaError_t loss_tc_fwd(const LossProblem& p, float* losses, float* stats, void*
 }
 
 cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_scale, void* const* dh,
-                        float* const* dW, int accumulate, void* ws, cudaStream_t st) {
-  __nv_bfloat16* G = static_cast<__nv_bfloat16*>(ws);
-  LossArgs a = base_args(p);
-  a.stats = const_cast<float*>(stats);
-  a.G = G;
-  const bool tgrad = p.teacher_grad != 0 && p.M > 1;
-  cudaError_t err = tgrad ? (p.distill == 1   ? run_loss_tiles<kModeGrad, 1, true>(p, a, st)
-                             : p.distill == 2 ? run_loss_tiles<kModeGrad, 2, true>(p, a, st)
-                             : p.distill == 3 ? run_loss_tiles<kModeGrad, 3, true>(p, a, st)
-                                              : run_loss_tiles<kModeGrad, 0, true>(p, a, st))
-                    : p.distill == 1 ? run_loss_tiles<kModeGrad, 1>(p, a, st)
-                    : p.distill == 2 ? run_loss_tiles<kModeGrad, 2>(p, a, st)
-                    : p.distill == 3 ? run_loss_tiles<kModeGrad, 3>(p, a, st)
-                                     : run_loss_tiles<kModeGrad, 0>(p, a, st);
-  if (err != cudaSuccess) return err;
-  // Tokens grouped by target, for the exact one-hot part of dW.
-  SegIndexDev ix;
-  err = build_segindex(p.y, p.T, p.V, static_cast<char*>(ws) + align_up(g_bytes(p)), &ix, st);
-  if (err != cudaSuccess) return err;
+                        float* const* dW, int accumulate, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const BwdPlan plan = choose_plan(p, ws_bytes);
+  if (plan.Tb == 0) return cudaErrorInvalidValue;       // the caller checked the minimum size
+  char* base = static_cast<char*>(ws);
+  __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(base);
+  float* acc = plan.acc_bytes ? reinterpret_cast<float*>(base + plan.g_bytes) : nullptr;
+  void* seg_ws = base + plan.g_bytes + plan.acc_bytes;
   const float alpha = grad_scale / static_cast<float>(p.T);
-  switch (pick_bn(p)) {
-    case 256: err = run_dh_all<256>(p, G, dh, alpha, st); break;
-    case 128: err = run_dh_all<128>(p, G, dh, alpha, st); break;
-    default: err = run_dh_all<64>(p, G, dh, alpha, st); break;
+  const int bn = pick_bn(p);
+  cudaError_t err = cudaSuccess;
+  for (int64_t t0 = 0; t0 < p.T && err == cudaSuccess; t0 += plan.Tb) {
+    for (int64_t v0 = 0; v0 < p.V && err == cudaSuccess; v0 += plan.Vc) {
+      BwdChunk c;
+      c.t0 = t0;
+      c.Tb = t0 + plan.Tb <= p.T ? plan.Tb : p.T - t0;
+      c.v0 = v0;
+      c.Vc = v0 + plan.Vc <= p.V ? plan.Vc : p.V - v0;
+      c.first_v = v0 == 0;
+      c.last_v = v0 + c.Vc >= p.V;
+      c.first_t = t0 == 0;
+      c.G = G;
+      c.acc = acc;
+      err = run_grad_chunk(p, c, stats, st);
+      if (err != cudaSuccess) break;
+      switch (bn) {
+        case 256: err = run_dh_chunk<256>(p, c, dh, alpha, st); break;
+        case 128: err = run_dh_chunk<128>(p, c, dh, alpha, st); break;
+        default: err = run_dh_chunk<64>(p, c, dh, alpha, st); break;
+      }
+      if (err != cudaSuccess) break;
+      switch (bn) {
+        case 256: err = run_dw_chunk<256>(p, c, dW, alpha, accumulate, st); break;
+        case 128: err = run_dw_chunk<128>(p, c, dW, alpha, accumulate, st); break;
+        default: err = run_dw_chunk<64>(p, c, dW, alpha, accumulate, st); break;
+      }
+    }
   }
   if (err != cudaSuccess) return err;
-  switch (pick_bn(p)) {
-    case 256: err = run_dw_all<256>(p, G, dW, alpha, accumulate, st); break;
-    case 128: err = run_dw_all<128>(p, G, dW, alpha, accumulate, st); break;
-    default: err = run_dw_all<64>(p, G, dW, alpha, accumulate, st); break;
-  }
+  // one-hot part of dW over every token: (1 - alpha_d) for students, 1 for the
+  // teacher; tokens grouped by target, every exit in one launch pair
+  SegIndexDev ix;
+  err = build_segindex(p.y, p.T, p.V, seg_ws, &ix, st);
   if (err != cudaSuccess) return err;
-  // one-hot part of dW: (1 - alpha_d) for students, 1 for the teacher; every exit in one launch pair
   int d_vec[kMaxExits];
   float scale[kMaxExits];
   for (int m = 0; m < p.M; ++m) {
-    const float c = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
+    const float cm = (m == p.M - 1) ? 1.f : 1.f - p.alpha_d;
     d_vec[m] = static_cast<int>(p.D[m] / 8);
-    scale[m] = alpha * p.exit_w[m] * c;
+    scale[m] = alpha * p.exit_w[m] * cm;
   }
   return scatter_target_rows(ix, p.M, p.h, d_vec, dW, scale, st);
 }

@@ -45,10 +45,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Gives up
-// when another role of the CTA has set *abort, or after kWaitLimitNs; in the
-// latter case it sets *abort and MLS_DEVFLAG_TIMEOUT.  Returns false on give-up.
+// when another role of the CTA has set *abort, or after limit_ns (default
+// kWaitLimitNs); in the latter case it sets *abort and MLS_DEVFLAG_TIMEOUT.
+// Returns false on give-up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* dev_status) {
+                                          int32_t* dev_status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
@@ -56,7 +57,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         set_flag(dev_status, MLS_DEVFLAG_TIMEOUT);
         return false;

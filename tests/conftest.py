@@ -11,12 +11,13 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: long CPU work (full-size oracle)")
-    # The boundary tests load libmls.so; build it in-tree when it is missing
-    # (nvcc cross-compiles without a GPU).
+    # The boundary and GPU tests load libmls.so; build it in-tree when it is
+    # missing or was built from other sources than the ones in the tree (a
+    # content hash, so a copied tree keeps its library; nvcc cross-compiles
+    # without a GPU).
     try:
         from lm_head_loss_junction_b200 import build
-        if not os.path.exists(build.LIB):
-            build.build(force=True)
+        build.build()
     except Exception as exc:  # the tests that need the library then fail with its error
         sys.stderr.write(f"libmls.so could not be built: {exc}\n")
 

@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import oracle
-from lm_head_loss_junction_b200 import multiexit_loss_bwd, multiexit_loss_fwd, new_status, status_read
+from lm_head_loss_junction_b200 import (multiexit_loss_bwd, multiexit_loss_bwd_plan, multiexit_loss_fwd, new_status,
+                                        status_read)
 from lm_head_loss_junction_b200 import workloads as wl
 from tests.helpers import assert_grad_close, assert_loss_close, assert_stats_close, f64
 
@@ -33,15 +34,19 @@ def _losses_expected(r, M):
     return np.concatenate([r["ce_lm"], r["ce_kd"], [r["loss"]]])
 
 
-def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce", teacher_grad=False):
+def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce", teacher_grad=False, bwd_ws_bytes=None):
+    """Every output against the oracle.  bwd_ws_bytes: the backward call's workspace
+    size (None: the size the workspace query returns), which sets how the call
+    splits its work into token blocks and vocabulary chunks."""
     cfg = d.cfg
     M = cfg.M
     y, h, W = _gpu_inputs(d)
     st = new_status()
     losses, stats = multiexit_loss_fwd(y, h, W, alpha, status=st, exit_weights=exit_weights, distill=distill,
                                        teacher_grad=teacher_grad)
+    ws = None if bwd_ws_bytes is None else torch.empty(bwd_ws_bytes, dtype=torch.uint8, device="cuda")
     dh, dW = multiexit_loss_bwd(y, h, W, stats, alpha, grad_scale, status=st, exit_weights=exit_weights,
-                                distill=distill, teacher_grad=teacher_grad)
+                                distill=distill, teacher_grad=teacher_grad, workspace=ws)
     assert status_read(st) == (0, 0)
     r = _oracle(d, alpha, grad_scale, exit_weights=exit_weights, distill=distill, teacher_grad=teacher_grad)
     assert_loss_close(losses, _losses_expected(r, M), "losses")
@@ -78,6 +83,70 @@ def test_bf16_tensor_core_path_small(name, small):
     cfg = wl.small_variant(wl.CONFIGS[name], **small)
     d = wl.make_inputs(cfg, with_tables=False)
     _check_all(d, cfg.alpha_d, grad_scale=1.0)
+
+
+def _pieces(cfg, ws_bytes):
+    Tb, Vc, _ = multiexit_loss_bwd_plan(cfg.T, cfg.D, cfg.V, torch.bfloat16, ws_bytes)
+    return Tb, Vc, -(-cfg.T // Tb), -(-cfg.V // Vc)
+
+
+# Small workspaces force the backward pass into many token blocks and
+# vocabulary chunks: ragged last blocks (T not a multiple of 128), a half-tile
+# last chunk (V = 640), first / middle / last chunks of the dh partial sums and
+# the dW additions of later blocks.
+CHUNKED = [
+    ("main3", dict(batch=1, seq=300, V=1024)),
+    ("proxy2", dict(batch=2, seq=97, V=2048)),
+    ("suite4", dict(batch=1, seq=200, V=512)),
+    ("main3_aligned", dict(batch=1, seq=256, V=640)),
+]
+
+
+@pytest.mark.parametrize("name,small", CHUNKED)
+def test_chunked_backward_smallest_workspace(name, small):
+    cfg = wl.small_variant(wl.CONFIGS[name], **small)
+    d = wl.make_inputs(cfg, with_tables=False)
+    _, _, mn = multiexit_loss_bwd_plan(cfg.T, cfg.D, cfg.V, torch.bfloat16, 0)
+    Tb, Vc, nT, nV = _pieces(cfg, mn)
+    assert Tb == 128 and nT > 1
+    _check_all(d, cfg.alpha_d, grad_scale=1.0, bwd_ws_bytes=mn)
+    # a middle size: fewer, larger pieces, same results within the tolerance
+    mid = mn
+    while _pieces(cfg, mid)[2:] == (nT, nV):
+        mid = mid * 5 // 4
+    _check_all(d, cfg.alpha_d, grad_scale=1.0, bwd_ws_bytes=mid)
+
+
+@pytest.mark.parametrize("distill,teacher_grad", [("ce", True), ("reverse_kl", False), ("js", True),
+                                                  ("accept", False)])
+def test_chunked_backward_options(distill, teacher_grad):
+    cfg = wl.small_variant(wl.CONFIGS["main3"], batch=1, seq=300, V=1024)
+    d = wl.make_inputs(cfg, with_tables=False)
+    _, _, mn = multiexit_loss_bwd_plan(cfg.T, cfg.D, cfg.V, torch.bfloat16, 0)
+    assert _pieces(cfg, mn)[3] > 2
+    _check_all(d, 0.6, 2.0, exit_weights=[1.5, 0.7, 0.8], distill=distill, teacher_grad=teacher_grad,
+               bwd_ws_bytes=mn)
+
+
+def test_chunked_backward_accumulate_and_determinism():
+    cfg = wl.small_variant(wl.CONFIGS["suite4"], batch=1, seq=200, V=512)
+    d = wl.make_inputs(cfg, with_tables=False)
+    y, h, W = _gpu_inputs(d)
+    _, _, mn = multiexit_loss_bwd_plan(cfg.T, cfg.D, cfg.V, torch.bfloat16, 0)
+    ws = torch.empty(mn, dtype=torch.uint8, device="cuda")
+    _, stats = multiexit_loss_fwd(y, h, W, 0.3)
+    r = oracle.multiexit_loss(d.y, d.o, d.W, alpha_d=0.3)
+    base = [torch.randn(w.shape, dtype=torch.float32, device="cuda") for w in W]
+    dW = [b.clone() for b in base]
+    dh1, _ = multiexit_loss_bwd(y, h, W, stats, 0.3, dW=dW, accumulate_dW=True, workspace=ws)
+    for m in range(cfg.M):
+        assert_grad_close(dW[m] - base[m], r["dW"][m], f"accumulated dW[{m}]")
+    g1 = multiexit_loss_bwd(y, h, W, stats, 0.3, workspace=ws)
+    g2 = multiexit_loss_bwd(y, h, W, stats, 0.3, workspace=ws)
+    for a, b in zip(g1[0] + g1[1], g2[0] + g2[1]):
+        assert torch.equal(a, b)
+    for a, b in zip(dh1, g1[0]):
+        assert torch.equal(a, b)
 
 
 def test_alpha_and_grad_scale_are_runtime_arguments():

@@ -1,12 +1,13 @@
 """The allocation-free junction backward entry point, called through the C ABI.
 
-mls_junction_bwd_noalloc serves callers that cannot give the library a device
-buffer (for example while a stream is being captured into a CUDA graph, where
-cudaMalloc is not allowed): it takes its scratch from a fixed array inside the
-library.  This test runs it twice in a row on different shapes -- so stale
-scratch contents from the first call would show in the second -- and checks
-each result against the ordinary entry point with a caller-supplied workspace.
-The file name makes pytest collect it last.
+mls_junction_bwd_noalloc serves callers that cannot allocate device memory at
+the point of the call -- programs whose device memory is owned by another
+allocator, or latency-critical code that must not call cudaMalloc/cudaFree
+(both can synchronise the device): it takes its scratch from a fixed array
+inside the library.  This test runs it twice in a row on different shapes --
+so stale scratch contents from the first call would show in the second -- and
+checks each result against the ordinary entry point with a caller-supplied
+workspace.  The file name makes pytest collect it last.
 """
 import pytest
 import torch
@@ -63,8 +64,14 @@ def test_noalloc_rejects_sizes_beyond_its_array():
     T, D = o.shape
     V_big = 4 << 20                       # the id tables alone would exceed the fixed array
     dE = torch.zeros(1, dtype=torch.float32, device="cuda")
-    code = _lib.lib().mls_junction_bwd_noalloc(
+    lib = _lib.lib()
+    stream = torch.cuda.current_stream().cuda_stream
+    code = lib.mls_junction_bwd_noalloc(
         x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V_big, E.shape[1], dy.data_ptr(),
-        torch.empty_like(o).data_ptr(), None, dE.data_ptr(), 0, _lib.MLS_BF16, None,
-        torch.cuda.current_stream().cuda_stream)
+        torch.empty_like(o).data_ptr(), None, dE.data_ptr(), 0, _lib.MLS_BF16, None, stream)
     assert code == 2                      # MLS_ERR_UNSUPPORTED, nothing launched
+    # argument errors are reported first, as mls_junction_bwd reports them
+    code = lib.mls_junction_bwd_noalloc(
+        x.data_ptr(), T, o.data_ptr(), D, E.data_ptr(), V_big, E.shape[1], None,
+        torch.empty_like(o).data_ptr(), None, dE.data_ptr(), 0, _lib.MLS_BF16, None, stream)
+    assert code == 1                      # MLS_ERR_INVALID_ARG: dy is NULL
