@@ -140,7 +140,8 @@ class Step:
         bb = bwd_ws_bytes or bb               # the query's bounded size unless asked otherwise
         self.ws_loss = torch.empty(max(fb, bb), dtype=torch.uint8, device=device)
         self.bwd_plan = api.multiexit_loss_bwd_plan(T, list(c.D), V, dt, max(fb, bb))
-        self.ws_j = torch.empty(api.junction_bwd_workspace(T, V), dtype=torch.uint8, device=device)
+        self.ws_j = torch.empty(api.junction_bwd_multi_workspace(T, V, M - 1) if M > 1 else 1, dtype=torch.uint8,
+                                device=device)
         self.status = api.new_status(device)
 
     def phases(self):
@@ -150,9 +151,9 @@ class Step:
         M = c.M
 
         def junction_fwd(stream):
-            for j in range(M - 1):
-                a.junction_fwd(self.x, self.o[j], self.E[j + 1], out=self.jy[j], scale_out=self.jscale[j],
-                               status=self.status, stream=stream)
+            if M > 1:    # every junction of the suite in one call (one launch for bf16)
+                a.junction_fwd_multi(self.x, self.o[:M - 1], self.E[1:], out=self.jy, scale_out=self.jscale,
+                                     status=self.status, stream=stream)
 
         def loss_fwd(stream):
             a.multiexit_loss_fwd(self.y, self.o, self.W, c.alpha_d, losses=self.losses, stats=self.stats,
@@ -163,10 +164,10 @@ class Step:
                                  workspace=self.ws_loss, status=self.status, stream=stream)
 
         def junction_bwd(stream):
-            for j in range(M - 1):
-                a.junction_bwd(self.x, self.o[j], self.E[j + 1], self.dh[j + 1], do_out=self.do[j],
-                               de_out=self.de[j], dE=self.dE[j], accumulate_dE=False, workspace=self.ws_j,
-                               status=self.status, stream=stream)
+            if M > 1:    # every junction in one call: one id grouping for all table gradients
+                a.junction_bwd_multi(self.x, self.o[:M - 1], self.E[1:], self.dh[1:], do_out=self.do,
+                                     de_out=self.de, dE=self.dE, accumulate_dE=False, workspace=self.ws_j,
+                                     status=self.status, stream=stream)
 
         return [junction_fwd, loss_fwd, loss_bwd, junction_bwd]
 
@@ -189,7 +190,13 @@ class Step:
         return 8.0 * c.T * c.V * sum(c.D)
 
     def junction_bytes(self):
-        """(forward, backward) algorithmic HBM bytes over all junctions of the step."""
+        """(forward, backward) algorithmic HBM bytes over all junctions of the step.
+
+        Backward: the row pass (dy, o, e row in; do, de rows, coefficient out;
+        id) plus the table gradient in overwrite mode: every row of each fp32
+        table dE written once, and the g_e part of dy and the coefficients
+        read again by the id-grouped sums.  (The embedding rows of the ids
+        present are read again too; not counted, so the rate is a lower bound.)"""
         c = self.cfg
         b = 2 if c.dtype == "bf16" else 4
         fwd = bwd = 0
@@ -197,6 +204,7 @@ class Step:
             D, dl, Dn = c.D[j], c.deltas[j + 1], c.D[j + 1]
             fwd += c.T * ((D + dl + Dn) * b + 4 + 4)                 # o, e row, y; id; scale
             bwd += c.T * ((Dn + D + dl + D + dl) * b + 4 + 4)        # dy, o, e row, do, de; id; coef
+            bwd += c.V * dl * 4 + c.T * (dl * b + 4)                 # dE table; g_e and coef re-read
         return fwd, bwd
 
 
@@ -274,6 +282,81 @@ def cpu_oracle_sample(d: wl.SuiteInputs, n_tokens: int):
     return time.perf_counter() - t0, n_tokens
 
 
+def measure_workload(name, device, stream, peaks, K, eager, cpu_tokens):
+    """One of the other workloads at its full size: the same step (junctions
+    fwd, loss fwd, loss bwd, junctions bwd), captured and replayed the same way,
+    K timed steps with CUDA events between phases; its loss-forward roofline
+    fraction; and the fp64 oracle timed on the first cpu_tokens tokens on the
+    host cores.  Returns a dict for the bench line's extras."""
+    cfg = wl.CONFIGS[name]
+    step = Step(cfg, device)
+    for _ in range(3):
+        step.run(stream)
+    torch.cuda.synchronize(device)
+    code, word = step.api.status_read(step.status, stream)
+    if code != 0:
+        raise RuntimeError(f"{name}: device status after warm-up: {code} ({word})")
+    fns = step.phases()
+    if eager:
+        runners = [lambda f=f: f(stream) for f in fns]
+        graphs = []
+    else:
+        graphs = []
+        for f in fns:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                f(None)
+            graphs.append(g)
+        runners = [g.replay for g in graphs]
+    for _ in range(2):
+        for r in runners:
+            r()
+    torch.cuda.synchronize(device)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(len(runners) + 1)] for _ in range(K)]
+    with ClockSampler(device.index) as clocks:
+        for k in range(K):
+            for i, r in enumerate(runners):
+                marks[k][i].record(stream)
+                r()
+            marks[k][-1].record(stream)
+        torch.cuda.synchronize(device)
+    ms = [statistics.mean(marks[k][i].elapsed_time(marks[k][i + 1]) for k in range(K)) for i in range(len(runners))]
+    code, word = step.api.status_read(step.status, stream)
+    if code != 0:
+        raise RuntimeError(f"{name}: device status after timing: {code} ({word})")
+    c = step.cfg
+    ms_step = sum(ms)
+    fl_fwd = 2.0 * c.T * c.V * sum(c.D)
+    out = {"workload": c.name, "T": c.T, "steps": K, "ms_per_step": ms_step,
+           "tokens_per_s": c.T / (ms_step / 1000.0),
+           "phases_ms": {"junction_fwd": ms[0], "loss_fwd": ms[1], "loss_bwd": ms[2], "junction_bwd": ms[3]},
+           "loss_bwd_pieces": {"token_block": step.bwd_plan[0], "vocab_chunk": step.bwd_plan[1]}}
+    if c.dtype == "bf16":
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        out["roofline"] = {"bound": "tensor", "kernel": "loss_tile_kernel<stats> (mls_multiexit_loss_fwd call)",
+                           "achieved": fl_fwd / (ms[1] / 1000.0) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                           "frac": fl_fwd / (ms[1] / 1000.0) / 1e12 / peak}
+        out["loss_executed_frac_of_peak"] = step.loss_flops_executed() / ((ms[1] + ms[2]) / 1000.0) / 1e12 / peak
+    else:
+        peak_fma = 148 * 128 * 2 * 1.965e9 / 1e12
+        out["roofline"] = {"bound": "alu", "kernel": "simt_stats_kernel (fp32 CUDA-core path)",
+                           "achieved": fl_fwd / (ms[1] / 1000.0) / 1e12, "peak": peak_fma, "unit": "TFLOP/s",
+                           "frac": fl_fwd / (ms[1] / 1000.0) / 1e12 / peak_fma}
+    if c.M > 1:
+        jf, jb = step.junction_bytes()
+        out["junction_fwd_frac_of_hbm"] = jf / (ms[0] / 1000.0) / 1e9 / peaks["hbm_gbs"]
+        out["junction_bwd_frac_of_hbm"] = jb / (ms[3] / 1000.0) / 1e9 / peaks["hbm_gbs"]
+    out["clocks"] = clocks.summary()
+    n = min(cpu_tokens, c.T)
+    sec, n = cpu_oracle_sample(step.host, n)
+    out["cpu_baseline"] = {"value": n / sec, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+                           "sample": f"first {n} tokens: junctions fwd+bwd and the {c.M}-exit loss fwd+bwd over "
+                                     f"the full vocabulary, fp64 numpy ({sec:.1f} s)"}
+    del graphs, runners, step
+    torch.cuda.empty_cache()
+    return out
+
+
 def _cores():
     try:
         import threadpoolctl
@@ -329,6 +412,8 @@ def main():
                     help="run the workload with this many tokens per GPU instead of its own batch")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step from Python instead of replaying a captured CUDA graph")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other four workloads (measured after the headline on one GPU by default)")
     ap.add_argument("--bwd-ws-gb", type=float, default=0.0,
                     help="workspace of the loss backward call in GB (default: the size the workspace query "
                          "returns); a larger one lets the call use fewer token blocks and vocabulary chunks")
@@ -584,7 +669,9 @@ def main():
         "loss_algorithmic_frac_of_peak": step.loss_flops_algorithmic() / ((ms_fwd + ms_bwd) / 1000.0) / 1e12 / peak_tc,
         "junction_fwd_gbs": jf_bytes / (phase_ms[0] / 1000.0) / 1e9 if c.M > 1 else None,
         "junction_fwd_frac_of_hbm": jf_bytes / (phase_ms[0] / 1000.0) / 1e9 / hbm if c.M > 1 else None,
-        "junction_bwd_gbs_incl_scatter": jb_bytes / (phase_ms[3] / 1000.0) / 1e9 if c.M > 1 else None,
+        "junction_bwd_gbs": jb_bytes / (phase_ms[3] / 1000.0) / 1e9 if c.M > 1 else None,
+        "junction_bwd_frac_of_hbm": jb_bytes / (phase_ms[3] / 1000.0) / 1e9 / hbm if c.M > 1 else None,
+        "junction_bytes": {"fwd": jf_bytes, "bwd_rows_and_tables": jb_bytes},
     }
     if sync_on:
         gbytes = sum(t.numel() * t.element_size() for t in grads)
@@ -611,6 +698,16 @@ def main():
         cpu = {"value": n / sec, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
                "sample": f"first {n} tokens of {cfg.name}: both junctions fwd+bwd and the {c.M}-exit loss "
                          f"fwd+bwd over the full vocabulary, fp64 numpy ({sec:.1f} s)"}
+
+    if rank == 0 and ws == 1 and not args.no_workloads and not args.tokens:
+        # the other workloads, each at its full size with the oracle beside it
+        others = []
+        for name in wl.CONFIG_ORDER:
+            if wl.CONFIGS[name].name == c.name:
+                continue
+            others.append(measure_workload(name, device, stream, peaks, max(5, min(K, 20)), args.eager,
+                                           256 if name == "tiny3" else 64))
+        extras["workloads"] = others
 
     if rank == 0:
         line = {

@@ -160,6 +160,41 @@ mls_status mls_junction_bwd_variant(const int32_t* x, int64_t T,
 mls_status mls_junction_bwd_workspace(int64_t T, int64_t V, size_t* bytes);
 
 /*
+ * Every junction of a suite in one call: J junctions (1 <= J <= 3) that share
+ * the token ids x, T and V, with widths D (HOST int64 [J+1], strictly
+ * increasing).  Junction k maps o[k] (dt [T, D[k]]) and e_next[k]
+ * (dt [V, D[k+1] - D[k]]) to y[k] (dt [T, D[k+1]]), exactly as
+ * mls_junction_fwd; the arrays o, e_next, y and scale_out are HOST arrays of
+ * J device pointers (scale_out may be NULL, or hold NULL entries).  In a
+ * training step the junctions' inputs come from different blocks, so this
+ * call fits where all of them are at hand (recomputation, the benchmark's
+ * hot-path step); the results equal J separate calls.  MLS_BF16 runs every
+ * junction in one launch whose blocks are divided among the junctions.
+ * Standard junction only (no variant bits).
+ */
+mls_status mls_junction_fwd_multi(const int32_t* x, int64_t T, int64_t V, int J, const int64_t* D,
+                                  const void* const* o, const void* const* e_next,
+                                  void* const* y, float* const* scale_out,
+                                  mls_dtype dt, int32_t* dev_status, void* stream);
+
+/*
+ * The backward pass of mls_junction_fwd_multi: results equal J calls of
+ * mls_junction_bwd with the same accumulate_dE.  dy, do_m: HOST arrays of J
+ * device pointers; de_rows and dE_table: HOST arrays of J device pointers
+ * (NULL entries allowed) or NULL.  The tokens are grouped by id once for all
+ * table gradients.  workspace >= mls_junction_bwd_multi_workspace(T, V, J)
+ * when any dE_table entry is non-NULL.
+ */
+mls_status mls_junction_bwd_multi_workspace(int64_t T, int64_t V, int J, size_t* bytes);
+
+mls_status mls_junction_bwd_multi(const int32_t* x, int64_t T, int64_t V, int J, const int64_t* D,
+                                  const void* const* o, const void* const* e_next,
+                                  const void* const* dy, void* const* do_m, void* const* de_rows,
+                                  float* const* dE_table, int accumulate_dE,
+                                  void* workspace, size_t ws_bytes,
+                                  mls_dtype dt, int32_t* dev_status, void* stream);
+
+/*
  * mls_junction_bwd_noalloc -- mls_junction_bwd without a workspace argument.
  * The paper has no counterpart: this is a convenience of this library.
  *

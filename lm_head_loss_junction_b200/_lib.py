@@ -49,6 +49,12 @@ PROTOTYPES = {
     "mls_junction_bwd_variant": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _int,
                                         _vp, _sz, _u32, _int, _vp, _vp]),
     "mls_junction_bwd_workspace": (_int, [_i64, _i64, ctypes.POINTER(_sz)]),
+    "mls_junction_fwd_multi": (_int, [_vp, _i64, _i64, _int, ctypes.POINTER(_i64), ctypes.POINTER(_vp),
+                                      ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int, _vp, _vp]),
+    "mls_junction_bwd_multi_workspace": (_int, [_i64, _i64, _int, ctypes.POINTER(_sz)]),
+    "mls_junction_bwd_multi": (_int, [_vp, _i64, _i64, _int, ctypes.POINTER(_i64), ctypes.POINTER(_vp),
+                                      ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                      ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int, _vp, _sz, _int, _vp, _vp]),
     "mls_junction_bwd_noalloc": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _int,
                                         _int, _vp, _vp]),
     "mls_multiexit_loss_workspace": (_int, [_int, _i64, ctypes.POINTER(_i64), _i64, _int,

@@ -115,6 +115,75 @@ def junction_bwd(x: torch.Tensor, o: torch.Tensor, E: torch.Tensor, dy: torch.Te
     return do, de, dE
 
 
+def junction_fwd_multi(x: torch.Tensor, o: Sequence[torch.Tensor], E: Sequence[torch.Tensor], *, out=None,
+                       scale_out=None, status=None, stream=None) -> List[torch.Tensor]:
+    """Every junction of a suite in one call: y[k] = junction(o[k], E[k]) (see mls_junction_fwd_multi)."""
+    J = len(o)
+    if len(E) != J or J < 1:
+        raise ValueError("o and E must be non-empty lists of the same length")
+    _need(x, "x", torch.int32, 1)
+    T = x.shape[0]
+    V = E[0].shape[0]
+    D = [o[0].shape[1]]
+    for k in range(J):
+        _need(o[k], f"o[{k}]", o[0].dtype, 2)
+        _need(E[k], f"E[{k}]", o[0].dtype, 2)
+        if o[k].shape[0] != T or E[k].shape[0] != V or o[k].shape[1] != D[k]:
+            raise ValueError(f"junction {k}: o must be [T, D_k] (D_k the previous junction's output width)")
+        D.append(D[k] + E[k].shape[1])
+    y = out if out is not None else [torch.empty((T, D[k + 1]), dtype=o[0].dtype, device=x.device)
+                                     for k in range(J)]
+    for k in range(J):
+        _need(y[k], f"out[{k}]", o[0].dtype, 2)
+    sc = None
+    if scale_out is not None:
+        sc = ptr_array([_ptr(t) for t in scale_out])
+    code = lib().mls_junction_fwd_multi(x.data_ptr(), T, V, J, i64_array(D), ptr_array([t.data_ptr() for t in o]),
+                                        ptr_array([t.data_ptr() for t in E]), ptr_array([t.data_ptr() for t in y]),
+                                        sc, _dtype_code(o[0]), _ptr(status), _stream_ptr(stream))
+    check("mls_junction_fwd_multi", code)
+    return y
+
+
+def junction_bwd_multi_workspace(T: int, V: int, J: int) -> int:
+    n = ctypes.c_size_t()
+    check("mls_junction_bwd_multi_workspace", lib().mls_junction_bwd_multi_workspace(T, V, J, ctypes.byref(n)))
+    return n.value
+
+
+def junction_bwd_multi(x: torch.Tensor, o: Sequence[torch.Tensor], E: Sequence[torch.Tensor],
+                       dy: Sequence[torch.Tensor], *, do_out=None, de_out=None, dE=None, accumulate_dE=False,
+                       workspace=None, status=None, stream=None):
+    """Backward of every junction of a suite in one call (see mls_junction_bwd_multi).
+    de_out / dE: lists (entries may be None) or None.  Returns (do list, de list, dE list)."""
+    J = len(o)
+    _need(x, "x", torch.int32, 1)
+    T = x.shape[0]
+    V = E[0].shape[0]
+    D = [o[0].shape[1]] + [o[0].shape[1]] * J
+    for k in range(J):
+        D[k + 1] = D[k] + E[k].shape[1]
+        if tuple(dy[k].shape) != (T, D[k + 1]):
+            raise ValueError(f"dy[{k}] must be [T, D_k+1]")
+    do = do_out if do_out is not None else [torch.empty_like(t) for t in o]
+    de = de_out if de_out is not None else [None] * J
+    tables = dE if dE is not None else [None] * J
+    ws_bytes = 0
+    if any(t is not None for t in tables):
+        ws_bytes = junction_bwd_multi_workspace(T, V, J)
+        if workspace is None:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    code = lib().mls_junction_bwd_multi(x.data_ptr(), T, V, J, i64_array(D), ptr_array([t.data_ptr() for t in o]),
+                                        ptr_array([t.data_ptr() for t in E]), ptr_array([t.data_ptr() for t in dy]),
+                                        ptr_array([t.data_ptr() for t in do]), ptr_array([_ptr(t) for t in de]),
+                                        ptr_array([_ptr(t) for t in tables]), int(bool(accumulate_dE)),
+                                        _ptr(workspace), ws_bytes, _dtype_code(o[0]), _ptr(status),
+                                        _stream_ptr(stream))
+    check("mls_junction_bwd_multi", code)
+    return do, de, tables
+
+
 # ---------------------------------------------------------------- multi-exit loss
 def multiexit_loss_workspace(T: int, D: Sequence[int], V: int, dtype: torch.dtype) -> Tuple[int, int]:
     f = ctypes.c_size_t()

@@ -246,6 +246,97 @@ mls_status mls_junction_bwd_variant(const int32_t* x, int64_t T, const void* o_m
   return from_cuda(mls::launch_junction_bwd(a, static_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Shared checks of the multi-junction calls; fills the per-junction shapes.
+mls_status check_multi(const int32_t* x, int64_t T, int64_t V, int J, const int64_t* D, const void* const* o,
+                       const void* const* e_next, mls_dtype dt, mls::JunctionArgs* js, int32_t* status) {
+  if (J < 1 || J > mls::kMaxExits - 1) return J < 1 ? MLS_ERR_INVALID_ARG : MLS_ERR_UNSUPPORTED;
+  if (D == nullptr || o == nullptr || e_next == nullptr) return MLS_ERR_INVALID_ARG;
+  for (int k = 0; k < J; ++k) {
+    if (D[k + 1] <= D[k]) return MLS_ERR_INVALID_ARG;
+    const mls_status st = check_junction_shape(x, T, o[k], D[k], e_next[k], V, D[k + 1] - D[k], dt);
+    if (st != MLS_OK) return st;
+    js[k] = mls::JunctionArgs{};
+    js[k].bf16 = dt == MLS_BF16;
+    js[k].x = x;
+    js[k].T = T;
+    js[k].D = D[k];
+    js[k].V = V;
+    js[k].delta = D[k + 1] - D[k];
+    js[k].o = o[k];
+    js[k].E = e_next[k];
+    js[k].status = status;
+  }
+  return MLS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mls_status mls_junction_fwd_multi(const int32_t* x, int64_t T, int64_t V, int J, const int64_t* D,
+                                  const void* const* o, const void* const* e_next, void* const* y,
+                                  float* const* scale_out, mls_dtype dt, int32_t* dev_status, void* stream) {
+  mls::JunctionArgs js[mls::kMaxExits - 1];
+  mls_status st = check_multi(x, T, V, J, D, o, e_next, dt, js, dev_status);
+  if (st != MLS_OK) return st;
+  if (y == nullptr) return MLS_ERR_INVALID_ARG;
+  for (int k = 0; k < J; ++k) {
+    if (y[k] == nullptr) return MLS_ERR_INVALID_ARG;
+    if (!aligned16(y[k])) return MLS_ERR_UNSUPPORTED;
+    js[k].y = y[k];
+    js[k].scale_out = scale_out != nullptr ? scale_out[k] : nullptr;
+  }
+  if ((st = device_ok()) != MLS_OK) return st;
+  return from_cuda(mls::launch_junction_fwd_multi(js, J, static_cast<cudaStream_t>(stream)));
+}
+
+mls_status mls_junction_bwd_multi_workspace(int64_t T, int64_t V, int J, size_t* bytes) {
+  if (bytes == nullptr || T <= 0 || V <= 0 || J < 1) return MLS_ERR_INVALID_ARG;
+  if (J > mls::kMaxExits - 1) return MLS_ERR_UNSUPPORTED;
+  *bytes = mls::junction_multi_scatter_bytes(T, V, J);
+  return MLS_OK;
+}
+
+mls_status mls_junction_bwd_multi(const int32_t* x, int64_t T, int64_t V, int J, const int64_t* D,
+                                  const void* const* o, const void* const* e_next, const void* const* dy,
+                                  void* const* do_m, void* const* de_rows, float* const* dE_table, int accumulate_dE,
+                                  void* workspace, size_t ws_bytes, mls_dtype dt, int32_t* dev_status, void* stream) {
+  mls::JunctionArgs js[mls::kMaxExits - 1];
+  mls_status st = check_multi(x, T, V, J, D, o, e_next, dt, js, dev_status);
+  if (st != MLS_OK) return st;
+  if (dy == nullptr || do_m == nullptr) return MLS_ERR_INVALID_ARG;
+  if (T > INT_MAX) return MLS_ERR_UNSUPPORTED;
+  bool any_table = false;
+  for (int k = 0; k < J; ++k) {
+    void* de = de_rows != nullptr ? de_rows[k] : nullptr;
+    float* dE = dE_table != nullptr ? dE_table[k] : nullptr;
+    if (dy[k] == nullptr || do_m[k] == nullptr) return MLS_ERR_INVALID_ARG;
+    if (!aligned16(dy[k]) || !aligned16(do_m[k]) || (de != nullptr && !aligned16(de)) ||
+        (dE != nullptr && !aligned16(dE)))
+      return MLS_ERR_UNSUPPORTED;
+    js[k].dy = dy[k];
+    js[k].do_out = do_m[k];
+    js[k].de_out = de;
+    js[k].dE = dE;
+    js[k].accumulate_dE = accumulate_dE;
+    any_table = any_table || dE != nullptr;
+  }
+  if (any_table) {
+    if (workspace == nullptr || ws_bytes < mls::junction_multi_scatter_bytes(T, V, J)) return MLS_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLS_ERR_UNSUPPORTED;
+  }
+  if ((st = device_ok()) != MLS_OK) return st;
+  return from_cuda(mls::launch_junction_bwd_multi(js, J, any_table, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+extern "C" {
+
 mls_status mls_multiexit_loss_workspace(int M, int64_t T, const int64_t* D, int64_t V, mls_dtype dt,
                                         size_t* fwd_bytes, size_t* bwd_bytes) {
   if (fwd_bytes == nullptr || bwd_bytes == nullptr) return MLS_ERR_INVALID_ARG;

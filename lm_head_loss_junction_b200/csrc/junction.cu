@@ -114,17 +114,15 @@ constexpr uint32_t kNoRescale = 1, kZeroFill = 2, kStopGrad = 4;
 // output: it does not depend on the scale) while accumulating both squared
 // norms; pass 2 writes the rescaled block output from registers.  Columns
 // beyond CAP*32 vectors are re-read in pass 2.
+// Warps warp0, warp0 + nwarps, ... of the launch (or of its share of a launch) take tokens t = warp0 + k nwarps.
 template <bool BF16, int CAP>
-__global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __restrict__ x, int64_t T,
-                                                           const uint4* __restrict__ o, int d_vec,
-                                                           const uint4* __restrict__ E, int64_t V,
-                                                           int dl_vec, uint4* __restrict__ y,
-                                                           float* __restrict__ scale_out,
-                                                           int32_t* __restrict__ status, uint32_t variant) {
+__device__ __forceinline__ void fwd_rows_body(int64_t warp0, int64_t nwarps, const int32_t* __restrict__ x,
+                                              int64_t T, const uint4* __restrict__ o, int d_vec,
+                                              const uint4* __restrict__ E, int64_t V, int dl_vec,
+                                              uint4* __restrict__ y, float* __restrict__ scale_out,
+                                              int32_t* __restrict__ status, uint32_t variant) {
   const int lane = threadIdx.x & 31;
   const bool zero_fill = (variant & kZeroFill) != 0;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int dp_vec = d_vec + dl_vec;
   const uint4 zero = make_uint4(0, 0, 0, 0);
   for (int64_t t = warp0; t < T; t += nwarps) {
@@ -180,22 +178,32 @@ __global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __r
   }
 }
 
+template <bool BF16, int CAP>
+__global__ void __launch_bounds__(256, 2) junction_fwd_kernel(const int32_t* __restrict__ x, int64_t T,
+                                                           const uint4* __restrict__ o, int d_vec,
+                                                           const uint4* __restrict__ E, int64_t V,
+                                                           int dl_vec, uint4* __restrict__ y,
+                                                           float* __restrict__ scale_out,
+                                                           int32_t* __restrict__ status, uint32_t variant) {
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  fwd_rows_body<BF16, CAP>(warp0, nwarps, x, T, o, d_vec, E, V, dl_vec, y, scale_out, status, variant);
+}
+
 // Short rows (at most CAP = 4 vectors of o and ECAP = 6 of e per lane): a
 // persistent grid of warps that each walk several tokens and load token
 // t + nwarps's id, block-output row and embedding row into registers while
 // token t is reduced and stored, so every warp keeps a row's worth of loads in
 // flight and the launch has no partial last wave.
 template <bool BF16, int CAP, int ECAP>
-__global__ void __launch_bounds__(256, 2) junction_fwd_pipe_kernel(const int32_t* __restrict__ x, int64_t T,
-                                                                  const uint4* __restrict__ o, int d_vec,
-                                                                  const uint4* __restrict__ E, int64_t V,
-                                                                  int dl_vec, uint4* __restrict__ y,
-                                                                  float* __restrict__ scale_out,
-                                                                  int32_t* __restrict__ status, uint32_t variant) {
+__device__ __forceinline__ void fwd_pipe_body(int64_t warp0, int64_t nwarps, const int32_t* __restrict__ x,
+                                              int64_t T, const uint4* __restrict__ o, int d_vec,
+                                              const uint4* __restrict__ E, int64_t V, int dl_vec,
+                                              uint4* __restrict__ y, float* __restrict__ scale_out,
+                                              int32_t* __restrict__ status, uint32_t variant) {
   const int lane = threadIdx.x & 31;
   const bool zero_fill = (variant & kZeroFill) != 0;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  int64_t t = warp0;
   if (t >= T) return;
   const int dp_vec = d_vec + dl_vec;
   const uint4 zero = make_uint4(0, 0, 0, 0);
@@ -256,6 +264,58 @@ __global__ void __launch_bounds__(256, 2) junction_fwd_pipe_kernel(const int32_t
 #pragma unroll
     for (int j = 0; j < ECAP; ++j) ec[j] = en[j];
   }
+}
+
+template <bool BF16, int CAP, int ECAP>
+__global__ void __launch_bounds__(256, 2) junction_fwd_pipe_kernel(const int32_t* __restrict__ x, int64_t T,
+                                                                  const uint4* __restrict__ o, int d_vec,
+                                                                  const uint4* __restrict__ E, int64_t V,
+                                                                  int dl_vec, uint4* __restrict__ y,
+                                                                  float* __restrict__ scale_out,
+                                                                  int32_t* __restrict__ status, uint32_t variant) {
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  fwd_pipe_body<BF16, CAP, ECAP>(warp0, nwarps, x, T, o, d_vec, E, V, dl_vec, y, scale_out, status, variant);
+}
+
+// Every junction of a suite in one persistent launch.  The launch's blocks are
+// divided among the junctions in proportion to their bytes; each junction's
+// share runs the prefetching body (short rows: at most PCAP vectors of o and
+// PECAP of the embedding per lane) or the whole-row body (RCAP vectors of o
+// per lane in registers), so no junction waits for another's tail.
+struct MultiFwdJob {
+  const uint4* o;
+  const uint4* E;
+  uint4* y;
+  float* scale_out;
+  int d_vec, dl_vec;
+  int pipe;          // 1: prefetching body, 0: whole-row body
+  int blk0;          // first block of this junction's share
+};
+struct MultiFwdArgs {
+  MultiFwdJob j[kMaxExits - 1];
+  int njobs;
+  int blk_end;       // one past the last job's blocks
+  const int32_t* x;
+  int64_t T, V;
+  int32_t* status;
+};
+
+template <int PCAP, int PECAP, int RCAP>
+__global__ void __launch_bounds__(256, 2) junction_fwd_multi_kernel(const __grid_constant__ MultiFwdArgs a) {
+  const int b = static_cast<int>(blockIdx.x);
+  int k = 0;
+  while (k + 1 < a.njobs && b >= a.j[k + 1].blk0) ++k;
+  const MultiFwdJob& jb = a.j[k];
+  const int b1 = (k + 1 < a.njobs) ? a.j[k + 1].blk0 : a.blk_end;
+  const int64_t warp0 = (static_cast<int64_t>(b - jb.blk0) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(b1 - jb.blk0) * blockDim.x) >> 5;
+  if (jb.pipe)
+    fwd_pipe_body<true, PCAP, PECAP>(warp0, nwarps, a.x, a.T, jb.o, jb.d_vec, jb.E, a.V, jb.dl_vec, jb.y,
+                                     jb.scale_out, a.status, 0u);
+  else
+    fwd_rows_body<true, RCAP>(warp0, nwarps, a.x, a.T, jb.o, jb.d_vec, jb.E, a.V, jb.dl_vec, jb.y, jb.scale_out,
+                              a.status, 0u);
 }
 
 // ---------------------------------------------------------------- backward
@@ -594,8 +654,10 @@ cudaError_t launch_fwd_t(const JunctionArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// The row kernels of one junction backward: do, de rows, and (coef != NULL)
+// the per-token coefficients of the table gradient.
 template <bool BF16>
-cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
+cudaError_t launch_bwd_rows_t(const JunctionArgs& a, float* coef, cudaStream_t st) {
   constexpr int N = Elt<BF16>::kPerVec;
   const int d_vec = static_cast<int>(a.D / N), dl_vec = static_cast<int>(a.delta / N);
   const int cap = pick_cap(d_vec);
@@ -605,8 +667,6 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
   auto* dy = static_cast<const uint4*>(a.dy);
   auto* dout = static_cast<uint4*>(a.do_out);
   auto* deo = static_cast<uint4*>(a.de_out);
-  float* coef = nullptr;
-  if (a.dE != nullptr) coef = static_cast<float*>(a.workspace);
   // Measured on the B200 (fraction of the copy bandwidth, T = 8192 .. 32768):
   //  - rows of <= 2 vectors per lane: the prefetching persistent kernel
   //    (512 -> 1024: 0.71 against 0.50-0.56);
@@ -646,22 +706,112 @@ cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
 #undef MLS_JB
   }
   note_launches(1);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess || a.dE == nullptr) return err;
+  return cudaGetLastError();
+}
 
+size_t coef_bytes(int64_t T) { return (static_cast<size_t>(T) * 4 + 255) & ~size_t(255); }
+
+template <bool BF16>
+cudaError_t launch_bwd_t(const JunctionArgs& a, cudaStream_t st) {
+  float* coef = a.dE != nullptr ? static_cast<float*>(a.workspace) : nullptr;
+  cudaError_t err = launch_bwd_rows_t<BF16>(a, coef, st);
+  if (err != cudaSuccess || a.dE == nullptr) return err;
   // Table gradient: tokens grouped by id, fixed-order row sums.
+  constexpr int N = Elt<BF16>::kPerVec;
   SegIndexDev ix;
-  void* ix_ws = static_cast<char*>(a.workspace) + ((static_cast<size_t>(a.T) * 4 + 255) & ~size_t(255));
-  err = build_segindex(a.x, a.T, a.V, ix_ws, &ix, st);
+  err = build_segindex(a.x, a.T, a.V, static_cast<char*>(a.workspace) + coef_bytes(a.T), &ix, st);
   if (err != cudaSuccess) return err;
   const float ge = (a.variant & kZeroFill) ? 0.f : 1.f;
-  return scatter_table_grad(ix, BF16, a.dy, d_vec, dl_vec, coef, ge, a.E, a.dE, a.accumulate_dE != 0, st);
+  return scatter_table_grad(ix, BF16, a.dy, static_cast<int>(a.D / N), static_cast<int>(a.delta / N), coef, ge, a.E,
+                            a.dE, a.accumulate_dE != 0, st);
 }
 
 }  // namespace
 
-size_t junction_scatter_bytes(int64_t T, int64_t V) {
-  return ((static_cast<size_t>(T) * 4 + 255) & ~size_t(255)) + segindex_bytes(T, V);
+size_t junction_scatter_bytes(int64_t T, int64_t V) { return coef_bytes(T) + segindex_bytes(T, V); }
+
+size_t junction_multi_scatter_bytes(int64_t T, int64_t V, int J) {
+  return coef_bytes(T) * static_cast<size_t>(J) + segindex_bytes(T, V);
+}
+
+// All junctions of a suite (they share the ids x and T).  bf16: one launch
+// whose blocks are split among the junctions; fp32: one launch per junction.
+cudaError_t launch_junction_fwd_multi(const JunctionArgs* js, int J, cudaStream_t st) {
+  if (!js[0].bf16) {
+    for (int k = 0; k < J; ++k) {
+      const cudaError_t err = launch_fwd_t<false>(js[k], st);
+      if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+  }
+  constexpr int N = 8;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int total_blocks = 2 * sms;              // two 8-warp blocks per SM, persistent
+  const int64_t T = js[0].T;
+  const int64_t need = (T + 7) / 8;              // blocks that give every token a warp
+  MultiFwdArgs m{};
+  m.njobs = J;
+  m.x = js[0].x;
+  m.T = T;
+  m.V = js[0].V;
+  m.status = js[0].status;
+  double bytes[kMaxExits - 1], sum = 0.0;
+  int rcap = 1;
+  for (int k = 0; k < J; ++k) {
+    const JunctionArgs& a = js[k];
+    MultiFwdJob& jb = m.j[k];
+    jb.o = static_cast<const uint4*>(a.o);
+    jb.E = static_cast<const uint4*>(a.E);
+    jb.y = static_cast<uint4*>(a.y);
+    jb.scale_out = a.scale_out;
+    jb.d_vec = static_cast<int>(a.D / N);
+    jb.dl_vec = static_cast<int>(a.delta / N);
+    jb.pipe = (pick_cap(jb.d_vec) <= 4 && pick_cap(jb.dl_vec) <= 6) ? 1 : 0;
+    if (!jb.pipe) rcap = pick_cap(jb.d_vec) > rcap ? pick_cap(jb.d_vec) : rcap;
+    bytes[k] = static_cast<double>(2 * jb.d_vec + 2 * jb.dl_vec);
+    sum += bytes[k];
+  }
+  int next = 0;
+  for (int k = 0; k < J; ++k) {
+    int64_t nb = static_cast<int64_t>(total_blocks * bytes[k] / sum + 0.5);
+    nb = nb < 1 ? 1 : (nb > need ? need : nb);
+    m.j[k].blk0 = next;
+    next += static_cast<int>(nb);
+  }
+  m.blk_end = next;
+  if (rcap <= 1) junction_fwd_multi_kernel<4, 6, 1><<<next, 256, 0, st>>>(m);
+  else if (rcap <= 9) junction_fwd_multi_kernel<4, 6, 9><<<next, 256, 0, st>>>(m);
+  else junction_fwd_multi_kernel<4, 6, 16><<<next, 256, 0, st>>>(m);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// The row kernels of every junction, then one id grouping shared by all table
+// gradients and one launch set of zero and segmented-sum passes over all tables.
+cudaError_t launch_junction_bwd_multi(const JunctionArgs* js, int J, bool any_table, void* ws, cudaStream_t st) {
+  const bool bf16 = js[0].bf16;
+  const int64_t T = js[0].T;
+  float* coef[kMaxExits - 1] = {};
+  for (int k = 0; k < J; ++k) {
+    coef[k] = js[k].dE != nullptr ? reinterpret_cast<float*>(static_cast<char*>(ws) + coef_bytes(T) * k) : nullptr;
+    const cudaError_t err = bf16 ? launch_bwd_rows_t<true>(js[k], coef[k], st) : launch_bwd_rows_t<false>(js[k], coef[k], st);
+    if (err != cudaSuccess) return err;
+  }
+  if (!any_table) return cudaSuccess;
+  SegIndexDev ix;
+  cudaError_t err = build_segindex(js[0].x, T, js[0].V, static_cast<char*>(ws) + coef_bytes(T) * J, &ix, st);
+  if (err != cudaSuccess) return err;
+  const int N = bf16 ? 8 : 4;
+  TableGradJob jobs[kMaxExits - 1];
+  int n = 0;
+  for (int k = 0; k < J; ++k) {
+    if (js[k].dE == nullptr) continue;
+    jobs[n++] = TableGradJob{js[k].dy, static_cast<int>(js[k].D / N), static_cast<int>(js[k].delta / N), coef[k],
+                             1.f, js[k].E, js[k].dE};
+  }
+  return scatter_table_grads(ix, bf16, n, jobs, js[0].accumulate_dE != 0, st);
 }
 
 cudaError_t launch_junction_fwd(const JunctionArgs& a, cudaStream_t st) {

@@ -38,6 +38,10 @@ mls_status check_junction_bwd_args(const int32_t* x, int64_t T, const void* o_m,
 size_t junction_scatter_bytes(int64_t T, int64_t V);
 cudaError_t launch_junction_fwd(const JunctionArgs& a, cudaStream_t st);
 cudaError_t launch_junction_bwd(const JunctionArgs& a, cudaStream_t st);
+// J junctions sharing x, T and V (standard junction; dtype of js[0] for all).
+size_t junction_multi_scatter_bytes(int64_t T, int64_t V, int J);
+cudaError_t launch_junction_fwd_multi(const JunctionArgs* js, int J, cudaStream_t st);
+cudaError_t launch_junction_bwd_multi(const JunctionArgs* js, int J, bool any_table, void* ws, cudaStream_t st);
 
 // ------------------------------------------------------------------ id-grouped row sums
 // Tokens grouped by id (stable in t): the tokens of id v are
@@ -61,6 +65,17 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
 cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
                                const float* coef, float ge, const void* E, float* dE, bool accumulate,
                                cudaStream_t st);
+// The same for several tables that share the ids (the junctions of one suite), one launch set for all.
+struct TableGradJob {
+  const void* dy;
+  int d_vec, dl_vec;
+  const float* coef;
+  float ge;
+  const void* E;
+  float* dE;
+};
+cudaError_t scatter_table_grads(const SegIndexDev& ix, bool bf16, int njobs, const TableGradJob* jobs, bool accumulate,
+                                cudaStream_t st);
 // For every job z < njobs (at most kMaxExits; one launch pair for all):
 //   dW[z][v] -= scale[z] * sum_{t: y_t = v} h[z]_t  (bf16 rows of d_vec[z] 16-byte vectors).
 cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,

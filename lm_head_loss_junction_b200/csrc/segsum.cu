@@ -224,6 +224,7 @@ struct SegJob {
   const uint4* E;
   float* out;
   float scale;
+  const float* coef;     // table mode: per-token coefficient of E[v]
 };
 struct SegJobs {
   SegJob j[kMaxExits];
@@ -232,10 +233,10 @@ struct SegJobs {
 // Light rows: warp w of block (x, y, z) takes light ids x*8 + w, x*8 + w + 8*gridDim.x, ...
 // and their slice y of 32 vectors (one 16-byte vector per lane) of job z.
 template <bool BF16, bool TABLE>
-__global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix, const SegJobs jobs,
-                                                           const float* __restrict__ coef, int accumulate) {
+__global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix, const SegJobs jobs, int accumulate) {
   constexpr int N = Vec8<BF16>::N;
   const SegJob& jb = jobs.j[blockIdx.z];
+  const float* __restrict__ coef = jb.coef;
   const uint4* __restrict__ src = jb.src;
   const int64_t src_ld = jb.src_ld;
   const int src_off = jb.src_off;
@@ -274,13 +275,15 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
 }
 
 // Overwrite mode of the table gradient: the rows of absent ids are zero.  One
-// warp per row; rows of present ids are left to the light and heavy kernels.
-__global__ void __launch_bounds__(256) zero_absent_rows_kernel(const SegIndexDev ix, float4* __restrict__ out,
-                                                               int f4_per_row) {
+// warp per row of table blockIdx.y (a job); rows of present ids are left to
+// the light and heavy kernels.
+__global__ void __launch_bounds__(256) zero_absent_rows_kernel(const SegIndexDev ix, const SegJobs jobs, int f4_mult) {
   const int lane = threadIdx.x & 31;
   const int64_t v = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (v >= ix.V || ix.ends[v] != 0) return;               // present ids have ends > 0
-  float4* o = out + v * f4_per_row;
+  const SegJob& jb = jobs.j[blockIdx.y];
+  const int f4_per_row = jb.n_vec * f4_mult;
+  float4* o = reinterpret_cast<float4*>(jb.out) + v * f4_per_row;
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int i = lane; i < f4_per_row; i += 32) o[i] = z;
 }
@@ -289,12 +292,12 @@ __global__ void __launch_bounds__(256) zero_absent_rows_kernel(const SegIndexDev
 // tokens round-robin and are combined in warp order.
 template <bool BF16, bool TABLE>
 __global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(const SegIndexDev ix, const SegJobs jobs,
-                                                                        const float* __restrict__ coef,
                                                                         int accumulate) {
   constexpr int N = Vec8<BF16>::N;
   __shared__ float part[kHeavyWarps][32 * N];
   __shared__ float cpart[kHeavyWarps];
   const SegJob& jb = jobs.j[blockIdx.z];
+  const float* __restrict__ coef = jb.coef;
   const uint4* __restrict__ src = jb.src;
   const int64_t src_ld = jb.src_ld;
   const int src_off = jb.src_off;
@@ -353,13 +356,12 @@ __global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(const Se
 }
 
 template <bool BF16, bool TABLE>
-cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs, const float* coef,
-                          int accumulate, cudaStream_t st) {
+cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs, int accumulate, cudaStream_t st) {
   constexpr int N = Vec8<BF16>::N;
   if (TABLE && !accumulate) {
     const int64_t blocks = (ix.V * 32 + 255) / 256;
-    zero_absent_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        ix, reinterpret_cast<float4*>(jobs.j[0].out), jobs.j[0].n_vec * N / 4);
+    zero_absent_rows_kernel<<<dim3(static_cast<unsigned>(blocks), static_cast<unsigned>(njobs)), 256, 0, st>>>(
+        ix, jobs, N / 4);
     note_launches(1);
   }
   int slices = 0, total_slices = 0;
@@ -376,9 +378,9 @@ cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs,
   const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(want, (ix.max_light + 7) / 8));
   segsum_light_kernel<BF16, TABLE>
       <<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices), static_cast<unsigned>(njobs)), 256, 0, st>>>(
-          ix, jobs, coef, accumulate);
+          ix, jobs, accumulate);
   dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>(slices), static_cast<unsigned>(njobs));
-  segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, jobs, coef, accumulate);
+  segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, jobs, accumulate);
   note_launches(2);
   return cudaGetLastError();
 }
@@ -450,21 +452,29 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
   return cudaGetLastError();
 }
 
+cudaError_t scatter_table_grads(const SegIndexDev& ix, bool bf16, int njobs, const TableGradJob* tj, bool accumulate,
+                                cudaStream_t st) {
+  SegJobs jobs{};
+  for (int z = 0; z < njobs; ++z)
+    jobs.j[z] = SegJob{static_cast<const uint4*>(tj[z].dy), tj[z].d_vec + tj[z].dl_vec, tj[z].d_vec, tj[z].dl_vec,
+                       static_cast<const uint4*>(tj[z].E), tj[z].dE, tj[z].ge, tj[z].coef};
+  return bf16 ? launch_segsum<true, true>(ix, jobs, njobs, accumulate, st)
+              : launch_segsum<false, true>(ix, jobs, njobs, accumulate, st);
+}
+
 cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
                                const float* coef, float ge, const void* E, float* dE, bool accumulate,
                                cudaStream_t st) {
-  SegJobs jobs{};
-  jobs.j[0] = SegJob{static_cast<const uint4*>(dy), d_vec + dl_vec, d_vec, dl_vec, static_cast<const uint4*>(E), dE, ge};
-  return bf16 ? launch_segsum<true, true>(ix, jobs, 1, coef, accumulate, st)
-              : launch_segsum<false, true>(ix, jobs, 1, coef, accumulate, st);
+  const TableGradJob j{dy, d_vec, dl_vec, coef, ge, E, dE};
+  return scatter_table_grads(ix, bf16, 1, &j, accumulate, st);
 }
 
 cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,
                                 float* const* dW, const float* scale, cudaStream_t st) {
   SegJobs jobs{};
   for (int z = 0; z < njobs; ++z)
-    jobs.j[z] = SegJob{static_cast<const uint4*>(h[z]), d_vec[z], 0, d_vec[z], nullptr, dW[z], scale[z]};
-  return launch_segsum<true, false>(ix, jobs, njobs, nullptr, 1, st);
+    jobs.j[z] = SegJob{static_cast<const uint4*>(h[z]), d_vec[z], 0, d_vec[z], nullptr, dW[z], scale[z], nullptr};
+  return launch_segsum<true, false>(ix, jobs, njobs, 1, st);
 }
 
 }  // namespace mls

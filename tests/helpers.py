@@ -14,6 +14,9 @@ Tolerances (fixed by the method's problem statement for this path):
     u = 2^-8 for bf16 (unit roundoff of an 8-bit significand), 2^-23 for f32,
     plus the fp32 error of the scale (a few ulp).
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -31,6 +34,28 @@ def unit_roundoff(dtype) -> float:
     return 2.0 ** -8 if dtype == torch.bfloat16 else 2.0 ** -23
 
 
+def _log_grad_error(name, got, exp, rtol, rms, scale, nrm, err):
+    """With MLS_GRAD_ERR_LOG set, appends one JSON line per compared tensor: the
+    worst element's error as a fraction of the per-element bound with the
+    tensor-rms term alone and with the row term, and the Frobenius error as a
+    fraction of its bound (a value above 1 would fail that bound)."""
+    path = os.environ.get("MLS_GRAD_ERR_LOG")
+    if not path or not exp.size:
+        return
+    d = np.abs(got - exp)
+    rec = {
+        "test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "tensor": name,
+        "shape": list(exp.shape), "rms": float(rms),
+        "worst_abs": float(d.max()),
+        "worst_frac_tensor_bound": float(np.max(d / (rtol * np.abs(exp) + rtol * rms + 1e-300))),
+        "worst_frac_row_bound": float(np.max(d / (rtol * np.abs(exp) + rtol * scale + 1e-300))),
+        "n_outside_tensor_bound": int(np.sum(d > rtol * np.abs(exp) + rtol * rms)),
+        "frobenius_frac": float(err / (rtol * nrm + 1e-300)),
+    }
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def assert_grad_close(got, exp, name="grad", rtol=GRAD_RTOL):
     got = f64(got)
     exp = f64(exp)
@@ -38,11 +63,12 @@ def assert_grad_close(got, exp, name="grad", rtol=GRAD_RTOL):
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
     nrm = np.linalg.norm(exp)
     err = np.linalg.norm(got - exp)
-    assert err <= rtol * nrm + 1e-30, f"{name}: Frobenius rel err {err / max(nrm, 1e-300):.3e} > {rtol}"
     rms = np.sqrt(np.mean(exp * exp)) if exp.size else 0.0
     scale = rms
     if exp.ndim == 2 and exp.size:
         scale = np.maximum(np.sqrt(np.mean(exp * exp, axis=1, keepdims=True)), rms)
+    _log_grad_error(name, got, exp, rtol, rms, scale, nrm, err)
+    assert err <= rtol * nrm + 1e-30, f"{name}: Frobenius rel err {err / max(nrm, 1e-300):.3e} > {rtol}"
     bad = np.abs(got - exp) > rtol * np.abs(exp) + rtol * scale
     assert not bad.any(), (f"{name}: {int(bad.sum())} elements outside tolerance; worst "
                            f"{np.max(np.abs(got - exp)):.3e} (rms {rms:.3e})")

@@ -64,8 +64,12 @@ def test_algorithmic_counts_of_the_main_suite():
     step = object.__new__(bench.Step)          # the counts need only the config
     step.cfg = c
     fwd, bwd = step.junction_bytes()
-    # per token: forward (D + delta + D_next) * 2 + 8 bytes, backward (D_next + 2D + 2 delta) * 2 + 8
+    # per token: forward (D + delta + D_next) * 2 + 8 bytes, backward rows (D_next + 2D + 2 delta) * 2 + 8
     assert fwd == c.T * ((1024 + 1280 + 2304) * 2 + 8 + (2304 + 2048 + 4352) * 2 + 8)
-    assert bwd == c.T * ((2304 + 2 * 1024 + 2 * 1280) * 2 + 8 + (4352 + 2 * 2304 + 2 * 2048) * 2 + 8)
+    rows = c.T * ((2304 + 2 * 1024 + 2 * 1280) * 2 + 8 + (4352 + 2 * 2304 + 2 * 2048) * 2 + 8)
+    # plus the fp32 tables written once (V x delta x 4) and g_e, coef read again (T x (delta * 2 + 4))
+    tables = c.V * (1280 + 2048) * 4 + c.T * ((1280 + 2048) * 2 + 8)
+    assert bwd == rows + tables
+    assert 1.0e9 < bwd < 1.1e9                 # about 1.04 GB per step at T = 8192
     assert step.loss_flops_algorithmic() == 6.0 * c.T * c.V * (1024 + 2304 + 4352)
     assert step.loss_flops_executed() == 8.0 * c.T * c.V * (1024 + 2304 + 4352)

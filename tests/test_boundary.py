@@ -130,3 +130,29 @@ def test_workspace_queries():
     assert junction_bwd_workspace(32768, 49152) >= 5 * 32768 * 4
     with pytest.raises(_lib.MLSError):
         multiexit_loss_workspace(10, [64, 64], 128, torch.bfloat16)
+
+
+def test_multi_junction_argument_errors():
+    lib = _lib.lib()
+    D = _lib.i64_array([64, 128, 192])
+    P = lambda *v: _lib.ptr_array(list(v))   # noqa: E731
+    f = lib.mls_junction_fwd_multi
+    ok = (FAKE, 8, 10, 2, D, P(FAKE, FAKE), P(FAKE, FAKE), P(FAKE, FAKE), None, _lib.MLS_BF16, None, None)
+    assert f(*ok) == 7 or f(*ok) == 0                                  # valid: no device here
+    assert f(FAKE, 8, 10, 0, D, P(FAKE), P(FAKE), P(FAKE), None, _lib.MLS_BF16, None, None) == 1
+    assert f(FAKE, 8, 10, 4, D, P(FAKE), P(FAKE), P(FAKE), None, _lib.MLS_BF16, None, None) == 2
+    assert f(FAKE, 8, 10, 2, _lib.i64_array([64, 64, 192]), P(FAKE, FAKE), P(FAKE, FAKE), P(FAKE, FAKE), None,
+             _lib.MLS_BF16, None, None) == 1                            # widths must increase
+    assert f(FAKE, 8, 10, 2, D, P(FAKE, FAKE), P(FAKE, FAKE), P(FAKE, None), None, _lib.MLS_BF16, None,
+             None) == 1                                                 # missing output
+    assert f(FAKE, 8, 10, 2, D, P(FAKE, FAKE + 4), P(FAKE, FAKE), P(FAKE, FAKE), None, _lib.MLS_BF16, None,
+             None) == 2                                                 # misaligned input
+    b = lib.mls_junction_bwd_multi
+    # a table gradient without workspace
+    assert b(FAKE, 8, 10, 2, D, P(FAKE, FAKE), P(FAKE, FAKE), P(FAKE, FAKE), P(FAKE, FAKE), None,
+             P(None, FAKE), 0, None, 0, _lib.MLS_BF16, None, None) == 3
+    n = ctypes.c_size_t()
+    assert lib.mls_junction_bwd_multi_workspace(8192, 49152, 2, ctypes.byref(n)) == 0
+    single = ctypes.c_size_t()
+    lib.mls_junction_bwd_workspace(8192, 49152, ctypes.byref(single))
+    assert single.value < n.value < 2 * single.value                   # one id grouping for both tables
