@@ -268,7 +268,7 @@ mls_status mls_junction_bwd_noalloc(const int32_t* x, int64_t T,
  * MLS_BF16 backward: the dense logit gradient G' is formed and consumed one
  * block of tokens x one chunk of the vocabulary at a time, so its workspace
  * does not grow with T x V.  *bwd_bytes is the workspace of the split chosen
- * for a 1 GiB budget (or of the whole problem in one piece, when that is
+ * for a 1.5 GiB budget (or of the whole problem in one piece, when that is
  * smaller); mls_multiexit_loss_bwd accepts any workspace of at least
  * mls_multiexit_loss_bwd_plan's minimum and splits the work to fit the size
  * it is given (a larger workspace means fewer, larger pieces).
@@ -314,12 +314,16 @@ mls_status mls_multiexit_loss_fwd(int M, int64_t T, int64_t V, const int64_t* D,
  *   stats is the forward call's output for the same inputs.
  * MLS_BF16: the logits are computed again tile by tile (never stored) and
  * the dense part of G (q_m - alpha_d p_M, or p_M for the largest exit) is
- * written in bf16 for one token block x vocabulary chunk at a time into the
- * workspace (see mls_multiexit_loss_bwd_plan), then multiplied out on the
- * tensor cores; the one-hot part is applied exactly in fp32.  dh rows of a
- * block are summed over the chunks in fp32 (fixed order), dW rows of a chunk
- * over the blocks in fp32 (fixed order): results are deterministic for a
- * given workspace size.
+ * written in fp16 (11-bit significand; entries beyond +-65504, which finite
+ * logits do not produce, saturate) for one token block x vocabulary chunk at
+ * a time into the workspace (see mls_multiexit_loss_bwd_plan), then
+ * multiplied on the tensor cores with fp16 copies of the block's h rows and
+ * the chunk's W rows (exact for values in fp16's normal range; a tensor whose
+ * largest magnitude is 2^15 or more, or below 2^-10, is copied scaled by a
+ * power of two that the result undoes); the one-hot part is applied exactly
+ * in fp32 from the bf16 inputs.  dh rows of a block are summed over the
+ * chunks in fp32 (fixed order), dW rows of a chunk over the blocks in fp32
+ * (fixed order): results are deterministic for a given workspace size.
  */
 mls_status mls_multiexit_loss_bwd(int M, int64_t T, int64_t V, const int64_t* D,
                                   const int32_t* y_targets,

@@ -106,7 +106,7 @@ size_t loss_simt_bwd_bytes(const LossProblem& p);
 
 // Tensor-core (bf16) path.  The backward pass runs in (token block x vocabulary
 // chunk) pieces sized to the workspace it is given: loss_tc_bwd_bytes is the
-// size of the plan for a 1 GiB budget (or of the whole problem, when smaller),
+// size of the plan for a 1.5 GiB budget (or of the whole problem, when smaller),
 // loss_tc_bwd_min_bytes the smallest workspace any plan fits in.
 size_t loss_tc_bwd_min_bytes(const LossProblem& p);
 void loss_tc_bwd_plan(const LossProblem& p, size_t ws_bytes, int64_t* Tb, int64_t* Vc);

@@ -14,11 +14,15 @@
 // Backward.  The same mainloop recomputes each tile's logits; the epilogue forms
 // the dense part of the logit gradient
 //   G'_m = q_m - alpha_d p_T   (students),   G'_T = p_T   (teacher, stop-gradient)
-// in bf16 into a workspace, and two tensor-core GEMMs per exit produce
+// in fp16 into a workspace, one block of tokens x one chunk of the vocabulary
+// at a time, and two tensor-core GEMMs per exit (fp16 operands: G' and fp16
+// copies of the chunk's W rows and the block's h rows) produce
 //   dh_m = a (G'_m W^m - c_m W^m[y_t])   and   dW^m (+)= a G'_m^T h_m - a c_m sum_{t: y_t = v} h_t,
 // a = grad_scale/T, c_m = 1 - alpha_d (students) or 1 (teacher).  The one-hot
 // term is applied exactly in fp32 (a row gather in the dh epilogue and an
-// id-grouped row sum for dW) instead of being rounded into the bf16 G'.
+// id-grouped row sum for dW) instead of being rounded into G'.  fp16 holds
+// G' with an 11-bit significand where bf16 holds 8: the rounding of the large
+// entries of peaked rows, which dominates the error of dW, is 8x smaller.
 //
 // Definitions: "Matryoshka Language Model Suites" (agihunt.info summary,
 // distillation paragraph), "Is nesting the cheapest way to build a model
@@ -30,6 +34,21 @@
 
 #include "kernels.h"
 #include "umma.cuh"
+
+// Raster groups.  Grouped GEMMs: tile rows (of 256 on CTA pairs) per group;
+// consecutive tiles go down a group's rows before moving to the next column,
+// so a wave of CTAs shares the group's A panels and a few B panels in L2.
+// Loss tile kernel: 128-token tiles per group; a group's h panels stay in L2
+// while the heads stream past them.
+#ifndef MLS_DH_GROUP_M
+#define MLS_DH_GROUP_M 8
+#endif
+#ifndef MLS_DW_GROUP_M
+#define MLS_DW_GROUP_M 8
+#endif
+#ifndef MLS_LOSS_GROUP_TT
+#define MLS_LOSS_GROUP_TT 16
+#endif
 
 namespace mls {
 
@@ -74,7 +93,7 @@ struct LossArgs {
   float student_wsum;          // sum of the smaller exits' weights
   float* partial;              // forward: [2 n_vt][2M-1][T]
   float* stats;                // forward: target rows written; backward: lse read
-  __nv_bfloat16* G;            // backward: [M][T][V] of the launch's tokens and columns
+  __half* G;                   // backward: fp16 G' [M][T][V] of the launch's tokens and columns
   int32_t* status;
   uint64_t wait_ns;            // limit of every barrier wait (the library default, or a test's)
   int withhold_loads;          // test of the bounded waits: the producer issues no loads
@@ -148,6 +167,15 @@ __device__ __forceinline__ uint32_t pack_p2(float lo, float hi) {
 
 __device__ __forceinline__ float2 unpack_p2(uint32_t u) { return __half22float2(*reinterpret_cast<__half2*>(&u)); }
 
+// G' is stored in fp16 (11-bit significand, 8x finer than bf16's): round to
+// nearest, and values beyond the largest finite fp16 (65504, far outside any
+// logit gradient of finite logits) saturate instead of becoming infinite.
+__device__ __forceinline__ uint32_t pack_g2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // acc + w * x on fp16 pairs (the teacher-gradient accumulator).
 __device__ __forceinline__ uint32_t hfma_p2(uint32_t w, uint32_t x, uint32_t acc) {
   __half2 r = __hfma2(*reinterpret_cast<__half2*>(&w), *reinterpret_cast<__half2*>(&x),
@@ -172,11 +200,11 @@ __device__ __forceinline__ void job_slot(bool hold_teacher, int M, uint32_t tile
   }
 }
 
-// One 32-column chunk of G' (this lane's row: 16 packed bf16 pairs) through the
+// One 32-column chunk of G' (this lane's row: 16 packed fp16 pairs) through the
 // warp's staging rows, so that each store instruction writes 8 rows x 64
 // contiguous bytes (full sectors).  Rows at or past T are not stored.
 __device__ __forceinline__ void store_g_chunk(uint8_t* stage, int lane, const uint32_t (&packed)[16],
-                                              __nv_bfloat16* G, int row0, int T, int V, int col) {
+                                              __half* G, int row0, int T, int V, int col) {
   uint4* mine = reinterpret_cast<uint4*>(stage + lane * kStageRowBytes);
 #pragma unroll
   for (int u = 0; u < 4; ++u)
@@ -648,7 +676,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                   if (TGRAD)                       // sum_m w_m (l_m - S_m)
                     pt[c][k / 2] = hfma_p2(wm2, pack_p2(r[kk] - klt, r[kk + 1] - klt), pt[c][k / 2]);
                 }
-                packed[k / 2] = bad ? 0u : pack_bf16x2(g0, g1);
+                packed[k / 2] = bad ? 0u : pack_g2(g0, g1);
               }
               }
               store_g_chunk(stage, lane, packed, a.G + static_cast<int64_t>(m) * a.T * a.V, row0, a.T, a.V,
@@ -687,7 +715,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                     g0 = p0 * fmaf(-al, acc.x, cp);
                     g1 = p1 * fmaf(-al, acc.y, cp);
                   }
-                  packed[k / 2] = bad ? 0u : pack_bf16x2(g0, g1);
+                  packed[k / 2] = bad ? 0u : pack_g2(g0, g1);
                 }
               }
               store_g_chunk(stage, lane, packed, a.G + static_cast<int64_t>(M - 1) * a.T * a.V, row0, a.T, a.V,
@@ -956,6 +984,8 @@ struct GemmArgs {
   // Optional fp32 partial sums (bf16 output only): out_p = alpha acc + addend_p (same layout as out_p)
   // before the one-hot term and the rounding; the earlier vocabulary chunks of dh.
   const float* addend[kMaxExits];
+  int f16;                         // 1: A and B hold fp16 (else bf16)
+  const float* bscale[kMaxExits];  // optional device factor on alpha: 1/s of a rescaled fp16 copy of B
 };
 
 template <int BN>
@@ -1066,7 +1096,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, BN, A_MN, B_MN);
+      const uint32_t idesc = g.f16 ? idesc_f16(kBM, BN, A_MN, B_MN) : idesc_bf16(kBM, BN, A_MN, B_MN);
       // K step of one tcgen05.mma: +32 B inside the swizzled row (K-major) or
       // +16 rows of 128 B (MN-major).
       constexpr uint32_t a_step = A_MN ? (kUK * 128) >> 4 : (kUK * 2) >> 4;
@@ -1117,8 +1147,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const int32_t k = __ldg(g.onehot_idx + row);
         if (k >= 0 && k < g.onehot_limit) onehot_row = k;
       }
-      const float alpha = g.alpha[p];
-      const float oh_scale = alpha * g.onehot_coef[p];
+      const float alpha = g.alpha[p] * (g.bscale[p] != nullptr ? *g.bscale[p] : 1.f);
+      const float oh_scale = g.alpha[p] * g.onehot_coef[p];
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float r[32];
@@ -1289,7 +1319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_bf16(2 * kBM, BN, A_MN, B_MN);
+      const uint32_t idesc = g.f16 ? idesc_f16(2 * kBM, BN, A_MN, B_MN) : idesc_bf16(2 * kBM, BN, A_MN, B_MN);
       constexpr uint32_t a_step = A_MN ? (kUK * 128) >> 4 : (kUK * 2) >> 4;
       constexpr uint32_t b_step = B_MN ? (kUK * 128) >> 4 : (kUK * 2) >> 4;
       constexpr uint32_t a_lbo = A_MN ? 64 * kBK * 2 : 16;
@@ -1344,8 +1374,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int32_t k = __ldg(g.onehot_idx + row);
         if (k >= 0 && k < g.onehot_limit) onehot_row = k;
       }
-      const float alpha = g.alpha[p];
-      const float oh_scale = alpha * g.onehot_coef[p];
+      const float alpha = g.alpha[p] * (g.bscale[p] != nullptr ? *g.bscale[p] : 1.f);
+      const float oh_scale = g.alpha[p] * g.onehot_coef[p];
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float r[32];
@@ -1408,6 +1438,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ fp16 operand copies
+// tcgen05.mma kind::f16 takes A and B in the same format, so the backward
+// GEMMs, whose A is the fp16 G', read fp16 copies of the chunk's rows of W and
+// the block's rows of h.  The copy is unscaled when the tensor's largest
+// magnitude m lies in [2^-10, 2^15): every bf16 value there converts exactly
+// (bf16's 8 significant bits fit in fp16's 11), and the few values below
+// fp16's normal range keep an absolute error under 3e-8.  Otherwise a second
+// pass copies x * s with s a power of two that puts m in [2^13, 2^14), and the
+// GEMM epilogue multiplies by 1/s; powers of two change no significand.
+struct HalfJob {
+  const uint4* src;          // bf16, 8 per vector
+  uint4* dst;                // fp16, 8 per vector
+  int64_t n_vec;
+  unsigned int* maxbits;     // largest |x| as float bits (non-negative floats order as unsigned ints)
+  float* inv_scale;          // 1/s, for the GEMM epilogue
+};
+struct HalfJobs {
+  HalfJob j[kMaxExits];
+};
+
+__device__ __forceinline__ uint4 bf16x8_to_half8(const uint4& u, float s, float& mx) {
+  float f[8];
+  bf16x8_to_f32(u, f);
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    mx = fmaxf(mx, fmaxf(fabsf(f[2 * k]), fabsf(f[2 * k + 1])));
+    __half2 h = __floats2half2_rn(f[2 * k] * s, f[2 * k + 1] * s);   // beyond the range: infinite, as in the input
+    w[k] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// First pass: the unscaled copy and the largest magnitude (job = blockIdx.y).
+__global__ void __launch_bounds__(256) half_copy_kernel(const __grid_constant__ HalfJobs jobs) {
+  const HalfJob& jb = jobs.j[blockIdx.y];
+  float mx = 0.f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < jb.n_vec; i += 4 * stride) {
+    uint4 u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = __ldg(jb.src + i + k * stride);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) jb.dst[i + k * stride] = bf16x8_to_half8(u[k], 1.f, mx);
+  }
+  for (; i < jb.n_vec; i += stride) jb.dst[i] = bf16x8_to_half8(__ldg(jb.src + i), 1.f, mx);
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0 && mx > 0.f) atomicMax(jb.maxbits, __float_as_uint(mx));
+}
+
+// Second pass: the scale from the largest magnitude, and the scaled copy when
+// the unscaled one does not serve.
+__global__ void __launch_bounds__(256) half_rescale_kernel(const __grid_constant__ HalfJobs jobs) {
+  const HalfJob& jb = jobs.j[blockIdx.y];
+  const float mx = __uint_as_float(*jb.maxbits);
+  float s = 1.f;
+  if (mx <= 3.4e38f && (mx >= 32768.f || (mx > 0.f && mx < 1.f / 1024.f))) {
+    int e = 13 - ilogbf(mx);
+    e = e < -126 ? -126 : (e > 126 ? 126 : e);
+    s = ldexpf(1.f, e);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *jb.inv_scale = 1.f / s;
+  if (s == 1.f) return;
+  float unused = 0.f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < jb.n_vec; i += stride)
+    jb.dst[i] = bf16x8_to_half8(__ldg(jb.src + i), s, unused);
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1426,16 +1526,18 @@ EncodeTiledFn get_encoder() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer][inner] (inner contiguous), 128-byte swizzled boxes.
+// 2-D tensor of 16-bit elements [outer][inner] (inner contiguous; bf16 unless
+// fp16 is set), 128-byte swizzled boxes.
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer) {
+              uint32_t box_outer, bool fp16 = false) {
   EncodeTiledFn enc = get_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {inner * 2};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return enc(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1474,22 +1576,28 @@ int resident_pairs(Kernel fn, int threads, size_t smem) {
 size_t align_up(size_t b) { return (b + 255) & ~size_t(255); }
 
 // ------------------------------------------------------------------ backward chunk plan
-// The backward pass writes the dense logit gradient G' of every exit for one
-// block of tokens x one chunk of the vocabulary at a time into the workspace,
-// then consumes it with the two GEMMs.  dW rows of a chunk are complete after
-// their chunk (K runs over the block's tokens; token blocks after the first
-// add into dW), dh rows of a block after the block's last chunk (K runs over
-// the chunk's columns; the chunks before the last leave fp32 partial sums in
-// the workspace).  Workspace: [G' chunk: M x Tb x Vc bf16][dh partials:
-// Tb x sum(D) f32, only with more than one chunk][targets grouped by id].
+// The backward pass writes the dense logit gradient G' (fp16) of every exit
+// for one block of tokens x one chunk of the vocabulary at a time into the
+// workspace, then consumes it with the two GEMMs.  dW rows of a chunk are
+// complete after their chunk (K runs over the block's tokens; token blocks
+// after the first add into dW), dh rows of a block after the block's last
+// chunk (K runs over the chunk's columns; the chunks before the last leave
+// fp32 partial sums in the workspace).  Workspace: [G' chunk: M x Tb x Vc f16]
+// [dh partials: Tb x sum(D) f32, only with more than one chunk][targets
+// grouped by id][fp16 copy of the block's h rows: Tb x sum(D)][fp16 copy of
+// the chunk's W rows: Vc x sum(D)][copy scales].
 struct BwdPlan {
   int64_t Tb, Vc;          // tokens per block (last block shorter), columns per chunk (last chunk shorter)
   int64_t nT, nV;
-  size_t g_bytes, acc_bytes, seg_bytes;
-  size_t total() const { return g_bytes + acc_bytes + seg_bytes; }
+  size_t g_bytes, acc_bytes, seg_bytes, h16_bytes, w16_bytes, aux_bytes;
+  size_t total() const { return g_bytes + acc_bytes + seg_bytes + h16_bytes + w16_bytes + aux_bytes; }
 };
 
-constexpr size_t kDefaultBwdBudget = size_t(1) << 30;   // 1 GiB
+// The workspace the query returns is the plan for this budget.  At the 3-exit
+// main suite (T = 8192) it holds three vocabulary chunks of 16384 in one token
+// block; 1 GiB would need five, whose extra dh partials (0.5 GB of fp32
+// read-modify-write per extra chunk) measured 0.5 ms per step slower.
+constexpr size_t kDefaultBwdBudget = size_t(3) << 29;   // 1.5 GiB
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
@@ -1506,20 +1614,26 @@ BwdPlan plan_shape(const LossProblem& p, int64_t Tb, int64_t Vc) {
   b.Vc = Vc;
   b.nT = ceil_div(p.T, Tb);
   b.nV = ceil_div(p.V, Vc);
-  b.g_bytes = align_up(static_cast<size_t>(p.M) * Tb * Vc * sizeof(__nv_bfloat16));
-  b.acc_bytes = b.nV > 1 ? align_up(static_cast<size_t>(Tb) * sum_d(p) * sizeof(float)) : 0;
+  const size_t sd = static_cast<size_t>(sum_d(p));
+  b.g_bytes = align_up(static_cast<size_t>(p.M) * Tb * Vc * 2);
+  b.acc_bytes = b.nV > 1 ? align_up(static_cast<size_t>(Tb) * sd * sizeof(float)) : 0;
   b.seg_bytes = align_up(segindex_bytes(p.T, p.V));
+  b.h16_bytes = align_up(static_cast<size_t>(Tb) * sd * 2);
+  b.w16_bytes = align_up(static_cast<size_t>(Vc) * sd * 2);
+  b.aux_bytes = 256;
   return b;
 }
 
 // Bytes the plan moves beyond one pass over G': the dW read-modify-write of
 // every token block after the first, the dh partials of every chunk but the
-// last, and a fixed charge per (block, chunk) for its three launches' ramps.
+// last, the fp16 copies of W (once per block) and h, and a fixed charge per
+// (block, chunk) for its launches' ramps.
 double plan_cost(const LossProblem& p, const BwdPlan& b) {
   const double sd = static_cast<double>(sum_d(p));
   const double dw_rmw = static_cast<double>(b.nT - 1) * 8.0 * static_cast<double>(p.V) * sd;
   const double dh_part = static_cast<double>(b.nT) * static_cast<double>(b.nV - 1) * 8.0 * static_cast<double>(b.Tb) * sd;
-  return dw_rmw + dh_part + 3.0e8 * static_cast<double>(b.nT * b.nV);
+  const double copies = 4.0 * sd * (static_cast<double>(b.nT) * static_cast<double>(p.V) + static_cast<double>(p.T));
+  return dw_rmw + dh_part + copies + 3.0e8 * static_cast<double>(b.nT * b.nV);
 }
 
 // The cheapest plan whose workspace fits in `budget` bytes (Tb = 0 when none fits).
@@ -1540,8 +1654,9 @@ BwdPlan choose_plan(const LossProblem& p, size_t budget) {
         continue;
       }
       // widest chunk (a multiple of the tile width) that fits, then equal chunks of at most that width
-      const size_t fixed = probe.acc_bytes + probe.seg_bytes;
-      int64_t vmax = static_cast<int64_t>((budget - fixed) / (static_cast<size_t>(p.M) * Tb * 2)) / kLossBN * kLossBN;
+      const size_t fixed = probe.acc_bytes + probe.seg_bytes + probe.h16_bytes + probe.aux_bytes;
+      const size_t per_col = static_cast<size_t>(p.M) * Tb * 2 + static_cast<size_t>(sum_d(p)) * 2;
+      int64_t vmax = static_cast<int64_t>((budget - fixed) / per_col) / kLossBN * kLossBN;
       while (vmax > kLossBN && plan_shape(p, Tb, vmax).total() > budget) vmax -= kLossBN;
       if (vmax < kLossBN) vmax = kLossBN;
       const int64_t nV = ceil_div(p.V, vmax);
@@ -1601,7 +1716,7 @@ LossArgs base_args(const LossProblem& p) {
   a.n_tt = static_cast<int>((p.T + kBM - 1) / kBM);
   a.n_vt = loss_n_vt(p);
   a.num_tiles = a.n_tt * a.n_vt;
-  a.group_tt = 16;
+  a.group_tt = MLS_LOSS_GROUP_TT;
   a.y = p.y;
   a.alpha = p.alpha_d;
   a.distill = p.distill;
@@ -1615,13 +1730,13 @@ LossArgs base_args(const LossProblem& p) {
 }
 
 template <bool A_MN, bool B_MN, int BN, bool OUT_BF16>
-cudaError_t run_gemm(const GemmMaps& maps, GemmArgs g, cudaStream_t st) {
+cudaError_t run_gemm(const GemmMaps& maps, GemmArgs g, int group_rows, cudaStream_t st) {
   // 256-wide N tiles run on CTA pairs (256 x 256 output tiles), narrower ones on single CTAs.
   constexpr bool kPair = (BN == 256);
   const int rows_per_tile = kPair ? 2 * kBM : kBM;
   g.n_mt = (g.Mdim + rows_per_tile - 1) / rows_per_tile;
   g.kblocks = (g.Kdim + kBK - 1) / kBK;
-  g.group_m = kPair ? 8 : 16;
+  g.group_m = kPair ? group_rows : 2 * group_rows;
   g.tile_start[0] = 0;
   for (int p = 0; p < g.nprob; ++p) {
     g.n_nt[p] = (g.Ndim[p] + BN - 1) / BN;     // the last N tile may be ragged (zero-filled by TMA)
@@ -1658,20 +1773,27 @@ int pick_bn(const LossProblem& p) {
 }
 
 // One (token block, vocabulary chunk) of the backward pass: its tokens [t0, t0 + Tb)
-// and columns [v0, v0 + Vc), with G' = [M][Tb][Vc] bf16.
+// and columns [v0, v0 + Vc), with G' = [M][Tb][Vc] fp16 and the fp16 copies of
+// the chunk's W rows ([Vc][D_m] per exit, exits one after another) and of the
+// block's h rows ([Tb][D_m] per exit).
 struct BwdChunk {
   int64_t t0, Tb, v0, Vc;
   bool first_v, last_v;    // first / last chunk of the block
   bool first_t;            // first block
-  const __nv_bfloat16* G;
+  const __half* G;
   float* acc;              // dh partial sums [Tb][sum D] (NULL with a single chunk)
+  const __half* w16;
+  const float* w16_inv;    // [M]: 1/s of each exit's copy
+  const __half* h16;
+  const float* h16_inv;    // [M]
 };
 
 // dh_m[Tb x D_m] (+)= a G'_m[Tb x Vc] W^m[v0 : v0 + Vc] for every exit in one launch:
-// A = G'_m (K = Vc contiguous), B = the chunk's rows of W^m (N = D_m contiguous).
-// The last chunk of a block adds the earlier chunks' fp32 partials, subtracts
-// the one-hot row a c_m W^m[y_t] exactly and writes bf16 dh; the others write
-// (first) or add to (later) the fp32 partials.
+// A = G'_m (K = Vc contiguous), B = the fp16 copy of the chunk's rows of W^m
+// (N = D_m contiguous).  The last chunk of a block adds the earlier chunks'
+// fp32 partials, subtracts the one-hot row a c_m W^m[y_t] exactly (from the
+// bf16 W) and writes bf16 dh; the others write (first) or add to (later) the
+// fp32 partials.
 template <int BN>
 cudaError_t run_dh_chunk(const LossProblem& p, const BwdChunk& c, void* const* dh, float alpha, cudaStream_t st) {
   GemmMaps maps;
@@ -1679,6 +1801,7 @@ cudaError_t run_dh_chunk(const LossProblem& p, const BwdChunk& c, void* const* d
   g.nprob = p.M;
   g.Mdim = static_cast<int>(c.Tb);
   g.Kdim = static_cast<int>(c.Vc);
+  g.f16 = 1;
   for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
   const bool tgrad = p.teacher_grad != 0 && p.M > 1;
   if (tgrad) g.alpha[p.M - 1] = alpha;             // the teacher's G' already carries w_T
@@ -1686,12 +1809,13 @@ cudaError_t run_dh_chunk(const LossProblem& p, const BwdChunk& c, void* const* d
   g.onehot_idx = p.y + c.t0;
   g.onehot_limit = static_cast<int>(p.V);
   g.accumulate = c.first_v ? 0 : 1;
-  int64_t acc_off = 0;
+  int64_t acc_off = 0, w_off = 0;
   for (int m = 0; m < p.M; ++m) {
-    const __nv_bfloat16* Gm = c.G + static_cast<int64_t>(m) * c.Tb * c.Vc;
-    const __nv_bfloat16* Wc = static_cast<const __nv_bfloat16*>(p.W[m]) + c.v0 * p.D[m];
-    if (!make_map(&maps.a[m], Gm, c.Vc, c.Tb, kBK, kBM)) return cudaErrorInvalidValue;
-    if (!make_map(&maps.b[m], Wc, p.D[m], c.Vc, 64, kBK)) return cudaErrorInvalidValue;
+    const __half* Gm = c.G + static_cast<int64_t>(m) * c.Tb * c.Vc;
+    if (!make_map(&maps.a[m], Gm, c.Vc, c.Tb, kBK, kBM, true)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.b[m], c.w16 + w_off, p.D[m], c.Vc, 64, kBK, true)) return cudaErrorInvalidValue;
+    w_off += c.Vc * p.D[m];
+    g.bscale[m] = c.w16_inv + m;
     g.Ndim[m] = static_cast<int>(p.D[m]);
     float* acc_m = c.acc != nullptr ? c.acc + acc_off : nullptr;
     acc_off += c.Tb * p.D[m];
@@ -1704,13 +1828,14 @@ cudaError_t run_dh_chunk(const LossProblem& p, const BwdChunk& c, void* const* d
       g.out[m] = acc_m;
     }
   }
-  if (c.last_v) return run_gemm<false, true, BN, true>(maps, g, st);
-  return run_gemm<false, true, BN, false>(maps, g, st);
+  if (c.last_v) return run_gemm<false, true, BN, true>(maps, g, MLS_DH_GROUP_M, st);
+  return run_gemm<false, true, BN, false>(maps, g, MLS_DH_GROUP_M, st);
 }
 
 // dW^m[v0 : v0 + Vc] (+)= a G'_m^T h_m[t0 : t0 + Tb] for every exit in one launch:
-// A = G'^T (M = Vc contiguous), B = the block's rows of h_m (N = D_m contiguous),
-// K = Tb.  Blocks after the first (and every block with accumulate) add.
+// A = G'^T (M = Vc contiguous), B = the fp16 copy of the block's rows of h_m
+// (N = D_m contiguous), K = Tb.  Blocks after the first (and every block with
+// accumulate) add.
 template <int BN>
 cudaError_t run_dw_chunk(const LossProblem& p, const BwdChunk& c, float* const* dW, float alpha, int accumulate,
                          cudaStream_t st) {
@@ -1719,19 +1844,22 @@ cudaError_t run_dw_chunk(const LossProblem& p, const BwdChunk& c, float* const* 
   g.nprob = p.M;
   g.Mdim = static_cast<int>(c.Vc);
   g.Kdim = static_cast<int>(c.Tb);
+  g.f16 = 1;
   for (int m = 0; m < p.M; ++m) g.alpha[m] = alpha * p.exit_w[m];
   if (p.teacher_grad != 0 && p.M > 1) g.alpha[p.M - 1] = alpha;   // the teacher's G' already carries w_T
   g.accumulate = (accumulate || !c.first_t) ? 1 : 0;
   g.status = p.status;
+  int64_t h_off = 0;
   for (int m = 0; m < p.M; ++m) {
-    const __nv_bfloat16* Gm = c.G + static_cast<int64_t>(m) * c.Tb * c.Vc;
-    const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(p.h[m]) + c.t0 * p.D[m];
-    if (!make_map(&maps.a[m], Gm, c.Vc, c.Tb, 64, kBK)) return cudaErrorInvalidValue;
-    if (!make_map(&maps.b[m], hb, p.D[m], c.Tb, 64, kBK)) return cudaErrorInvalidValue;
+    const __half* Gm = c.G + static_cast<int64_t>(m) * c.Tb * c.Vc;
+    if (!make_map(&maps.a[m], Gm, c.Vc, c.Tb, 64, kBK, true)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.b[m], c.h16 + h_off, p.D[m], c.Tb, 64, kBK, true)) return cudaErrorInvalidValue;
+    h_off += c.Tb * p.D[m];
+    g.bscale[m] = c.h16_inv + m;
     g.Ndim[m] = static_cast<int>(p.D[m]);
     g.out[m] = dW[m] + c.v0 * p.D[m];
   }
-  return run_gemm<true, true, BN, false>(maps, g, st);
+  return run_gemm<true, true, BN, false>(maps, g, MLS_DW_GROUP_M, st);
 }
 
 // G' of one (token block, vocabulary chunk): the tile kernel on the block's
@@ -1750,7 +1878,7 @@ cudaError_t run_grad_chunk(const LossProblem& p, const BwdChunk& c, const float*
   a.Vtot = static_cast<int>(p.V);
   a.ldS = static_cast<int>(p.T);
   a.stats = const_cast<float*>(stats) + c.t0;
-  a.G = const_cast<__nv_bfloat16*>(c.G);
+  a.G = const_cast<__half*>(c.G);
   const bool tgrad = p.teacher_grad != 0 && p.M > 1;
   return tgrad ? (p.distill == 1   ? run_loss_tiles<kModeGrad, 1, true>(q, a, st)
                   : p.distill == 2 ? run_loss_tiles<kModeGrad, 2, true>(q, a, st)
@@ -1760,6 +1888,30 @@ cudaError_t run_grad_chunk(const LossProblem& p, const BwdChunk& c, const float*
          : p.distill == 2 ? run_loss_tiles<kModeGrad, 2>(q, a, st)
          : p.distill == 3 ? run_loss_tiles<kModeGrad, 3>(q, a, st)
                           : run_loss_tiles<kModeGrad, 0>(q, a, st);
+}
+
+// fp16 copies of rows [r0, r0 + n) of every exit's bf16 matrix src[m] ([*][D_m])
+// into dst (exits one after another), with their scales in inv[0 .. M).
+cudaError_t run_half_copies(const LossProblem& p, const void* const* src, int64_t r0, int64_t n, __half* dst,
+                            unsigned int* maxbits, float* inv, cudaStream_t st) {
+  cudaError_t err = cudaMemsetAsync(maxbits, 0, sizeof(unsigned int) * p.M, st);
+  if (err != cudaSuccess) return err;
+  HalfJobs jobs{};
+  int64_t off = 0, most = 0;
+  for (int m = 0; m < p.M; ++m) {
+    const int64_t nv = n * p.D[m] / 8;
+    jobs.j[m] = HalfJob{reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(src[m]) + r0 * p.D[m]),
+                        reinterpret_cast<uint4*>(dst + off), nv, maxbits + m, inv + m};
+    off += n * p.D[m];
+    most = nv > most ? nv : most;
+  }
+  const int64_t want = ceil_div(most, 256 * 4);
+  const int64_t cap = 2 * static_cast<int64_t>(num_sms());
+  const dim3 grid(static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap)), static_cast<unsigned>(p.M));
+  half_copy_kernel<<<grid, 256, 0, st>>>(jobs);
+  half_rescale_kernel<<<grid, 256, 0, st>>>(jobs);
+  note_launches(2);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -1855,17 +2007,28 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   const BwdPlan plan = choose_plan(p, ws_bytes);
   if (plan.Tb == 0) return cudaErrorInvalidValue;       // the caller checked the minimum size
   char* base = static_cast<char*>(ws);
-  __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(base);
-  float* acc = plan.acc_bytes ? reinterpret_cast<float*>(base + plan.g_bytes) : nullptr;
-  void* seg_ws = base + plan.g_bytes + plan.acc_bytes;
+  __half* G = reinterpret_cast<__half*>(base);
+  char* q = base + plan.g_bytes;
+  float* acc = plan.acc_bytes ? reinterpret_cast<float*>(q) : nullptr;
+  q += plan.acc_bytes;
+  void* seg_ws = q;
+  q += plan.seg_bytes;
+  __half* h16 = reinterpret_cast<__half*>(q);
+  q += plan.h16_bytes;
+  __half* w16 = reinterpret_cast<__half*>(q);
+  q += plan.w16_bytes;
+  unsigned int* maxbits = reinterpret_cast<unsigned int*>(q);     // [0, M) W, [M, 2M) h
+  float* inv = reinterpret_cast<float*>(q + 2 * kMaxExits * sizeof(unsigned int));
   const float alpha = grad_scale / static_cast<float>(p.T);
   const int bn = pick_bn(p);
   cudaError_t err = cudaSuccess;
   for (int64_t t0 = 0; t0 < p.T && err == cudaSuccess; t0 += plan.Tb) {
+    const int64_t Tb = t0 + plan.Tb <= p.T ? plan.Tb : p.T - t0;
+    err = run_half_copies(p, p.h, t0, Tb, h16, maxbits + p.M, inv + p.M, st);
     for (int64_t v0 = 0; v0 < p.V && err == cudaSuccess; v0 += plan.Vc) {
       BwdChunk c;
       c.t0 = t0;
-      c.Tb = t0 + plan.Tb <= p.T ? plan.Tb : p.T - t0;
+      c.Tb = Tb;
       c.v0 = v0;
       c.Vc = v0 + plan.Vc <= p.V ? plan.Vc : p.V - v0;
       c.first_v = v0 == 0;
@@ -1873,6 +2036,12 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
       c.first_t = t0 == 0;
       c.G = G;
       c.acc = acc;
+      c.w16 = w16;
+      c.w16_inv = inv;
+      c.h16 = h16;
+      c.h16_inv = inv + p.M;
+      err = run_half_copies(p, p.W, v0, c.Vc, w16, maxbits, inv, st);
+      if (err != cudaSuccess) break;
       err = run_grad_chunk(p, c, stats, st);
       if (err != cudaSuccess) break;
       switch (bn) {

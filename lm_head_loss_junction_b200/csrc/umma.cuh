@@ -134,6 +134,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool a_mn_major,
          | (static_cast<uint32_t>(m >> 4) << 24);    // M / 16
 }
 
+// The same with fp16 A and B (format code 0 in both fields).
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16(m, n, a_mn_major, b_mn_major) & ~((7u << 7) | (7u << 10));
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm100 version bits.
 //   K-major tile: rows of 64 bf16 (128 B), 8-row groups 1024 B apart (SBO).
 //   MN-major tile: each K row holds 64 MN-contiguous bf16 (128 B); 8-row K

@@ -122,8 +122,8 @@ def test_workspace_queries():
     import torch
     from lm_head_loss_junction_b200 import junction_bwd_workspace, multiexit_loss_workspace
     f, b = multiexit_loss_workspace(8192, [1024, 2304, 4352], 49152, torch.bfloat16)
-    # a bounded piece of the bf16 G' (one 16384-column chunk of every exit), not all of it
-    assert 3 * 8192 * 16384 * 2 <= b <= 1 << 30
+    # a bounded piece of G' (one 16384-column chunk of every exit), not all of it
+    assert 3 * 8192 * 16384 * 2 <= b <= 3 << 29
     assert f >= (49152 // 128) * 5 * 8192 * 4
     f32f, f32b = multiexit_loss_workspace(256, [64, 128, 192], 512, torch.float32)
     assert f32b == 3 * 256 * 512 * 4

@@ -11,7 +11,7 @@ import oracle
 from lm_head_loss_junction_b200 import (multiexit_loss_bwd, multiexit_loss_bwd_plan, multiexit_loss_fwd, new_status,
                                         status_read)
 from lm_head_loss_junction_b200 import workloads as wl
-from tests.helpers import assert_grad_close, assert_loss_close, assert_stats_close, f64
+from tests.helpers import acceptance_tie_mass, assert_grad_close, assert_loss_close, assert_stats_close, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -54,12 +54,13 @@ def _check_all(d, alpha, grad_scale=1.0, exit_weights=None, distill="ce", teache
     assert_stats_close(s[:M], r["lse"], "lse")
     assert_stats_close(s[M:2 * M], r["tgt"], "target logits")
     if M > 1:
+        slack = acceptance_tie_mass(d.y, d.o, d.W) if distill == "accept" else None
         assert_stats_close(s[2 * M:3 * M - 1],
                            {"ce": r["S"], "reverse_kl": r["R"], "js": r["J"], "accept": r["A"]}[distill],
-                           "distillation statistic")
+                           "distillation statistic", slack=slack)
         if distill in ("js", "accept") and teacher_grad:
             assert_stats_close(s[3 * M - 1:], {"js": r["Jp"], "accept": r["B"]}[distill],
-                               "teacher-side distillation statistic")
+                               "teacher-side distillation statistic", slack=slack)
     for m in range(M):
         assert_grad_close(dh[m], r["dh"][m], f"dh[{m}]")
         assert_grad_close(dW[m], r["dW"][m], f"dW[{m}]")
