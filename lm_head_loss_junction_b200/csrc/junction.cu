@@ -794,15 +794,24 @@ cudaError_t launch_junction_bwd_multi(const JunctionArgs* js, int J, bool any_ta
   const bool bf16 = js[0].bf16;
   const int64_t T = js[0].T;
   float* coef[kMaxExits - 1] = {};
-  for (int k = 0; k < J; ++k) {
-    coef[k] = js[k].dE != nullptr ? reinterpret_cast<float*>(static_cast<char*>(ws) + coef_bytes(T) * k) : nullptr;
-    const cudaError_t err = bf16 ? launch_bwd_rows_t<true>(js[k], coef[k], st) : launch_bwd_rows_t<false>(js[k], coef[k], st);
+  SegIndexDev ix;
+  cudaError_t err = cudaSuccess;
+  {
+    // the id grouping (latency-bound, reads only x) beside the row kernels
+    SideScope side(st);
+    if (any_table) {
+      err = build_segindex(js[0].x, T, js[0].V, static_cast<char*>(ws) + coef_bytes(T) * J, &ix, side.stream());
+      if (err != cudaSuccess) return err;
+    }
+    for (int k = 0; k < J; ++k) {
+      coef[k] = js[k].dE != nullptr ? reinterpret_cast<float*>(static_cast<char*>(ws) + coef_bytes(T) * k) : nullptr;
+      err = bf16 ? launch_bwd_rows_t<true>(js[k], coef[k], st) : launch_bwd_rows_t<false>(js[k], coef[k], st);
+      if (err != cudaSuccess) return err;
+    }
+    err = side.join();
     if (err != cudaSuccess) return err;
   }
   if (!any_table) return cudaSuccess;
-  SegIndexDev ix;
-  cudaError_t err = build_segindex(js[0].x, T, js[0].V, static_cast<char*>(ws) + coef_bytes(T) * J, &ix, st);
-  if (err != cudaSuccess) return err;
   const int N = bf16 ? 8 : 4;
   TableGradJob jobs[kMaxExits - 1];
   int n = 0;

@@ -59,6 +59,24 @@ struct SegIndexDev {
   int64_t max_light;
 };
 
+// A per-device side stream for latency-bound work that does not depend on
+// the bandwidth-bound kernels of the same call (the id sort): forked from the
+// caller's stream with an event, joined back into it with another, so under
+// graph capture it becomes a parallel branch.  One scope at a time per
+// process (a mutex held from the fork to the join); without a side stream
+// (creation failed) stream() is the caller's stream and join() does nothing.
+class SideScope {
+ public:
+  explicit SideScope(cudaStream_t st);
+  ~SideScope();
+  cudaStream_t stream() const { return side_; }
+  cudaError_t join();
+ private:
+  cudaStream_t main_, side_;
+  void* slot_;
+  bool joined_;
+};
+
 size_t segindex_bytes(int64_t T, int64_t V);
 cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, SegIndexDev* out, cudaStream_t st);
 // dE[v] (+)= ge sum_t g_e,t + (sum_t coef_t) E[v]; g_e is the tail of each dy row.

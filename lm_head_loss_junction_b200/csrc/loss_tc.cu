@@ -85,7 +85,8 @@ struct LossArgs {
   int Vtot;                    // the vocabulary size (targets outside [0, Vtot) are invalid)
   int ldS;                     // row stride of stats (the call's token count)
   int kblocks[kMaxExits];      // D_m / kBK
-  int n_tt, n_vt, num_tiles, group_tt;
+  int n_tt, n_vt, num_tiles;
+  int group_tt;                // token tiles per raster group (W streams once per group)
   const int32_t* y;
   float alpha;                 // alpha_d
   int distill;                 // 0: cross-entropy, 1: KL(q_m || p_M), 2: Jensen-Shannon, 3: 1 - sum min(q, p)
@@ -131,6 +132,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 // log(1 + e^x), without overflow for large x.
 __device__ __forceinline__ float softplus(float x) { return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))); }
 
+// Tile i of the launch -> (token tile, vocabulary tile).  Tiles are visited in
+// groups of group_tt token tiles x every vocabulary tile, vocabulary tiles
+// outer, so the group's h rows stay in L2 while the heads stream past (W is
+// read once per token group).
 __device__ __forceinline__ void loss_tile_coords(int i, const LossArgs& a, int& tt, int& vt) {
   const int per_group = a.group_tt * a.n_vt;
   const int g = i / per_group;
@@ -2022,6 +2027,12 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   const float alpha = grad_scale / static_cast<float>(p.T);
   const int bn = pick_bn(p);
   cudaError_t err = cudaSuccess;
+  // tokens grouped by target, for the exact one-hot part of dW: on the side
+  // stream, beside the chunk loop (it reads only the targets)
+  SegIndexDev ix;
+  SideScope side(st);
+  err = build_segindex(p.y, p.T, p.V, seg_ws, &ix, side.stream());
+  if (err != cudaSuccess) return err;
   for (int64_t t0 = 0; t0 < p.T && err == cudaSuccess; t0 += plan.Tb) {
     const int64_t Tb = t0 + plan.Tb <= p.T ? plan.Tb : p.T - t0;
     err = run_half_copies(p, p.h, t0, Tb, h16, maxbits + p.M, inv + p.M, st);
@@ -2058,11 +2069,10 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
     }
   }
   if (err != cudaSuccess) return err;
-  // one-hot part of dW over every token: (1 - alpha_d) for students, 1 for the
-  // teacher; tokens grouped by target, every exit in one launch pair
-  SegIndexDev ix;
-  err = build_segindex(p.y, p.T, p.V, seg_ws, &ix, st);
+  err = side.join();
   if (err != cudaSuccess) return err;
+  // one-hot part of dW over every token: (1 - alpha_d) for students, 1 for the
+  // teacher; every exit in one launch pair
   int d_vec[kMaxExits];
   float scale[kMaxExits];
   for (int m = 0; m < p.M; ++m) {

@@ -11,11 +11,70 @@
 // that no warp is spent on absent ids; each row slice is still summed by one
 // warp in token order, so the list order does not change any result.
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
 
 namespace mls {
+
+// ------------------------------------------------------------------ side stream
+namespace {
+struct SideSlot {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool tried = false;
+};
+constexpr int kMaxSideDevices = 64;
+SideSlot g_side[kMaxSideDevices];
+std::mutex g_side_mu;
+}  // namespace
+
+// Compile with -DMLS_SIDE_STREAM=0 to run the side work on the caller's stream.
+#ifndef MLS_SIDE_STREAM
+#define MLS_SIDE_STREAM 1
+#endif
+
+SideScope::SideScope(cudaStream_t st) : main_(st), side_(st), slot_(nullptr), joined_(true) {
+  if (!MLS_SIDE_STREAM) return;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) {
+    (void)cudaGetLastError();
+    return;
+  }
+  g_side_mu.lock();
+  SideSlot& sl = g_side[dev];
+  if (!sl.tried) {
+    sl.tried = true;
+    if (cudaStreamCreateWithFlags(&sl.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sl.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sl.join, cudaEventDisableTiming) != cudaSuccess) {
+      (void)cudaGetLastError();
+      sl.s = nullptr;
+    }
+  }
+  if (sl.s == nullptr || cudaEventRecord(sl.fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(sl.s, sl.fork, 0) != cudaSuccess) {
+    (void)cudaGetLastError();
+    g_side_mu.unlock();
+    return;
+  }
+  side_ = sl.s;
+  slot_ = &sl;
+  joined_ = false;
+}
+
+cudaError_t SideScope::join() {
+  if (joined_) return cudaSuccess;
+  joined_ = true;
+  SideSlot& sl = *static_cast<SideSlot*>(slot_);
+  cudaError_t err = cudaEventRecord(sl.join, side_);
+  if (err == cudaSuccess) err = cudaStreamWaitEvent(main_, sl.join, 0);
+  g_side_mu.unlock();
+  return err;
+}
+
+SideScope::~SideScope() { (void)join(); }
 
 namespace {
 
@@ -274,18 +333,70 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
   }
 }
 
-// Overwrite mode of the table gradient: the rows of absent ids are zero.  One
-// warp per row of table blockIdx.y (a job); rows of present ids are left to
-// the light and heavy kernels.
-__global__ void __launch_bounds__(256) zero_absent_rows_kernel(const SegIndexDev ix, const SegJobs jobs, int f4_mult) {
+// Overwrite mode of the table gradients, in one pass over every row of every
+// table: warp tasks (row v, 32-vector slice of one table's row) in a
+// grid-stride loop, consecutive tasks covering row v of every table slice by
+// slice; rows of absent ids get zeros, rows of light ids (at most kHeavy
+// tokens) the sum of their tokens' rows in token order (the same order and
+// arithmetic as segsum_light_kernel), rows of heavy ids are left to
+// segsum_heavy_kernel.  The zero writes of the many absent rows hide the
+// latency of the light rows' gathers, which are spread over all warps.
+// Launched with one warp per task (the loop covers larger grids' leftovers).
+template <bool BF16>
+__global__ void __launch_bounds__(256) table_rows_kernel(const __grid_constant__ SegIndexDev ix,
+                                                         const __grid_constant__ SegJobs jobs, int njobs,
+                                                         int row_slices, int v_begin, int v_end) {
+  constexpr int N = Vec8<BF16>::N;
   const int lane = threadIdx.x & 31;
-  const int64_t v = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (v >= ix.V || ix.ends[v] != 0) return;               // present ids have ends > 0
-  const SegJob& jb = jobs.j[blockIdx.y];
-  const int f4_per_row = jb.n_vec * f4_mult;
-  float4* o = reinterpret_cast<float4*>(jb.out) + v * f4_per_row;
-  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i = lane; i < f4_per_row; i += 32) o[i] = z;
+  const unsigned warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const unsigned nwarps = (gridDim.x * blockDim.x) >> 5;
+  const unsigned ntasks = static_cast<unsigned>(v_end - v_begin) * static_cast<unsigned>(row_slices);
+  for (unsigned task = warp0; task < ntasks; task += nwarps) {
+    const unsigned rv = task / static_cast<unsigned>(row_slices);
+    const int v = v_begin + static_cast<int>(rv);
+    int sl = static_cast<int>(task - rv * static_cast<unsigned>(row_slices));
+    int z = 0;
+    while (z + 1 < njobs && sl * 32 >= jobs.j[z].n_vec) {   // which table this slice belongs to
+      sl -= (jobs.j[z].n_vec + 31) / 32;
+      ++z;
+    }
+    const SegJob& jb = jobs.j[z];
+    const int n_vec = jb.n_vec;
+    const int vi = sl * 32 + lane;
+    const bool active = vi < n_vec;
+    const int32_t end = ix.ends[v];
+    float* out_row = jb.out + static_cast<int64_t>(v) * n_vec * N;
+    if (end == 0) {                                      // absent id: zeros
+      if (active) {
+        float4* o = reinterpret_cast<float4*>(out_row + vi * N);
+#pragma unroll
+        for (int q = 0; q < N / 4; ++q) o[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      continue;
+    }
+    const int32_t off = ix.offsets[v];
+    const int32_t cnt = end - off;
+    if (cnt > kHeavy) continue;                          // heavy id: its own kernel
+    float cs = 0.f;
+    for (int p = 0; p < cnt; ++p) cs += jb.coef[ix.toks[off + p]];
+    if (!active) continue;
+    const uint4* __restrict__ src = jb.src;
+    float acc[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) acc[k] = 0.f;
+    int p = 0;
+    for (; p + 4 <= cnt; p += 4) {
+      uint4 u[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        u[b] = __ldg(src + static_cast<int64_t>(ix.toks[off + p + b]) * jb.src_ld + jb.src_off + vi);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) Vec8<BF16>::add(acc, u[b]);
+    }
+    for (; p < cnt; ++p)
+      Vec8<BF16>::add(acc, __ldg(src + static_cast<int64_t>(ix.toks[off + p]) * jb.src_ld + jb.src_off + vi));
+    emit<BF16, true>(out_row, vi, acc, cs, jb.E + static_cast<int64_t>(v) * n_vec, jb.scale, false);
+  }
 }
 
 // One block per (heavy row, slice of 32 vectors, job); warps split the row's
@@ -357,31 +468,41 @@ __global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(const Se
 
 template <bool BF16, bool TABLE>
 cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs, int accumulate, cudaStream_t st) {
-  constexpr int N = Vec8<BF16>::N;
-  if (TABLE && !accumulate) {
-    const int64_t blocks = (ix.V * 32 + 255) / 256;
-    zero_absent_rows_kernel<<<dim3(static_cast<unsigned>(blocks), static_cast<unsigned>(njobs)), 256, 0, st>>>(
-        ix, jobs, N / 4);
-    note_launches(1);
-  }
   int slices = 0, total_slices = 0;
   for (int z = 0; z < njobs; ++z) {
     const int sz = (jobs.j[z].n_vec + 31) / 32;
     slices = std::max(slices, sz);
     total_slices += sz;
   }
-  // light rows: about one full wave of 8-warp blocks over (light ids) x (32-vector slices of every job)
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (static_cast<int64_t>(sms) * 8 + total_slices - 1) / total_slices;
-  const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(want, (ix.max_light + 7) / 8));
-  segsum_light_kernel<BF16, TABLE>
-      <<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices), static_cast<unsigned>(njobs)), 256, 0, st>>>(
-          ix, jobs, accumulate);
+  if (TABLE && !accumulate) {
+    // every row of every table in one pass: zeros for absent ids, sums for light ones
+    // (row ranges of at most 2^31 warp tasks per launch: 32-bit task indices)
+    const int64_t rows_per_launch = std::max<int64_t>(1, ((int64_t(1) << 31) - 1) / total_slices);
+    for (int64_t v0 = 0; v0 < ix.V; v0 += rows_per_launch) {
+      const int64_t v1 = std::min<int64_t>(ix.V, v0 + rows_per_launch);
+      // one warp per task: every task starts with a dependent load of its row's
+      // segment bounds, so latency is hidden by the number of warps in flight
+      const int64_t tasks = (v1 - v0) * total_slices;
+      const int64_t blocks = std::max<int64_t>(1, (tasks + 7) / 8);
+      table_rows_kernel<BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(ix, jobs, njobs, total_slices,
+                                                                             static_cast<int>(v0), static_cast<int>(v1));
+      note_launches(1);
+    }
+  } else {
+    // light rows: about one full wave of 8-warp blocks over (light ids) x (32-vector slices of every job)
+    const int64_t want = (static_cast<int64_t>(sms) * 8 + total_slices - 1) / total_slices;
+    const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(want, (ix.max_light + 7) / 8));
+    segsum_light_kernel<BF16, TABLE>
+        <<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices), static_cast<unsigned>(njobs)), 256, 0, st>>>(
+            ix, jobs, accumulate);
+    note_launches(1);
+  }
   dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>(slices), static_cast<unsigned>(njobs));
   segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, jobs, accumulate);
-  note_launches(2);
+  note_launches(1);
   return cudaGetLastError();
 }
 
