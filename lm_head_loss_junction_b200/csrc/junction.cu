@@ -789,29 +789,27 @@ cudaError_t launch_junction_fwd_multi(const JunctionArgs* js, int J, cudaStream_
 }
 
 // The row kernels of every junction, then one id grouping shared by all table
-// gradients and one launch set of zero and segmented-sum passes over all tables.
+// gradients and one launch set of row-sum passes over all tables.  On the
+// side stream: the id grouping (latency-bound, reads only x) beside the row
+// kernels, then the heavy rows' sums beside the pass over the other rows.
 cudaError_t launch_junction_bwd_multi(const JunctionArgs* js, int J, bool any_table, void* ws, cudaStream_t st) {
   const bool bf16 = js[0].bf16;
   const int64_t T = js[0].T;
   float* coef[kMaxExits - 1] = {};
   SegIndexDev ix;
+  SideScope side(st);
   cudaError_t err = cudaSuccess;
-  {
-    // the id grouping (latency-bound, reads only x) beside the row kernels
-    SideScope side(st);
-    if (any_table) {
-      err = build_segindex(js[0].x, T, js[0].V, static_cast<char*>(ws) + coef_bytes(T) * J, &ix, side.stream());
-      if (err != cudaSuccess) return err;
-    }
-    for (int k = 0; k < J; ++k) {
-      coef[k] = js[k].dE != nullptr ? reinterpret_cast<float*>(static_cast<char*>(ws) + coef_bytes(T) * k) : nullptr;
-      err = bf16 ? launch_bwd_rows_t<true>(js[k], coef[k], st) : launch_bwd_rows_t<false>(js[k], coef[k], st);
-      if (err != cudaSuccess) return err;
-    }
-    err = side.join();
+  if (any_table) {
+    err = build_segindex(js[0].x, T, js[0].V, static_cast<char*>(ws) + coef_bytes(T) * J, &ix, side.stream());
     if (err != cudaSuccess) return err;
   }
-  if (!any_table) return cudaSuccess;
+  for (int k = 0; k < J; ++k) {
+    coef[k] = js[k].dE != nullptr ? reinterpret_cast<float*>(static_cast<char*>(ws) + coef_bytes(T) * k) : nullptr;
+    err = bf16 ? launch_bwd_rows_t<true>(js[k], coef[k], st) : launch_bwd_rows_t<false>(js[k], coef[k], st);
+    if (err != cudaSuccess) return err;
+  }
+  err = side.join();
+  if (err != cudaSuccess || !any_table) return err;
   const int N = bf16 ? 8 : 4;
   TableGradJob jobs[kMaxExits - 1];
   int n = 0;
@@ -820,7 +818,11 @@ cudaError_t launch_junction_bwd_multi(const JunctionArgs* js, int J, bool any_ta
     jobs[n++] = TableGradJob{js[k].dy, static_cast<int>(js[k].D / N), static_cast<int>(js[k].delta / N), coef[k],
                              1.f, js[k].E, js[k].dE};
   }
-  return scatter_table_grads(ix, bf16, n, jobs, js[0].accumulate_dE != 0, st);
+  err = side.fork();
+  if (err != cudaSuccess) return err;
+  err = scatter_table_grads(ix, bf16, n, jobs, js[0].accumulate_dE != 0, st, side.stream());
+  if (err != cudaSuccess) return err;
+  return side.join();
 }
 
 cudaError_t launch_junction_fwd(const JunctionArgs& a, cudaStream_t st) {

@@ -59,17 +59,21 @@ struct SegIndexDev {
   int64_t max_light;
 };
 
-// A per-device side stream for latency-bound work that does not depend on
-// the bandwidth-bound kernels of the same call (the id sort): forked from the
-// caller's stream with an event, joined back into it with another, so under
-// graph capture it becomes a parallel branch.  One scope at a time per
-// process (a mutex held from the fork to the join); without a side stream
-// (creation failed) stream() is the caller's stream and join() does nothing.
+// A per-device side stream for work that does not depend on the kernels the
+// caller's stream runs meanwhile (the id sort beside the junction row kernels,
+// the fp16 operand copies beside the loss backward's tensor-core kernels):
+// forked from the caller's stream with an event (at construction and at each
+// fork()), joined back into it with another (join(), and at destruction), so
+// under graph capture it becomes parallel branches.  One scope at a time per
+// process (a mutex held for the scope's life); without a side stream
+// (creation failed, or built with MLS_SIDE_STREAM=0) stream() is the caller's
+// stream and fork()/join() do nothing.
 class SideScope {
  public:
   explicit SideScope(cudaStream_t st);
   ~SideScope();
   cudaStream_t stream() const { return side_; }
+  cudaError_t fork();
   cudaError_t join();
  private:
   cudaStream_t main_, side_;
@@ -92,8 +96,9 @@ struct TableGradJob {
   const void* E;
   float* dE;
 };
+// The rows of ids with many tokens go to heavy_st (disjoint rows; it may be st).
 cudaError_t scatter_table_grads(const SegIndexDev& ix, bool bf16, int njobs, const TableGradJob* jobs, bool accumulate,
-                                cudaStream_t st);
+                                cudaStream_t st, cudaStream_t heavy_st);
 // For every job z < njobs (at most kMaxExits; one launch pair for all):
 //   dW[z][v] -= scale[z] * sum_{t: y_t = v} h[z]_t  (bf16 rows of d_vec[z] 16-byte vectors).
 cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,

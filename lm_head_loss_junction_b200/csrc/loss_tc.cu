@@ -2027,15 +2027,28 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   const float alpha = grad_scale / static_cast<float>(p.T);
   const int bn = pick_bn(p);
   cudaError_t err = cudaSuccess;
-  // tokens grouped by target, for the exact one-hot part of dW: on the side
-  // stream, beside the chunk loop (it reads only the targets)
+  // On the side stream, beside the tensor-core kernels on the caller's stream:
+  // the tokens grouped by target (for the exact one-hot part of dW; it reads
+  // only the targets), the first block's fp16 h rows and the first piece's
+  // fp16 W rows (beside the first gradient tile kernel, which reads the bf16
+  // originals), and each next piece's W rows once the current piece's dh GEMM
+  // is done with the copy (beside its dW GEMM and the next gradient tile
+  // kernel).  The next block's h rows are copied on the caller's stream, after
+  // the block before has finished with them.
   SegIndexDev ix;
   SideScope side(st);
   err = build_segindex(p.y, p.T, p.V, seg_ws, &ix, side.stream());
   if (err != cudaSuccess) return err;
+  err = run_half_copies(p, p.h, 0, plan.Tb <= p.T ? plan.Tb : p.T, h16, maxbits + p.M, inv + p.M, side.stream());
+  if (err != cudaSuccess) return err;
+  err = run_half_copies(p, p.W, 0, plan.Vc <= p.V ? plan.Vc : p.V, w16, maxbits, inv, side.stream());
+  if (err != cudaSuccess) return err;
   for (int64_t t0 = 0; t0 < p.T && err == cudaSuccess; t0 += plan.Tb) {
     const int64_t Tb = t0 + plan.Tb <= p.T ? plan.Tb : p.T - t0;
-    err = run_half_copies(p, p.h, t0, Tb, h16, maxbits + p.M, inv + p.M, st);
+    if (t0 > 0) {
+      err = run_half_copies(p, p.h, t0, Tb, h16, maxbits + p.M, inv + p.M, st);
+      if (err != cudaSuccess) break;
+    }
     for (int64_t v0 = 0; v0 < p.V && err == cudaSuccess; v0 += plan.Vc) {
       BwdChunk c;
       c.t0 = t0;
@@ -2051,9 +2064,9 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
       c.w16_inv = inv;
       c.h16 = h16;
       c.h16_inv = inv + p.M;
-      err = run_half_copies(p, p.W, v0, c.Vc, w16, maxbits, inv, st);
-      if (err != cudaSuccess) break;
       err = run_grad_chunk(p, c, stats, st);
+      if (err != cudaSuccess) break;
+      err = side.join();                      // this piece's fp16 copies are done
       if (err != cudaSuccess) break;
       switch (bn) {
         case 256: err = run_dh_chunk<256>(p, c, dh, alpha, st); break;
@@ -2061,6 +2074,15 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
         default: err = run_dh_chunk<64>(p, c, dh, alpha, st); break;
       }
       if (err != cudaSuccess) break;
+      // the next piece's W rows (the next chunk, or the next block's first chunk)
+      const bool more = !(c.last_v && t0 + Tb >= p.T);
+      if (more) {
+        const int64_t nv0 = c.last_v ? 0 : v0 + plan.Vc;
+        const int64_t nVc = nv0 + plan.Vc <= p.V ? plan.Vc : p.V - nv0;
+        err = side.fork();
+        if (err == cudaSuccess) err = run_half_copies(p, p.W, nv0, nVc, w16, maxbits, inv, side.stream());
+        if (err != cudaSuccess) break;
+      }
       switch (bn) {
         case 256: err = run_dw_chunk<256>(p, c, dW, alpha, accumulate, st); break;
         case 128: err = run_dw_chunk<128>(p, c, dW, alpha, accumulate, st); break;

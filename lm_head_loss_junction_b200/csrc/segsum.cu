@@ -53,28 +53,44 @@ SideScope::SideScope(cudaStream_t st) : main_(st), side_(st), slot_(nullptr), jo
       sl.s = nullptr;
     }
   }
-  if (sl.s == nullptr || cudaEventRecord(sl.fork, st) != cudaSuccess ||
-      cudaStreamWaitEvent(sl.s, sl.fork, 0) != cudaSuccess) {
-    (void)cudaGetLastError();
+  if (sl.s == nullptr) {
     g_side_mu.unlock();
     return;
   }
   side_ = sl.s;
   slot_ = &sl;
-  joined_ = false;
+  if (fork() != cudaSuccess) {
+    (void)cudaGetLastError();
+    side_ = st;
+    slot_ = nullptr;
+    g_side_mu.unlock();
+  }
+}
+
+cudaError_t SideScope::fork() {
+  if (slot_ == nullptr) return cudaSuccess;
+  // (forking again while forked makes the side stream also wait for the
+  // caller's work enqueued since the last fork)
+  SideSlot& sl = *static_cast<SideSlot*>(slot_);
+  cudaError_t err = cudaEventRecord(sl.fork, main_);
+  if (err == cudaSuccess) err = cudaStreamWaitEvent(side_, sl.fork, 0);
+  if (err == cudaSuccess) joined_ = false;
+  return err;
 }
 
 cudaError_t SideScope::join() {
-  if (joined_) return cudaSuccess;
+  if (slot_ == nullptr || joined_) return cudaSuccess;
   joined_ = true;
   SideSlot& sl = *static_cast<SideSlot*>(slot_);
   cudaError_t err = cudaEventRecord(sl.join, side_);
   if (err == cudaSuccess) err = cudaStreamWaitEvent(main_, sl.join, 0);
-  g_side_mu.unlock();
   return err;
 }
 
-SideScope::~SideScope() { (void)join(); }
+SideScope::~SideScope() {
+  (void)join();
+  if (slot_ != nullptr) g_side_mu.unlock();
+}
 
 namespace {
 
@@ -334,44 +350,33 @@ __global__ void __launch_bounds__(256) segsum_light_kernel(const SegIndexDev ix,
 }
 
 // Overwrite mode of the table gradients, in one pass over every row of every
-// table: warp tasks (row v, 32-vector slice of one table's row) in a
-// grid-stride loop, consecutive tasks covering row v of every table slice by
-// slice; rows of absent ids get zeros, rows of light ids (at most kHeavy
-// tokens) the sum of their tokens' rows in token order (the same order and
+// table: one warp per (row v, table) task, consecutive tasks covering row v
+// of every table; rows of absent ids get zeros (every store 512 contiguous
+// bytes), rows of light ids (at most kHeavy tokens) the sum of their tokens'
+// rows in token order, 32 vectors (one per lane) at a time (the same order and
 // arithmetic as segsum_light_kernel), rows of heavy ids are left to
 // segsum_heavy_kernel.  The zero writes of the many absent rows hide the
-// latency of the light rows' gathers, which are spread over all warps.
-// Launched with one warp per task (the loop covers larger grids' leftovers).
+// latency of the light rows' gathers.
 template <bool BF16>
 __global__ void __launch_bounds__(256) table_rows_kernel(const __grid_constant__ SegIndexDev ix,
                                                          const __grid_constant__ SegJobs jobs, int njobs,
-                                                         int row_slices, int v_begin, int v_end) {
+                                                         int v_begin, int v_end) {
   constexpr int N = Vec8<BF16>::N;
   const int lane = threadIdx.x & 31;
   const unsigned warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const unsigned nwarps = (gridDim.x * blockDim.x) >> 5;
-  const unsigned ntasks = static_cast<unsigned>(v_end - v_begin) * static_cast<unsigned>(row_slices);
+  const unsigned ntasks = static_cast<unsigned>(v_end - v_begin) * static_cast<unsigned>(njobs);
   for (unsigned task = warp0; task < ntasks; task += nwarps) {
-    const unsigned rv = task / static_cast<unsigned>(row_slices);
+    const unsigned rv = task / static_cast<unsigned>(njobs);
     const int v = v_begin + static_cast<int>(rv);
-    int sl = static_cast<int>(task - rv * static_cast<unsigned>(row_slices));
-    int z = 0;
-    while (z + 1 < njobs && sl * 32 >= jobs.j[z].n_vec) {   // which table this slice belongs to
-      sl -= (jobs.j[z].n_vec + 31) / 32;
-      ++z;
-    }
-    const SegJob& jb = jobs.j[z];
+    const SegJob& jb = jobs.j[task - rv * static_cast<unsigned>(njobs)];
     const int n_vec = jb.n_vec;
-    const int vi = sl * 32 + lane;
-    const bool active = vi < n_vec;
     const int32_t end = ix.ends[v];
     float* out_row = jb.out + static_cast<int64_t>(v) * n_vec * N;
     if (end == 0) {                                      // absent id: zeros
-      if (active) {
-        float4* o = reinterpret_cast<float4*>(out_row + vi * N);
-#pragma unroll
-        for (int q = 0; q < N / 4; ++q) o[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      float4* o = reinterpret_cast<float4*>(out_row);
+      const int n4 = n_vec * (N / 4);
+      for (int k = lane; k < n4; k += 32) o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
       continue;
     }
     const int32_t off = ix.offsets[v];
@@ -379,23 +384,25 @@ __global__ void __launch_bounds__(256) table_rows_kernel(const __grid_constant__
     if (cnt > kHeavy) continue;                          // heavy id: its own kernel
     float cs = 0.f;
     for (int p = 0; p < cnt; ++p) cs += jb.coef[ix.toks[off + p]];
-    if (!active) continue;
     const uint4* __restrict__ src = jb.src;
-    float acc[N];
+    const uint4* E_row = jb.E + static_cast<int64_t>(v) * n_vec;
+    for (int vi = lane; vi < n_vec; vi += 32) {
+      float acc[N];
 #pragma unroll
-    for (int k = 0; k < N; ++k) acc[k] = 0.f;
-    int p = 0;
-    for (; p + 4 <= cnt; p += 4) {
-      uint4 u[4];
+      for (int k = 0; k < N; ++k) acc[k] = 0.f;
+      int p = 0;
+      for (; p + 4 <= cnt; p += 4) {
+        uint4 u[4];
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
-        u[b] = __ldg(src + static_cast<int64_t>(ix.toks[off + p + b]) * jb.src_ld + jb.src_off + vi);
+        for (int b = 0; b < 4; ++b)
+          u[b] = __ldg(src + static_cast<int64_t>(ix.toks[off + p + b]) * jb.src_ld + jb.src_off + vi);
 #pragma unroll
-      for (int b = 0; b < 4; ++b) Vec8<BF16>::add(acc, u[b]);
+        for (int b = 0; b < 4; ++b) Vec8<BF16>::add(acc, u[b]);
+      }
+      for (; p < cnt; ++p)
+        Vec8<BF16>::add(acc, __ldg(src + static_cast<int64_t>(ix.toks[off + p]) * jb.src_ld + jb.src_off + vi));
+      emit<BF16, true>(out_row, vi, acc, cs, E_row, jb.scale, false);
     }
-    for (; p < cnt; ++p)
-      Vec8<BF16>::add(acc, __ldg(src + static_cast<int64_t>(ix.toks[off + p]) * jb.src_ld + jb.src_off + vi));
-    emit<BF16, true>(out_row, vi, acc, cs, jb.E + static_cast<int64_t>(v) * n_vec, jb.scale, false);
   }
 }
 
@@ -466,8 +473,11 @@ __global__ void __launch_bounds__(kHeavyWarps * 32) segsum_heavy_kernel(const Se
   }
 }
 
+// Row sums of every job; the heavy rows go to heavy_st (rows disjoint from the
+// others, so they may run beside them on another stream).
 template <bool BF16, bool TABLE>
-cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs, int accumulate, cudaStream_t st) {
+cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs, int accumulate, cudaStream_t st,
+                          cudaStream_t heavy_st) {
   int slices = 0, total_slices = 0;
   for (int z = 0; z < njobs; ++z) {
     const int sz = (jobs.j[z].n_vec + 31) / 32;
@@ -478,17 +488,15 @@ cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs,
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (TABLE && !accumulate) {
-    // every row of every table in one pass: zeros for absent ids, sums for light ones
-    // (row ranges of at most 2^31 warp tasks per launch: 32-bit task indices)
-    const int64_t rows_per_launch = std::max<int64_t>(1, ((int64_t(1) << 31) - 1) / total_slices);
+    // every row of every table in one pass: zeros for absent ids, sums for light ones;
+    // one warp per (row, table) task (row ranges of at most 2^31 tasks per launch)
+    const int64_t rows_per_launch = std::max<int64_t>(1, ((int64_t(1) << 31) - 1) / njobs);
     for (int64_t v0 = 0; v0 < ix.V; v0 += rows_per_launch) {
       const int64_t v1 = std::min<int64_t>(ix.V, v0 + rows_per_launch);
-      // one warp per task: every task starts with a dependent load of its row's
-      // segment bounds, so latency is hidden by the number of warps in flight
-      const int64_t tasks = (v1 - v0) * total_slices;
+      const int64_t tasks = (v1 - v0) * njobs;
       const int64_t blocks = std::max<int64_t>(1, (tasks + 7) / 8);
-      table_rows_kernel<BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(ix, jobs, njobs, total_slices,
-                                                                             static_cast<int>(v0), static_cast<int>(v1));
+      table_rows_kernel<BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(ix, jobs, njobs, static_cast<int>(v0),
+                                                                             static_cast<int>(v1));
       note_launches(1);
     }
   } else {
@@ -501,7 +509,7 @@ cudaError_t launch_segsum(const SegIndexDev& ix, const SegJobs& jobs, int njobs,
     note_launches(1);
   }
   dim3 grid(static_cast<unsigned>(ix.max_heavy), static_cast<unsigned>(slices), static_cast<unsigned>(njobs));
-  segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, st>>>(ix, jobs, accumulate);
+  segsum_heavy_kernel<BF16, TABLE><<<grid, kHeavyWarps * 32, 0, heavy_st>>>(ix, jobs, accumulate);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -574,20 +582,20 @@ cudaError_t build_segindex(const int32_t* ids, int64_t T, int64_t V, void* ws, S
 }
 
 cudaError_t scatter_table_grads(const SegIndexDev& ix, bool bf16, int njobs, const TableGradJob* tj, bool accumulate,
-                                cudaStream_t st) {
+                                cudaStream_t st, cudaStream_t heavy_st) {
   SegJobs jobs{};
   for (int z = 0; z < njobs; ++z)
     jobs.j[z] = SegJob{static_cast<const uint4*>(tj[z].dy), tj[z].d_vec + tj[z].dl_vec, tj[z].d_vec, tj[z].dl_vec,
                        static_cast<const uint4*>(tj[z].E), tj[z].dE, tj[z].ge, tj[z].coef};
-  return bf16 ? launch_segsum<true, true>(ix, jobs, njobs, accumulate, st)
-              : launch_segsum<false, true>(ix, jobs, njobs, accumulate, st);
+  return bf16 ? launch_segsum<true, true>(ix, jobs, njobs, accumulate, st, heavy_st)
+              : launch_segsum<false, true>(ix, jobs, njobs, accumulate, st, heavy_st);
 }
 
 cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy, int d_vec, int dl_vec,
                                const float* coef, float ge, const void* E, float* dE, bool accumulate,
                                cudaStream_t st) {
   const TableGradJob j{dy, d_vec, dl_vec, coef, ge, E, dE};
-  return scatter_table_grads(ix, bf16, 1, &j, accumulate, st);
+  return scatter_table_grads(ix, bf16, 1, &j, accumulate, st, st);
 }
 
 cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,
@@ -595,7 +603,7 @@ cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* co
   SegJobs jobs{};
   for (int z = 0; z < njobs; ++z)
     jobs.j[z] = SegJob{static_cast<const uint4*>(h[z]), d_vec[z], 0, d_vec[z], nullptr, dW[z], scale[z], nullptr};
-  return launch_segsum<true, false>(ix, jobs, njobs, 1, st);
+  return launch_segsum<true, false>(ix, jobs, njobs, 1, st, st);
 }
 
 }  // namespace mls
