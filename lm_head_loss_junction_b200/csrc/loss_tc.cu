@@ -188,6 +188,19 @@ __device__ __forceinline__ uint32_t hfma_p2(uint32_t w, uint32_t x, uint32_t acc
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
+// r[i] of this lane's 32 register values, through the lane's own row of
+// shared memory (an indexed read of the registers would move the whole array
+// to local memory, and a tree of selects needs 16 more live registers).  The
+// row holds 16 values; only this lane reads or writes it.
+__device__ __forceinline__ float pick32(const float (&r)[32], int i, float4* row) {
+  const int h = i >> 4;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    row[u] = h ? make_float4(r[16 + 4 * u], r[17 + 4 * u], r[18 + 4 * u], r[19 + 4 * u])
+               : make_float4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+  return reinterpret_cast<const float*>(row)[i & 15];
+}
+
 // TMEM region and use count of job j (exit M-1-j) of the tile_iter-th tile of a CTA.
 // By default consecutive jobs alternate the two regions.  When the epilogue
 // needs the teacher's logits at every element of a student's tile (the
@@ -356,6 +369,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
     const int q = warp & 3;                          // TMEM lane quadrant this warp may access
     const int half = (warp - 2) >> 2;                // which 128-column split of the tile
     const int row = q * 32 + lane;
+    float4* tgt_row = reinterpret_cast<float4*>(s.gstage[warp - 2] + lane * kStageRowBytes);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * kSplitCols;
     const int Q = 2 * M - 1;
     const float al = a.alpha;
@@ -398,9 +412,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
 #pragma unroll
                 for (int k = 0; k < 32; ++k) mx = fmaxf(mx, r[k]);
                 if (has_tgt && (yl >> 5) == c) {
-#pragma unroll
-                  for (int k = 0; k < 32; ++k)
-                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = r[k];
+                  a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = pick32(r, yl & 31, tgt_row);
                 }
               }
               const float mxs = mx * kLog2e;
@@ -445,9 +457,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 B = B * rs + bc;
                 ms = mn;
                 if (has_tgt && (yl >> 5) == c) {
-#pragma unroll
-                  for (int k = 0; k < 32; ++k)
-                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = r[k];
+                  a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = pick32(r, yl & 31, tgt_row);
                 }
               }
               lse_part = ms + logf(zs);
@@ -475,9 +485,7 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
                 zs = zs * exp2f((ms - mn) * kLog2e) + zc;
                 ms = mn;
                 if (has_tgt && (yl >> 5) == c) {
-#pragma unroll
-                  for (int k = 0; k < 32; ++k)
-                    if (k == (yl & 31)) a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = r[k];
+                  a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = pick32(r, yl & 31, tgt_row);
                 }
               }
               lse_part = ms + logf(zs);
