@@ -783,19 +783,23 @@ __global__ void __launch_bounds__(32 * kLossMergeRows) loss_merge_kernel(const f
   float mT = -INFINITY, zT = 0.f;
   float A[S] = {0.f, 0.f, 0.f}, ms[S] = {-INFINITY, -INFINITY, -INFINITY}, zs[S] = {0.f, 0.f, 0.f};
   if (t < T) {
+#pragma unroll 4
     for (int i = i0; i < i1; ++i) {
       const float* pi = partial + static_cast<int64_t>(i) * Q * T + t;
       const float l = pi[static_cast<int64_t>(M - 1) * T];
       if (l > mT) {
         const float r = __expf(mT - l);
         zT *= r;
-        if (distill != 1)
-          for (int s = 0; s < M - 1; ++s) A[s] *= r;   // teacher-weighted sums follow the teacher's max
+        if (distill != 1) {   // teacher-weighted sums follow the teacher's max
+#pragma unroll
+          for (int s = 0; s < S; ++s) if (s < M - 1) A[s] *= r;
+        }
         mT = l;
       }
       const float w = (l == -INFINITY) ? 0.f : __expf(l - mT);
       zT += w;
-      for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+      for (int s = 0; s < S; ++s) if (s < M - 1) {
         const float ls = pi[static_cast<int64_t>(s) * T];
         const float ab = pi[static_cast<int64_t>(M + s) * T];
         if (distill != 1) A[s] = fmaf(w, ab, A[s]);
@@ -815,6 +819,7 @@ __global__ void __launch_bounds__(32 * kLossMergeRows) loss_merge_kernel(const f
   }
   st_mT[rowi][lane] = mT;
   st_zT[rowi][lane] = zT;
+#pragma unroll
   for (int s = 0; s < S; ++s) {
     st_A[rowi][s][lane] = A[s];
     st_ms[rowi][s][lane] = ms[s];
@@ -828,7 +833,8 @@ __global__ void __launch_bounds__(32 * kLossMergeRows) loss_merge_kernel(const f
     const float r1 = (mT == -INFINITY) ? 0.f : __expf(mT - mm);
     const float r2 = (m2 == -INFINITY) ? 0.f : __expf(m2 - mm);
     zT = zT * r1 + z2 * r2;
-    for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) if (s < M - 1) {
       const float n2 = st_ms[r][s][lane], y2 = st_zs[r][s][lane];
       const float mn = fmaxf(ms[s], n2);
       const float q1 = (ms[s] == -INFINITY) ? 0.f : __expf(ms[s] - mn);
@@ -846,7 +852,8 @@ __global__ void __launch_bounds__(32 * kLossMergeRows) loss_merge_kernel(const f
   stats[static_cast<int64_t>(M - 1) * T + t] = lseT;
   if (bad) stats[static_cast<int64_t>(2 * M - 1) * T + t] = 0.f;
   terms[static_cast<int64_t>(M - 1) * T + t] = bad ? 0.f : lseT - stats[static_cast<int64_t>(2 * M - 1) * T + t];
-  for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+  for (int s = 0; s < S; ++s) if (s < M - 1) {
     const float lse = ms[s] + logf(zs[s]);
     // cross-entropy: S = sum p_T l_m (teacher-weighted); reverse KL: R = sum q_m (l_m - l_T).
     // (Jensen-Shannon: S and the cross-entropy term here; its own pass overwrites both.)
@@ -883,29 +890,38 @@ __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const floa
   float mx[kMaxExits] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   int ix[kMaxExits] = {-1, -1, -1, -1};
   if (t < T) {
+#pragma unroll 4
     for (int i = i0; i < i1; ++i) {
       const float* pi = partial + static_cast<int64_t>(i) * QA * T + t;
-      for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+      for (int s = 0; s < S; ++s) if (s < M - 1) {
         b[s] += pi[static_cast<int64_t>(s) * T];
         kl[s] += pi[static_cast<int64_t>(M - 1 + s) * T];
       }
-      for (int m = 0; m < M; ++m) {
+#pragma unroll
+      for (int m = 0; m < kMaxExits; ++m) if (m < M) {
         const float v = pi[static_cast<int64_t>(2 * (M - 1) + m) * T];
         if (v > mx[m]) { mx[m] = v; ix[m] = __float_as_int(pi[static_cast<int64_t>(3 * M - 2 + m) * T]); }
       }
     }
   }
+#pragma unroll
   for (int s = 0; s < S; ++s) { sh_b[rowi][s][lane] = b[s]; sh_k[rowi][s][lane] = kl[s]; }
+#pragma unroll
   for (int m = 0; m < kMaxExits; ++m) { sh_mx[rowi][m][lane] = mx[m]; sh_ix[rowi][m][lane] = ix[m]; }
   __syncthreads();
   if (rowi != 0 || t >= T) return;
   for (int r = 1; r < kMergeRows; ++r) {
-    for (int s = 0; s < M - 1; ++s) { b[s] += sh_b[r][s][lane]; kl[s] += sh_k[r][s][lane]; }
-    for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int s = 0; s < S; ++s) if (s < M - 1) { b[s] += sh_b[r][s][lane]; kl[s] += sh_k[r][s][lane]; }
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M)
       if (sh_mx[r][m][lane] > mx[m]) { mx[m] = sh_mx[r][m][lane]; ix[m] = sh_ix[r][m][lane]; }
   }
-  for (int m = 0; m < M; ++m) top1[static_cast<int64_t>(m) * T + t] = ix[m];
-  for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) top1[static_cast<int64_t>(m) * T + t] = ix[m];
+#pragma unroll
+  for (int s = 0; s < S; ++s) if (s < M - 1) {
     terms[static_cast<int64_t>(s) * T + t] = b[s];
     terms[static_cast<int64_t>(M - 1 + s) * T + t] = kl[s];
     terms[static_cast<int64_t>(2 * (M - 1) + s) * T + t] = (ix[s] == ix[M - 1]) ? 1.f : 0.f;
@@ -931,22 +947,27 @@ __global__ void __launch_bounds__(32 * kMergeRows) js_merge_kernel(const float* 
   const int i0 = min(n_splits, rowi * per), i1 = min(n_splits, i0 + per);
   float jq[S] = {0.f, 0.f, 0.f}, jp[S] = {0.f, 0.f, 0.f};
   if (t < T) {
+#pragma unroll 4
     for (int i = i0; i < i1; ++i) {
       const float* pi = partial + static_cast<int64_t>(i) * QJ * T + t;
-      for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+      for (int s = 0; s < S; ++s) if (s < M - 1) {
         jq[s] += pi[static_cast<int64_t>(s) * T];
         jp[s] += pi[static_cast<int64_t>(M - 1 + s) * T];
       }
     }
   }
+#pragma unroll
   for (int s = 0; s < S; ++s) { sh_q[rowi][s][lane] = jq[s]; sh_p[rowi][s][lane] = jp[s]; }
   __syncthreads();
   if (rowi != 0 || t >= T) return;
   for (int r = 1; r < kMergeRows; ++r)
-    for (int s = 0; s < M - 1; ++s) { jq[s] += sh_q[r][s][lane]; jp[s] += sh_p[r][s][lane]; }
+#pragma unroll
+    for (int s = 0; s < S; ++s) if (s < M - 1) { jq[s] += sh_q[r][s][lane]; jp[s] += sh_p[r][s][lane]; }
   const int yt = y[t];
   const bool bad = yt < 0 || yt >= V;
-  for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+  for (int s = 0; s < S; ++s) if (s < M - 1) {
     if (kind == 3) {
       // acceptance: A into the statistics row, 1 - beta = 1 - (A + B) as the term, B for the teacher
       stats[static_cast<int64_t>(2 * M + s) * T + t] = jq[s];
