@@ -783,36 +783,54 @@ __global__ void __launch_bounds__(32 * kLossMergeRows) loss_merge_kernel(const f
   float mT = -INFINITY, zT = 0.f;
   float A[S] = {0.f, 0.f, 0.f}, ms[S] = {-INFINITY, -INFINITY, -INFINITY}, zs[S] = {0.f, 0.f, 0.f};
   if (t < T) {
-#pragma unroll 4
-    for (int i = i0; i < i1; ++i) {
-      const float* pi = partial + static_cast<int64_t>(i) * Q * T + t;
-      const float l = pi[static_cast<int64_t>(M - 1) * T];
-      if (l > mT) {
-        const float r = __expf(mT - l);
-        zT *= r;
-        if (distill != 1) {   // teacher-weighted sums follow the teacher's max
+    // The partials of kB splits are loaded before any of them is merged, so a
+    // thread has that many independent loads in flight; padding splits past i1
+    // read as empty (-inf, weight 0) and leave every sum unchanged.
+    constexpr int kB = 4;
+    for (int i = i0; i < i1; i += kB) {
+      float lt[kB], lsv[kB][S], abv[kB][S];
 #pragma unroll
-          for (int s = 0; s < S; ++s) if (s < M - 1) A[s] *= r;
+      for (int u = 0; u < kB; ++u) {
+        const bool in = i + u < i1;
+        const float* pi = partial + static_cast<int64_t>(in ? i + u : i0) * Q * T + t;
+        lt[u] = in ? pi[static_cast<int64_t>(M - 1) * T] : -INFINITY;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+          const bool ok = in && s < M - 1;
+          lsv[u][s] = ok ? pi[static_cast<int64_t>(s) * T] : -INFINITY;
+          abv[u][s] = ok ? pi[static_cast<int64_t>(M + s) * T] : 0.f;
         }
-        mT = l;
       }
-      const float w = (l == -INFINITY) ? 0.f : __expf(l - mT);
-      zT += w;
 #pragma unroll
-      for (int s = 0; s < S; ++s) if (s < M - 1) {
-        const float ls = pi[static_cast<int64_t>(s) * T];
-        const float ab = pi[static_cast<int64_t>(M + s) * T];
-        if (distill != 1) A[s] = fmaf(w, ab, A[s]);
-        if (ls > ms[s]) {
-          const float r = __expf(ms[s] - ls);
-          zs[s] *= r;
-          if (distill == 1) A[s] *= r;          // reverse KL: weights are the student's own
-          ms[s] = ls;
+      for (int u = 0; u < kB; ++u) {
+        const float l = lt[u];
+        if (l > mT) {
+          const float r = __expf(mT - l);
+          zT *= r;
+          if (distill != 1) {   // teacher-weighted sums follow the teacher's max
+#pragma unroll
+            for (int s = 0; s < S; ++s) if (s < M - 1) A[s] *= r;
+          }
+          mT = l;
         }
-        if (ls != -INFINITY) {
-          const float ws = __expf(ls - ms[s]);
-          zs[s] += ws;
-          if (distill == 1) A[s] = fmaf(ws, ab, A[s]);
+        const float w = (l == -INFINITY) ? 0.f : __expf(l - mT);
+        zT += w;
+#pragma unroll
+        for (int s = 0; s < S; ++s) if (s < M - 1) {
+          const float ls = lsv[u][s];
+          const float ab = abv[u][s];
+          if (distill != 1) A[s] = fmaf(w, ab, A[s]);
+          if (ls > ms[s]) {
+            const float r = __expf(ms[s] - ls);
+            zs[s] *= r;
+            if (distill == 1) A[s] *= r;          // reverse KL: weights are the student's own
+            ms[s] = ls;
+          }
+          if (ls != -INFINITY) {
+            const float ws = __expf(ls - ms[s]);
+            zs[s] += ws;
+            if (distill == 1) A[s] = fmaf(ws, ab, A[s]);
+          }
         }
       }
     }
@@ -890,18 +908,40 @@ __global__ void __launch_bounds__(32 * kMergeRows) agree_merge_kernel(const floa
   float mx[kMaxExits] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   int ix[kMaxExits] = {-1, -1, -1, -1};
   if (t < T) {
-#pragma unroll 4
-    for (int i = i0; i < i1; ++i) {
-      const float* pi = partial + static_cast<int64_t>(i) * QA * T + t;
+    // kB splits' partials are loaded before any is merged (independent loads in
+    // flight); padding splits past i1 add zeros and never beat a maximum.
+    constexpr int kB = 4;
+    for (int i = i0; i < i1; i += kB) {
+      float bv[kB][S], kv[kB][S], mv[kB][kMaxExits];
+      int iv[kB][kMaxExits];
 #pragma unroll
-      for (int s = 0; s < S; ++s) if (s < M - 1) {
-        b[s] += pi[static_cast<int64_t>(s) * T];
-        kl[s] += pi[static_cast<int64_t>(M - 1 + s) * T];
+      for (int u = 0; u < kB; ++u) {
+        const bool in = i + u < i1;
+        const float* pi = partial + static_cast<int64_t>(in ? i + u : i0) * QA * T + t;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+          const bool ok = in && s < M - 1;
+          bv[u][s] = ok ? pi[static_cast<int64_t>(s) * T] : 0.f;
+          kv[u][s] = ok ? pi[static_cast<int64_t>(M - 1 + s) * T] : 0.f;
+        }
+#pragma unroll
+        for (int m = 0; m < kMaxExits; ++m) {
+          const bool ok = in && m < M;
+          mv[u][m] = ok ? pi[static_cast<int64_t>(2 * (M - 1) + m) * T] : -INFINITY;
+          iv[u][m] = ok ? __float_as_int(pi[static_cast<int64_t>(3 * M - 2 + m) * T]) : -1;
+        }
       }
 #pragma unroll
-      for (int m = 0; m < kMaxExits; ++m) if (m < M) {
-        const float v = pi[static_cast<int64_t>(2 * (M - 1) + m) * T];
-        if (v > mx[m]) { mx[m] = v; ix[m] = __float_as_int(pi[static_cast<int64_t>(3 * M - 2 + m) * T]); }
+      for (int u = 0; u < kB; ++u) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) if (s < M - 1) {
+          b[s] += bv[u][s];
+          kl[s] += kv[u][s];
+        }
+#pragma unroll
+        for (int m = 0; m < kMaxExits; ++m) if (m < M) {
+          if (mv[u][m] > mx[m]) { mx[m] = mv[u][m]; ix[m] = iv[u][m]; }
+        }
       }
     }
   }
