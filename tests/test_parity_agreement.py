@@ -72,6 +72,15 @@ def test_agreement_bf16_small(name, small):
     _check(wl.make_inputs(wl.small_variant(wl.CONFIGS[name], **small), with_tables=False))
 
 
+# Vocabulary sizes whose split counts give the agreement merge's thread rows
+# (16 per 32-token block, four splits loaded per batch) a full batch and a
+# partial one (V = 10240: 80 splits, 5 per row) or exact batches (V = 24576:
+# 192 splits, 12 per row).
+@pytest.mark.parametrize("V", [10240, 24576])
+def test_agreement_merge_split_batches(V):
+    _check(wl.make_inputs(wl.small_variant(wl.CONFIGS["main3"], batch=1, seq=130, V=V), with_tables=False))
+
+
 @pytest.mark.parametrize("name", ["main3", "main3_aligned"])
 def test_agreement_full_size_sampled(name):
     d = wl.make_inputs(wl.CONFIGS[name], with_tables=False)

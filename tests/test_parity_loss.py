@@ -86,6 +86,27 @@ def test_bf16_tensor_core_path_small(name, small):
     _check_all(d, cfg.alpha_d, grad_scale=1.0)
 
 
+# Vocabulary sizes whose split counts leave the loss merge's thread rows (32
+# per 32-token block, four splits loaded per batch) partial batches:
+# V = 10240 is 80 splits (3 per row, one row of 2, the last five rows empty),
+# V = 24576 is 192 splits (6 per row: a full batch and a partial one).
+@pytest.mark.parametrize("V", [10240, 24576])
+def test_forward_merge_split_batches(V):
+    cfg = wl.small_variant(wl.CONFIGS["main3"], batch=1, seq=130, V=V)
+    d = wl.make_inputs(cfg, with_tables=False)
+    y, h, W = _gpu_inputs(d)
+    st = new_status()
+    losses, stats = multiexit_loss_fwd(y, h, W, cfg.alpha_d, status=st)
+    assert status_read(st) == (0, 0)
+    r = _oracle(d, cfg.alpha_d, need_grad=False)
+    M = cfg.M
+    assert_loss_close(losses, _losses_expected(r, M), "losses")
+    s = f64(stats)
+    assert_stats_close(s[:M], r["lse"], "lse")
+    assert_stats_close(s[M:2 * M], r["tgt"], "target logits")
+    assert_stats_close(s[2 * M:3 * M - 1], r["S"], "distillation statistic")
+
+
 def _pieces(cfg, ws_bytes):
     Tb, Vc, _ = multiexit_loss_bwd_plan(cfg.T, cfg.D, cfg.V, torch.bfloat16, ws_bytes)
     return Tb, Vc, -(-cfg.T // Tb), -(-cfg.V // Vc)
