@@ -32,6 +32,7 @@ struct SimtDev {
   int32_t* status;
   float* dh[kMaxExits];
   float* dW[kMaxExits];
+  int vec;                   // every width a multiple of 4 and every W row 16-byte aligned: float4 loads
 };
 
 __device__ __forceinline__ void merge_max_sum(float& m1, float& z1, float m2, float z2) {
@@ -46,9 +47,52 @@ constexpr float kLn2 = 0.6931471805599453f;
 // log(1 + e^x), without overflow for large x.
 __device__ __forceinline__ float softplus(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
 
+// a[i] of a per-exit register array by selects (an indexed read with a
+// run-time i would move the array to local memory).
+__device__ __forceinline__ float exit_at(const float (&a)[kMaxExits], int i) {
+  float r = a[0];
+#pragma unroll
+  for (int k = 1; k < kMaxExits; ++k) r = (i == k) ? a[k] : r;
+  return r;
+}
+
+// One logit: the staged h row (shared memory) against one W row (global
+// memory), with four independent partial sums so that the row's loads are not
+// serialised behind one chain of dependent FMAs; float4 loads when p.vec.
+__device__ __forceinline__ float dot_row(const float* __restrict__ hh, const float* __restrict__ w, int64_t D,
+                                         int vec) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int64_t k = 0;
+  if (vec) {
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    const float4* h4 = reinterpret_cast<const float4*>(hh);
+    const int64_t n4 = D >> 2;
+#pragma unroll 4
+    for (int64_t i = 0; i < n4; ++i) {
+      const float4 x = __ldg(w4 + i);
+      const float4 y = h4[i];
+      a0 = fmaf(y.x, x.x, a0);
+      a1 = fmaf(y.y, x.y, a1);
+      a2 = fmaf(y.z, x.z, a2);
+      a3 = fmaf(y.w, x.w, a3);
+    }
+    k = n4 << 2;
+  } else {
+#pragma unroll 1
+    for (; k + 4 <= D; k += 4) {
+      a0 = fmaf(hh[k], __ldg(w + k), a0);
+      a1 = fmaf(hh[k + 1], __ldg(w + k + 1), a1);
+      a2 = fmaf(hh[k + 2], __ldg(w + k + 2), a2);
+      a3 = fmaf(hh[k + 3], __ldg(w + k + 3), a3);
+    }
+  }
+  for (; k < D; ++k) a0 = fmaf(hh[k], __ldg(w + k), a0);
+  return (a0 + a1) + (a2 + a3);
+}
+
 // Quantities per thread, in shared memory for the tree merge:
 //   [0] m_T  [1] z_T  [2..2+M-2] A_s  then per student (m_s, z_s), then tgt[M]
-__global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev p, float* __restrict__ stats,
+__global__ void __launch_bounds__(kSimtThreads, 1) simt_stats_kernel(const SimtDev p, float* __restrict__ stats,
                                                                   float* __restrict__ terms) {
   extern __shared__ float sm[];
   __shared__ float lse_sh[kMaxExits];
@@ -58,9 +102,11 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
   const int tid = threadIdx.x;
   float* hrow = sm;
   int64_t hsum = 0;
-  for (int m = 0; m < M; ++m) hsum += p.D[m];
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) hsum += p.D[m];
   float* red = sm + hsum;  // [Q][kSimtThreads]
-  for (int m = 0; m < M; ++m)
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M)
     for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) hrow[p.Doff[m] + k] = p.h[m][t * p.D[m] + k];
   __syncthreads();
 
@@ -73,24 +119,24 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
 
   for (int64_t v = tid; v < p.V; v += kSimtThreads) {
     float l[kMaxExits];
-    for (int m = 0; m < M; ++m) {
-      const float* w = p.W[m] + v * p.D[m];
-      const float* hh = hrow + p.Doff[m];
-      float acc = 0.f;
-      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
-      l[m] = acc;
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) {
+      l[m] = dot_row(hrow + p.Doff[m], p.W[m] + v * p.D[m], p.D[m], p.vec);
     }
-    const float lT = l[M - 1];
+    const float lT = exit_at(l, M - 1);
     if (lT > mT) {
       const float r = __expf(mT - lT);
       zT *= r;
-      if (p.distill != 1)
-        for (int s = 0; s < S; ++s) A[s] *= r;
+      if (p.distill != 1) {
+#pragma unroll
+        for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) A[s] *= r;
+      }
       mT = lT;
     }
     const float pt = __expf(lT - mT);
     zT += pt;
-    for (int s = 0; s < S; ++s) {
+#pragma unroll
+    for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
       if (p.distill != 1) A[s] = fmaf(pt, l[s], A[s]);
       if (l[s] > ms[s]) {
         const float r = __expf(ms[s] - l[s]);
@@ -102,19 +148,24 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       zs[s] += qs;
       if (p.distill == 1) A[s] = fmaf(qs, l[s] - lT, A[s]);
     }
-    if (v == yt)
-      for (int m = 0; m < M; ++m) tgt[m] = l[m];
+    if (v == yt) {
+#pragma unroll
+      for (int m = 0; m < kMaxExits; ++m) if (m < M) tgt[m] = l[m];
+    }
   }
 
   // stage per-thread partials
   red[0 * kSimtThreads + tid] = mT;
   red[1 * kSimtThreads + tid] = zT;
-  for (int s = 0; s < S; ++s) red[(2 + s) * kSimtThreads + tid] = A[s];
-  for (int s = 0; s < S; ++s) {
+#pragma unroll
+  for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) red[(2 + s) * kSimtThreads + tid] = A[s];
+#pragma unroll
+  for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
     red[(2 + S + 2 * s) * kSimtThreads + tid] = ms[s];
     red[(2 + S + 2 * s + 1) * kSimtThreads + tid] = zs[s];
   }
-  for (int m = 0; m < M; ++m) red[(2 + 3 * S + m) * kSimtThreads + tid] = tgt[m];
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) red[(2 + 3 * S + m) * kSimtThreads + tid] = tgt[m];
   __syncthreads();
   for (int stride = kSimtThreads / 2; stride > 0; stride >>= 1) {
     if (tid < stride) {
@@ -126,7 +177,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       const float r2 = (m2 == -INFINITY) ? 0.f : __expf(m2 - mm);
       red[tid] = mm;
       red[kSimtThreads + tid] = z1 * r1 + z2 * r2;
-      for (int s = 0; s < S; ++s) {
+#pragma unroll
+      for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
         float* a = red + (2 + s) * kSimtThreads;
         float* msp = red + (2 + S + 2 * s) * kSimtThreads;
         float* zsp = msp + kSimtThreads;
@@ -143,13 +195,15 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
         msp[tid] = mA;
         zsp[tid] = zA;
       }
-      for (int m = 0; m < M; ++m) red[(2 + 3 * S + m) * kSimtThreads + tid] += red[(2 + 3 * S + m) * kSimtThreads + o];
+#pragma unroll
+      for (int m = 0; m < kMaxExits; ++m) if (m < M) red[(2 + 3 * S + m) * kSimtThreads + tid] += red[(2 + 3 * S + m) * kSimtThreads + o];
     }
     __syncthreads();
   }
   if (tid == 0) {
     const float lseT = red[0] + logf(red[kSimtThreads]);
-    for (int m = 0; m < M; ++m) {
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) {
       float lse;
       if (m == M - 1) {
         lse = lseT;
@@ -161,7 +215,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       stats[(M + m) * p.T + t] = bad ? 0.f : tg;
       terms[m * p.T + t] = bad ? 0.f : lse - tg;
     }
-    for (int s = 0; s < S; ++s) {
+#pragma unroll
+    for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
       const float zsum = red[(2 + S + 2 * s + 1) * kSimtThreads];
       const float lse = red[(2 + S + 2 * s) * kSimtThreads] + logf(zsum);
       // cross-entropy: S = sum p_T l_m; reverse KL: R = sum q_m (l_m - l_T)
@@ -170,7 +225,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       terms[(M + s) * p.T + t] = bad ? 0.f : (p.distill != 1 ? lse - Sv : Sv - lse + lseT);
     }
     if (bad) set_flag(p.status, MLS_DEVFLAG_BAD_ID);
-    for (int m = 0; m < M; ++m) lse_sh[m] = stats[m * p.T + t];
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) lse_sh[m] = stats[m * p.T + t];
   }
   if ((p.distill != 2 && p.distill != 3) || S == 0) return;
   // Jensen-Shannon or acceptance: second walk over the vocabulary with the final
@@ -178,21 +234,21 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
   // acceptance sums q where q < p (A) and p where q >= p (B).
   __syncthreads();
   float lse[kMaxExits];
-  for (int m = 0; m < M; ++m) lse[m] = lse_sh[m];
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) lse[m] = lse_sh[m];
+  const float lseT = exit_at(lse, M - 1);
   float jq[kMaxExits - 1], jp[kMaxExits - 1];
   for (int s = 0; s < kMaxExits - 1; ++s) { jq[s] = 0.f; jp[s] = 0.f; }
   for (int64_t v = tid; v < p.V; v += kSimtThreads) {
     float l[kMaxExits];
-    for (int m = 0; m < M; ++m) {
-      const float* w = p.W[m] + v * p.D[m];
-      const float* hh = hrow + p.Doff[m];
-      float acc = 0.f;
-      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
-      l[m] = acc;
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) {
+      l[m] = dot_row(hrow + p.Doff[m], p.W[m] + v * p.D[m], p.D[m], p.vec);
     }
-    const float lp = l[M - 1] - lse[M - 1];
+    const float lp = exit_at(l, M - 1) - lseT;
     const float pv = expf(lp);
-    for (int s = 0; s < S; ++s) {
+#pragma unroll
+    for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
       const float lq = l[s] - lse[s];
       if (p.distill == 3) {
         if (lq < lp) jq[s] += expf(lq);
@@ -204,7 +260,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
       }
     }
   }
-  for (int s = 0; s < S; ++s) {
+#pragma unroll
+  for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
     red[(2 * s) * kSimtThreads + tid] = jq[s];
     red[(2 * s + 1) * kSimtThreads + tid] = jp[s];
   }
@@ -215,7 +272,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
     __syncthreads();
   }
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
+#pragma unroll
+    for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
       const float a = red[(2 * s) * kSimtThreads], b = red[(2 * s + 1) * kSimtThreads];
       if (p.distill == 3) {                 // A, then B for the teacher; the term is 1 - (A + B)
         stats[(2 * M + s) * p.T + t] = a;
@@ -232,36 +290,39 @@ __global__ void __launch_bounds__(kSimtThreads) simt_stats_kernel(const SimtDev 
 
 // Backward, one block per token: G'_m[t, :] into the workspace, then
 // dh_m[t] = alpha * G'_m[t, :] W^m.
-__global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p, const float* __restrict__ stats,
+__global__ void __launch_bounds__(kSimtThreads, 1) simt_grad_kernel(const SimtDev p, const float* __restrict__ stats,
                                                                  float alpha, float* __restrict__ G) {
   extern __shared__ float sm[];
   const int M = p.M;
   const int64_t t = blockIdx.x;
   const int tid = threadIdx.x;
   float* hrow = sm;
-  for (int m = 0; m < M; ++m)
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M)
     for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) hrow[p.Doff[m] + k] = p.h[m][t * p.D[m] + k];
   __syncthreads();
   const int32_t yt = p.y[t];
   const bool bad = yt < 0 || yt >= p.V;
   float lse[kMaxExits], kl[kMaxExits];
-  for (int m = 0; m < M; ++m) lse[m] = stats[m * p.T + t];
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) lse[m] = stats[m * p.T + t];
+  const float lseT = exit_at(lse, M - 1);
   // reverse KL: KL(q_m || p_T) = R - lse_m + lse_T; Jensen-Shannon: K = KL(q_m || mu)/2 as stored
-  for (int m = 0; m < M - 1; ++m)
-    kl[m] = (p.distill >= 2) ? stats[(2 * M + m) * p.T + t] : stats[(2 * M + m) * p.T + t] - lse[m] + lse[M - 1];
+#pragma unroll
+  for (int m = 0; m < kMaxExits - 1; ++m) if (m < M - 1)
+    kl[m] = (p.distill >= 2) ? stats[(2 * M + m) * p.T + t] : stats[(2 * M + m) * p.T + t] - lse[m] + lseT;
   const float a = p.alpha_d;
   for (int64_t v = tid; v < p.V; v += kSimtThreads) {
     float l[kMaxExits];
-    for (int m = 0; m < M; ++m) {
-      const float* w = p.W[m] + v * p.D[m];
-      const float* hh = hrow + p.Doff[m];
-      float acc = 0.f;
-      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
-      l[m] = acc;
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) {
+      l[m] = dot_row(hrow + p.Doff[m], p.W[m] + v * p.D[m], p.D[m], p.vec);
     }
-    const float pT = __expf(l[M - 1] - lse[M - 1]);
+    const float lT = exit_at(l, M - 1);
+    const float pT = __expf(lT - lseT);
     const float hot = (v == yt) ? 1.f : 0.f;
-    for (int m = 0; m < M; ++m) {
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) {
       float g;
       if (m == M - 1) {
         g = pT - hot;
@@ -271,15 +332,16 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
           //   Jensen-Shannon p_T (log(p_T/mu_s)/2 - K^p_s), log(p/mu) = ln 2 - softplus(log q - log p);
           //   acceptance p_T (B_s - [q_s >= p_T])
           float extra = 0.f;
-          for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+          for (int s = 0; s < kMaxExits - 1; ++s) if (s < M - 1) {
             float ts;
             if (p.distill == 1) {
               ts = pT - __expf(l[s] - lse[s]);
             } else if (p.distill == 2) {
-              const float lq = l[s] - lse[s], lp = l[M - 1] - lse[M - 1];
+              const float lq = l[s] - lse[s], lp = lT - lseT;
               ts = pT * (0.5f * (kLn2 - softplus(lq - lp)) - stats[(3 * M - 1 + s) * p.T + t]);
             } else if (p.distill == 3) {    // acceptance: p_T (B_s - [q_s >= p_T])
-              const float lq = l[s] - lse[s], lp = l[M - 1] - lse[M - 1];
+              const float lq = l[s] - lse[s], lp = lT - lseT;
               ts = pT * (stats[(3 * M - 1 + s) * p.T + t] - ((lq < lp) ? 0.f : 1.f));
             } else {
               ts = -pT * (l[s] - stats[(2 * M + s) * p.T + t]);
@@ -293,42 +355,64 @@ __global__ void __launch_bounds__(kSimtThreads) simt_grad_kernel(const SimtDev p
         g = __expf(l[m] - lse[m]) - a * pT - (1.f - a) * hot;
       } else if (p.distill == 1) {
         const float q = __expf(l[m] - lse[m]);
-        const float d = (l[m] - lse[m]) - (l[M - 1] - lse[M - 1]) - kl[m];
+        const float d = (l[m] - lse[m]) - (lT - lseT) - kl[m];
         g = (1.f - a) * (q - hot) + a * q * d;
       } else if (p.distill == 2) {
         const float q = __expf(l[m] - lse[m]);
-        const float d = 0.5f * (kLn2 - softplus((l[M - 1] - lse[M - 1]) - (l[m] - lse[m]))) - kl[m];
+        const float d = 0.5f * (kLn2 - softplus((lT - lseT) - (l[m] - lse[m]))) - kl[m];
         g = (1.f - a) * (q - hot) + a * q * d;
       } else {                              // acceptance: q (A - [q < p])
         const float q = __expf(l[m] - lse[m]);
-        const float ind = ((l[m] - lse[m]) < (l[M - 1] - lse[M - 1])) ? 1.f : 0.f;
+        const float ind = ((l[m] - lse[m]) < (lT - lseT)) ? 1.f : 0.f;
         g = (1.f - a) * (q - hot) + a * q * (kl[m] - ind);
       }
       G[(static_cast<int64_t>(m) * p.T + t) * p.V + v] = bad ? 0.f : p.exit_w[m] * g;
     }
   }
   __syncthreads();
-  for (int m = 0; m < M; ++m) {
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) {
     const float* g = G + (static_cast<int64_t>(m) * p.T + t) * p.V;
-    for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) {
-      float acc = 0.f;
-      for (int64_t v = 0; v < p.V; ++v) acc = fmaf(g[v], p.W[m][v * p.D[m] + k], acc);
-      p.dh[m][t * p.D[m] + k] = bad ? 0.f : alpha * acc;
+    const float* __restrict__ Wm = p.W[m];
+    const int64_t D = p.D[m];
+    for (int64_t k = tid; k < D; k += kSimtThreads) {
+      // four partial sums over the vocabulary (independent loads in flight)
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      int64_t v = 0;
+      for (; v + 4 <= p.V; v += 4) {
+        a0 = fmaf(g[v], __ldg(Wm + v * D + k), a0);
+        a1 = fmaf(g[v + 1], __ldg(Wm + (v + 1) * D + k), a1);
+        a2 = fmaf(g[v + 2], __ldg(Wm + (v + 2) * D + k), a2);
+        a3 = fmaf(g[v + 3], __ldg(Wm + (v + 3) * D + k), a3);
+      }
+      for (; v < p.V; ++v) a0 = fmaf(g[v], __ldg(Wm + v * D + k), a0);
+      p.dh[m][t * D + k] = bad ? 0.f : alpha * ((a0 + a1) + (a2 + a3));
     }
   }
   if (tid == 0 && bad) set_flag(p.status, MLS_DEVFLAG_BAD_ID);
 }
 
 // dW^m[v] (+)= alpha * sum_t G'_m[t, v] h_m[t], one block per (v, m).
-__global__ void __launch_bounds__(kSimtThreads) simt_dw_kernel(const SimtDev p, float alpha, const float* __restrict__ G,
+__global__ void __launch_bounds__(kSimtThreads, 1) simt_dw_kernel(const SimtDev p, float alpha, const float* __restrict__ G,
                                                                int accumulate) {
   const int64_t v = blockIdx.x;
   const int m = blockIdx.y;
   const float* g = G + static_cast<int64_t>(m) * p.T * p.V + v;
-  for (int64_t k = threadIdx.x; k < p.D[m]; k += kSimtThreads) {
-    float acc = 0.f;
-    for (int64_t t = 0; t < p.T; ++t) acc = fmaf(g[t * p.V], p.h[m][t * p.D[m] + k], acc);
-    float* out = p.dW[m] + v * p.D[m] + k;
+  const float* __restrict__ hm = p.h[m];
+  const int64_t D = p.D[m], V = p.V;
+  for (int64_t k = threadIdx.x; k < D; k += kSimtThreads) {
+    // four partial sums over the tokens (independent loads in flight)
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int64_t t = 0;
+    for (; t + 4 <= p.T; t += 4) {
+      a0 = fmaf(g[t * V], __ldg(hm + t * D + k), a0);
+      a1 = fmaf(g[(t + 1) * V], __ldg(hm + (t + 1) * D + k), a1);
+      a2 = fmaf(g[(t + 2) * V], __ldg(hm + (t + 2) * D + k), a2);
+      a3 = fmaf(g[(t + 3) * V], __ldg(hm + (t + 3) * D + k), a3);
+    }
+    for (; t < p.T; ++t) a0 = fmaf(g[t * V], __ldg(hm + t * D + k), a0);
+    const float acc = (a0 + a1) + (a2 + a3);
+    float* out = p.dW[m] + v * D + k;
     *out = accumulate ? *out + alpha * acc : alpha * acc;
   }
 }
@@ -358,8 +442,10 @@ __global__ void __launch_bounds__(1024) loss_reduce_kernel(const float* __restri
   }
   if (tid == 0) {
     float L = ew.w[M - 1] * tot[M - 1];
-    for (int m = 0; m < M; ++m) losses[m] = tot[m];
-    for (int s = 0; s < M - 1; ++s) {
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) losses[m] = tot[m];
+#pragma unroll
+    for (int s = 0; s < kMaxExits - 1; ++s) if (s < M - 1) {
       losses[M + s] = tot[M + s];
       L += ew.w[s] * ((1.f - alpha_d) * tot[s] + alpha_d * tot[M + s]);
     }
@@ -387,7 +473,7 @@ __global__ void __launch_bounds__(1024) row_means_kernel(const float* __restrict
 // Agreement of every smaller exit with the largest, one block per token, with
 // the normalisers from the forward statistics: sum_v min(q_m, p_T),
 // sum_v p_T l_m, sum_v p_T l_T and the first maximum of each exit's logits.
-__global__ void __launch_bounds__(kSimtThreads) simt_agree_kernel(const SimtDev p, const float* __restrict__ stats,
+__global__ void __launch_bounds__(kSimtThreads, 1) simt_agree_kernel(const SimtDev p, const float* __restrict__ stats,
                                                                   float* __restrict__ terms,
                                                                   int32_t* __restrict__ top1) {
   extern __shared__ float sm[];
@@ -397,40 +483,45 @@ __global__ void __launch_bounds__(kSimtThreads) simt_agree_kernel(const SimtDev 
   const int tid = threadIdx.x;
   float* hrow = sm;
   int64_t hsum = 0;
-  for (int m = 0; m < M; ++m) hsum += p.D[m];
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) hsum += p.D[m];
   float* red = sm + hsum;                     // [2S + 1 + M][kSimtThreads] floats
   int* redi = reinterpret_cast<int*>(red + (2 * S + 1 + M) * kSimtThreads);   // [M][kSimtThreads]
-  for (int m = 0; m < M; ++m)
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M)
     for (int64_t k = tid; k < p.D[m]; k += kSimtThreads) hrow[p.Doff[m] + k] = p.h[m][t * p.D[m] + k];
   __syncthreads();
   float lse[kMaxExits];
-  for (int m = 0; m < M; ++m) lse[m] = stats[m * p.T + t];
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) lse[m] = stats[m * p.T + t];
+  const float lseT = exit_at(lse, M - 1);
   float beta[kMaxExits - 1] = {0.f, 0.f, 0.f}, sl[kMaxExits - 1] = {0.f, 0.f, 0.f}, st = 0.f;
   float mx[kMaxExits] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   int ix[kMaxExits] = {-1, -1, -1, -1};
   for (int64_t v = tid; v < p.V; v += kSimtThreads) {
     float l[kMaxExits];
-    for (int m = 0; m < M; ++m) {
-      const float* w = p.W[m] + v * p.D[m];
-      const float* hh = hrow + p.Doff[m];
-      float acc = 0.f;
-      for (int64_t k = 0; k < p.D[m]; ++k) acc = fmaf(hh[k], w[k], acc);
-      l[m] = acc;
-      if (acc > mx[m]) { mx[m] = acc; ix[m] = static_cast<int>(v); }
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) {
+      l[m] = dot_row(hrow + p.Doff[m], p.W[m] + v * p.D[m], p.D[m], p.vec);
+      if (l[m] > mx[m]) { mx[m] = l[m]; ix[m] = static_cast<int>(v); }
     }
-    const float pT = __expf(l[M - 1] - lse[M - 1]);
-    st = fmaf(pT, l[M - 1], st);
-    for (int s = 0; s < S; ++s) {
+    const float lT = exit_at(l, M - 1);
+    const float pT = __expf(lT - lseT);
+    st = fmaf(pT, lT, st);
+#pragma unroll
+    for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
       beta[s] += fminf(__expf(l[s] - lse[s]), pT);
       sl[s] = fmaf(pT, l[s], sl[s]);
     }
   }
-  for (int s = 0; s < S; ++s) {
+#pragma unroll
+  for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
     red[s * kSimtThreads + tid] = beta[s];
     red[(S + s) * kSimtThreads + tid] = sl[s];
   }
   red[2 * S * kSimtThreads + tid] = st;
-  for (int m = 0; m < M; ++m) {
+#pragma unroll
+  for (int m = 0; m < kMaxExits; ++m) if (m < M) {
     red[(2 * S + 1 + m) * kSimtThreads + tid] = mx[m];
     redi[m * kSimtThreads + tid] = ix[m];
   }
@@ -439,7 +530,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_agree_kernel(const SimtDev 
     if (tid < stride) {
       const int o = tid + stride;
       for (int q = 0; q < 2 * S + 1; ++q) red[q * kSimtThreads + tid] += red[q * kSimtThreads + o];
-      for (int m = 0; m < M; ++m) {
+#pragma unroll
+      for (int m = 0; m < kMaxExits; ++m) if (m < M) {
         float* mv = red + (2 * S + 1 + m) * kSimtThreads;
         int* iv = redi + m * kSimtThreads;
         // larger value wins; on equal values the smaller vocabulary index
@@ -452,11 +544,13 @@ __global__ void __launch_bounds__(kSimtThreads) simt_agree_kernel(const SimtDev 
     __syncthreads();
   }
   if (tid == 0) {
-    for (int m = 0; m < M; ++m) top1[m * p.T + t] = redi[m * kSimtThreads];
+#pragma unroll
+    for (int m = 0; m < kMaxExits; ++m) if (m < M) top1[m * p.T + t] = redi[m * kSimtThreads];
     const float stT = red[2 * S * kSimtThreads];
-    for (int s = 0; s < S; ++s) {
+#pragma unroll
+    for (int s = 0; s < kMaxExits - 1; ++s) if (s < S) {
       terms[s * p.T + t] = red[s * kSimtThreads];
-      terms[(S + s) * p.T + t] = (stT - red[(S + s) * kSimtThreads]) + (lse[s] - lse[M - 1]);
+      terms[(S + s) * p.T + t] = (stT - red[(S + s) * kSimtThreads]) + (lse[s] - lseT);
       terms[(2 * S + s) * p.T + t] = (redi[s * kSimtThreads] == redi[(M - 1) * kSimtThreads]) ? 1.f : 0.f;
     }
   }
@@ -481,6 +575,9 @@ SimtDev make_dev(const LossProblem& p) {
   d.teacher_grad = (p.teacher_grad != 0 && p.M > 1) ? 1 : 0;
   for (int m = 0; m < kMaxExits; ++m) d.exit_w[m] = p.exit_w[m];
   d.status = p.status;
+  d.vec = 1;
+  for (int m = 0; m < p.M; ++m)
+    if (p.D[m] % 4 != 0 || reinterpret_cast<uintptr_t>(p.W[m]) % 16 != 0) d.vec = 0;
   return d;
 }
 
