@@ -101,8 +101,9 @@ cudaError_t scatter_table_grads(const SegIndexDev& ix, bool bf16, int njobs, con
                                 cudaStream_t st, cudaStream_t heavy_st);
 // For every job z < njobs (at most kMaxExits; one launch pair for all):
 //   dW[z][v] -= scale[z] * sum_{t: y_t = v} h[z]_t  (bf16 rows of d_vec[z] 16-byte vectors).
+// The rows of ids with many tokens go to heavy_st (disjoint rows; it may be st).
 cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,
-                                float* const* dW, const float* scale, cudaStream_t st);
+                                float* const* dW, const float* scale, cudaStream_t st, cudaStream_t heavy_st);
 
 // ------------------------------------------------------------------ loss
 struct LossProblem {

@@ -2163,7 +2163,8 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
   err = side.join();
   if (err != cudaSuccess) return err;
   // one-hot part of dW over every token: (1 - alpha_d) for students, 1 for the
-  // teacher; every exit in one launch pair
+  // teacher; every exit in one launch pair, the heavy rows on the side stream
+  // beside the others (disjoint rows of dW)
   int d_vec[kMaxExits];
   float scale[kMaxExits];
   for (int m = 0; m < p.M; ++m) {
@@ -2171,7 +2172,11 @@ cudaError_t loss_tc_bwd(const LossProblem& p, const float* stats, float grad_sca
     d_vec[m] = static_cast<int>(p.D[m] / 8);
     scale[m] = alpha * p.exit_w[m] * cm;
   }
-  return scatter_target_rows(ix, p.M, p.h, d_vec, dW, scale, st);
+  err = side.fork();
+  if (err != cudaSuccess) return err;
+  err = scatter_target_rows(ix, p.M, p.h, d_vec, dW, scale, st, side.stream());
+  if (err != cudaSuccess) return err;
+  return side.join();
 }
 
 }  // namespace mls

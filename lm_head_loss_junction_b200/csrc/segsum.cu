@@ -599,11 +599,11 @@ cudaError_t scatter_table_grad(const SegIndexDev& ix, bool bf16, const void* dy,
 }
 
 cudaError_t scatter_target_rows(const SegIndexDev& ix, int njobs, const void* const* h, const int* d_vec,
-                                float* const* dW, const float* scale, cudaStream_t st) {
+                                float* const* dW, const float* scale, cudaStream_t st, cudaStream_t heavy_st) {
   SegJobs jobs{};
   for (int z = 0; z < njobs; ++z)
     jobs.j[z] = SegJob{static_cast<const uint4*>(h[z]), d_vec[z], 0, d_vec[z], nullptr, dW[z], scale[z], nullptr};
-  return launch_segsum<true, false>(ix, jobs, njobs, 1, st, st);
+  return launch_segsum<true, false>(ix, jobs, njobs, 1, st, heavy_st);
 }
 
 }  // namespace mls
