@@ -107,6 +107,55 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def cublas_calibration(step, run_loss_fwd, stream, device, seconds=1.0):
+    """The forward's logits GEMMs through cuBLAS (torch.matmul: the same bf16
+    operands, fp32 accumulation, bf16 logits out) against the library's loss
+    forward call, each repeated for about `seconds` (a sustained load under
+    the power cap, like the step), interleaved twice, with the SM clock
+    sampled during each.  A same-box, same-clock denominator for the
+    forward's fraction; cuBLAS is timed here only, never on the path."""
+    c = step.cfg
+    outs = [torch.empty(c.T, c.V, dtype=torch.bfloat16, device=device) for _ in range(c.M)]
+
+    def cublas():
+        for m in range(c.M):
+            torch.matmul(step.o[m], step.W[m].t(), out=outs[m])
+
+    flops = 2.0 * c.T * c.V * sum(c.D)
+
+    def sustained(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        n = max(3, int(seconds * 1000.0 / max(e0.elapsed_time(e1), 1e-3)))
+        with ClockSampler(device.index) as clk:
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / n, clk.summary()["sm_mhz"]
+
+    arms = {"cublas": [], "loss_fwd": []}
+    for _ in range(2):
+        arms["cublas"].append(sustained(cublas))
+        arms["loss_fwd"].append(sustained(run_loss_fwd))
+    del outs
+    out = {"what": "the forward's logits GEMMs through cuBLAS (bf16, fp32 accumulation) against "
+                   "mls_multiexit_loss_fwd, each sustained for ~1 s, interleaved twice"}
+    for k, v in arms.items():
+        ms = statistics.mean(t for t, _ in v)
+        mhz = [f for _, f in v if f is not None]
+        out[k] = {"ms": ms, "tflops": flops / (ms / 1000.0) / 1e12,
+                  "sm_mhz": statistics.mean(mhz) if mhz else None}
+    out["loss_fwd_vs_cublas"] = out["cublas"]["ms"] / out["loss_fwd"]["ms"]
+    return out
+
+
 # ---------------------------------------------------------------- the step
 class Step:
     """Device-resident inputs, outputs and workspaces of one hot-path step."""
@@ -601,6 +650,11 @@ def main():
             "ms": ms_a, "tflops": 2.0 * c.T * c.V * sum(c.D) / (ms_a / 1000.0) / 1e12,
             "beta_mean": vals[:S], "kl_mean": vals[S:2 * S], "top1_agree_mean": vals[2 * S:],
             "what": "each smaller exit vs the largest: acceptance sum_v min(q,p), KL(p||q), top-1 agreement"}
+
+    # ---------------- the forward against cuBLAS GEMMs of the same shapes, same box
+    if ws == 1 and c.dtype == "bf16":
+        extras["cublas_calibration"] = cublas_calibration(step, runners[1], stream, device)
+        barrier()
 
     # ---------------- each junction kernel alone: 24 back-to-back launches rotating
     # over enough copies of the streamed rows (o, dy in; y, do, de out) that they
