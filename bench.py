@@ -107,19 +107,29 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def cublas_calibration(step, run_loss_fwd, stream, device, seconds=1.0):
-    """The forward's logits GEMMs through cuBLAS (torch.matmul: the same bf16
-    operands, fp32 accumulation, bf16 logits out) against the library's loss
-    forward call, each repeated for about `seconds` (a sustained load under
-    the power cap, like the step), interleaved twice, with the SM clock
-    sampled during each.  A same-box, same-clock denominator for the
-    forward's fraction; cuBLAS is timed here only, never on the path."""
+def cublas_calibration(step, run_loss_fwd, run_loss_bwd, stream, device, seconds=1.0):
+    """cuBLAS GEMMs of the loss's shapes (torch.matmul: the same bf16 operands,
+    fp32 accumulation, bf16 out) against the library's calls, each repeated
+    for about `seconds` (a sustained load under the power cap, like the
+    step), interleaved twice, with the SM clock sampled during each.
+    Forward: the logits GEMM of every exit against mls_multiexit_loss_fwd.
+    Backward: per exit the logits GEMM, G W (dh) and G^T h (dW), with the
+    logits standing in for G, against mls_multiexit_loss_bwd.  A same-box,
+    same-clock denominator; cuBLAS is timed here only, never on the path."""
     c = step.cfg
     outs = [torch.empty(c.T, c.V, dtype=torch.bfloat16, device=device) for _ in range(c.M)]
+    dh = [torch.empty(c.T, d, dtype=torch.bfloat16, device=device) for d in c.D]
+    dW = [torch.empty(c.V, d, dtype=torch.bfloat16, device=device) for d in c.D]
 
     def cublas():
         for m in range(c.M):
             torch.matmul(step.o[m], step.W[m].t(), out=outs[m])
+
+    def cublas_bwd():
+        for m in range(c.M):
+            torch.matmul(step.o[m], step.W[m].t(), out=outs[m])
+            torch.matmul(outs[m], step.W[m], out=dh[m])
+            torch.matmul(outs[m].t(), step.o[m], out=dW[m])
 
     flops = 2.0 * c.T * c.V * sum(c.D)
 
@@ -140,19 +150,24 @@ def cublas_calibration(step, run_loss_fwd, stream, device, seconds=1.0):
             torch.cuda.synchronize(device)
         return e0.elapsed_time(e1) / n, clk.summary()["sm_mhz"]
 
-    arms = {"cublas": [], "loss_fwd": []}
+    arms = {"cublas": [], "loss_fwd": [], "cublas_bwd": [], "loss_bwd": []}
     for _ in range(2):
         arms["cublas"].append(sustained(cublas))
         arms["loss_fwd"].append(sustained(run_loss_fwd))
-    del outs
-    out = {"what": "the forward's logits GEMMs through cuBLAS (bf16, fp32 accumulation) against "
-                   "mls_multiexit_loss_fwd, each sustained for ~1 s, interleaved twice"}
+        arms["cublas_bwd"].append(sustained(cublas_bwd))
+        arms["loss_bwd"].append(sustained(run_loss_bwd))
+    del outs, dh, dW
+    out = {"what": "cuBLAS bf16 GEMMs of the loss's shapes (forward: the logits of every exit; backward: "
+                   "logits, dh and dW of every exit) against mls_multiexit_loss_fwd / _bwd, each sustained "
+                   "for ~1 s, interleaved twice"}
     for k, v in arms.items():
         ms = statistics.mean(t for t, _ in v)
         mhz = [f for _, f in v if f is not None]
-        out[k] = {"ms": ms, "tflops": flops / (ms / 1000.0) / 1e12,
+        n = 3.0 if k.endswith("bwd") else 1.0
+        out[k] = {"ms": ms, "tflops": n * flops / (ms / 1000.0) / 1e12,
                   "sm_mhz": statistics.mean(mhz) if mhz else None}
     out["loss_fwd_vs_cublas"] = out["cublas"]["ms"] / out["loss_fwd"]["ms"]
+    out["loss_bwd_vs_cublas"] = out["cublas_bwd"]["ms"] / out["loss_bwd"]["ms"]
     return out
 
 
@@ -653,7 +668,7 @@ def main():
 
     # ---------------- the forward against cuBLAS GEMMs of the same shapes, same box
     if ws == 1 and c.dtype == "bf16":
-        extras["cublas_calibration"] = cublas_calibration(step, runners[1], stream, device)
+        extras["cublas_calibration"] = cublas_calibration(step, runners[1], runners[2], stream, device)
         barrier()
 
     # ---------------- each junction kernel alone: 24 back-to-back launches rotating
