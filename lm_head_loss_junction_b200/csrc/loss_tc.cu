@@ -403,24 +403,36 @@ __global__ void __launch_bounds__(kLossThreads, 1) loss_tile_kernel(const __grid
           float lse_part = -INFINITY, abar = 0.f;
           if (live) {
             if (j == 0) {
-              // teacher: split max, then p~ = exp(l - max) (fp16 pairs in registers) and their sum
-              float mx = -INFINITY;
+              // teacher, one pass over TMEM: online split max; p~ = exp(l - max) as fp16 pairs
+              // in registers, the pairs of earlier chunks (and their sum) rescaled by the same
+              // fp16 factor when a larger maximum appears
+              float mx = -INFINITY, z = 0.f;
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 float r[32];
                 tmem_ld32(base + c * 32, r);
+                float cm = r[0];
 #pragma unroll
-                for (int k = 0; k < 32; ++k) mx = fmaxf(mx, r[k]);
+                for (int k = 1; k < 32; ++k) cm = fmaxf(cm, r[k]);
                 if (has_tgt && (yl >> 5) == c) {
                   a.stats[static_cast<int64_t>(M + m) * a.ldS + t] = pick32(r, yl & 31, tgt_row);
                 }
-              }
-              const float mxs = mx * kLog2e;
-              float z = 0.f;
+                if (cm > mx) {
+                  const uint32_t sc2 = pack_p2(exp2f((mx - cm) * kLog2e), 0.f);
+                  z *= unpack_p2(sc2).x;
+                  const uint32_t scc = __byte_perm(sc2, sc2, 0x1010);
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                float r[32];
-                tmem_ld32(base + c * 32, r);
+                  for (int c2 = 0; c2 < c; ++c2) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                      uint32_t v;
+                      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(v) : "r"(pt[c2][k]), "r"(scc));
+                      pt[c2][k] = v;
+                    }
+                  }
+                  mx = cm;
+                }
+                const float mxs = mx * kLog2e;
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
                   const float e0 = exp2f(fmaf(r[k], kLog2e, -mxs));
